@@ -1,0 +1,452 @@
+"""Benchmark of the paged decode path on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload C] [--block-size BS]
+    python bench.py --impl reference ...     # the fp64 CPU oracle, same metric
+
+One step = one decode iteration of the whole hot path over one batch:
+pa_reshape_and_cache of each sequence's newest token, then pa_decode over all
+(sequence, head) pairs (and, for the shared-prefix workload, the copy-on-write
+pa_copy_blocks before them).  The default workload is the LLaMA-13B-shaped
+single-layer decode batch (B=32, H=40, D=128, bs=16, context U[256, 2048]).
+
+Under torchrun each rank runs its own batch (a different seed) on its own GPU:
+sequences are independent, so there is no collective on the data path
+("weak" scaling); rank 0 prints one JSON line with the whole-job throughput.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import statistics
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "paged decode attention: KV-cache GB/s (% of HBM peak), seq-heads/s"
+FALLBACK_HBM_GBS = 6650.0
+L2_BYTES = 126 * 2**20
+
+
+def _peak_hbm():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            return float(json.load(f)["hbm_gbs"]), "measured"
+    except Exception:
+        return FALLBACK_HBM_GBS, "fallback"
+
+
+def _decode_kernel_hash():
+    h = hashlib.sha256()
+    for rel in ("paged_kv_cache_481_b200/csrc/decode_kernel.cuh",
+                "paged_kv_cache_481_b200/csrc/ptx.cuh",
+                "paged_kv_cache_481_b200/csrc/pa.cu"):
+        with open(os.path.join(ROOT, rel), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()
+
+
+def _recorded_traffic(workload: str):
+    """DRAM bytes per decode launch from the committed ncu summary, only if
+    it was taken on the current kernel source and this workload."""
+    path = os.path.join(ROOT, "profiles", "decode_traffic.json")
+    try:
+        with open(path) as f:
+            rec = json.load(f)
+    except Exception:
+        return None
+    if rec.get("kernel_sha256") != _decode_kernel_hash() or rec.get("workload") != workload:
+        return None
+    return rec.get("dram_bytes_per_launch")
+
+
+class ClockSampler:
+    """Polls the GPU's SM clock and clock-event reasons through NVML (read
+    only) from a background thread."""
+    REASONS = {0x1: "gpu_idle", 0x2: "applications_clocks_setting", 0x4: "sw_power_cap",
+               0x8: "hw_slowdown", 0x10: "sync_boost", 0x20: "sw_thermal_slowdown",
+               0x40: "hw_thermal_slowdown", 0x80: "hw_power_brake_slowdown",
+               0x100: "display_clock_setting"}
+
+    def __init__(self, device_index: int, period_s: float = 0.005):
+        self.samples = []
+        self.max_mhz = None
+        self.error = None
+        self._stop = threading.Event()
+        self._period = period_s
+        try:
+            import pynvml
+            import torch
+            pynvml.nvmlInit()
+            props = torch.cuda.get_device_properties(device_index)
+            handle = None
+            uuid = getattr(props, "uuid", None)
+            if uuid is not None:
+                try:
+                    handle = pynvml.nvmlDeviceGetHandleByUUID(f"GPU-{uuid}")
+                except Exception:
+                    handle = None
+            if handle is None:
+                handle = pynvml.nvmlDeviceGetHandleByIndex(device_index)
+            self._nvml, self._h = pynvml, handle
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(handle, pynvml.NVML_CLOCK_SM)
+            self._reasons_fn = getattr(pynvml, "nvmlDeviceGetCurrentClocksEventReasons", None) \
+                or pynvml.nvmlDeviceGetCurrentClocksThrottleReasons
+        except Exception as e:  # no NVML: report that instead of guessing
+            self.error = f"{type(e).__name__}: {e}"
+            self._h = None
+        self._thread = threading.Thread(target=self._run, daemon=True)
+
+    def _run(self):
+        while not self._stop.is_set():
+            try:
+                mhz = self._nvml.nvmlDeviceGetClockInfo(self._h, self._nvml.NVML_CLOCK_SM)
+                reasons = int(self._reasons_fn(self._h))
+                self.samples.append((time.perf_counter(), mhz, reasons))
+            except Exception as e:
+                self.error = f"{type(e).__name__}: {e}"
+                return
+            time.sleep(self._period)
+
+    def start(self):
+        if self._h is not None:
+            self._thread.start()
+        return self
+
+    def stop(self):
+        self._stop.set()
+        if self._thread.is_alive():
+            self._thread.join()
+
+    def summary(self, t0: float, t1: float):
+        inside = [s for s in self.samples if t0 <= s[0] <= t1]
+        if not inside:   # very short timed region: fall back to the whole window
+            inside = self.samples
+        if not inside:
+            return {"sm_mhz": None, "sm_max_mhz": self.max_mhz, "reasons": [],
+                    "samples": 0, "error": self.error}
+        bits = 0
+        for s in inside:
+            bits |= s[2]
+        names = [n for b, n in self.REASONS.items() if bits & b and n != "gpu_idle"]
+        return {"sm_mhz": statistics.median(s[1] for s in inside), "sm_max_mhz": self.max_mhz,
+                "reasons": names, "samples": len(inside)}
+
+
+def _workload_desc(wl, cfg):
+    from paged_kv_cache_481_b200 import workloads
+    return {
+        "workload": workloads.WORKLOAD_NAMES[cfg] if cfg != 5 else
+        f"{workloads.WORKLOAD_NAMES[5]} (bs={wl.block_size})",
+        "num_seqs": wl.num_seqs, "num_heads": wl.num_heads, "head_dim": wl.head_dim,
+        "block_size": wl.block_size, "num_blocks": wl.num_blocks,
+        "mean_context_len": float(np.mean(wl.context_lens)),
+        "max_context_len": wl.max_context_len, "seed": wl.seed,
+    }
+
+
+def _cpu_sample(wl, max_units: int, seqs=None):
+    """Host inputs for the oracle on a bounded sample: the first sequences'
+    blocks extracted from the pool (renumbered), and the first `max_units`
+    (sequence, head) pairs of them."""
+    import torch
+    if seqs is None:
+        seqs = np.arange(min(wl.num_seqs, max(1, math.ceil(max_units / wl.num_heads))))
+    tables = wl.block_tables[seqs]
+    ids = np.unique(tables[tables >= 0])
+    remap = np.full(wl.num_blocks, -1, np.int64)
+    remap[ids] = np.arange(len(ids))
+    sub_tables = np.where(tables >= 0, remap[np.maximum(tables, 0)], -1).astype(np.int32)
+    idx = torch.from_numpy(ids).to(wl.k_cache.device)
+    kc = wl.k_cache.index_select(0, idx).cpu().numpy()
+    vc = wl.v_cache.index_select(0, idx).cpu().numpy()
+    return dict(q=wl.q[seqs].cpu().numpy(), kc=kc, vc=vc, tables=sub_tables,
+                lens=wl.context_lens[seqs].copy(), scale=wl.scale)
+
+
+def _time_oracle(sample, reps: int = 1):
+    import oracle
+    t = []
+    for _ in range(reps):
+        t0 = time.perf_counter()
+        oracle.paged_decode(sample["q"], sample["kc"], sample["vc"], sample["tables"],
+                            sample["lens"], sample["scale"])
+        t.append(time.perf_counter() - t0)
+    return statistics.median(t)
+
+
+def cpu_baseline(wl, target_s: float = 10.0):
+    """The oracle as it stands, on the host cores, on a bounded sample of the
+    same workload; GB/s over the sample's algorithmic bytes."""
+    import oracle
+    from paged_kv_cache_481_b200 import accounting
+    probe = _cpu_sample(wl, wl.num_heads)                       # one sequence
+    t1 = _time_oracle(probe)
+    per_seq = max(t1, 1e-4)
+    nseq = int(min(wl.num_seqs, max(1, target_s / per_seq)))
+    sample = _cpu_sample(wl, nseq * wl.num_heads)
+    t = _time_oracle(sample)
+    nbytes = accounting.decode_bytes(sample["lens"], wl.num_heads, wl.head_dim)
+    return {"value": nbytes / t / 1e9, "unit": "GB/s", "cores": oracle.num_threads(),
+            "kind": "oracle",
+            "sample": f"first {len(sample['lens'])} of {wl.num_seqs} sequences x {wl.num_heads} "
+                      f"heads (decode only, fp64), {t:.2f} s wall"}
+
+
+def run_reference(args):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return 0
+    import oracle
+    from paged_kv_cache_481_b200 import accounting, workloads
+    import torch
+    cfg = args.workload
+    wl = workloads.make_workload(cfg, device="cpu" if not torch.cuda.is_available() else "cuda",
+                                 seed=cfg, block_size=args.block_size)
+    # size each step's sample so that warm-up + timed steps stay within ~2 min
+    probe = _cpu_sample(wl, wl.num_heads)
+    t1 = max(_time_oracle(probe), 1e-4)
+    budget = 120.0 / max(1, args.steps + args.warmup)
+    nseq = int(max(1, min(wl.num_seqs, budget / t1)))
+    if nseq == 1 and t1 > budget:
+        units = max(1, int(wl.num_heads * budget / t1))
+        sample = _cpu_sample(wl, units, seqs=np.arange(1))
+        sample["q"] = sample["q"][:, :units].copy()
+        sample["kc"] = np.ascontiguousarray(sample["kc"][:, :units])
+        sample["vc"] = np.ascontiguousarray(sample["vc"][:, :units])
+        heads = units
+    else:
+        sample = _cpu_sample(wl, nseq * wl.num_heads)
+        heads = wl.num_heads
+    for _ in range(args.warmup):
+        _time_oracle(sample)
+    times = [_time_oracle(sample) for _ in range(args.steps)]
+    total = sum(times)
+    nbytes = accounting.decode_bytes(sample["lens"], heads, wl.head_dim)
+    value = nbytes * args.steps / total / 1e9
+    desc = (f"per step: {len(sample['lens'])} of {wl.num_seqs} sequences x {heads} heads "
+            f"(decode only, fp64 oracle)")
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "GB/s",
+        "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": total / args.steps * 1e3, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": _workload_desc(wl, cfg),
+        "seq_heads_per_s": len(sample["lens"]) * heads * args.steps / total,
+        "cpu_baseline": {"value": value, "unit": "GB/s", "cores": oracle.num_threads(),
+                         "kind": "oracle", "sample": desc},
+        "e2e": {"value": value, "unit": "GB/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def run_gpu(args):
+    import torch
+    import torch.distributed as dist
+    from paged_kv_cache_481_b200 import accounting, binding, build, workloads
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world != args.gpus:
+        raise SystemExit(f"--gpus {args.gpus} but WORLD_SIZE={world}")
+    torch.cuda.set_device(local)
+    if world > 1:
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+    build.build()
+    binding.load()
+
+    cfg = args.workload
+    wl = workloads.make_workload(cfg, device="cuda", seed=cfg + 100 * rank,
+                                 block_size=args.block_size)
+    dev = torch.device("cuda", local)
+    stream = torch.cuda.Stream(device=dev)
+    b, h, d = wl.num_seqs, wl.num_heads, wl.head_dim
+    q = wl.q
+    kc, vc = wl.k_cache, wl.v_cache
+    key, value = wl.new_key, wl.new_value
+    slots = torch.from_numpy(wl.slot_mapping).to(dev)
+    tables = torch.from_numpy(np.ascontiguousarray(wl.block_tables)).to(dev)
+    lens = torch.from_numpy(wl.context_lens).to(dev)
+    pairs = torch.from_numpy(wl.copy_pairs).to(dev) if len(wl.copy_pairs) else None
+    out = torch.empty_like(q)
+    mcl = wl.max_context_len
+    ws = binding.new_workspace(b, h, d, mcl, device=dev)
+    torch.cuda.synchronize()
+
+    def step(ev_pair=None):
+        if pairs is not None:
+            binding.pa_copy_blocks(kc, vc, pairs, stream=stream)
+        binding.pa_reshape_and_cache(key, value, kc, vc, slots, stream=stream)
+        if ev_pair is not None:
+            ev_pair[0].record(stream)
+        binding.pa_decode(out, q, kc, vc, tables, lens, mcl, wl.scale, ws, stream=stream)
+        if ev_pair is not None:
+            ev_pair[1].record(stream)
+
+    launches_per_step = 2 + (1 if pairs is not None else 0)
+    with torch.cuda.stream(stream):
+        for _ in range(args.warmup):
+            step()
+    torch.cuda.synchronize()
+    assert binding.pa_get_last_device_error() == 0
+
+    sampler = ClockSampler(local).start()
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+           for _ in range(args.steps)]
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    w0 = time.perf_counter()
+    start.record(stream)
+    with torch.cuda.stream(stream):
+        for i in range(args.steps):
+            step(evs[i])
+    end.record(stream)
+    torch.cuda.synchronize()
+    w1 = time.perf_counter()
+    if world > 1:
+        dist.barrier()
+    sampler.stop()
+    ms = start.elapsed_time(end)
+    decode_ms = [a.elapsed_time(z) for a, z in evs]
+    assert binding.pa_get_last_device_error() == 0
+
+    # end to end: per-step inputs from pinned host buffers, output back to host
+    h_q = q.cpu().pin_memory()
+    h_key, h_value = key.cpu().pin_memory(), value.cpu().pin_memory()
+    h_slots = slots.cpu().pin_memory()
+    h_tables, h_lens = tables.cpu().pin_memory(), lens.cpu().pin_memory()
+    h_out = torch.empty(out.shape, dtype=out.dtype, pin_memory=True)
+    d_q, d_key, d_value = torch.empty_like(q), torch.empty_like(key), torch.empty_like(value)
+    d_slots, d_tables, d_lens = (torch.empty_like(slots), torch.empty_like(tables),
+                                 torch.empty_like(lens))
+    h2d = sum(t.numel() * t.element_size() for t in (h_q, h_key, h_value, h_slots, h_tables,
+                                                     h_lens))
+    d2h = h_out.numel() * h_out.element_size()
+
+    def e2e_step():
+        for dst, src in ((d_q, h_q), (d_key, h_key), (d_value, h_value), (d_slots, h_slots),
+                         (d_tables, h_tables), (d_lens, h_lens)):
+            dst.copy_(src, non_blocking=True)
+        if pairs is not None:
+            binding.pa_copy_blocks(kc, vc, pairs, stream=stream)
+        binding.pa_reshape_and_cache(d_key, d_value, kc, vc, d_slots, stream=stream)
+        binding.pa_decode(out, d_q, kc, vc, d_tables, d_lens, mcl, wl.scale, ws, stream=stream)
+        h_out.copy_(out, non_blocking=True)
+
+    with torch.cuda.stream(stream):
+        for _ in range(max(3, args.warmup)):
+            e2e_step()
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    with torch.cuda.stream(stream):
+        for _ in range(args.steps):
+            e2e_step()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = e0.elapsed_time(e1)
+    if world > 1:
+        dist.barrier()
+
+    dec_bytes = accounting.decode_bytes(wl.context_lens, h, d)
+    step_bytes = dec_bytes + accounting.cache_write_bytes(b, h, d)
+    if pairs is not None:
+        step_bytes += accounting.copy_blocks_bytes(len(wl.copy_pairs), h, d, wl.block_size)
+
+    # max over ranks of the device-timed regions; totals over ranks
+    stats = torch.tensor([ms, e2e_ms], dtype=torch.float64, device=dev)
+    tot = torch.tensor([float(step_bytes), float(b * h)], dtype=torch.float64, device=dev)
+    if world > 1:
+        dist.all_reduce(stats, op=dist.ReduceOp.MAX)
+        dist.all_reduce(tot, op=dist.ReduceOp.SUM)
+    ms, e2e_ms = stats.tolist()
+    total_bytes, total_units = tot.tolist()
+
+    result = None
+    if rank == 0:
+        peak, peak_kind = _peak_hbm()
+        mean_dec_ms = statistics.fmean(decode_ms)
+        achieved = dec_bytes / (mean_dec_ms * 1e-3) / 1e9
+        clocks = sampler.summary(w0, w1)
+        desc = _workload_desc(wl, cfg)
+        kv_bytes = dec_bytes
+        desc.update({
+            "step": ("pa_copy_blocks + " if pairs is not None else "")
+                    + f"pa_reshape_and_cache({b} tokens) + pa_decode",
+            "l2": f"inputs larger than L2: {kv_bytes / 1e9:.2f} GB of K/V read per step "
+                  f"vs {L2_BYTES / 2**20:.0f} MiB L2 (no flush)",
+            "partition_size": binding.pa_decode_partition_size(b, h, d, mcl),
+            "parallelism": f"dp{world} (independent batches per GPU)",
+        })
+        result = {
+            "metric": METRIC,
+            "value": total_bytes * args.steps / (ms * 1e-3) / 1e9,
+            "unit": "GB/s",
+            "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": ms / args.steps,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "dtype": "f32", "storage_dtype": "f16", "data": "synthetic",
+            "config": desc,
+            "seq_heads_per_s": total_units * args.steps / (ms * 1e-3),
+            "hbm_frac": achieved / peak,
+            "decode_us_mean": mean_dec_ms * 1e3,
+            "decode_us_median": statistics.median(decode_ms) * 1e3,
+            "roofline": {
+                "kernel": "paged_decode_kernel", "bound": "hbm", "achieved": achieved,
+                "peak": peak, "peak_kind": f"{peak_kind} (hbm_gbs)", "unit": "GB/s",
+                "frac": achieved / peak, "traffic": _recorded_traffic(desc["workload"]),
+                "algorithmic_bytes_per_launch": dec_bytes,
+            },
+            "e2e": {"value": total_bytes * args.steps / (e2e_ms * 1e-3) / 1e9, "unit": "GB/s",
+                    "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+                    "ms_per_step": e2e_ms / args.steps},
+            "gpu_launches": launches_per_step * args.steps,
+            "clocks": clocks,
+        }
+        if world == 1 and not args.no_cpu_baseline:
+            result["cpu_baseline"] = cpu_baseline(wl, target_s=args.cpu_seconds)
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    if result is not None:
+        print(json.dumps(result), flush=True)
+    return 0
+
+
+def main(argv=None):
+    ap = argparse.ArgumentParser(description=__doc__.splitlines()[0])
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=1000)
+    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", type=int, default=2, choices=[1, 2, 3, 4, 5])
+    ap.add_argument("--block-size", type=int, default=None)
+    ap.add_argument("--cpu-seconds", type=float, default=10.0)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args(argv)
+    if args.warmup < 3:
+        raise SystemExit("--warmup must be >= 3")
+    if args.impl == "reference":
+        return run_reference(args)
+    return run_gpu(args)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

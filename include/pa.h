@@ -1,0 +1,160 @@
+/*
+ * pa.h — C ABI of libpa, the B200 (sm_100a) PagedAttention decode path.
+ *
+ * The operations follow the pages on PagedAttention:
+ *   - comfyai.app "6.4 PagedAttention", 6.4.1 Mechanism: each sequence's
+ *     K/V cache is split into blocks of a fixed number of tokens; a block
+ *     table maps the sequence's logically contiguous blocks onto physically
+ *     non-contiguous blocks of one pool.
+ *   - polomodov.tech "vLLM and PagedAttention", slide 9 (the attention kernel
+ *     fetches K and V from non-contiguous blocks by their addresses), slide 10
+ *     (block table, logical -> physical), slide 11 (a new token goes into the
+ *     next free slot; a new block is taken only when the last one is full),
+ *     slide 13 (copy-on-write duplicates only the last block).
+ *   - brentwoodlivery.com "5.3.18 LLM serving, vLLM, quantized inference":
+ *     paging changes only the memory layout, not the attention arithmetic.
+ *
+ * Layouts (row-major, fp16 = IEEE binary16):
+ *   q, out            [num_seqs, num_heads, head_dim]           fp16
+ *   key, value        [num_tokens, num_heads, head_dim]         fp16
+ *   k_cache, v_cache  [num_blocks, num_heads, block_size, head_dim] fp16
+ *                     element (p, h, j, d) at ((p*H + h)*bs + j)*D + d
+ *   block_tables      [num_seqs, max_blocks_per_seq]            int32
+ *   context_lens      [num_seqs]                                int32
+ *   slot_mapping      [num_tokens]   int64, slot = block*bs + offset, <0 = skip
+ *   block_mapping     [num_pairs, 2] int64, (src, dst) physical block ids
+ *
+ * Ownership and execution: every array argument is a DEVICE pointer owned by
+ * the caller, and must stay valid until the work on `stream` has finished.
+ * The library never allocates device memory.  Calls only validate arguments
+ * on the host and enqueue kernels on `stream` (asynchronous); PA_OK means the
+ * launch was accepted.  fp16 arrays and the workspace must be 16-byte aligned.
+ *
+ * Errors: host-detectable problems return a status and launch nothing.
+ * Out-of-range indices found on the device (block id >= num_blocks, slot past
+ * the pool, context_lens[b] outside [0, max_context_len], a bad copy pair) are
+ * never dereferenced: the access is skipped, the affected result is
+ * unspecified, and a bit is set in a per-device error word read (and
+ * cleared) by pa_get_last_device_error().
+ */
+#ifndef PA_H
+#define PA_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define PA_API __attribute__((visibility("default")))
+#else
+#define PA_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Same type as the CUDA runtime's cudaStream_t; NULL = legacy default stream. */
+typedef struct CUstream_st *pa_stream_t;
+
+typedef enum pa_status {
+    PA_OK = 0,
+    PA_ERR_INVALID_ARG = 1,  /* null pointer, negative size, misalignment, lengths too long */
+    PA_ERR_UNSUPPORTED = 2,  /* head_dim not in {64,128} or block_size not in {8,16,32,64,128} */
+    PA_ERR_CUDA = 3,         /* the CUDA runtime refused the launch */
+    PA_ERR_WORKSPACE = 4     /* workspace null or smaller than pa_decode_workspace_size() */
+} pa_status;
+
+/* Bits of the device error word (pa_get_last_device_error). */
+#define PA_DEVERR_BLOCK_ID    1u   /* decode: block table entry outside [0, num_blocks) */
+#define PA_DEVERR_CONTEXT_LEN 2u   /* decode: context_lens[b] < 0 or > max_context_len */
+#define PA_DEVERR_SLOT        4u   /* cache write: slot >= num_blocks * block_size */
+#define PA_DEVERR_COPY_PAIR   8u   /* copy: src or dst outside [0, num_blocks) */
+#define PA_DEVERR_TIMEOUT     16u  /* decode: a shared-memory transfer did not arrive in ~1 s */
+
+/*
+ * Cache write (polomodov.tech slide 11; comfyai.app 6.4.1).  For every token i
+ * with slot = slot_mapping[i] >= 0, copy key[i, h, :] to
+ * k_cache[slot / block_size, h, slot % block_size, :] and value[i, h, :] to
+ * v_cache at the same place, for all heads h.  Negative slots (padding) are
+ * skipped.  Bit-exact copy.  Slots within one call must be distinct (else
+ * which token lands is unspecified).  num_tokens == 0 is a no-op.
+ */
+PA_API pa_status pa_reshape_and_cache(const void *key, const void *value, void *k_cache,
+                               void *v_cache, const int64_t *slot_mapping,
+                               int num_tokens, int num_heads, int head_dim,
+                               int block_size, int num_blocks, pa_stream_t stream);
+
+/*
+ * Bytes of workspace pa_decode needs for these sizes (split-K partial
+ * results and one merge counter per (sequence, head)).  Never 0.
+ */
+PA_API size_t pa_decode_workspace_size(int num_seqs, int num_heads, int head_dim,
+                                int max_context_len);
+
+/*
+ * Zero the workspace's merge counters (a cudaMemsetAsync on `stream`).  Call
+ * once on a fresh workspace before its first pa_decode, and again after
+ * pa_get_last_device_error reported PA_DEVERR_TIMEOUT.  pa_decode leaves the
+ * counters at zero when it completes, so a workspace is reusable across calls
+ * of any size that fits it.
+ */
+PA_API pa_status pa_decode_workspace_init(void *workspace, size_t workspace_bytes,
+                                   pa_stream_t stream);
+
+/*
+ * Tokens per context partition (split-K chunk) pa_decode uses for these
+ * sizes; a sequence of length L is split into ceil(L / partition) partitions.
+ */
+PA_API int pa_decode_partition_size(int num_seqs, int num_heads, int head_dim,
+                             int max_context_len);
+
+/*
+ * Paged single-token decode attention (comfyai.app 6.4.1; polomodov.tech
+ * slides 9-10; brentwoodlivery.com 5.3.18).  For every sequence b and head h,
+ * with L = context_lens[b] and, for t < L,
+ *     K_t = k_cache[block_tables[b][t / bs], h, t % bs, :]   (V_t likewise)
+ *     s_t = scale * sum_d q[b,h,d] * K_t[d]
+ *     out[b,h,:] = sum_t exp(s_t - max s) V_t / sum_t exp(s_t - max s)
+ * computed with fp32 accumulation and written as fp16 (round to nearest even).
+ * L == 0 writes zeros.  Only block_tables[b][0 .. ceil(L/bs)) is read; cache
+ * rows at positions >= L are never used.  max_context_len is a host-side
+ * upper bound of context_lens (it sizes the grid); it must not exceed
+ * max_blocks_per_seq * block_size.  `workspace` (workspace_bytes >=
+ * pa_decode_workspace_size(...), counters zeroed by pa_decode_workspace_init)
+ * holds split-K partials; calls that share a workspace must not overlap on
+ * the GPU.  Results are deterministic (fixed reduction order, no float
+ * atomics), so aliased and copied blocks give bit-identical outputs.
+ */
+PA_API pa_status pa_decode(void *out, const void *q, const void *k_cache, const void *v_cache,
+                    const int32_t *block_tables, int max_blocks_per_seq,
+                    const int32_t *context_lens, int max_context_len, int num_seqs,
+                    int num_heads, int head_dim, int block_size, int num_blocks,
+                    float scale, void *workspace, size_t workspace_bytes,
+                    pa_stream_t stream);
+
+/*
+ * Copy-on-write block copy (comfyai.app 6.4.2-6.4.3; polomodov.tech slide
+ * 13).  For each pair (src, dst): k_cache[dst] = k_cache[src] and
+ * v_cache[dst] = v_cache[src], all num_heads * block_size * head_dim
+ * elements, bit-exact.  dst ids must be distinct and no dst may also be a
+ * src in the same call.  num_pairs == 0 is a no-op.
+ */
+PA_API pa_status pa_copy_blocks(void *k_cache, void *v_cache, const int64_t *block_mapping,
+                         int num_pairs, int num_heads, int head_dim, int block_size,
+                         int num_blocks, pa_stream_t stream);
+
+/* Static description of a status code. */
+PA_API const char *pa_status_string(pa_status status);
+
+/*
+ * Read and clear the current device's error word (PA_DEVERR_* bits; 0 = no
+ * error).  Synchronises with the device.  Returns PA_ERR_CUDA if the read
+ * fails, PA_ERR_INVALID_ARG if code is NULL.
+ */
+PA_API pa_status pa_get_last_device_error(unsigned int *code);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* PA_H */

@@ -36,6 +36,7 @@
  * Return codes: 0 ok, 1 invalid argument, 2 out-of-range block id or slot.
  */
 #include <math.h>
+#include <pthread.h>
 #include <stdint.h>
 #include <stdlib.h>
 #include <string.h>
@@ -61,6 +62,22 @@ double oracle_half_to_double(uint16_t bits)
     else
         v = ldexp((double)(frac + 1024), expo - 25);
     return sign ? -v : v;
+}
+
+/* All 65536 binary16 values, decoded once by oracle_half_to_double (so the
+ * table is that definition evaluated, not a second decoder). */
+static double half_table[1 << 16];
+static pthread_once_t half_table_once = PTHREAD_ONCE_INIT;
+
+static void fill_half_table(void)
+{
+    for (uint32_t i = 0; i < (1u << 16); ++i)
+        half_table[i] = oracle_half_to_double((uint16_t)i);
+}
+
+static inline double h2d(uint16_t bits)
+{
+    return half_table[bits];
 }
 
 /* KV cache size in bytes, brentwoodlivery.com 5.3.18 ("KV cache size bytes
@@ -158,7 +175,7 @@ static int decode_one(double *out, double *probs, double *scores,
         const uint16_t *k = k_cache + ((p * H + h) * bs + t % bs) * D;
         double dot = 0.0;
         for (int64_t d = 0; d < D; ++d)
-            dot += oracle_half_to_double(q[d]) * oracle_half_to_double(k[d]);
+            dot += h2d(q[d]) * h2d(k[d]);
         scores[t] = scale * dot;
         if (scores[t] > m)
             m = scores[t];
@@ -174,7 +191,7 @@ static int decode_one(double *out, double *probs, double *scores,
         int64_t p = table[t / bs];
         const uint16_t *v = v_cache + ((p * H + h) * bs + t % bs) * D;
         for (int64_t d = 0; d < D; ++d)
-            out[d] += scores[t] * oracle_half_to_double(v[d]);
+            out[d] += scores[t] * h2d(v[d]);
     }
     for (int64_t d = 0; d < D; ++d)
         out[d] /= l;
@@ -209,6 +226,7 @@ int oracle_paged_decode(double *out, double *probs, int64_t probs_stride,
             return ORACLE_ERR_ARG;
     }
 
+    pthread_once(&half_table_once, fill_half_table);
     int status = ORACLE_OK;
     const int64_t units = (int64_t)num_seqs * H;
 #pragma omp parallel for schedule(dynamic, 1) reduction(max : status)

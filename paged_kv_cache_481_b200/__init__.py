@@ -6,16 +6,9 @@
 ``pa_copy_blocks`` (copy-on-write block copy).  ``binding`` is a thin ctypes
 layer over it with the same names; it only marshals arguments.
 
-The native library is loaded on first use and there is no fallback: if it
+The native library is loaded on first call and there is no fallback: if it
 is missing or no CUDA device is present, the call raises.
 """
-from . import accounting, workloads  # noqa: F401  (host-side only, no GPU needed)
+from . import accounting, binding, workloads  # noqa: F401
 
-__all__ = ["accounting", "workloads", "binding"]
-
-
-def __getattr__(name):
-    if name == "binding":
-        from . import binding
-        return binding
-    raise AttributeError(name)
+__all__ = ["accounting", "binding", "workloads"]

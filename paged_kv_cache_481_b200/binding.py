@@ -1,0 +1,168 @@
+"""Thin ctypes binding over libpa.so with the C ABI's names.
+
+Argument marshalling only: shapes are read off the tensors, raw device
+pointers and sizes are passed to the C functions declared in include/pa.h,
+and a non-OK status raises ``PAError``.  Every step of the path runs in the
+library's CUDA kernels; there is no CPU or PyTorch fallback, and loading
+fails loudly when libpa.so is missing.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import threading
+
+import torch
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "libpa.so")
+
+PA_OK, PA_ERR_INVALID_ARG, PA_ERR_UNSUPPORTED, PA_ERR_CUDA, PA_ERR_WORKSPACE = range(5)
+PA_DEVERR_BLOCK_ID = 1
+PA_DEVERR_CONTEXT_LEN = 2
+PA_DEVERR_SLOT = 4
+PA_DEVERR_COPY_PAIR = 8
+PA_DEVERR_TIMEOUT = 16
+
+# every symbol include/pa.h declares
+EXPORTED = ("pa_reshape_and_cache", "pa_decode_workspace_size", "pa_decode_workspace_init",
+            "pa_decode_partition_size", "pa_decode", "pa_copy_blocks", "pa_status_string",
+            "pa_get_last_device_error")
+
+_lock = threading.Lock()
+_lib = None
+
+
+class PAError(RuntimeError):
+    def __init__(self, status: int, what: str):
+        self.status = status
+        super().__init__(f"{what}: {status_string(status)} (status {status})")
+
+
+def load(path: str | None = None):
+    """Load libpa.so (once).  Raises if the library is absent."""
+    global _lib
+    with _lock:
+        if _lib is not None and path is None:
+            return _lib
+        p = path or LIB_PATH
+        if not os.path.exists(p):
+            raise RuntimeError(f"libpa.so not built at {p}: run "
+                               "`python -m paged_kv_cache_481_b200.build`")
+        lib = ctypes.CDLL(p)
+        vp, i32, sz = ctypes.c_void_p, ctypes.c_int, ctypes.c_size_t
+        lib.pa_reshape_and_cache.argtypes = [vp, vp, vp, vp, vp, i32, i32, i32, i32, i32, vp]
+        lib.pa_reshape_and_cache.restype = i32
+        lib.pa_decode_workspace_size.argtypes = [i32, i32, i32, i32]
+        lib.pa_decode_workspace_size.restype = sz
+        lib.pa_decode_workspace_init.argtypes = [vp, sz, vp]
+        lib.pa_decode_workspace_init.restype = i32
+        lib.pa_decode_partition_size.argtypes = [i32, i32, i32, i32]
+        lib.pa_decode_partition_size.restype = i32
+        lib.pa_decode.argtypes = [vp, vp, vp, vp, vp, i32, vp, i32, i32, i32, i32, i32, i32,
+                                  ctypes.c_float, vp, sz, vp]
+        lib.pa_decode.restype = i32
+        lib.pa_copy_blocks.argtypes = [vp, vp, vp, i32, i32, i32, i32, i32, vp]
+        lib.pa_copy_blocks.restype = i32
+        lib.pa_status_string.argtypes = [i32]
+        lib.pa_status_string.restype = ctypes.c_char_p
+        lib.pa_get_last_device_error.argtypes = [ctypes.POINTER(ctypes.c_uint)]
+        lib.pa_get_last_device_error.restype = i32
+        if path is None:
+            _lib = lib
+        return lib
+
+
+def status_string(status: int) -> str:
+    return load().pa_status_string(int(status)).decode()
+
+
+def _check(status: int, what: str):
+    if status != PA_OK:
+        raise PAError(status, what)
+
+
+def _stream(stream) -> ctypes.c_void_p:
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return ctypes.c_void_p(stream.cuda_stream if isinstance(stream, torch.cuda.Stream)
+                           else int(stream))
+
+
+def _ptr(t: torch.Tensor | None) -> ctypes.c_void_p:
+    if t is None:
+        return ctypes.c_void_p(None)
+    if not t.is_cuda:
+        raise ValueError("libpa takes device tensors")
+    if not t.is_contiguous():
+        raise ValueError("libpa takes contiguous tensors")
+    return ctypes.c_void_p(t.data_ptr())
+
+
+def pa_reshape_and_cache(key, value, k_cache, v_cache, slot_mapping, stream=None):
+    """Write each token's K/V row at its slot (negative slots skipped)."""
+    n, h, d = key.shape
+    nb, hk, bs, dk = k_cache.shape
+    assert key.dtype == value.dtype == k_cache.dtype == v_cache.dtype == torch.float16
+    assert slot_mapping.dtype == torch.int64 and slot_mapping.numel() == n
+    assert (hk, dk) == (h, d) and value.shape == key.shape and v_cache.shape == k_cache.shape
+    _check(load().pa_reshape_and_cache(_ptr(key), _ptr(value), _ptr(k_cache), _ptr(v_cache),
+                                       _ptr(slot_mapping), n, h, d, bs, nb, _stream(stream)),
+           "pa_reshape_and_cache")
+
+
+def pa_decode_workspace_size(num_seqs, num_heads, head_dim, max_context_len) -> int:
+    return int(load().pa_decode_workspace_size(num_seqs, num_heads, head_dim, max_context_len))
+
+
+def pa_decode_partition_size(num_seqs, num_heads, head_dim, max_context_len) -> int:
+    return int(load().pa_decode_partition_size(num_seqs, num_heads, head_dim, max_context_len))
+
+
+def pa_decode_workspace_init(workspace: torch.Tensor, stream=None):
+    _check(load().pa_decode_workspace_init(_ptr(workspace), workspace.numel()
+                                           * workspace.element_size(), _stream(stream)),
+           "pa_decode_workspace_init")
+
+
+def new_workspace(num_seqs, num_heads, head_dim, max_context_len, device=None) -> torch.Tensor:
+    """Allocate (through torch) and initialise a decode workspace."""
+    n = pa_decode_workspace_size(num_seqs, num_heads, head_dim, max_context_len)
+    ws = torch.empty(n, dtype=torch.uint8, device=device or "cuda")
+    pa_decode_workspace_init(ws)
+    return ws
+
+
+def pa_decode(out, q, k_cache, v_cache, block_tables, context_lens, max_context_len,
+              scale, workspace, stream=None):
+    """Paged decode attention: out[b, h] = softmax(scale q.K) V over the
+    sequence's blocks.  max_context_len is a host-side bound on context_lens."""
+    b, h, d = q.shape
+    nb, hk, bs, dk = k_cache.shape
+    assert q.dtype == out.dtype == k_cache.dtype == v_cache.dtype == torch.float16
+    assert out.shape == q.shape and (hk, dk) == (h, d) and v_cache.shape == k_cache.shape
+    assert block_tables.dtype == torch.int32 and block_tables.dim() == 2
+    assert context_lens.dtype == torch.int32 and context_lens.numel() == b
+    _check(load().pa_decode(_ptr(out), _ptr(q), _ptr(k_cache), _ptr(v_cache),
+                            _ptr(block_tables), block_tables.shape[1], _ptr(context_lens),
+                            int(max_context_len), b, h, d, bs, nb, float(scale),
+                            _ptr(workspace), workspace.numel() * workspace.element_size(),
+                            _stream(stream)),
+           "pa_decode")
+
+
+def pa_copy_blocks(k_cache, v_cache, block_mapping, stream=None):
+    """Copy whole blocks src -> dst for each (src, dst) row of block_mapping."""
+    nb, h, bs, d = k_cache.shape
+    assert block_mapping.dtype == torch.int64
+    pairs = block_mapping.numel() // 2
+    _check(load().pa_copy_blocks(_ptr(k_cache), _ptr(v_cache), _ptr(block_mapping) if pairs
+                                 else ctypes.c_void_p(None), pairs, h, d, bs, nb,
+                                 _stream(stream)),
+           "pa_copy_blocks")
+
+
+def pa_get_last_device_error() -> int:
+    code = ctypes.c_uint(0)
+    _check(load().pa_get_last_device_error(ctypes.byref(code)), "pa_get_last_device_error")
+    return int(code.value)

@@ -1,0 +1,249 @@
+// libpa: C ABI over the sm_100a PagedAttention kernels.  Host code here only
+// validates arguments, sizes grids and launches; all of the path's arithmetic
+// and data movement runs in the kernels of decode_kernel.cuh and
+// cache_kernels.cuh.  Nothing here allocates device memory.
+#include <cuda_runtime.h>
+
+#include <atomic>
+#include <cmath>
+#include <cstdint>
+
+#include "../../include/pa.h"
+#include "cache_kernels.cuh"
+#include "decode_kernel.cuh"
+
+namespace {
+
+constexpr int kMaxDevices = 64;
+
+bool aligned16(const void *p)
+{
+    return (reinterpret_cast<uintptr_t>(p) & 15u) == 0;
+}
+
+bool supported_head_dim(int d)
+{
+    return d == 64 || d == 128;
+}
+
+bool supported_block_size(int bs)
+{
+    return bs == 8 || bs == 16 || bs == 32 || bs == 64 || bs == 128;
+}
+
+size_t align256(size_t x)
+{
+    return (x + 255) & ~size_t(255);
+}
+
+// Tokens per split-K partition.  A multiple of every tile height (16 or 32
+// rows) and every supported block size, with at most 512/8 + 1 table entries
+// per partition.
+int partition_size_for(int /*num_seqs*/, int /*num_heads*/, int /*head_dim*/, int /*max_context_len*/)
+{
+    return 512;
+}
+
+struct WorkspaceLayout {
+    size_t o_off, ml_off, count_off, total;
+    int max_parts;
+};
+
+WorkspaceLayout workspace_layout(int num_seqs, int num_heads, int head_dim, int max_context_len)
+{
+    WorkspaceLayout w{};
+    const int P = partition_size_for(num_seqs, num_heads, head_dim, max_context_len);
+    w.max_parts = max_context_len > 0 ? (max_context_len + P - 1) / P : 1;
+    const size_t units = size_t(num_seqs) * size_t(num_heads);
+    const size_t parts = w.max_parts > 1 ? size_t(w.max_parts) : 0;
+    w.o_off = 0;
+    w.ml_off = align256(units * parts * size_t(head_dim) * sizeof(float));
+    w.count_off = w.ml_off + align256(units * parts * 2 * sizeof(float));
+    w.total = w.count_off + align256((units > 0 ? units : 1) * sizeof(unsigned));
+    return w;
+}
+
+template <int D, int NW, int S>
+pa_status launch_decode(const pa::DecodeParams &p, int num_seqs, cudaStream_t stream)
+{
+    using Sm = pa::DecodeSmem<D, NW, S>;
+    static std::atomic<bool> configured[kMaxDevices];
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices)
+        return PA_ERR_CUDA;
+    if (!configured[dev].load(std::memory_order_acquire)) {
+        if (cudaFuncSetAttribute(pa::paged_decode_kernel<D, NW, S>,
+                                 cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 int(Sm::kBytes)) != cudaSuccess)
+            return PA_ERR_CUDA;
+        configured[dev].store(true, std::memory_order_release);
+    }
+    const dim3 grid(unsigned(p.max_parts), unsigned(p.num_heads), unsigned(num_seqs));
+    pa::paged_decode_kernel<D, NW, S><<<grid, NW * 32, Sm::kBytes, stream>>>(p);
+    return cudaGetLastError() == cudaSuccess ? PA_OK : PA_ERR_CUDA;
+}
+
+constexpr int kDecodeWarps = 4;
+constexpr int kDecodeStages = 3;
+
+} // namespace
+
+extern "C" {
+
+const char *pa_status_string(pa_status status)
+{
+    switch (status) {
+    case PA_OK: return "ok";
+    case PA_ERR_INVALID_ARG: return "invalid argument";
+    case PA_ERR_UNSUPPORTED: return "unsupported head_dim or block_size";
+    case PA_ERR_CUDA: return "CUDA runtime error";
+    case PA_ERR_WORKSPACE: return "workspace missing or too small";
+    }
+    return "unknown status";
+}
+
+pa_status pa_get_last_device_error(unsigned int *code)
+{
+    if (!code)
+        return PA_ERR_INVALID_ARG;
+    if (cudaDeviceSynchronize() != cudaSuccess)
+        return PA_ERR_CUDA;
+    unsigned int v = 0, zero = 0;
+    if (cudaMemcpyFromSymbol(&v, pa::g_device_error, sizeof(v)) != cudaSuccess)
+        return PA_ERR_CUDA;
+    if (cudaMemcpyToSymbol(pa::g_device_error, &zero, sizeof(zero)) != cudaSuccess)
+        return PA_ERR_CUDA;
+    *code = v;
+    return PA_OK;
+}
+
+pa_status pa_reshape_and_cache(const void *key, const void *value, void *k_cache, void *v_cache,
+                               const int64_t *slot_mapping, int num_tokens, int num_heads,
+                               int head_dim, int block_size, int num_blocks, pa_stream_t stream)
+{
+    if (num_tokens < 0 || num_heads <= 0 || num_blocks <= 0)
+        return PA_ERR_INVALID_ARG;
+    if (!supported_head_dim(head_dim) || !supported_block_size(block_size))
+        return PA_ERR_UNSUPPORTED;
+    if (num_tokens == 0)
+        return PA_OK;
+    if (!key || !value || !k_cache || !v_cache || !slot_mapping)
+        return PA_ERR_INVALID_ARG;
+    if (!aligned16(key) || !aligned16(value) || !aligned16(k_cache) || !aligned16(v_cache) ||
+        (reinterpret_cast<uintptr_t>(slot_mapping) & 7u))
+        return PA_ERR_INVALID_ARG;
+    const dim3 grid(unsigned(num_tokens), 2);
+    pa::reshape_and_cache_kernel<<<grid, 128, 0, reinterpret_cast<cudaStream_t>(stream)>>>(
+        static_cast<const uint4 *>(key), static_cast<const uint4 *>(value),
+        static_cast<uint4 *>(k_cache), static_cast<uint4 *>(v_cache), slot_mapping, num_heads,
+        head_dim / 8, block_size, num_blocks);
+    return cudaGetLastError() == cudaSuccess ? PA_OK : PA_ERR_CUDA;
+}
+
+pa_status pa_copy_blocks(void *k_cache, void *v_cache, const int64_t *block_mapping, int num_pairs,
+                         int num_heads, int head_dim, int block_size, int num_blocks,
+                         pa_stream_t stream)
+{
+    if (num_pairs < 0 || num_heads <= 0 || num_blocks <= 0)
+        return PA_ERR_INVALID_ARG;
+    if (!supported_head_dim(head_dim) || !supported_block_size(block_size))
+        return PA_ERR_UNSUPPORTED;
+    if (num_pairs == 0)
+        return PA_OK;
+    if (!k_cache || !v_cache || !block_mapping)
+        return PA_ERR_INVALID_ARG;
+    if (!aligned16(k_cache) || !aligned16(v_cache) ||
+        (reinterpret_cast<uintptr_t>(block_mapping) & 7u))
+        return PA_ERR_INVALID_ARG;
+    const int64_t block_vecs = int64_t(num_heads) * block_size * head_dim / 8;
+    const int64_t per_cta = int64_t(pa::kCopyThreads) * pa::kCopyUnroll;
+    const int64_t chunks = (block_vecs + per_cta - 1) / per_cta;
+    if (chunks > 65535)
+        return PA_ERR_INVALID_ARG;
+    const dim3 grid(unsigned(num_pairs), 2, unsigned(chunks));
+    pa::copy_blocks_kernel<<<grid, pa::kCopyThreads, 0, reinterpret_cast<cudaStream_t>(stream)>>>(
+        static_cast<uint4 *>(k_cache), static_cast<uint4 *>(v_cache), block_mapping, block_vecs,
+        num_blocks);
+    return cudaGetLastError() == cudaSuccess ? PA_OK : PA_ERR_CUDA;
+}
+
+int pa_decode_partition_size(int num_seqs, int num_heads, int head_dim, int max_context_len)
+{
+    return partition_size_for(num_seqs, num_heads, head_dim, max_context_len);
+}
+
+size_t pa_decode_workspace_size(int num_seqs, int num_heads, int head_dim, int max_context_len)
+{
+    if (num_seqs < 0 || num_heads < 0 || head_dim < 0 || max_context_len < 0)
+        return 0;
+    return workspace_layout(num_seqs, num_heads, head_dim, max_context_len).total;
+}
+
+pa_status pa_decode_workspace_init(void *workspace, size_t workspace_bytes, pa_stream_t stream)
+{
+    if (!workspace || workspace_bytes == 0)
+        return PA_ERR_INVALID_ARG;
+    // The whole workspace is cleared: the counters are all that must start
+    // at zero, but zeroing everything keeps the call independent of sizes.
+    return cudaMemsetAsync(workspace, 0, workspace_bytes, reinterpret_cast<cudaStream_t>(stream)) ==
+                   cudaSuccess
+               ? PA_OK
+               : PA_ERR_CUDA;
+}
+
+pa_status pa_decode(void *out, const void *q, const void *k_cache, const void *v_cache,
+                    const int32_t *block_tables, int max_blocks_per_seq, const int32_t *context_lens,
+                    int max_context_len, int num_seqs, int num_heads, int head_dim, int block_size,
+                    int num_blocks, float scale, void *workspace, size_t workspace_bytes,
+                    pa_stream_t stream)
+{
+    if (num_seqs < 0 || num_heads <= 0 || num_blocks <= 0 || max_context_len < 0 ||
+        max_blocks_per_seq < 0)
+        return PA_ERR_INVALID_ARG;
+    if (!supported_head_dim(head_dim) || !supported_block_size(block_size))
+        return PA_ERR_UNSUPPORTED;
+    if (int64_t(max_context_len) > int64_t(max_blocks_per_seq) * block_size)
+        return PA_ERR_INVALID_ARG;
+    if (!std::isfinite(scale))
+        return PA_ERR_INVALID_ARG;
+    if (num_seqs == 0)
+        return PA_OK;
+    if (!out || !q || !k_cache || !v_cache || !block_tables || !context_lens)
+        return PA_ERR_INVALID_ARG;
+    if (!aligned16(out) || !aligned16(q) || !aligned16(k_cache) || !aligned16(v_cache) ||
+        (reinterpret_cast<uintptr_t>(block_tables) & 3u) ||
+        (reinterpret_cast<uintptr_t>(context_lens) & 3u))
+        return PA_ERR_INVALID_ARG;
+    if (num_seqs > 65535 || num_heads > 65535)
+        return PA_ERR_INVALID_ARG;
+    const WorkspaceLayout w = workspace_layout(num_seqs, num_heads, head_dim, max_context_len);
+    if (!workspace || workspace_bytes < w.total || !aligned16(workspace))
+        return PA_ERR_WORKSPACE;
+
+    unsigned char *ws = static_cast<unsigned char *>(workspace);
+    pa::DecodeParams p{};
+    p.out = static_cast<__half *>(out);
+    p.q = static_cast<const __half *>(q);
+    p.k_cache = static_cast<const __half *>(k_cache);
+    p.v_cache = static_cast<const __half *>(v_cache);
+    p.block_tables = block_tables;
+    p.context_lens = context_lens;
+    p.ws_o = reinterpret_cast<float *>(ws + w.o_off);
+    p.ws_ml = reinterpret_cast<float *>(ws + w.ml_off);
+    p.ws_count = reinterpret_cast<unsigned *>(ws + w.count_off);
+    p.max_blocks_per_seq = max_blocks_per_seq;
+    p.max_context_len = max_context_len;
+    p.num_heads = num_heads;
+    p.block_size = block_size;
+    p.num_blocks = num_blocks;
+    p.partition_size = partition_size_for(num_seqs, num_heads, head_dim, max_context_len);
+    p.max_parts = w.max_parts;
+    p.qk_scale_log2 = float(double(scale) * 1.4426950408889634);  // scale * log2(e)
+
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    if (head_dim == 128)
+        return launch_decode<128, kDecodeWarps, kDecodeStages>(p, num_seqs, s);
+    return launch_decode<64, kDecodeWarps, kDecodeStages>(p, num_seqs, s);
+}
+
+} // extern "C"
