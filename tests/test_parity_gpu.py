@@ -275,10 +275,15 @@ def test_shared_prefix_config_aliased_equals_copied():
     binding.pa_copy_blocks(t["k_cache"], t["v_cache"], torch.from_numpy(wl.copy_pairs).cuda())
     out_cow = gpu_decode(wl, t)
     assert torch.equal(out_alias.view(torch.int16), out_cow.view(torch.int16))
-    ref, okc, ovc = oracle_write_and_decode(wl)
+    # oracle: the same write, then the copy, then decode through the copies
+    okc, ovc = oracle.reshape_and_cache(wl.new_key.cpu().numpy(), wl.new_value.cpu().numpy(),
+                                        wl.k_cache.cpu().numpy(), wl.v_cache.cpu().numpy(),
+                                        wl.slot_mapping, wl.block_size)
     okc, ovc = oracle.copy_blocks(okc, ovc, wl.copy_pairs)
     assert np.array_equal(_bits(t["k_cache"]), okc.view(np.uint16))
     assert np.array_equal(_bits(t["v_cache"]), ovc.view(np.uint16))
+    ref = oracle.paged_decode(wl.q.cpu().numpy(), okc, ovc, wl.block_tables, wl.context_lens,
+                              wl.scale)
     assert max_abs_err(out_cow, ref) <= ATOL
     _assert_no_device_error()
 
