@@ -141,6 +141,24 @@ class ClockSampler:
                 "reasons": names, "samples": len(inside)}
 
 
+def rank_seed(cfg: int, rank: int) -> int:
+    """Each rank decodes its own batch: same recipe, a rank-specific seed."""
+    return cfg + 100 * rank
+
+
+def reduce_over_ranks(max_vals, sum_vals, device):
+    """Max of the device-timed regions and sum of the work over all ranks
+    (identity on one process).  Runs outside any timed region."""
+    import torch
+    import torch.distributed as dist
+    mx = torch.tensor([float(v) for v in max_vals], dtype=torch.float64, device=device)
+    sm = torch.tensor([float(v) for v in sum_vals], dtype=torch.float64, device=device)
+    if dist.is_available() and dist.is_initialized() and dist.get_world_size() > 1:
+        dist.all_reduce(mx, op=dist.ReduceOp.MAX)
+        dist.all_reduce(sm, op=dist.ReduceOp.SUM)
+    return mx.tolist(), sm.tolist()
+
+
 def _workload_desc(wl, cfg):
     from paged_kv_cache_481_b200 import workloads
     return {
@@ -154,9 +172,10 @@ def _workload_desc(wl, cfg):
 
 
 def _cpu_sample(wl, max_units: int, seqs=None):
-    """Host inputs for the oracle on a bounded sample: the first sequences'
-    blocks extracted from the pool (renumbered), and the first `max_units`
-    (sequence, head) pairs of them."""
+    """Host inputs for the oracle on a bounded sample, cut from the pool as
+    generated (before any GPU work): the first sequences' blocks, renumbered,
+    completed by the oracle's own cache write of their newest tokens."""
+    import oracle
     import torch
     if seqs is None:
         seqs = np.arange(min(wl.num_seqs, max(1, math.ceil(max_units / wl.num_heads))))
@@ -168,6 +187,11 @@ def _cpu_sample(wl, max_units: int, seqs=None):
     idx = torch.from_numpy(ids).to(wl.k_cache.device)
     kc = wl.k_cache.index_select(0, idx).cpu().numpy()
     vc = wl.v_cache.index_select(0, idx).cpu().numpy()
+    bs = wl.block_size
+    slots = wl.slot_mapping[seqs]
+    kc, vc = oracle.reshape_and_cache(wl.new_key[seqs].cpu().numpy(),
+                                      wl.new_value[seqs].cpu().numpy(), kc, vc,
+                                      remap[slots // bs] * bs + slots % bs, bs)
     return dict(q=wl.q[seqs].cpu().numpy(), kc=kc, vc=vc, tables=sub_tables,
                 lens=wl.context_lens[seqs].copy(), scale=wl.scale)
 
@@ -183,16 +207,20 @@ def _time_oracle(sample, reps: int = 1):
     return statistics.median(t)
 
 
-def cpu_baseline(wl, target_s: float = 10.0):
+def cpu_baseline_sample(wl, target_s: float = 10.0):
+    """Size and cut the CPU-baseline sample (call before any GPU work touches
+    the pool): about target_s seconds of oracle decode."""
+    probe = _cpu_sample(wl, wl.num_heads)                       # one sequence
+    per_seq = max(_time_oracle(probe), 1e-4)
+    nseq = int(min(wl.num_seqs, max(1, target_s / per_seq)))
+    return _cpu_sample(wl, nseq * wl.num_heads)
+
+
+def cpu_baseline(wl, sample):
     """The oracle as it stands, on the host cores, on a bounded sample of the
     same workload; GB/s over the sample's algorithmic bytes."""
     import oracle
     from paged_kv_cache_481_b200 import accounting
-    probe = _cpu_sample(wl, wl.num_heads)                       # one sequence
-    t1 = _time_oracle(probe)
-    per_seq = max(t1, 1e-4)
-    nseq = int(min(wl.num_seqs, max(1, target_s / per_seq)))
-    sample = _cpu_sample(wl, nseq * wl.num_heads)
     t = _time_oracle(sample)
     nbytes = accounting.decode_bytes(sample["lens"], wl.num_heads, wl.head_dim)
     return {"value": nbytes / t / 1e9, "unit": "GB/s", "cores": oracle.num_threads(),
@@ -269,9 +297,12 @@ def run_gpu(args):
     binding.load()
 
     cfg = args.workload
-    wl = workloads.make_workload(cfg, device="cuda", seed=cfg + 100 * rank,
+    wl = workloads.make_workload(cfg, device="cuda", seed=rank_seed(cfg, rank),
                                  block_size=args.block_size)
     dev = torch.device("cuda", local)
+    cpu_sample = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        cpu_sample = cpu_baseline_sample(wl, target_s=args.cpu_seconds)
     stream = torch.cuda.Stream(device=dev)
     b, h, d = wl.num_seqs, wl.num_heads, wl.head_dim
     q = wl.q
@@ -371,13 +402,8 @@ def run_gpu(args):
         step_bytes += accounting.copy_blocks_bytes(len(wl.copy_pairs), h, d, wl.block_size)
 
     # max over ranks of the device-timed regions; totals over ranks
-    stats = torch.tensor([ms, e2e_ms], dtype=torch.float64, device=dev)
-    tot = torch.tensor([float(step_bytes), float(b * h)], dtype=torch.float64, device=dev)
-    if world > 1:
-        dist.all_reduce(stats, op=dist.ReduceOp.MAX)
-        dist.all_reduce(tot, op=dist.ReduceOp.SUM)
-    ms, e2e_ms = stats.tolist()
-    total_bytes, total_units = tot.tolist()
+    (ms, e2e_ms), (total_bytes, total_units) = reduce_over_ranks(
+        [ms, e2e_ms], [step_bytes, b * h], dev)
 
     result = None
     if rank == 0:
@@ -408,6 +434,8 @@ def run_gpu(args):
             "hbm_frac": achieved / peak,
             "decode_us_mean": mean_dec_ms * 1e3,
             "decode_us_median": statistics.median(decode_ms) * 1e3,
+            "decode_us_max": max(decode_ms) * 1e3,
+            "decode_us_argmax": int(np.argmax(decode_ms)),
             "roofline": {
                 "kernel": "paged_decode_kernel", "bound": "hbm", "achieved": achieved,
                 "peak": peak, "peak_kind": f"{peak_kind} (hbm_gbs)", "unit": "GB/s",
@@ -420,8 +448,8 @@ def run_gpu(args):
             "gpu_launches": launches_per_step * args.steps,
             "clocks": clocks,
         }
-        if world == 1 and not args.no_cpu_baseline:
-            result["cpu_baseline"] = cpu_baseline(wl, target_s=args.cpu_seconds)
+        if cpu_sample is not None:
+            result["cpu_baseline"] = cpu_baseline(wl, cpu_sample)
     if world > 1:
         dist.barrier()
         dist.destroy_process_group()
