@@ -143,6 +143,32 @@ PA_API pa_status pa_copy_blocks(void *k_cache, void *v_cache, const int64_t *blo
                          int num_pairs, int num_heads, int head_dim, int block_size,
                          int num_blocks, pa_stream_t stream);
 
+/*
+ * pa_decode without a caller-supplied workspace, for callers that cannot
+ * allocate device memory at decode time (for example a serving engine that
+ * has reserved nearly all free HBM for its KV block pool, or a loop that
+ * must not let cudaMalloc/cudaFree synchronise the device).  There is no
+ * counterpart on the pages: it is a library convenience.  Same arguments and
+ * results as pa_decode minus workspace/workspace_bytes.
+ *   - Scratch is a static 8 MiB device array inside libpa, present on every
+ *     GPU that loads the library until the process exits; no device memory
+ *     is allocated by this call.
+ *   - Sizes whose pa_decode_workspace_size() exceeds 8 MiB return
+ *     PA_ERR_WORKSPACE (use pa_decode with your own workspace instead).
+ *   - The first call on each device looks up the array's device address
+ *     (cudaGetSymbolAddress) with that device current; make that first call
+ *     before any stream capture.  Each call clears the merge counters with a
+ *     cudaMemsetAsync on `stream`.
+ *   - All calls on a device share the one array: calls that overlap on the
+ *     GPU (other streams, other host threads) race and give wrong results.
+ */
+PA_API pa_status pa_decode_no_alloc(void *out, const void *q, const void *k_cache,
+                                    const void *v_cache, const int32_t *block_tables,
+                                    int max_blocks_per_seq, const int32_t *context_lens,
+                                    int max_context_len, int num_seqs, int num_heads,
+                                    int head_dim, int block_size, int num_blocks, float scale,
+                                    pa_stream_t stream);
+
 /* Static description of a status code. */
 PA_API const char *pa_status_string(pa_status status);
 

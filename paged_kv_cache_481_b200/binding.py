@@ -27,7 +27,7 @@ PA_DEVERR_TIMEOUT = 16
 # every symbol include/pa.h declares
 EXPORTED = ("pa_reshape_and_cache", "pa_decode_workspace_size", "pa_decode_workspace_init",
             "pa_decode_partition_size", "pa_decode", "pa_copy_blocks", "pa_status_string",
-            "pa_get_last_device_error")
+            "pa_get_last_device_error", "pa_decode_no_alloc")
 
 _lock = threading.Lock()
 _lib = None
@@ -62,6 +62,9 @@ def load(path: str | None = None):
         lib.pa_decode.argtypes = [vp, vp, vp, vp, vp, i32, vp, i32, i32, i32, i32, i32, i32,
                                   ctypes.c_float, vp, sz, vp]
         lib.pa_decode.restype = i32
+        lib.pa_decode_no_alloc.argtypes = [vp, vp, vp, vp, vp, i32, vp, i32, i32, i32, i32, i32,
+                                           i32, ctypes.c_float, vp]
+        lib.pa_decode_no_alloc.restype = i32
         lib.pa_copy_blocks.argtypes = [vp, vp, vp, i32, i32, i32, i32, i32, vp]
         lib.pa_copy_blocks.restype = i32
         lib.pa_status_string.argtypes = [i32]
@@ -149,6 +152,26 @@ def pa_decode(out, q, k_cache, v_cache, block_tables, context_lens, max_context_
                             _ptr(workspace), workspace.numel() * workspace.element_size(),
                             _stream(stream)),
            "pa_decode")
+
+
+def pa_decode_no_alloc(out, q, k_cache, v_cache, block_tables, context_lens, max_context_len,
+                       scale, stream=None):
+    """pa_decode with the library's static device scratch instead of a
+    workspace, for callers that cannot allocate device memory at decode time
+    (e.g. when the KV block pool has taken the free HBM).  Raises PAError
+    (PA_ERR_WORKSPACE) for sizes past the 8 MiB scratch.  Calls sharing a
+    device must not overlap on the GPU."""
+    b, h, d = q.shape
+    nb, hk, bs, dk = k_cache.shape
+    assert q.dtype == out.dtype == k_cache.dtype == v_cache.dtype == torch.float16
+    assert out.shape == q.shape and (hk, dk) == (h, d) and v_cache.shape == k_cache.shape
+    assert block_tables.dtype == torch.int32 and block_tables.dim() == 2
+    assert context_lens.dtype == torch.int32 and context_lens.numel() == b
+    _check(load().pa_decode_no_alloc(_ptr(out), _ptr(q), _ptr(k_cache), _ptr(v_cache),
+                                     _ptr(block_tables), block_tables.shape[1],
+                                     _ptr(context_lens), int(max_context_len), b, h, d, bs, nb,
+                                     float(scale), _stream(stream)),
+           "pa_decode_no_alloc")
 
 
 def pa_copy_blocks(k_cache, v_cache, block_mapping, stream=None):

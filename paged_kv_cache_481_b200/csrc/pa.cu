@@ -247,3 +247,73 @@ pa_status pa_decode(void *out, const void *q, const void *k_cache, const void *v
 }
 
 } // extern "C"
+
+// ---------------------------------------------------------------------------
+// Allocation-free variant of pa_decode.
+//
+// Some callers cannot allocate device memory when they call the decode: a
+// serving engine typically reserves almost all free HBM for its KV block
+// pool at start-up, so a later cudaMalloc for a workspace fails, and
+// cudaMalloc/cudaFree can also synchronise the device in the middle of a
+// latency-critical decode loop.  For them the split-K workspace lives in the
+// file-scope device array below, which the CUDA module reserves on every GPU
+// that loads this library and keeps until the process exits.
+
+namespace {
+
+constexpr size_t kNoAllocScratchBytes = size_t(8) << 20;  // 8 MiB per GPU
+
+// In host code this name is only a host-side stand-in for the array, never a
+// device address: kernels get the address from cudaGetSymbolAddress.
+static __device__ __align__(256) unsigned char g_no_alloc_scratch[kNoAllocScratchBytes];
+
+std::atomic<void *> g_no_alloc_scratch_addr[kMaxDevices];
+
+// Device address of g_no_alloc_scratch on the current device; looked up once
+// per device (with that device current) on the first call there.
+pa_status no_alloc_scratch_address(void **addr)
+{
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices)
+        return PA_ERR_CUDA;
+    void *p = g_no_alloc_scratch_addr[dev].load(std::memory_order_acquire);
+    if (!p) {
+        if (cudaGetSymbolAddress(&p, g_no_alloc_scratch) != cudaSuccess || !p)
+            return PA_ERR_CUDA;
+        g_no_alloc_scratch_addr[dev].store(p, std::memory_order_release);
+    }
+    *addr = p;
+    return PA_OK;
+}
+
+} // namespace
+
+extern "C" pa_status pa_decode_no_alloc(void *out, const void *q, const void *k_cache,
+                                        const void *v_cache, const int32_t *block_tables,
+                                        int max_blocks_per_seq, const int32_t *context_lens,
+                                        int max_context_len, int num_seqs, int num_heads,
+                                        int head_dim, int block_size, int num_blocks, float scale,
+                                        pa_stream_t stream)
+{
+    if (num_seqs < 0 || num_heads <= 0 || head_dim < 0 || max_context_len < 0)
+        return PA_ERR_INVALID_ARG;
+    const size_t need = pa_decode_workspace_size(num_seqs, num_heads, head_dim, max_context_len);
+    if (need > kNoAllocScratchBytes)
+        return PA_ERR_WORKSPACE;  // sizes beyond the static scratch: use pa_decode
+    void *scratch = nullptr;
+    const pa_status st = no_alloc_scratch_address(&scratch);
+    if (st != PA_OK)
+        return st;
+    // The merge tickets must start at zero; the array keeps whatever the last
+    // call (or an aborted one) left there, so clear them on every call.
+    if (num_seqs > 0 && supported_head_dim(head_dim)) {
+        const WorkspaceLayout w = workspace_layout(num_seqs, num_heads, head_dim, max_context_len);
+        if (cudaMemsetAsync(static_cast<unsigned char *>(scratch) + w.count_off, 0,
+                            size_t(num_seqs) * size_t(num_heads) * sizeof(unsigned),
+                            reinterpret_cast<cudaStream_t>(stream)) != cudaSuccess)
+            return PA_ERR_CUDA;
+    }
+    return pa_decode(out, q, k_cache, v_cache, block_tables, max_blocks_per_seq, context_lens,
+                     max_context_len, num_seqs, num_heads, head_dim, block_size, num_blocks, scale,
+                     scratch, kNoAllocScratchBytes, stream);
+}
