@@ -356,23 +356,28 @@ def run_gpu(args):
     decode_ms = [a.elapsed_time(z) for a, z in evs]
     assert binding.pa_get_last_device_error() == 0
 
-    # end to end: per-step inputs from pinned host buffers, output back to host
-    h_q = q.cpu().pin_memory()
-    h_key, h_value = key.cpu().pin_memory(), value.cpu().pin_memory()
-    h_slots = slots.cpu().pin_memory()
-    h_tables, h_lens = tables.cpu().pin_memory(), lens.cpu().pin_memory()
+    # end to end: each step's inputs (q, the new tokens' K/V, slots, block
+    # tables, context lengths) leave one pinned host buffer in one copy, and
+    # out comes back to pinned host memory; the KV pool stays resident.
+    parts = [q, key, value, slots, tables, lens]
+    offs, total = [], 0
+    for t in parts:
+        offs.append(total)
+        total += (t.numel() * t.element_size() + 255) // 256 * 256
+    h_stage = torch.empty(total, dtype=torch.uint8, pin_memory=True)
+    d_stage = torch.empty(total, dtype=torch.uint8, device=dev)
+    views = []
+    for t, o in zip(parts, offs):
+        n = t.numel() * t.element_size()
+        h_stage[o:o + n].copy_(t.reshape(-1).view(torch.uint8).cpu())
+        views.append(d_stage[o:o + n].view(t.dtype).view(t.shape))
+    d_q, d_key, d_value, d_slots, d_tables, d_lens = views
     h_out = torch.empty(out.shape, dtype=out.dtype, pin_memory=True)
-    d_q, d_key, d_value = torch.empty_like(q), torch.empty_like(key), torch.empty_like(value)
-    d_slots, d_tables, d_lens = (torch.empty_like(slots), torch.empty_like(tables),
-                                 torch.empty_like(lens))
-    h2d = sum(t.numel() * t.element_size() for t in (h_q, h_key, h_value, h_slots, h_tables,
-                                                     h_lens))
+    h2d = sum(t.numel() * t.element_size() for t in parts)
     d2h = h_out.numel() * h_out.element_size()
 
     def e2e_step():
-        for dst, src in ((d_q, h_q), (d_key, h_key), (d_value, h_value), (d_slots, h_slots),
-                         (d_tables, h_tables), (d_lens, h_lens)):
-            dst.copy_(src, non_blocking=True)
+        d_stage.copy_(h_stage, non_blocking=True)
         if pairs is not None:
             binding.pa_copy_blocks(kc, vc, pairs, stream=stream)
         binding.pa_reshape_and_cache(d_key, d_value, kc, vc, d_slots, stream=stream)
@@ -418,7 +423,6 @@ def run_gpu(args):
                     + f"pa_reshape_and_cache({b} tokens) + pa_decode",
             "l2": f"inputs larger than L2: {kv_bytes / 1e9:.2f} GB of K/V read per step "
                   f"vs {L2_BYTES / 2**20:.0f} MiB L2 (no flush)",
-            "partition_size": binding.pa_decode_partition_size(b, h, d, mcl),
             "parallelism": f"dp{world} (independent batches per GPU)",
         })
         result = {

@@ -85,8 +85,10 @@ PA_API pa_status pa_reshape_and_cache(const void *key, const void *value, void *
                                int block_size, int num_blocks, pa_stream_t stream);
 
 /*
- * Bytes of workspace pa_decode needs for these sizes (split-K partial
- * results and one merge counter per (sequence, head)).  Never 0.
+ * Bytes of workspace pa_decode needs for these sizes: partial results of the
+ * (sequence, head) pairs whose context is split between workers (a fixed
+ * part, 2 * 4096 * (head_dim + 2) floats) and one merge ticket per
+ * (sequence, head).  Never 0; max_context_len does not change it.
  */
 PA_API size_t pa_decode_workspace_size(int num_seqs, int num_heads, int head_dim,
                                 int max_context_len);
@@ -100,13 +102,6 @@ PA_API size_t pa_decode_workspace_size(int num_seqs, int num_heads, int head_dim
  */
 PA_API pa_status pa_decode_workspace_init(void *workspace, size_t workspace_bytes,
                                    pa_stream_t stream);
-
-/*
- * Tokens per context partition (split-K chunk) pa_decode uses for these
- * sizes; a sequence of length L is split into ceil(L / partition) partitions.
- */
-PA_API int pa_decode_partition_size(int num_seqs, int num_heads, int head_dim,
-                             int max_context_len);
 
 /*
  * Paged single-token decode attention (comfyai.app 6.4.1; polomodov.tech

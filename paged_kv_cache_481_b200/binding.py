@@ -26,7 +26,7 @@ PA_DEVERR_TIMEOUT = 16
 
 # every symbol include/pa.h declares
 EXPORTED = ("pa_reshape_and_cache", "pa_decode_workspace_size", "pa_decode_workspace_init",
-            "pa_decode_partition_size", "pa_decode", "pa_copy_blocks", "pa_status_string",
+            "pa_decode", "pa_copy_blocks", "pa_status_string",
             "pa_get_last_device_error", "pa_decode_no_alloc")
 
 _lock = threading.Lock()
@@ -57,8 +57,6 @@ def load(path: str | None = None):
         lib.pa_decode_workspace_size.restype = sz
         lib.pa_decode_workspace_init.argtypes = [vp, sz, vp]
         lib.pa_decode_workspace_init.restype = i32
-        lib.pa_decode_partition_size.argtypes = [i32, i32, i32, i32]
-        lib.pa_decode_partition_size.restype = i32
         lib.pa_decode.argtypes = [vp, vp, vp, vp, vp, i32, vp, i32, i32, i32, i32, i32, i32,
                                   ctypes.c_float, vp, sz, vp]
         lib.pa_decode.restype = i32
@@ -116,10 +114,6 @@ def pa_reshape_and_cache(key, value, k_cache, v_cache, slot_mapping, stream=None
 
 def pa_decode_workspace_size(num_seqs, num_heads, head_dim, max_context_len) -> int:
     return int(load().pa_decode_workspace_size(num_seqs, num_heads, head_dim, max_context_len))
-
-
-def pa_decode_partition_size(num_seqs, num_heads, head_dim, max_context_len) -> int:
-    return int(load().pa_decode_partition_size(num_seqs, num_heads, head_dim, max_context_len))
 
 
 def pa_decode_workspace_init(workspace: torch.Tensor, stream=None):

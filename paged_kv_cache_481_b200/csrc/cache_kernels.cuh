@@ -17,6 +17,8 @@ __global__ void __launch_bounds__(256) reshape_and_cache_kernel(
     uint4 *__restrict__ v_cache, const int64_t *__restrict__ slot_mapping, int num_heads,
     int head_chunks, int block_size, int num_blocks)
 {
+    grid_dependency_wait();
+    allow_dependent_launch();
     const int i = blockIdx.x;
     const int64_t slot = slot_mapping[i];
     if (slot < 0)
@@ -48,6 +50,8 @@ __global__ void __launch_bounds__(kCopyThreads) copy_blocks_kernel(
     uint4 *__restrict__ k_cache, uint4 *__restrict__ v_cache, const int64_t *__restrict__ block_mapping,
     int64_t block_vecs, int num_blocks)
 {
+    grid_dependency_wait();
+    allow_dependent_launch();
     const int pair = blockIdx.x;
     const int64_t src = block_mapping[2 * pair], dst = block_mapping[2 * pair + 1];
     if (src < 0 || src >= num_blocks || dst < 0 || dst >= num_blocks) {

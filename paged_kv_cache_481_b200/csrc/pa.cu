@@ -36,55 +36,84 @@ size_t align256(size_t x)
     return (x + 255) & ~size_t(255);
 }
 
-// Tokens per split-K partition.  A multiple of every tile height (16 or 32
-// rows) and every supported block size, with at most 512/8 + 1 table entries
-// per partition.
-int partition_size_for(int /*num_seqs*/, int /*num_heads*/, int /*head_dim*/, int /*max_context_len*/)
+// Launch with programmatic stream serialisation: the grid may begin while the
+// previous kernel in the stream drains; every kernel here waits on
+// griddepcontrol.wait before it touches memory, so ordering is unchanged.
+template <typename... KArgs, typename... Args>
+cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem,
+                       cudaStream_t stream, Args... args)
 {
-    return 512;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, kernel, static_cast<KArgs>(args)...);
 }
 
+// Workspace: for each worker (warp) two partial-result slots (its first and
+// its last (sequence, head), the only ones that can straddle workers), then
+// one merge ticket per (sequence, head).
 struct WorkspaceLayout {
     size_t o_off, ml_off, count_off, total;
-    int max_parts;
 };
 
-WorkspaceLayout workspace_layout(int num_seqs, int num_heads, int head_dim, int max_context_len)
+WorkspaceLayout workspace_layout(int num_seqs, int num_heads, int head_dim)
 {
     WorkspaceLayout w{};
-    const int P = partition_size_for(num_seqs, num_heads, head_dim, max_context_len);
-    w.max_parts = max_context_len > 0 ? (max_context_len + P - 1) / P : 1;
     const size_t units = size_t(num_seqs) * size_t(num_heads);
-    const size_t parts = w.max_parts > 1 ? size_t(w.max_parts) : 0;
+    const size_t slots = size_t(pa::kMaxWorkers) * 2;
     w.o_off = 0;
-    w.ml_off = align256(units * parts * size_t(head_dim) * sizeof(float));
-    w.count_off = w.ml_off + align256(units * parts * 2 * sizeof(float));
+    w.ml_off = align256(slots * size_t(head_dim) * sizeof(float));
+    w.count_off = w.ml_off + align256(slots * 2 * sizeof(float));
     w.total = w.count_off + align256((units > 0 ? units : 1) * sizeof(unsigned));
     return w;
 }
 
 template <int D, int NW, int S>
-pa_status launch_decode(const pa::DecodeParams &p, int num_seqs, cudaStream_t stream)
+pa_status launch_decode(const pa::DecodeParams &p, cudaStream_t stream)
 {
     using Sm = pa::DecodeSmem<D, NW, S>;
-    static std::atomic<bool> configured[kMaxDevices];
+    static std::atomic<int> grid_for[kMaxDevices];  // 0 = not configured yet
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices)
         return PA_ERR_CUDA;
-    if (!configured[dev].load(std::memory_order_acquire)) {
+    int grid = grid_for[dev].load(std::memory_order_acquire);
+    if (grid == 0) {
         if (cudaFuncSetAttribute(pa::paged_decode_kernel<D, NW, S>,
                                  cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  int(Sm::kBytes)) != cudaSuccess)
             return PA_ERR_CUDA;
-        configured[dev].store(true, std::memory_order_release);
+        int sms = 0, per_sm = 0;
+        if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess ||
+            cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, pa::paged_decode_kernel<D, NW, S>,
+                                                          pa::DecodeSmem<D, NW, S>::kThreads,
+                                                          Sm::kBytes) != cudaSuccess)
+            return PA_ERR_CUDA;
+        grid = sms * (per_sm > 0 ? per_sm : 1);
+        if (grid * NW > pa::kMaxWorkers)
+            grid = pa::kMaxWorkers / NW;
+        grid_for[dev].store(grid, std::memory_order_release);
     }
-    const dim3 grid(unsigned(p.max_parts), unsigned(p.num_heads), unsigned(num_seqs));
-    pa::paged_decode_kernel<D, NW, S><<<grid, NW * 32, Sm::kBytes, stream>>>(p);
-    return cudaGetLastError() == cudaSuccess ? PA_OK : PA_ERR_CUDA;
+    return launch_pdl(pa::paged_decode_kernel<D, NW, S>, dim3(grid), dim3(Sm::kThreads),
+                      Sm::kBytes, stream, p) == cudaSuccess
+               ? PA_OK
+               : PA_ERR_CUDA;
 }
 
-constexpr int kDecodeWarps = 4;
-constexpr int kDecodeStages = 3;
+#ifndef PA_DECODE_WARPS
+#define PA_DECODE_WARPS 8
+#endif
+#ifndef PA_DECODE_STAGES
+#define PA_DECODE_STAGES 1
+#endif
+constexpr int kDecodeWarps = PA_DECODE_WARPS;
+constexpr int kDecodeStages = PA_DECODE_STAGES;
 
 } // namespace
 
@@ -133,11 +162,13 @@ pa_status pa_reshape_and_cache(const void *key, const void *value, void *k_cache
         (reinterpret_cast<uintptr_t>(slot_mapping) & 7u))
         return PA_ERR_INVALID_ARG;
     const dim3 grid(unsigned(num_tokens), 2);
-    pa::reshape_and_cache_kernel<<<grid, 128, 0, reinterpret_cast<cudaStream_t>(stream)>>>(
-        static_cast<const uint4 *>(key), static_cast<const uint4 *>(value),
-        static_cast<uint4 *>(k_cache), static_cast<uint4 *>(v_cache), slot_mapping, num_heads,
-        head_dim / 8, block_size, num_blocks);
-    return cudaGetLastError() == cudaSuccess ? PA_OK : PA_ERR_CUDA;
+    return launch_pdl(pa::reshape_and_cache_kernel, grid, dim3(128), 0,
+                      reinterpret_cast<cudaStream_t>(stream), static_cast<const uint4 *>(key),
+                      static_cast<const uint4 *>(value), static_cast<uint4 *>(k_cache),
+                      static_cast<uint4 *>(v_cache), slot_mapping, num_heads, head_dim / 8,
+                      block_size, num_blocks) == cudaSuccess
+               ? PA_OK
+               : PA_ERR_CUDA;
 }
 
 pa_status pa_copy_blocks(void *k_cache, void *v_cache, const int64_t *block_mapping, int num_pairs,
@@ -161,22 +192,20 @@ pa_status pa_copy_blocks(void *k_cache, void *v_cache, const int64_t *block_mapp
     if (chunks > 65535)
         return PA_ERR_INVALID_ARG;
     const dim3 grid(unsigned(num_pairs), 2, unsigned(chunks));
-    pa::copy_blocks_kernel<<<grid, pa::kCopyThreads, 0, reinterpret_cast<cudaStream_t>(stream)>>>(
-        static_cast<uint4 *>(k_cache), static_cast<uint4 *>(v_cache), block_mapping, block_vecs,
-        num_blocks);
-    return cudaGetLastError() == cudaSuccess ? PA_OK : PA_ERR_CUDA;
-}
-
-int pa_decode_partition_size(int num_seqs, int num_heads, int head_dim, int max_context_len)
-{
-    return partition_size_for(num_seqs, num_heads, head_dim, max_context_len);
+    return launch_pdl(pa::copy_blocks_kernel, grid, dim3(pa::kCopyThreads), 0,
+                      reinterpret_cast<cudaStream_t>(stream), static_cast<uint4 *>(k_cache),
+                      static_cast<uint4 *>(v_cache), block_mapping, block_vecs,
+                      num_blocks) == cudaSuccess
+               ? PA_OK
+               : PA_ERR_CUDA;
 }
 
 size_t pa_decode_workspace_size(int num_seqs, int num_heads, int head_dim, int max_context_len)
 {
     if (num_seqs < 0 || num_heads < 0 || head_dim < 0 || max_context_len < 0)
         return 0;
-    return workspace_layout(num_seqs, num_heads, head_dim, max_context_len).total;
+    (void)max_context_len;
+    return workspace_layout(num_seqs, num_heads, head_dim).total;
 }
 
 pa_status pa_decode_workspace_init(void *workspace, size_t workspace_bytes, pa_stream_t stream)
@@ -214,9 +243,7 @@ pa_status pa_decode(void *out, const void *q, const void *k_cache, const void *v
         (reinterpret_cast<uintptr_t>(block_tables) & 3u) ||
         (reinterpret_cast<uintptr_t>(context_lens) & 3u))
         return PA_ERR_INVALID_ARG;
-    if (num_seqs > 65535 || num_heads > 65535)
-        return PA_ERR_INVALID_ARG;
-    const WorkspaceLayout w = workspace_layout(num_seqs, num_heads, head_dim, max_context_len);
+    const WorkspaceLayout w = workspace_layout(num_seqs, num_heads, head_dim);
     if (!workspace || workspace_bytes < w.total || !aligned16(workspace))
         return PA_ERR_WORKSPACE;
 
@@ -231,19 +258,18 @@ pa_status pa_decode(void *out, const void *q, const void *k_cache, const void *v
     p.ws_o = reinterpret_cast<float *>(ws + w.o_off);
     p.ws_ml = reinterpret_cast<float *>(ws + w.ml_off);
     p.ws_count = reinterpret_cast<unsigned *>(ws + w.count_off);
+    p.num_seqs = num_seqs;
     p.max_blocks_per_seq = max_blocks_per_seq;
     p.max_context_len = max_context_len;
     p.num_heads = num_heads;
     p.block_size = block_size;
     p.num_blocks = num_blocks;
-    p.partition_size = partition_size_for(num_seqs, num_heads, head_dim, max_context_len);
-    p.max_parts = w.max_parts;
     p.qk_scale_log2 = float(double(scale) * 1.4426950408889634);  // scale * log2(e)
 
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
     if (head_dim == 128)
-        return launch_decode<128, kDecodeWarps, kDecodeStages>(p, num_seqs, s);
-    return launch_decode<64, kDecodeWarps, kDecodeStages>(p, num_seqs, s);
+        return launch_decode<128, kDecodeWarps, kDecodeStages>(p, s);
+    return launch_decode<64, kDecodeWarps, kDecodeStages>(p, s);
 }
 
 } // extern "C"
@@ -307,7 +333,7 @@ extern "C" pa_status pa_decode_no_alloc(void *out, const void *q, const void *k_
     // The merge tickets must start at zero; the array keeps whatever the last
     // call (or an aborted one) left there, so clear them on every call.
     if (num_seqs > 0 && supported_head_dim(head_dim)) {
-        const WorkspaceLayout w = workspace_layout(num_seqs, num_heads, head_dim, max_context_len);
+        const WorkspaceLayout w = workspace_layout(num_seqs, num_heads, head_dim);
         if (cudaMemsetAsync(static_cast<unsigned char *>(scratch) + w.count_off, 0,
                             size_t(num_seqs) * size_t(num_heads) * sizeof(unsigned),
                             reinterpret_cast<cudaStream_t>(stream)) != cudaSuccess)

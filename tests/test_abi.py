@@ -48,14 +48,15 @@ def test_status_strings(lib):
     assert binding.status_string(99) == "unknown status"
 
 
-def test_workspace_size_grows_with_partitions(lib):
-    one = binding.pa_decode_workspace_size(32, 40, 128, 512)
-    many = binding.pa_decode_workspace_size(32, 40, 128, 4096)
-    p = binding.pa_decode_partition_size(32, 40, 128, 4096)
-    assert one > 0 and many > one
-    parts = -(-4096 // p)
-    # partial outputs + (max, sum) + one counter per (sequence, head)
-    assert many >= 32 * 40 * parts * (128 + 2) * 4 + 32 * 40 * 4
+def test_workspace_size_covers_partials_and_tickets(lib):
+    small = binding.pa_decode_workspace_size(1, 1, 128, 512)
+    big = binding.pa_decode_workspace_size(256, 40, 128, 4096)
+    assert small > 0 and big > small
+    # two partial slots of (D + 2) floats per worker, one ticket per (seq, head)
+    assert small >= 2 * 4096 * (128 + 2) * 4
+    assert big - small >= (256 * 40 - 1) * 4 - 256
+    assert binding.pa_decode_workspace_size(256, 40, 128, 4096) == \
+        binding.pa_decode_workspace_size(256, 40, 128, 16)
 
 
 NULL = ctypes.c_void_p(None)

@@ -41,8 +41,8 @@ def _no_alloc(wl, t):
 
 
 def test_matches_workspace_entry_point_on_two_calls_in_a_row():
-    # several partitions per sequence, so the static scratch holds split-K
-    # partials and merge tickets; the second call sees what the first left
+    # contexts split between workers, so the static scratch holds partial
+    # results and merge tickets; the second call sees what the first left
     wl = workloads.make_random(301, [1500, 40, 2049, 700, 1], num_heads=6, head_dim=128,
                                block_size=16, keep_logical=False)
     t = _written(wl)
@@ -72,19 +72,18 @@ def test_second_call_with_other_sizes_and_the_13b_shape():
 def test_sizes_past_the_static_scratch_are_rejected_before_any_launch():
     lib = binding.load()
     null = ctypes.c_void_p(None)
-    # 256 sequences x 40 heads x 4096 tokens needs far more than the 8 MiB scratch
-    assert binding.pa_decode_workspace_size(256, 40, 128, 4096) > 8 << 20
-    rc = lib.pa_decode_no_alloc(null, null, null, null, null, 256, null, 4096, 256, 40, 128, 16,
+    # one merge ticket per (sequence, head): 65535 x 64 of them exceed 8 MiB
+    assert binding.pa_decode_workspace_size(65535, 64, 128, 16) > 8 << 20
+    rc = lib.pa_decode_no_alloc(null, null, null, null, null, 1, null, 16, 65535, 64, 128, 16,
                                 1, ctypes.c_float(1.0), null)
     assert rc == binding.PA_ERR_WORKSPACE
-    # and through the binding, with real (small) tensors but a long host bound
-    h, d = 64, 128
-    q = torch.zeros((4, h, d), dtype=torch.float16, device="cuda")
+    # and through the binding, with real tensors
+    b, h, d = 65535, 32, 64
+    assert binding.pa_decode_workspace_size(b, h, d, 16) > 8 << 20
+    q = torch.zeros((b, h, d), dtype=torch.float16, device="cuda")
     cache = torch.zeros((1, h, 16, d), dtype=torch.float16, device="cuda")
-    tables = torch.zeros((4, 4096), dtype=torch.int32, device="cuda")
-    lens = torch.ones(4, dtype=torch.int32, device="cuda")
-    assert binding.pa_decode_workspace_size(4, h, d, 16 * 4096) > 8 << 20
+    tables = torch.zeros((b, 1), dtype=torch.int32, device="cuda")
+    lens = torch.ones(b, dtype=torch.int32, device="cuda")
     with pytest.raises(binding.PAError) as e:
-        binding.pa_decode_no_alloc(torch.empty_like(q), q, cache, cache, tables, lens,
-                                   16 * 4096, 0.1)
+        binding.pa_decode_no_alloc(torch.empty_like(q), q, cache, cache, tables, lens, 16, 0.1)
     assert e.value.status == binding.PA_ERR_WORKSPACE
