@@ -60,7 +60,9 @@ def _load():
     with _lock:
         if _lib is not None:
             return _lib
-        lib = ctypes.CDLL(build())
+        # PA_ORACLE_LIB points the tests' mutation check at a deliberately
+        # broken copy of this oracle; normal use builds and loads pa_oracle.c.
+        lib = ctypes.CDLL(os.environ.get("PA_ORACLE_LIB") or build())
         vp, i32, i64 = ctypes.c_void_p, ctypes.c_int, ctypes.c_int64
         lib.oracle_half_to_double.argtypes = [ctypes.c_uint16]
         lib.oracle_half_to_double.restype = ctypes.c_double
