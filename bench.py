@@ -298,7 +298,7 @@ def run_gpu(args):
 
     cfg = args.workload
     wl = workloads.make_workload(cfg, device="cuda", seed=rank_seed(cfg, rank),
-                                 block_size=args.block_size)
+                                 block_size=args.block_size, placement=args.placement)
     dev = torch.device("cuda", local)
     cpu_sample = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
@@ -430,6 +430,7 @@ def run_gpu(args):
             "l2": f"inputs larger than L2: {kv_bytes / 1e9:.2f} GB of K/V read per step "
                   f"vs {L2_BYTES / 2**20:.0f} MiB L2 (no flush)",
             "parallelism": f"dp{world} (independent batches per GPU)",
+            "placement": args.placement,
         })
         result = {
             "metric": METRIC,
@@ -477,6 +478,8 @@ def main(argv=None):
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", type=int, default=2, choices=[1, 2, 3, 4, 5])
     ap.add_argument("--block-size", type=int, default=None)
+    ap.add_argument("--placement", choices=["shuffled", "sequential"], default="shuffled",
+                    help="physical block placement (sequential = contiguous-cache baseline)")
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     args = ap.parse_args(argv)

@@ -61,7 +61,8 @@ typedef enum pa_status {
     PA_ERR_INVALID_ARG = 1,  /* null pointer, negative size, misalignment, lengths too long */
     PA_ERR_UNSUPPORTED = 2,  /* head_dim not in {64,128} or block_size not in {8,16,32,64,128} */
     PA_ERR_CUDA = 3,         /* the CUDA runtime refused the launch */
-    PA_ERR_WORKSPACE = 4     /* workspace null or smaller than pa_decode_workspace_size() */
+    PA_ERR_WORKSPACE = 4,    /* workspace null or smaller than pa_decode_workspace_size() */
+    PA_ERR_OUT_OF_BLOCKS = 5 /* block manager: the free pool cannot cover the request */
 } pa_status;
 
 /* Bits of the device error word (pa_get_last_device_error). */
@@ -173,6 +174,16 @@ PA_API const char *pa_status_string(pa_status status);
  * fails, PA_ERR_INVALID_ARG if code is NULL.
  */
 PA_API pa_status pa_get_last_device_error(unsigned int *code);
+
+/*
+ * Self-test of failure detection (no counterpart on the pages).  Every wait
+ * inside the kernels is bounded; this launches one warp that waits on a
+ * barrier nothing ever completes, for limit_us microseconds (1 .. 2 000 000),
+ * after which it records PA_DEVERR_TIMEOUT in the device error word and
+ * exits.  It faults nothing and leaves the context usable.  Asynchronous on
+ * `stream`; read the result with pa_get_last_device_error().
+ */
+PA_API pa_status pa_selftest_bounded_wait(unsigned int limit_us, pa_stream_t stream);
 
 #ifdef __cplusplus
 }

@@ -17,7 +17,8 @@ import torch
 _PKG = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_PKG, "libpa.so")
 
-PA_OK, PA_ERR_INVALID_ARG, PA_ERR_UNSUPPORTED, PA_ERR_CUDA, PA_ERR_WORKSPACE = range(5)
+(PA_OK, PA_ERR_INVALID_ARG, PA_ERR_UNSUPPORTED, PA_ERR_CUDA, PA_ERR_WORKSPACE,
+ PA_ERR_OUT_OF_BLOCKS) = range(6)
 PA_DEVERR_BLOCK_ID = 1
 PA_DEVERR_CONTEXT_LEN = 2
 PA_DEVERR_SLOT = 4
@@ -27,7 +28,10 @@ PA_DEVERR_TIMEOUT = 16
 # every symbol include/pa.h declares
 EXPORTED = ("pa_reshape_and_cache", "pa_decode_workspace_size", "pa_decode_workspace_init",
             "pa_decode", "pa_copy_blocks", "pa_status_string",
-            "pa_get_last_device_error", "pa_decode_no_alloc")
+            "pa_get_last_device_error", "pa_decode_no_alloc", "pa_selftest_bounded_wait",
+            "pa_bm_create", "pa_bm_destroy", "pa_bm_num_free", "pa_bm_refcount",
+            "pa_bm_add_sequence", "pa_bm_fork", "pa_bm_free_sequence", "pa_bm_append_slots",
+            "pa_bm_block_tables")
 
 _lock = threading.Lock()
 _lib = None
@@ -63,6 +67,27 @@ def load(path: str | None = None):
         lib.pa_decode_no_alloc.argtypes = [vp, vp, vp, vp, vp, i32, vp, i32, i32, i32, i32, i32,
                                            i32, ctypes.c_float, vp]
         lib.pa_decode_no_alloc.restype = i32
+        lib.pa_selftest_bounded_wait.argtypes = [ctypes.c_uint, vp]
+        lib.pa_selftest_bounded_wait.restype = i32
+        i64, p64, p32 = ctypes.c_int64, ctypes.POINTER(ctypes.c_int64), ctypes.POINTER(ctypes.c_int32)
+        lib.pa_bm_create.argtypes = [i32, i32]
+        lib.pa_bm_create.restype = vp
+        lib.pa_bm_destroy.argtypes = [vp]
+        lib.pa_bm_destroy.restype = None
+        lib.pa_bm_num_free.argtypes = [vp]
+        lib.pa_bm_num_free.restype = i32
+        lib.pa_bm_refcount.argtypes = [vp, i32]
+        lib.pa_bm_refcount.restype = i32
+        lib.pa_bm_add_sequence.argtypes = [vp, i64, i32]
+        lib.pa_bm_add_sequence.restype = i32
+        lib.pa_bm_fork.argtypes = [vp, i64, i64]
+        lib.pa_bm_fork.restype = i32
+        lib.pa_bm_free_sequence.argtypes = [vp, i64]
+        lib.pa_bm_free_sequence.restype = i32
+        lib.pa_bm_append_slots.argtypes = [vp, vp, i32, vp, vp, ctypes.POINTER(ctypes.c_int)]
+        lib.pa_bm_append_slots.restype = i32
+        lib.pa_bm_block_tables.argtypes = [vp, vp, i32, vp, i32, vp]
+        lib.pa_bm_block_tables.restype = i32
         lib.pa_copy_blocks.argtypes = [vp, vp, vp, i32, i32, i32, i32, i32, vp]
         lib.pa_copy_blocks.restype = i32
         lib.pa_status_string.argtypes = [i32]
@@ -179,7 +204,78 @@ def pa_copy_blocks(k_cache, v_cache, block_mapping, stream=None):
            "pa_copy_blocks")
 
 
+def pa_selftest_bounded_wait(limit_us: int, stream=None):
+    """Launch the bounded-wait self-test (a wait nothing completes)."""
+    _check(load().pa_selftest_bounded_wait(int(limit_us), _stream(stream)),
+           "pa_selftest_bounded_wait")
+
+
 def pa_get_last_device_error() -> int:
     code = ctypes.c_uint(0)
     _check(load().pa_get_last_device_error(ctypes.byref(code)), "pa_get_last_device_error")
     return int(code.value)
+
+
+class BlockManager:
+    """Host KV block manager (C++ in libpa): shared free pool, reference
+    counts, slot allocation per decode step and copy-on-write decisions."""
+
+    def __init__(self, num_blocks: int, block_size: int):
+        self._lib = load()
+        self._h = self._lib.pa_bm_create(num_blocks, block_size)
+        if not self._h:
+            raise PAError(PA_ERR_INVALID_ARG, "pa_bm_create")
+        self.num_blocks, self.block_size = num_blocks, block_size
+
+    def close(self):
+        if self._h:
+            self._lib.pa_bm_destroy(self._h)
+            self._h = None
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass
+
+    def num_free(self) -> int:
+        return int(self._lib.pa_bm_num_free(self._h))
+
+    def refcount(self, block: int) -> int:
+        return int(self._lib.pa_bm_refcount(self._h, int(block)))
+
+    def add_sequence(self, seq: int, prompt_len: int):
+        _check(self._lib.pa_bm_add_sequence(self._h, int(seq), int(prompt_len)), "pa_bm_add_sequence")
+
+    def fork(self, parent: int, child: int):
+        _check(self._lib.pa_bm_fork(self._h, int(parent), int(child)), "pa_bm_fork")
+
+    def free_sequence(self, seq: int):
+        _check(self._lib.pa_bm_free_sequence(self._h, int(seq)), "pa_bm_free_sequence")
+
+    def append_slots(self, seqs):
+        """Reserve each sequence's next slot.  Returns (slots int64 [n],
+        cow_pairs int64 [p, 2])."""
+        import numpy as np
+        ids = np.ascontiguousarray(seqs, dtype=np.int64)
+        n = ids.shape[0]
+        slots = np.empty(n, dtype=np.int64)
+        pairs = np.empty((max(n, 1), 2), dtype=np.int64)
+        npairs = ctypes.c_int(0)
+        _check(self._lib.pa_bm_append_slots(self._h, ids.ctypes.data, n, slots.ctypes.data,
+                                            pairs.ctypes.data, ctypes.byref(npairs)),
+               "pa_bm_append_slots")
+        return slots, pairs[:npairs.value].copy()
+
+    def block_tables(self, seqs, max_blocks: int):
+        """(block_tables int32 [n, max_blocks] padded with -1, context_lens int32 [n])."""
+        import numpy as np
+        ids = np.ascontiguousarray(seqs, dtype=np.int64)
+        n = ids.shape[0]
+        tables = np.empty((n, max_blocks), dtype=np.int32)
+        lens = np.empty(n, dtype=np.int32)
+        _check(self._lib.pa_bm_block_tables(self._h, ids.ctypes.data, n, tables.ctypes.data,
+                                            int(max_blocks), lens.ctypes.data),
+               "pa_bm_block_tables")
+        return tables, lens
+

@@ -3,7 +3,7 @@
     python -m paged_kv_cache_481_b200.build [--force] [--verbose-ptxas]
 
 The library is compiled from csrc/pa.cu (which includes the kernel headers)
-for ``arch=compute_100a,code=sm_100a`` only, with the CUDA runtime linked
+and csrc/block_manager.cpp (host code) for ``arch=compute_100a,code=sm_100a`` only, with the CUDA runtime linked
 statically so the .so does not depend on the toolkit's libcudart at run time.
 """
 from __future__ import annotations
@@ -31,7 +31,8 @@ def _nvcc() -> str:
 
 def _sources():
     return sorted(glob.glob(os.path.join(CSRC, "*.cu")) + glob.glob(os.path.join(CSRC, "*.cuh"))
-                  + [os.path.join(ROOT, "include", "pa.h")])
+                  + glob.glob(os.path.join(CSRC, "*.cpp"))
+                  + glob.glob(os.path.join(ROOT, "include", "*.h")))
 
 
 def up_to_date() -> bool:
@@ -48,7 +49,7 @@ def build(force: bool = False, verbose_ptxas: bool = False) -> str:
     cmd = [_nvcc(), *ARCH_FLAGS, "-O3", "-lineinfo", "-std=c++17", "-shared",
            "-Xcompiler", "-fPIC", "-Xcompiler", "-fvisibility=hidden",
            "-cudart", "static", "-I", os.path.join(ROOT, "include"),
-           "-o", tmp, os.path.join(CSRC, "pa.cu")]
+           "-o", tmp, os.path.join(CSRC, "pa.cu"), os.path.join(CSRC, "block_manager.cpp")]
     if verbose_ptxas:
         cmd.insert(1, "-Xptxas=-v")
     subprocess.run(cmd, check=True)

@@ -78,4 +78,20 @@ __global__ void __launch_bounds__(kCopyThreads) copy_blocks_kernel(
     }
 }
 
+// Self-test of the bounded wait every kernel here relies on: one warp waits
+// on an mbarrier that nothing ever arrives at; the wait must give up after
+// limit_ns and record PA_DEVERR_TIMEOUT, leaving the context usable.
+__global__ void __launch_bounds__(32) bounded_wait_selftest_kernel(uint64_t limit_ns)
+{
+    __shared__ __align__(8) uint64_t bar;
+    if (threadIdx.x == 0) {
+        mbar_init(smem_u32(&bar), 1);
+        fence_mbar_init();
+    }
+    __syncwarp();
+    const bool ok = mbar_wait_bounded(smem_u32(&bar), 0u, limit_ns);
+    if (!__all_sync(kFullMask, ok) && threadIdx.x == 0)
+        raise_device_error(kErrTimeout);
+}
+
 } // namespace pa

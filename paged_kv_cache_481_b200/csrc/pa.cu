@@ -127,6 +127,7 @@ const char *pa_status_string(pa_status status)
     case PA_ERR_UNSUPPORTED: return "unsupported head_dim or block_size";
     case PA_ERR_CUDA: return "CUDA runtime error";
     case PA_ERR_WORKSPACE: return "workspace missing or too small";
+    case PA_ERR_OUT_OF_BLOCKS: return "no free blocks left in the pool";
     }
     return "unknown status";
 }
@@ -169,6 +170,15 @@ pa_status pa_reshape_and_cache(const void *key, const void *value, void *k_cache
                       block_size, num_blocks) == cudaSuccess
                ? PA_OK
                : PA_ERR_CUDA;
+}
+
+pa_status pa_selftest_bounded_wait(unsigned int limit_us, pa_stream_t stream)
+{
+    if (limit_us == 0 || limit_us > 2000000u)
+        return PA_ERR_INVALID_ARG;
+    pa::bounded_wait_selftest_kernel<<<1, 32, 0, reinterpret_cast<cudaStream_t>(stream)>>>(
+        uint64_t(limit_us) * 1000ull);
+    return cudaGetLastError() == cudaSuccess ? PA_OK : PA_ERR_CUDA;
 }
 
 pa_status pa_copy_blocks(void *k_cache, void *v_cache, const int64_t *block_mapping, int num_pairs,

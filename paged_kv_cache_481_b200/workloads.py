@@ -103,14 +103,21 @@ def _randn_half(shape, gen, device) -> torch.Tensor:
     return torch.randn(shape, generator=gen, device=device, dtype=torch.float32).half()
 
 
-def _place_sequences(lens, bs, num_blocks, rng):
-    """Give each sequence ceil(L/bs) distinct physical ids from a random
-    permutation of the pool, in order.  Returns the [B, MB] table (-1 unused)."""
+def _place_sequences(lens, bs, num_blocks, rng, placement="shuffled"):
+    """Give each sequence ceil(L/bs) distinct physical ids, in order, from a
+    random permutation of the pool ("shuffled") or from the pool in address
+    order ("sequential": each sequence's blocks are physically consecutive,
+    the contiguous-cache baseline).  Returns the [B, MB] table (-1 unused)."""
     nblk = [(int(x) + bs - 1) // bs for x in lens]
     need = sum(nblk)
     if need > num_blocks:
         raise ValueError(f"pool of {num_blocks} blocks cannot hold {need}")
-    perm = rng.permutation(num_blocks).astype(np.int32)
+    if placement == "sequential":
+        perm = np.arange(num_blocks, dtype=np.int32)
+    elif placement == "shuffled":
+        perm = rng.permutation(num_blocks).astype(np.int32)
+    else:
+        raise ValueError(placement)
     mb = max(max(nblk) if nblk else 1, 1)
     tables = np.full((len(lens), mb), -1, dtype=np.int32)
     off = 0
@@ -144,7 +151,7 @@ def _newest_token_slots(lens, tables, bs):
 
 def build_paged(name, seed, lens, num_heads, head_dim, block_size, num_blocks,
                 scale, device="cpu", rng=None, keep_logical=False,
-                logical_fn=None) -> PagedWorkload:
+                logical_fn=None, placement="shuffled") -> PagedWorkload:
     """Generic builder: lengths -> placement -> values -> canary-marked pool.
 
     Every sequence must have L >= 1 (its newest token is written by the cache
@@ -156,7 +163,7 @@ def build_paged(name, seed, lens, num_heads, head_dim, block_size, num_blocks,
     if (lens < 1).any():
         raise ValueError("every sequence needs at least its newest token")
     rng = rng if rng is not None else np.random.default_rng(seed)
-    tables = _place_sequences(lens, block_size, num_blocks, rng)
+    tables = _place_sequences(lens, block_size, num_blocks, rng, placement)
     gen = torch.Generator(device=device).manual_seed(seed)
     h, d, bs = num_heads, head_dim, block_size
     q = _randn_half((len(lens), h, d), gen, device)
@@ -203,10 +210,12 @@ def config_lengths(cfg: int, seed: int) -> np.ndarray:
 
 def make_workload(cfg: int, device="cpu", seed: int | None = None,
                   block_size: int | None = None, keep_logical: bool = False,
-                  num_seqs: int | None = None) -> PagedWorkload:
+                  num_seqs: int | None = None, placement: str = "shuffled") -> PagedWorkload:
     """Build standard configuration ``cfg`` (1..5).  ``seed`` defaults to the
     config index (use cfg + 10 for the second draw).  ``num_seqs`` truncates
-    the batch (smaller parity cases with the same length distribution)."""
+    the batch (smaller parity cases with the same length distribution);
+    ``placement="sequential"`` lays every sequence out in consecutive
+    physical blocks (same lengths and values)."""
     seed = cfg if seed is None else seed
     if cfg == 4:
         return make_shared_prefix(device=device, seed=seed, keep_logical=keep_logical,
@@ -230,7 +239,7 @@ def make_workload(cfg: int, device="cpu", seed: int | None = None,
     need = sum((int(x) + bs - 1) // bs for x in lens)
     nb = nb_fixed if nb_fixed is not None else int(math.ceil(factor * need))
     return build_paged(WORKLOAD_NAMES[cfg], seed, lens, h, d, bs, nb, 1.0 / math.sqrt(d),
-                       device=device, rng=rng, keep_logical=keep_logical)
+                       device=device, rng=rng, keep_logical=keep_logical, placement=placement)
 
 
 def make_shared_prefix(device="cpu", seed: int = 4, num_groups: int = 8,

@@ -1,6 +1,7 @@
 """The C-ABI library loads and exports every symbol include/pa.h declares;
 host-side validation answers without touching a GPU."""
 import ctypes
+import glob
 import os
 import re
 
@@ -19,9 +20,11 @@ def lib():
 
 
 def _declared_functions():
-    text = open(HEADER).read()
-    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
-    return sorted(set(re.findall(r"\b(pa_[a-z_]+)\s*\(", text)))
+    names = set()
+    for path in glob.glob(os.path.join(ROOT, "include", "*.h")):
+        text = re.sub(r"/\*.*?\*/", "", open(path).read(), flags=re.S)
+        names |= set(re.findall(r"\b(pa_[a-z_]+)\s*\(", text))
+    return sorted(names)
 
 
 def test_header_declares_the_binding_names():
@@ -46,6 +49,7 @@ def test_status_strings(lib):
     assert binding.status_string(0) == "ok"
     assert "workspace" in binding.status_string(4)
     assert binding.status_string(99) == "unknown status"
+    assert "free blocks" in binding.status_string(binding.PA_ERR_OUT_OF_BLOCKS)
 
 
 def test_workspace_size_covers_partials_and_tickets(lib):

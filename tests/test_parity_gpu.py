@@ -343,3 +343,24 @@ def test_opt66b_heads_block_size_sweep_sampled(bs):
     ref = _sampled_oracle(wl, seqs)
     assert max_abs_err(out[torch.from_numpy(seqs).cuda()], ref) <= ATOL
     _assert_no_device_error()
+
+
+# ------------------------------------------------------ failure detection
+
+def test_bounded_wait_gives_up_and_the_context_stays_usable():
+    """A wait that nothing completes ends after its limit with
+    PA_DEVERR_TIMEOUT in the error word; the next decode still matches."""
+    import time
+    torch.cuda.synchronize()
+    t0 = time.perf_counter()
+    binding.pa_selftest_bounded_wait(20000)           # 20 ms
+    assert binding.pa_get_last_device_error() == binding.PA_DEVERR_TIMEOUT
+    elapsed = time.perf_counter() - t0
+    assert 0.015 < elapsed < 5.0
+    assert binding.pa_get_last_device_error() == 0     # read clears it
+    wl = workloads.make_random(140, [300, 20], num_heads=2, head_dim=128, block_size=16,
+                               keep_logical=False)
+    out, _, _ = gpu_write_and_decode(wl)
+    ref, _, _ = oracle_write_and_decode(wl)
+    assert max_abs_err(out, ref) <= ATOL
+    _assert_no_device_error()

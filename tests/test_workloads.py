@@ -91,3 +91,12 @@ def test_unique_bytes_count_shared_blocks_once():
     unique = accounting.decode_unique_bytes(wl.alias_block_tables, wl.context_lens, 2, 64, 16)
     shared_rows = 2 * (4 - 1) * 64               # prefix rows read by the 3 other members
     assert logical - unique == shared_rows * accounting.kv_bytes_per_token(2, 64)
+
+
+def test_sequential_placement_keeps_values_and_makes_blocks_consecutive():
+    a = workloads.make_workload(1, keep_logical=True)
+    b = workloads.make_workload(1, keep_logical=True, placement="sequential")
+    for x, y in zip(a.logical_k, b.logical_k):
+        assert np.array_equal(x.numpy(), y.numpy())
+    ids = b.block_tables[b.block_tables >= 0]
+    assert np.array_equal(ids, np.arange(len(ids)))
