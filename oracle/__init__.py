@@ -75,6 +75,14 @@ def _load():
         lib.oracle_paged_decode.argtypes = [vp, vp, i64, vp, vp, vp, vp, i32, vp,
                                             i32, i32, i32, i32, i32, ctypes.c_double]
         lib.oracle_paged_decode.restype = i32
+        lib.oracle_quantize_rows.argtypes = [vp, i32, i32, i32, vp, vp]
+        lib.oracle_quantize_rows.restype = i32
+        lib.oracle_reshape_and_cache_int8.argtypes = [vp, vp, vp, vp, vp, vp, vp, i32, i32, i32,
+                                                      i32, i32]
+        lib.oracle_reshape_and_cache_int8.restype = i32
+        lib.oracle_paged_decode_int8.argtypes = [vp, vp, vp, vp, vp, vp, vp, i32, vp, i32, i32,
+                                                 i32, i32, i32, ctypes.c_double]
+        lib.oracle_paged_decode_int8.restype = i32
         lib.oracle_num_threads.argtypes = []
         lib.oracle_num_threads.restype = i32
         _lib = lib
@@ -172,3 +180,60 @@ def paged_decode(q, k_cache, v_cache, block_tables, context_lens, scale,
                                      b, h, d, bs, nb, float(scale))
     _check(rc, "paged_decode")
     return (out, probs) if return_probs else out
+
+
+# ---------------------------------------------------------------- int8 KV
+
+def quantize_rows(x, bits: int = 8):
+    """Affine quantization of each row of x ([n, D] fp16), brentwoodlivery.com
+    5.3.18: returns (codes uint8 [n, D], params float32 [n, 2] = (s, z))."""
+    x = _bits(x)
+    n, d = x.shape
+    codes = np.zeros((n, d), dtype=np.uint8)
+    params = np.zeros((n, 2), dtype=np.float32)
+    _check(_load().oracle_quantize_rows(_ptr(x), n, d, bits, _ptr(codes), _ptr(params)),
+           "quantize_rows")
+    return codes, params
+
+
+def dequantize(codes, params):
+    """r_hat = s (q - z), in float64."""
+    p = np.asarray(params, dtype=np.float64)
+    return p[..., 0:1] * (np.asarray(codes, dtype=np.float64) - p[..., 1:2])
+
+
+def reshape_and_cache_int8(key, value, k_codes, v_codes, k_params, v_params, slot_mapping,
+                           block_size):
+    """Return new (k_codes, v_codes, k_params, v_params) after quantizing each
+    token's rows into its slot (negative slots skipped).  Inputs unchanged."""
+    key, value = _bits(key), _bits(value)
+    kc, vc = np.ascontiguousarray(k_codes, np.uint8).copy(), np.ascontiguousarray(v_codes, np.uint8).copy()
+    kp, vp_ = np.ascontiguousarray(k_params, np.float32).copy(), np.ascontiguousarray(v_params, np.float32).copy()
+    slots = np.ascontiguousarray(slot_mapping, dtype=np.int64)
+    n, h, d = key.shape
+    nb = kc.shape[0]
+    assert kc.shape == (nb, h, block_size, d) and kp.shape == (nb, h, block_size, 2)
+    rc = _load().oracle_reshape_and_cache_int8(_ptr(key), _ptr(value), _ptr(kc), _ptr(vc),
+                                               _ptr(kp), _ptr(vp_), _ptr(slots), n, h, d,
+                                               block_size, nb)
+    _check(rc, "reshape_and_cache_int8")
+    return kc, vc, kp, vp_
+
+
+def paged_decode_int8(q, k_codes, v_codes, k_params, v_params, block_tables, context_lens, scale):
+    """fp64 paged decode over the dequantized int8 cache: out [B, H, D] float64."""
+    q = _bits(q)
+    kc, vc = np.ascontiguousarray(k_codes, np.uint8), np.ascontiguousarray(v_codes, np.uint8)
+    kp, vp_ = np.ascontiguousarray(k_params, np.float32), np.ascontiguousarray(v_params, np.float32)
+    tables = np.ascontiguousarray(block_tables, dtype=np.int32)
+    lens = np.ascontiguousarray(context_lens, dtype=np.int32)
+    b, h, d = q.shape
+    nb, hk, bs, dk = kc.shape
+    assert (hk, dk) == (h, d) and kp.shape == (nb, h, bs, 2)
+    out = np.zeros((b, h, d), dtype=np.float64)
+    rc = _load().oracle_paged_decode_int8(_ptr(out), _ptr(q), _ptr(kc), _ptr(vc), _ptr(kp),
+                                          _ptr(vp_), _ptr(tables), tables.shape[1], _ptr(lens),
+                                          b, h, d, bs, nb, float(scale))
+    _check(rc, "paged_decode_int8")
+    return out
+

@@ -249,6 +249,163 @@ int oracle_paged_decode(double *out, double *probs, int64_t probs_stride,
     return status;
 }
 
+/* ------------------------------------------------------------------------
+ * Low-bit KV cache (brentwoodlivery.com "5.3.18 LLM serving, vLLM, quantized
+ * inference": the KV cache can be kept in low-bit integer formats; affine
+ * quantization s = (r_max - r_min) / (2^b - 1), z = round(-r_min / s),
+ * q = round(r / s) + z, r_hat = s (q - z), with one (s, z) per group of
+ * values; the page uses groups of 128).  Here a group is one (token, head)
+ * row of head_dim values, b = 8, codes stored as uint8 (clamped to
+ * [0, 2^b - 1]).  The rounding decisions are taken in fp32, the precision
+ * the GPU kernel uses (the page fixes none); round = round half to even.
+ * A row whose values are all equal (r_max == r_min = c) has no spread: it
+ * uses s = |c| (or 1 when c is 0), so z = -sign(c), every code is 0 and
+ * s (0 - z) = c exactly.
+ */
+static void quantize_row_f32(const uint16_t *x, int64_t D, int bits, uint8_t *codes,
+                             float *s_out, float *z_out)
+{
+    const float qmax = (float)((1 << bits) - 1);
+    float rmin = INFINITY, rmax = -INFINITY;
+    for (int64_t d = 0; d < D; ++d) {
+        const float v = (float)h2d(x[d]);
+        if (v < rmin)
+            rmin = v;
+        if (v > rmax)
+            rmax = v;
+    }
+    float s = (rmax - rmin) / qmax;
+    if (s == 0.0f)
+        s = rmax != 0.0f ? fabsf(rmax) : 1.0f;
+    const float z = rintf(-rmin / s);
+    for (int64_t d = 0; d < D; ++d) {
+        float q = rintf((float)h2d(x[d]) / s) + z;
+        if (q < 0.0f)
+            q = 0.0f;
+        if (q > qmax)
+            q = qmax;
+        codes[d] = (uint8_t)q;
+    }
+    *s_out = s;
+    *z_out = z;
+}
+
+/* Quantize n rows of D fp16 values: codes [n, D] uint8, params [n, 2] (s, z). */
+int oracle_quantize_rows(const uint16_t *x, int n, int D, int bits, uint8_t *codes, float *params)
+{
+    if (n < 0 || D <= 0 || bits < 2 || bits > 8)
+        return ORACLE_ERR_ARG;
+    pthread_once(&half_table_once, fill_half_table);
+    for (int i = 0; i < n; ++i)
+        quantize_row_f32(x + (int64_t)i * D, D, bits, codes + (int64_t)i * D, &params[2 * i],
+                         &params[2 * i + 1]);
+    return ORACLE_OK;
+}
+
+/* Cache write into the int8 cache: token i's key/value row of head h is
+ * quantized and stored at (slot / bs, h, slot % bs).  Caches: codes
+ * [NB, H, bs, D] uint8, params [NB, H, bs, 2] float (s, z). */
+int oracle_reshape_and_cache_int8(const uint16_t *key, const uint16_t *value, uint8_t *k_codes,
+                                  uint8_t *v_codes, float *k_params, float *v_params,
+                                  const int64_t *slot_mapping, int num_tokens, int num_heads,
+                                  int head_dim, int block_size, int num_blocks)
+{
+    if (num_tokens < 0 || num_heads <= 0 || head_dim <= 0 || block_size <= 0 || num_blocks <= 0)
+        return ORACLE_ERR_ARG;
+    pthread_once(&half_table_once, fill_half_table);
+    const int64_t H = num_heads, D = head_dim, bs = block_size;
+    for (int i = 0; i < num_tokens; ++i) {
+        const int64_t slot = slot_mapping[i];
+        if (slot < 0)
+            continue;
+        if (slot >= (int64_t)num_blocks * bs)
+            return ORACLE_ERR_RANGE;
+        const int64_t row0 = (slot / bs) * H * bs + slot % bs;
+        for (int64_t h = 0; h < H; ++h) {
+            const int64_t row = row0 + h * bs;
+            quantize_row_f32(key + ((int64_t)i * H + h) * D, D, 8, k_codes + row * D,
+                             &k_params[2 * row], &k_params[2 * row + 1]);
+            quantize_row_f32(value + ((int64_t)i * H + h) * D, D, 8, v_codes + row * D,
+                             &v_params[2 * row], &v_params[2 * row + 1]);
+        }
+    }
+    return ORACLE_OK;
+}
+
+/* Paged decode over the int8 cache: each gathered row is dequantized exactly
+ * (r_hat = s (q - z) in double) and the attention is the same as
+ * oracle_paged_decode's. */
+int oracle_paged_decode_int8(double *out, const uint16_t *q, const uint8_t *k_codes,
+                             const uint8_t *v_codes, const float *k_params, const float *v_params,
+                             const int32_t *block_tables, int max_blocks_per_seq,
+                             const int32_t *context_lens, int num_seqs, int num_heads,
+                             int head_dim, int block_size, int num_blocks, double scale)
+{
+    if (num_seqs < 0 || num_heads <= 0 || head_dim <= 0 || block_size <= 0 ||
+        num_blocks <= 0 || max_blocks_per_seq < 0)
+        return ORACLE_ERR_ARG;
+    pthread_once(&half_table_once, fill_half_table);
+    const int64_t H = num_heads, D = head_dim, bs = block_size;
+    for (int b = 0; b < num_seqs; ++b)
+        if (context_lens[b] < 0 || (int64_t)context_lens[b] > (int64_t)max_blocks_per_seq * bs)
+            return ORACLE_ERR_ARG;
+    int status = ORACLE_OK;
+    const int64_t units = (int64_t)num_seqs * H;
+#pragma omp parallel for schedule(dynamic, 1) reduction(max : status)
+    for (int64_t u = 0; u < units; ++u) {
+        const int b = (int)(u / H), h = (int)(u % H);
+        const int len = context_lens[b];
+        const int32_t *table = block_tables + (int64_t)b * max_blocks_per_seq;
+        double *o = out + u * D;
+        for (int64_t d = 0; d < D; ++d)
+            o[d] = 0.0;
+        if (len == 0)
+            continue;
+        double *sc = (double *)malloc(sizeof(double) * (size_t)len);
+        if (!sc) {
+            status = status > ORACLE_ERR_ARG ? status : ORACLE_ERR_ARG;
+            continue;
+        }
+        double m = -INFINITY;
+        int rc = ORACLE_OK;
+        for (int t = 0; t < len && rc == ORACLE_OK; ++t) {
+            const int64_t p = table[t / bs];
+            if (p < 0 || p >= num_blocks) {
+                rc = ORACLE_ERR_RANGE;
+                break;
+            }
+            const int64_t row = (p * H + h) * bs + t % bs;
+            const double s = k_params[2 * row], z = k_params[2 * row + 1];
+            double dot = 0.0;
+            for (int64_t d = 0; d < D; ++d)
+                dot += h2d(q[u * D + d]) * (s * ((double)k_codes[row * D + d] - z));
+            sc[t] = scale * dot;
+            if (sc[t] > m)
+                m = sc[t];
+        }
+        if (rc == ORACLE_OK) {
+            double l = 0.0;
+            for (int t = 0; t < len; ++t) {
+                sc[t] = exp(sc[t] - m);
+                l += sc[t];
+            }
+            for (int t = 0; t < len; ++t) {
+                const int64_t p = table[t / bs];
+                const int64_t row = (p * H + h) * bs + t % bs;
+                const double s = v_params[2 * row], z = v_params[2 * row + 1];
+                for (int64_t d = 0; d < D; ++d)
+                    o[d] += sc[t] * (s * ((double)v_codes[row * D + d] - z));
+            }
+            for (int64_t d = 0; d < D; ++d)
+                o[d] /= l;
+        }
+        free(sc);
+        if (rc > status)
+            status = rc;
+    }
+    return status;
+}
+
 /* Number of OpenMP threads a parallel region would use (for reporting). */
 int oracle_num_threads(void)
 {

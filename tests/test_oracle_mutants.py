@@ -28,6 +28,11 @@ MUTANTS = {
                             "return batch * seq_len * layers * d_model * bytes_per_elem;"),
     "head_stride": ("const uint16_t *v = v_cache + ((p * H + h) * bs + t % bs) * D;",
                     "const uint16_t *v = v_cache + ((p * H + (h + 1) % H) * bs + t % bs) * D;"),
+    "quant_levels": ("const float qmax = (float)((1 << bits) - 1);",
+                     "const float qmax = (float)(1 << bits);"),
+    "quant_zero_point_unrounded": ("const float z = rintf(-rmin / s);", "const float z = -rmin / s;"),
+    "dequant_sign": ("dot += h2d(q[u * D + d]) * (s * ((double)k_codes[row * D + d] - z));",
+                     "dot += h2d(q[u * D + d]) * (s * ((double)k_codes[row * D + d] + z));"),
 }
 
 
@@ -43,6 +48,7 @@ def test_pins_catch_planted_mistake(name, tmp_path):
                     "-o", str(lib), str(mutant_c), "-lm"], check=True)
     env = dict(os.environ, PA_ORACLE_LIB=str(lib))
     r = subprocess.run([sys.executable, "-m", "pytest", "-x", "-q", "-p", "no:cacheprovider",
-                        os.path.join(ROOT, "tests", "test_oracle_pins.py")],
+                        os.path.join(ROOT, "tests", "test_oracle_pins.py"),
+                        os.path.join(ROOT, "tests", "test_quant_pins.py")],
                        cwd=ROOT, env=env, capture_output=True, text=True, timeout=600)
     assert r.returncode == 1, f"pins did not catch {name}:\n{r.stdout[-2000:]}"
