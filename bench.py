@@ -297,11 +297,13 @@ def run_gpu(args):
     binding.load()
 
     cfg = args.workload
+    int8 = args.kv_dtype == "int8"
     wl = workloads.make_workload(cfg, device="cuda", seed=rank_seed(cfg, rank),
-                                 block_size=args.block_size, placement=args.placement)
+                                 block_size=args.block_size, placement=args.placement,
+                                 keep_tokens=int8)
     dev = torch.device("cuda", local)
     cpu_sample = None
-    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+    if rank == 0 and world == 1 and not args.no_cpu_baseline and not int8:
         cpu_sample = cpu_baseline_sample(wl, target_s=args.cpu_seconds)
     stream = torch.cuda.Stream(device=dev)
     b, h, d = wl.num_seqs, wl.num_heads, wl.head_dim
@@ -315,19 +317,55 @@ def run_gpu(args):
     out = torch.empty_like(q)
     mcl = wl.max_context_len
     ws = binding.new_workspace(b, h, d, mcl, device=dev)
+    if int8:
+        # the int8 pool is filled by the int8 cache write of every context
+        # token; the fp16 pool is then released
+        nbk, bsz = wl.num_blocks, wl.block_size
+        kc = torch.zeros((nbk, h, bsz, d), dtype=torch.uint8, device=dev)
+        vc = torch.zeros_like(kc)
+        kp = torch.zeros((nbk, h, bsz, 2), dtype=torch.float32, device=dev)
+        vp = torch.zeros_like(kp)
+        all_k, all_v, all_s = workloads.all_token_writes(wl)
+        binding.pa_reshape_and_cache_int8(all_k, all_v, kc, vc, kp, vp,
+                                          torch.from_numpy(all_s).to(dev))
+        del all_k, all_v
+        wl.device_k = wl.device_v = None
+        torch.cuda.synchronize()
     torch.cuda.synchronize()
+
+    def write_step(d_key, d_value, d_slots):
+        if int8:
+            binding.pa_reshape_and_cache_int8(d_key, d_value, kc, vc, kp, vp, d_slots,
+                                              stream=stream)
+        else:
+            binding.pa_reshape_and_cache(d_key, d_value, kc, vc, d_slots, stream=stream)
+
+    def decode_step(d_out, d_q, d_tables, d_lens):
+        if int8:
+            binding.pa_decode_int8(d_out, d_q, kc, vc, kp, vp, d_tables, d_lens, mcl, wl.scale,
+                                   ws, stream=stream)
+        else:
+            binding.pa_decode(d_out, d_q, kc, vc, d_tables, d_lens, mcl, wl.scale, ws,
+                              stream=stream)
+
+    def copy_step():
+        if int8:
+            for cache in (kc, vc, kp, vp):
+                binding.pa_copy_blocks_raw(cache, pairs, stream=stream)
+        else:
+            binding.pa_copy_blocks(kc, vc, pairs, stream=stream)
 
     def step(ev_pair=None):
         if pairs is not None:
-            binding.pa_copy_blocks(kc, vc, pairs, stream=stream)
-        binding.pa_reshape_and_cache(key, value, kc, vc, slots, stream=stream)
+            copy_step()
+        write_step(key, value, slots)
         if ev_pair is not None:
             ev_pair[0].record(stream)
-        binding.pa_decode(out, q, kc, vc, tables, lens, mcl, wl.scale, ws, stream=stream)
+        decode_step(out, q, tables, lens)
         if ev_pair is not None:
             ev_pair[1].record(stream)
 
-    launches_per_step = 2 + (1 if pairs is not None else 0)
+    launches_per_step = 2 + ((4 if int8 else 1) if pairs is not None else 0)
     with torch.cuda.stream(stream):
         for _ in range(args.warmup):
             step()
@@ -379,9 +417,9 @@ def run_gpu(args):
     def e2e_step():
         d_stage.copy_(h_stage, non_blocking=True)
         if pairs is not None:
-            binding.pa_copy_blocks(kc, vc, pairs, stream=stream)
-        binding.pa_reshape_and_cache(d_key, d_value, kc, vc, d_slots, stream=stream)
-        binding.pa_decode(out, d_q, kc, vc, d_tables, d_lens, mcl, wl.scale, ws, stream=stream)
+            copy_step()
+        write_step(d_key, d_value, d_slots)
+        decode_step(out, d_q, d_tables, d_lens)
         h_out.copy_(out, non_blocking=True)
 
     with torch.cuda.stream(stream):
@@ -401,14 +439,16 @@ def run_gpu(args):
     if world > 1:
         dist.barrier()
 
-    dec_bytes = accounting.decode_bytes(wl.context_lens, h, d)
+    dec_bytes = (accounting.decode_bytes_int8(wl.context_lens, h, d) if int8
+                 else accounting.decode_bytes(wl.context_lens, h, d))
     # aliased blocks are read once from DRAM and then hit L2: the roofline uses
     # the bytes DRAM must deliver (each physical row once)
     roof_bytes = dec_bytes
-    if wl.alias_block_tables is not None:
+    if wl.alias_block_tables is not None and not int8:
         roof_bytes = accounting.decode_unique_bytes(wl.block_tables, wl.context_lens, h, d,
                                                     wl.block_size)
-    step_bytes = dec_bytes + accounting.cache_write_bytes(b, h, d)
+    step_bytes = dec_bytes + (b * h * (2 * d * 2 + 2 * (d + 8)) if int8
+                              else accounting.cache_write_bytes(b, h, d))
     if pairs is not None:
         step_bytes += accounting.copy_blocks_bytes(len(wl.copy_pairs), h, d, wl.block_size)
 
@@ -431,6 +471,7 @@ def run_gpu(args):
                   f"vs {L2_BYTES / 2**20:.0f} MiB L2 (no flush)",
             "parallelism": f"dp{world} (independent batches per GPU)",
             "placement": args.placement,
+            "kv_cache": ("int8 codes + fp32 (s, z) per row" if int8 else "fp16"),
         })
         result = {
             "metric": METRIC,
@@ -439,7 +480,7 @@ def run_gpu(args):
             "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
             "ms_per_step": ms / args.steps,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
-            "dtype": "f32", "storage_dtype": "f16", "data": "synthetic",
+            "dtype": "f32", "storage_dtype": "u8" if int8 else "f16", "data": "synthetic",
             "config": desc,
             "seq_heads_per_s": total_units * args.steps / (ms * 1e-3),
             "hbm_frac": achieved / peak,
@@ -448,7 +489,8 @@ def run_gpu(args):
             "decode_us_max": max(decode_ms) * 1e3,
             "decode_us_argmax": int(np.argmax(decode_ms)),
             "roofline": {
-                "kernel": "paged_decode_kernel", "bound": "hbm", "achieved": achieved,
+                "kernel": "paged_decode_kernel" + ("<int8>" if int8 else ""), "bound": "hbm",
+                "achieved": achieved,
                 "peak": peak, "peak_kind": f"{peak_kind} (hbm_gbs)", "unit": "GB/s",
                 "frac": achieved / peak, "traffic": _recorded_traffic(desc["workload"]),
                 "algorithmic_bytes_per_launch": roof_bytes,
@@ -480,6 +522,8 @@ def main(argv=None):
     ap.add_argument("--block-size", type=int, default=None)
     ap.add_argument("--placement", choices=["shuffled", "sequential"], default="shuffled",
                     help="physical block placement (sequential = contiguous-cache baseline)")
+    ap.add_argument("--kv-dtype", choices=["fp16", "int8"], default="fp16",
+                    help="KV cache storage (int8 = 8-bit affine codes per row)")
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     args = ap.parse_args(argv)

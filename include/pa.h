@@ -165,6 +165,52 @@ PA_API pa_status pa_decode_no_alloc(void *out, const void *q, const void *k_cach
                                     int head_dim, int block_size, int num_blocks, float scale,
                                     pa_stream_t stream);
 
+/*
+ * Low-bit KV cache (brentwoodlivery.com "5.3.18 LLM serving, vLLM, quantized
+ * inference": the KV cache kept in low-bit integer form with affine
+ * quantization s = (r_max - r_min) / (2^b - 1), z = round(-r_min / s),
+ * q = round(r / s) + z, r_hat = s (q - z), one (s, z) per group of values).
+ * Here b = 8 and a group is one (token, head) row of head_dim values:
+ *   k_codes, v_codes    [num_blocks, num_heads, block_size, head_dim] uint8
+ *   k_params, v_params  [num_blocks, num_heads, block_size, 2] float (s, z)
+ * Rounding decisions are taken in fp32 (IEEE division, round half to even);
+ * codes are clamped to [0, 255]; a row whose values are all equal (c) is
+ * stored with s = |c| (1 if c = 0) and reconstructs exactly.  Rows holding
+ * inf or NaN get unspecified codes.  All arrays are device pointers, 16-byte
+ * aligned.
+ *
+ * pa_reshape_and_cache_int8: quantize each token's key/value rows and store
+ * them at their slots (same slot rules as pa_reshape_and_cache).
+ */
+PA_API pa_status pa_reshape_and_cache_int8(const void *key, const void *value, void *k_codes,
+                                           void *v_codes, void *k_params, void *v_params,
+                                           const int64_t *slot_mapping, int num_tokens,
+                                           int num_heads, int head_dim, int block_size,
+                                           int num_blocks, pa_stream_t stream);
+
+/*
+ * pa_decode over the int8 cache: K_t and V_t are the dequantized rows
+ * s (q - z); otherwise identical to pa_decode (same arguments, workspace,
+ * tolerance and determinism).  Moves about half the bytes of pa_decode.
+ */
+PA_API pa_status pa_decode_int8(void *out, const void *q, const void *k_codes,
+                                const void *v_codes, const void *k_params, const void *v_params,
+                                const int32_t *block_tables, int max_blocks_per_seq,
+                                const int32_t *context_lens, int max_context_len, int num_seqs,
+                                int num_heads, int head_dim, int block_size, int num_blocks,
+                                float scale, void *workspace, size_t workspace_bytes,
+                                pa_stream_t stream);
+
+/*
+ * Copy-on-write copy of whole blocks of any per-block byte size (use it for
+ * the int8 codes and their parameter arrays): for each (src, dst) pair, the
+ * block_bytes bytes of block src are copied to block dst of `cache`
+ * ([num_blocks, block_bytes / elem] contiguous).  block_bytes must be a
+ * multiple of 16; same pair rules as pa_copy_blocks.
+ */
+PA_API pa_status pa_copy_blocks_raw(void *cache, size_t block_bytes, const int64_t *block_mapping,
+                                    int num_pairs, int num_blocks, pa_stream_t stream);
+
 /* Static description of a status code. */
 PA_API const char *pa_status_string(pa_status status);
 

@@ -53,3 +53,13 @@ def copy_blocks_bytes(num_pairs: int, num_heads: int, head_dim: int, block_size:
                       elem_bytes: int = FP16_BYTES) -> int:
     """Whole K and V blocks read from src and written to dst."""
     return 2 * num_pairs * block_size * kv_bytes_per_token(num_heads, head_dim, elem_bytes)
+
+
+def decode_bytes_int8(context_lens, num_heads: int, head_dim: int) -> int:
+    """Int8 cache: per context token and head, K and V codes (D bytes each)
+    and their (s, z) float pairs (8 bytes each), plus q read and out written
+    in fp16."""
+    lens = np.asarray(context_lens, dtype=np.int64)
+    per_head = lens * 2 * (head_dim + 8) + 2 * head_dim * FP16_BYTES
+    return int(num_heads * per_head.sum())
+

@@ -31,7 +31,8 @@ EXPORTED = ("pa_reshape_and_cache", "pa_decode_workspace_size", "pa_decode_works
             "pa_get_last_device_error", "pa_decode_no_alloc", "pa_selftest_bounded_wait",
             "pa_bm_create", "pa_bm_destroy", "pa_bm_num_free", "pa_bm_refcount",
             "pa_bm_add_sequence", "pa_bm_fork", "pa_bm_free_sequence", "pa_bm_append_slots",
-            "pa_bm_block_tables")
+            "pa_bm_block_tables", "pa_reshape_and_cache_int8", "pa_decode_int8",
+            "pa_copy_blocks_raw")
 
 _lock = threading.Lock()
 _lib = None
@@ -88,6 +89,14 @@ def load(path: str | None = None):
         lib.pa_bm_append_slots.restype = i32
         lib.pa_bm_block_tables.argtypes = [vp, vp, i32, vp, i32, vp]
         lib.pa_bm_block_tables.restype = i32
+        lib.pa_reshape_and_cache_int8.argtypes = [vp, vp, vp, vp, vp, vp, vp, i32, i32, i32, i32,
+                                                  i32, vp]
+        lib.pa_reshape_and_cache_int8.restype = i32
+        lib.pa_decode_int8.argtypes = [vp, vp, vp, vp, vp, vp, vp, i32, vp, i32, i32, i32, i32,
+                                       i32, i32, ctypes.c_float, vp, sz, vp]
+        lib.pa_decode_int8.restype = i32
+        lib.pa_copy_blocks_raw.argtypes = [vp, sz, vp, i32, i32, vp]
+        lib.pa_copy_blocks_raw.restype = i32
         lib.pa_copy_blocks.argtypes = [vp, vp, vp, i32, i32, i32, i32, i32, vp]
         lib.pa_copy_blocks.restype = i32
         lib.pa_status_string.argtypes = [i32]
@@ -208,6 +217,47 @@ def pa_selftest_bounded_wait(limit_us: int, stream=None):
     """Launch the bounded-wait self-test (a wait nothing completes)."""
     _check(load().pa_selftest_bounded_wait(int(limit_us), _stream(stream)),
            "pa_selftest_bounded_wait")
+
+
+def pa_reshape_and_cache_int8(key, value, k_codes, v_codes, k_params, v_params, slot_mapping,
+                              stream=None):
+    """Quantize each token's K/V rows (8-bit affine, per row) into its slot."""
+    n, h, d = key.shape
+    nb, hk, bs, dk = k_codes.shape
+    assert key.dtype == value.dtype == torch.float16 and k_codes.dtype == v_codes.dtype == torch.uint8
+    assert k_params.dtype == v_params.dtype == torch.float32 and k_params.shape == (nb, h, bs, 2)
+    assert slot_mapping.dtype == torch.int64 and slot_mapping.numel() == n and (hk, dk) == (h, d)
+    _check(load().pa_reshape_and_cache_int8(_ptr(key), _ptr(value), _ptr(k_codes), _ptr(v_codes),
+                                            _ptr(k_params), _ptr(v_params), _ptr(slot_mapping),
+                                            n, h, d, bs, nb, _stream(stream)),
+           "pa_reshape_and_cache_int8")
+
+
+def pa_decode_int8(out, q, k_codes, v_codes, k_params, v_params, block_tables, context_lens,
+                   max_context_len, scale, workspace, stream=None):
+    """pa_decode over the int8 cache (dequantized rows s (q - z))."""
+    b, h, d = q.shape
+    nb, hk, bs, dk = k_codes.shape
+    assert q.dtype == out.dtype == torch.float16 and k_codes.dtype == torch.uint8
+    assert out.shape == q.shape and (hk, dk) == (h, d) and k_params.shape == (nb, h, bs, 2)
+    assert block_tables.dtype == torch.int32 and context_lens.dtype == torch.int32
+    _check(load().pa_decode_int8(_ptr(out), _ptr(q), _ptr(k_codes), _ptr(v_codes), _ptr(k_params),
+                                 _ptr(v_params), _ptr(block_tables), block_tables.shape[1],
+                                 _ptr(context_lens), int(max_context_len), b, h, d, bs, nb,
+                                 float(scale), _ptr(workspace),
+                                 workspace.numel() * workspace.element_size(), _stream(stream)),
+           "pa_decode_int8")
+
+
+def pa_copy_blocks_raw(cache, block_mapping, stream=None):
+    """Copy whole blocks (dim 0 of `cache`) src -> dst for each mapping row."""
+    nb = cache.shape[0]
+    block_bytes = cache[0].numel() * cache.element_size()
+    pairs = block_mapping.numel() // 2
+    _check(load().pa_copy_blocks_raw(_ptr(cache), block_bytes,
+                                     _ptr(block_mapping) if pairs else ctypes.c_void_p(None),
+                                     pairs, nb, _stream(stream)),
+           "pa_copy_blocks_raw")
 
 
 def pa_get_last_device_error() -> int:

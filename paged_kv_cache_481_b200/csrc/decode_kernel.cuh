@@ -35,6 +35,13 @@
 //     contributions in worker order (deterministic) and writes out.
 //   * Every wait is bounded; on expiry the worker records PA_DEVERR_TIMEOUT,
 //     lets its copies in flight land and stops.
+//   * Storage: fp16 rows, or int8 codes with one affine (s, z) per (token,
+//     head) row (brentwoodlivery.com 5.3.18: r_hat = s (q - z)).  For int8 a
+//     tile is 32 rows; the codes are widened exactly to fp16 as (q - 128)
+//     with a byte permute, the QK dot runs on them with the same
+//     mixed-precision FMA, and the zero point enters once per row:
+//       q.K = s (sum_d q_d (c_d - 128) - (z - 128) sum_d q_d),
+//     sum_t w_t V_t = sum_t w_t s_t (c_t - 128) - sum_t w_t s_t (z_t - 128).
 #pragma once
 
 #include <cuda_fp16.h>
@@ -55,14 +62,16 @@ constexpr unsigned kErrBlockId = 1u << 0;
 constexpr unsigned kErrContextLen = 1u << 1;
 constexpr unsigned kErrTimeout = 1u << 4;
 
-constexpr int kTileBytes = 4096;  // one K (or V) tile in shared memory
+constexpr int kTileBytes = 4096;  // one fp16 K (or V) tile in shared memory
 constexpr int kMaxWorkers = 4096; // warps per grid; sizes the workspace
 
 struct DecodeParams {
     __half *out;
     const __half *q;
-    const __half *k_cache;
-    const __half *v_cache;
+    const void *k_cache;     // fp16 rows or int8 codes, [NB, H, bs, D]
+    const void *v_cache;
+    const float *k_params;   // int8 only: [NB, H, bs, 2] (s, z) per row
+    const float *v_params;
     const int32_t *block_tables;
     const int32_t *context_lens;
     float *ws_o;         // [kMaxWorkers, 2, D] partial outputs of straddling units
@@ -77,17 +86,30 @@ struct DecodeParams {
     float qk_scale_log2; // softmax scale * log2(e)
 };
 
-template <int D>
+constexpr int ilog2(int x)
+{
+    return x <= 1 ? 0 : 1 + ilog2(x / 2);
+}
+
+// Tile geometry for head_dim D and fp16 (kInt8 = false) or int8 storage.
+template <int D, bool kInt8>
 struct DecodeShape {
-    static constexpr int kTokens = kTileBytes / (D * 2);  // rows per tile
-    static constexpr int kChunks = D / 8;                 // 16-byte chunks per row
-    static constexpr int kRowsPerStep = 32 / kChunks;     // rows one warp load covers
-    static constexpr int kIters = kTokens / kRowsPerStep; // warp loads per tile
-    static constexpr int kLogChunks = kChunks == 16 ? 4 : 3;
-    static constexpr int kLogIters = kIters == 8 ? 3 : (kIters == 4 ? 2 : 1);
+    static constexpr bool kQuant = kInt8;
+    static constexpr int kElemBytes = kInt8 ? 1 : 2;
+    static constexpr int kRowBytes = D * kElemBytes;
+    static constexpr int kTokens = kInt8 ? 32 : kTileBytes / kRowBytes;  // rows per tile
+    static constexpr int kTileK = kTokens * kRowBytes;                  // bytes of a K (or V) tile
+    static constexpr int kChunks = kRowBytes / 16;                      // 16-byte chunks per row
+    static constexpr int kDims = 16 / kElemBytes;                       // dims per chunk
+    static constexpr int kRowsPerStep = 32 / kChunks;                   // rows one warp load covers
+    static constexpr int kIters = kTokens / kRowsPerStep;               // warp loads per tile
+    static constexpr int kLogChunks = ilog2(kChunks);
+    static constexpr int kLogIters = ilog2(kIters);
     // after the transposing reduction, kDup adjacent lanes hold the same row
     static constexpr int kDup = 1 << (kLogChunks - kLogIters);
-    static constexpr int kMaxIds = 4;                     // block ids one tile can span (bs >= 8)
+    static constexpr int kParamBytes = kInt8 ? kTokens * 8 : 0;         // (s, z) per row
+    static constexpr int kMaxIds = 4;                                   // blocks one tile can span
+    static constexpr int kQWords = kDims / 8;                           // uint4 of q per lane
     static_assert(kChunks * kRowsPerStep == 32, "a warp covers whole rows");
     static_assert(kLogChunks >= kLogIters, "reduction keeps one row per lane group");
     static_assert(kTokens / 8 <= kMaxIds, "tile spans at most kMaxIds blocks of 8");
@@ -100,14 +122,21 @@ struct TileMeta {
     long long k;       // global tile index
 };
 
-template <int D, int NW, int S>
+template <int D, bool kInt8, int NW, int S>
 struct DecodeSmem {
-    static constexpr size_t kStageBytes = 2 * kTileBytes + D * 2;  // K, V, q row
+    using Sh = DecodeShape<D, kInt8>;
+    // stage: K tile, V tile, K params, V params, q row
+    static constexpr size_t kOffV = Sh::kTileK;
+    static constexpr size_t kOffKP = 2 * Sh::kTileK;
+    static constexpr size_t kOffVP = kOffKP + Sh::kParamBytes;
+    static constexpr size_t kOffQ = kOffVP + Sh::kParamBytes;
+    static constexpr size_t kStageBytes = kOffQ + D * 2;
     static constexpr size_t kTiles = size_t(NW) * S * kStageBytes;
     static constexpr size_t kBars = size_t(NW) * S * sizeof(uint64_t);
     static constexpr size_t kMeta = size_t(NW) * S * sizeof(TileMeta);
     static constexpr size_t kBytes = kTiles + kBars + kMeta;
     static constexpr int kThreads = NW * 32;
+    static_assert(kStageBytes % 16 == 0, "bulk-copy destinations stay 16-byte aligned");
 };
 
 __device__ __forceinline__ float2 h2f(uint32_t bits)
@@ -116,43 +145,84 @@ __device__ __forceinline__ float2 h2f(uint32_t bits)
     return __half22float2(h);
 }
 
-// q . k over one 16-byte chunk (8 fp16 each), fp32 accumulation.
-__device__ __forceinline__ float dot8(const uint4 &q, const uint4 &k)
+// Two int8 codes of a packed word, widened exactly to fp16 as (code - 128):
+// the byte permute builds halves 0x64cc = 1024 + code, then 1152 is removed.
+__device__ __forceinline__ uint32_t codes_to_h2(uint32_t word, uint32_t selector)
 {
-    float s0 = fma2_f16_f32(q.x, k.x, 0.f);
-    float s1 = fma2_f16_f32(q.y, k.y, 0.f);
-    s0 = fma2_f16_f32(q.z, k.z, s0);
-    s1 = fma2_f16_f32(q.w, k.w, s1);
-    return s0 + s1;
+    const uint32_t biased = __byte_perm(word, 0x64646464u, selector);
+    const __half2 h = __hsub2(*reinterpret_cast<const __half2 *>(&biased),
+                              __half2(__float2half_rn(1152.f), __float2half_rn(1152.f)));
+    return *reinterpret_cast<const uint32_t *>(&h);
 }
 
-__device__ __forceinline__ void axpy8(float (&acc)[8], float w, const uint4 &u)
+// q . k over one 16-byte chunk: 8 fp16 of K, or 16 int8 codes (centred).
+template <bool kInt8>
+__device__ __forceinline__ float dot_chunk(const uint4 (&q)[kInt8 ? 2 : 1], const uint4 &k)
 {
-    const float2 a = h2f(u.x), b = h2f(u.y), c = h2f(u.z), d = h2f(u.w);
-    acc[0] = fmaf(w, a.x, acc[0]);
-    acc[1] = fmaf(w, a.y, acc[1]);
-    acc[2] = fmaf(w, b.x, acc[2]);
-    acc[3] = fmaf(w, b.y, acc[3]);
-    acc[4] = fmaf(w, c.x, acc[4]);
-    acc[5] = fmaf(w, c.y, acc[5]);
-    acc[6] = fmaf(w, d.x, acc[6]);
-    acc[7] = fmaf(w, d.y, acc[7]);
+    if constexpr (!kInt8) {
+        float s0 = fma2_f16_f32(q[0].x, k.x, 0.f);
+        float s1 = fma2_f16_f32(q[0].y, k.y, 0.f);
+        s0 = fma2_f16_f32(q[0].z, k.z, s0);
+        s1 = fma2_f16_f32(q[0].w, k.w, s1);
+        return s0 + s1;
+    } else {
+        float s0 = fma2_f16_f32(q[0].x, codes_to_h2(k.x, 0x5140u), 0.f);
+        float s1 = fma2_f16_f32(q[0].y, codes_to_h2(k.x, 0x5342u), 0.f);
+        s0 = fma2_f16_f32(q[0].z, codes_to_h2(k.y, 0x5140u), s0);
+        s1 = fma2_f16_f32(q[0].w, codes_to_h2(k.y, 0x5342u), s1);
+        s0 = fma2_f16_f32(q[1].x, codes_to_h2(k.z, 0x5140u), s0);
+        s1 = fma2_f16_f32(q[1].y, codes_to_h2(k.z, 0x5342u), s1);
+        s0 = fma2_f16_f32(q[1].z, codes_to_h2(k.w, 0x5140u), s0);
+        s1 = fma2_f16_f32(q[1].w, codes_to_h2(k.w, 0x5342u), s1);
+        return s0 + s1;
+    }
+}
+
+__device__ __forceinline__ void axpy_h2(float &a0, float &a1, float w, uint32_t h2)
+{
+    const float2 v = h2f(h2);
+    a0 = fmaf(w, v.x, a0);
+    a1 = fmaf(w, v.y, a1);
+}
+
+// acc += w * chunk (8 fp16 values, or 16 centred int8 codes).
+template <bool kInt8>
+__device__ __forceinline__ void axpy_chunk(float (&acc)[kInt8 ? 16 : 8], float w, const uint4 &u)
+{
+    if constexpr (!kInt8) {
+        axpy_h2(acc[0], acc[1], w, u.x);
+        axpy_h2(acc[2], acc[3], w, u.y);
+        axpy_h2(acc[4], acc[5], w, u.z);
+        axpy_h2(acc[6], acc[7], w, u.w);
+    } else {
+        axpy_h2(acc[0], acc[1], w, codes_to_h2(u.x, 0x5140u));
+        axpy_h2(acc[2], acc[3], w, codes_to_h2(u.x, 0x5342u));
+        axpy_h2(acc[4], acc[5], w, codes_to_h2(u.y, 0x5140u));
+        axpy_h2(acc[6], acc[7], w, codes_to_h2(u.y, 0x5342u));
+        axpy_h2(acc[8], acc[9], w, codes_to_h2(u.z, 0x5140u));
+        axpy_h2(acc[10], acc[11], w, codes_to_h2(u.z, 0x5342u));
+        axpy_h2(acc[12], acc[13], w, codes_to_h2(u.w, 0x5140u));
+        axpy_h2(acc[14], acc[15], w, codes_to_h2(u.w, 0x5342u));
+    }
 }
 
 // Consume one staged tile: scores, online-softmax update and PV accumulate.
 // Lane (r, c) = (lane / kChunks, lane % kChunks) handles rows i*kRowsPerStep + r
-// and dims [8c, 8c + 8).
-template <int D, bool kFull>
+// and dims [kDims c, kDims (c + 1)).  For int8, kp / vp are the tile's (s, z)
+// rows, qsum = sum_d q_d, and corr accumulates sum_t w_t s_t (z_t - 128).
+template <int D, bool kInt8, bool kFull>
 __device__ __forceinline__ void consume_tile(const uint4 *__restrict__ ks, const uint4 *__restrict__ vs,
-                                             int valid_rows, int r, int c, const uint4 &qh,
-                                             float qk_scale_log2, float &m, float &l_part,
-                                             float (&acc)[8])
+                                             const float2 *__restrict__ kp, const float2 *__restrict__ vp,
+                                             int valid_rows, int r, int c,
+                                             const uint4 (&qh)[DecodeShape<D, kInt8>::kQWords],
+                                             float qsum, float qk_scale_log2, float &m, float &l_part,
+                                             float (&acc)[DecodeShape<D, kInt8>::kDims], float &corr)
 {
-    using S = DecodeShape<D>;
+    using S = DecodeShape<D, kInt8>;
     float v[S::kIters];
 #pragma unroll
     for (int i = 0; i < S::kIters; ++i)
-        v[i] = dot8(qh, ks[(i * S::kRowsPerStep + r) * S::kChunks + c]);
+        v[i] = dot_chunk<kInt8>(qh, ks[(i * S::kRowsPerStep + r) * S::kChunks + c]);
 
     // Transposing reduction over the kChunks lanes of a row group: each step
     // halves the number of values a lane holds while summing across lanes.
@@ -173,7 +243,13 @@ __device__ __forceinline__ void consume_tile(const uint4 *__restrict__ ks, const
         }
     }
     const int my_row = (c / S::kDup) * S::kRowsPerStep + r;
-    float s = v[0] * qk_scale_log2;
+    float s;
+    if constexpr (kInt8) {
+        const float2 pz = kp[my_row];  // (s, z) of this lane's row
+        s = pz.x * fmaf(-(pz.y - 128.f), qsum, v[0]) * qk_scale_log2;
+    } else {
+        s = v[0] * qk_scale_log2;
+    }
     if (!kFull && my_row >= valid_rows)
         s = -INFINITY;
 
@@ -186,14 +262,25 @@ __device__ __forceinline__ void consume_tile(const uint4 *__restrict__ ks, const
     const float w = exp2f(s - m_new);
     l_part = l_part * alpha + ((c % S::kDup) == 0 ? w : 0.f);
 #pragma unroll
-    for (int k = 0; k < 8; ++k)
+    for (int k = 0; k < S::kDims; ++k)
         acc[k] *= alpha;
+    if constexpr (kInt8)
+        corr *= alpha;
 
 #pragma unroll
     for (int i = 0; i < S::kIters; ++i) {
         const float wi = __shfl_sync(kFullMask, w, r * S::kChunks + i * S::kDup);
-        if (kFull || i * S::kRowsPerStep + r < valid_rows)
-            axpy8(acc, wi, vs[(i * S::kRowsPerStep + r) * S::kChunks + c]);
+        const int row = i * S::kRowsPerStep + r;
+        if (kFull || row < valid_rows) {
+            if constexpr (kInt8) {
+                const float2 pz = vp[row];
+                const float ws = wi * pz.x;
+                corr = fmaf(ws, pz.y - 128.f, corr);
+                axpy_chunk<true>(acc, ws, vs[row * S::kChunks + c]);
+            } else {
+                axpy_chunk<false>(acc, wi, vs[row * S::kChunks + c]);
+            }
+        }
     }
     m = m_new;
 }
@@ -241,11 +328,10 @@ struct TileCursor {
 
 // Block ids of the tile under the cursor, loaded one tile ahead of their use;
 // they are range-checked when the copies are issued.
-template <int D>
+template <class Sh>
 __device__ __forceinline__ void load_tile_ids(const DecodeParams &p, const TileCursor &cur,
-                                              int (&ids)[DecodeShape<D>::kMaxIds])
+                                              int (&ids)[Sh::kMaxIds])
 {
-    using Sh = DecodeShape<D>;
     const int bs = p.block_size;
     const int t0 = cur.i * Sh::kTokens;
     const int nv = min(Sh::kTokens, cur.len - t0);
@@ -257,17 +343,49 @@ __device__ __forceinline__ void load_tile_ids(const DecodeParams &p, const TileC
         ids[s] = s < nsub ? row[first + s] : 0;
 }
 
-// Arm the stage's full barrier and issue the bulk copies of the tile under
-// the cursor (K rows, V rows, and the q row when `with_q`).  K and V are read
-// exactly once, so they go through L2 with an evict-first policy that keeps
-// the small reused data (block tables, q, split partials) resident.
-template <int D>
-__device__ __forceinline__ void issue_tile(const DecodeParams &p, const TileCursor &cur,
-                                           const int (&ids)[DecodeShape<D>::kMaxIds], bool with_q,
-                                           unsigned char *stage_buf, uint32_t bar, TileMeta *meta,
-                                           uint64_t stream_policy)
+// Copy `rows` rows starting at row `row0` of the (block, head) run into the
+// stage: K and V rows, and for int8 their (s, z) pairs (rounded up to an even
+// number of rows so every copy is a multiple of 16 bytes; the extra row lies
+// inside the same block and is never used).
+template <int D, bool kInt8, class Sm>
+__device__ __forceinline__ void copy_rows(const DecodeParams &p, size_t row0, int rows, uint32_t dst,
+                                          uint32_t dst_row, uint32_t bar, uint64_t policy)
 {
-    using Sh = DecodeShape<D>;
+    using Sh = DecodeShape<D, kInt8>;
+    const uint32_t bytes = uint32_t(rows) * Sh::kRowBytes;
+    const char *k = static_cast<const char *>(p.k_cache) + row0 * Sh::kRowBytes;
+    const char *v = static_cast<const char *>(p.v_cache) + row0 * Sh::kRowBytes;
+    bulk_copy_g2s_hint(dst + dst_row * Sh::kRowBytes, k, bytes, bar, policy);
+    bulk_copy_g2s_hint(dst + Sm::kOffV + dst_row * Sh::kRowBytes, v, bytes, bar, policy);
+    if constexpr (kInt8) {
+        const uint32_t pbytes = uint32_t((rows + 1) & ~1) * 8u;
+        bulk_copy_g2s(dst + Sm::kOffKP + dst_row * 8u, p.k_params + row0 * 2, pbytes, bar);
+        bulk_copy_g2s(dst + Sm::kOffVP + dst_row * 8u, p.v_params + row0 * 2, pbytes, bar);
+    }
+}
+
+template <int D, bool kInt8>
+__device__ __forceinline__ uint32_t rows_tx_bytes(int rows)
+{
+    using Sh = DecodeShape<D, kInt8>;
+    uint32_t b = 2u * uint32_t(rows) * Sh::kRowBytes;
+    if constexpr (kInt8)
+        b += 2u * uint32_t((rows + 1) & ~1) * 8u;
+    return b;
+}
+
+// Arm the stage's full barrier and issue the bulk copies of the tile under
+// the cursor (K rows, V rows, their int8 parameters, and the q row when
+// `with_q`).  K and V are read exactly once, so they go through L2 with an
+// evict-first policy that keeps the small reused data (block tables, q, split
+// partials) resident.
+template <int D, bool kInt8, class Sm>
+__device__ __forceinline__ void issue_tile(const DecodeParams &p, const TileCursor &cur,
+                                           const int (&ids)[DecodeShape<D, kInt8>::kMaxIds],
+                                           bool with_q, unsigned char *stage_buf, uint32_t bar,
+                                           TileMeta *meta, uint64_t stream_policy)
+{
+    using Sh = DecodeShape<D, kInt8>;
     const int bs = p.block_size;
     const int t0 = cur.i * Sh::kTokens;
     const int nv = min(Sh::kTokens, cur.len - t0);
@@ -277,10 +395,7 @@ __device__ __forceinline__ void issue_tile(const DecodeParams &p, const TileCurs
     meta->len = cur.len;
     meta->k = cur.k;
 
-    const uint32_t kdst = smem_u32(stage_buf);
-    const uint32_t vdst = kdst + kTileBytes;
-    const uint32_t qdst = kdst + 2 * kTileBytes;
-    const size_t head_stride = size_t(bs) * D;  // elements between heads of a block
+    const uint32_t dst = smem_u32(stage_buf);
     // an id outside the pool is recorded and its rows are not fetched
     bool ok[Sh::kMaxIds];
 #pragma unroll
@@ -290,7 +405,7 @@ __device__ __forceinline__ void issue_tile(const DecodeParams &p, const TileCurs
     bool bad = false;
     if (bs >= Sh::kTokens) {
         if (ok[0])
-            total += 2u * uint32_t(nv) * D * 2;
+            total += rows_tx_bytes<D, kInt8>(nv);
         else
             bad = true;
     } else {
@@ -299,7 +414,7 @@ __device__ __forceinline__ void issue_tile(const DecodeParams &p, const TileCurs
             if (s * bs >= nv)
                 break;
             if (ok[s])
-                total += 2u * uint32_t(min(bs, nv - s * bs)) * D * 2;
+                total += rows_tx_bytes<D, kInt8>(min(bs, nv - s * bs));
             else
                 bad = true;
         }
@@ -308,14 +423,11 @@ __device__ __forceinline__ void issue_tile(const DecodeParams &p, const TileCurs
         raise_device_error(kErrBlockId);
     mbar_arrive_expect_tx(bar, total);
     if (with_q)
-        bulk_copy_g2s(qdst, p.q + (size_t(cur.b) * p.num_heads + cur.h) * D, D * 2, bar);
+        bulk_copy_g2s(dst + Sm::kOffQ, p.q + (size_t(cur.b) * p.num_heads + cur.h) * D, D * 2, bar);
     if (bs >= Sh::kTokens) {
-        if (ok[0]) {
-            const uint32_t bytes = uint32_t(nv) * D * 2;
-            const size_t off = (size_t(ids[0]) * p.num_heads + cur.h) * head_stride + size_t(t0 % bs) * D;
-            bulk_copy_g2s_hint(kdst, p.k_cache + off, bytes, bar, stream_policy);
-            bulk_copy_g2s_hint(vdst, p.v_cache + off, bytes, bar, stream_policy);
-        }
+        if (ok[0])
+            copy_rows<D, kInt8, Sm>(p, (size_t(ids[0]) * p.num_heads + cur.h) * bs + size_t(t0 % bs),
+                                    nv, dst, 0, bar, stream_policy);
     } else {
 #pragma unroll
         for (int s = 0; s < Sh::kMaxIds; ++s) {
@@ -323,11 +435,8 @@ __device__ __forceinline__ void issue_tile(const DecodeParams &p, const TileCurs
                 break;
             if (!ok[s])
                 continue;
-            const uint32_t bytes = uint32_t(min(bs, nv - s * bs)) * D * 2;
-            const size_t off = (size_t(ids[s]) * p.num_heads + cur.h) * head_stride;
-            const uint32_t sub = uint32_t(s) * bs * D * 2;
-            bulk_copy_g2s_hint(kdst + sub, p.k_cache + off, bytes, bar, stream_policy);
-            bulk_copy_g2s_hint(vdst + sub, p.v_cache + off, bytes, bar, stream_policy);
+            copy_rows<D, kInt8, Sm>(p, (size_t(ids[s]) * p.num_heads + cur.h) * bs,
+                                    min(bs, nv - s * bs), dst, uint32_t(s * bs), bar, stream_policy);
         }
     }
 }
@@ -335,48 +444,53 @@ __device__ __forceinline__ void issue_tile(const DecodeParams &p, const TileCurs
 // Merge the partial results of a (sequence, head) whose tiles were split
 // between workers w_first..w_last, in worker order, and write out.  One pass:
 // each contribution rescales the running sums to the running maximum, so all
-// loads are independent.  Lanes with r == 0 each handle 8 dims.
-template <int D>
+// loads are independent.  Lanes with r == 0 each handle kDims dims.
+template <int D, int kDims>
 __device__ __forceinline__ void merge_partials(const DecodeParams &p, uint4 *out_row, int c,
                                                long long u_start, long long w_first,
                                                long long w_last, long long total,
                                                long long workers)
 {
     float gmax = -INFINITY, den = 0.f;
-    float num[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+    float num[kDims];
+#pragma unroll
+    for (int k = 0; k < kDims; ++k)
+        num[k] = 0.f;
     for (long long w = w_first; w <= w_last; ++w) {
         const size_t q = size_t(w) * 2 + (u_start <= range_start(w, total, workers) ? 0 : 1);
         const float mw = __ldcg(p.ws_ml + q * 2), lw = __ldcg(p.ws_ml + q * 2 + 1);
-        const float4 *po = reinterpret_cast<const float4 *>(p.ws_o + q * D + 8 * c);
-        const float4 x = __ldcg(po), y = __ldcg(po + 1);
+        const float4 *po = reinterpret_cast<const float4 *>(p.ws_o + q * D + kDims * c);
         const float m_new = fmaxf(gmax, mw);
         const float a = exp2f(gmax - m_new), f = exp2f(mw - m_new);
         gmax = m_new;
         den = fmaf(den, a, f * lw);
-        num[0] = fmaf(num[0], a, f * x.x);
-        num[1] = fmaf(num[1], a, f * x.y);
-        num[2] = fmaf(num[2], a, f * x.z);
-        num[3] = fmaf(num[3], a, f * x.w);
-        num[4] = fmaf(num[4], a, f * y.x);
-        num[5] = fmaf(num[5], a, f * y.y);
-        num[6] = fmaf(num[6], a, f * y.z);
-        num[7] = fmaf(num[7], a, f * y.w);
-    }
-    __half2 o[4];
 #pragma unroll
-    for (int k = 0; k < 4; ++k)
+        for (int k = 0; k < kDims / 4; ++k) {
+            const float4 x = __ldcg(po + k);
+            num[4 * k + 0] = fmaf(num[4 * k + 0], a, f * x.x);
+            num[4 * k + 1] = fmaf(num[4 * k + 1], a, f * x.y);
+            num[4 * k + 2] = fmaf(num[4 * k + 2], a, f * x.z);
+            num[4 * k + 3] = fmaf(num[4 * k + 3], a, f * x.w);
+        }
+    }
+    __half2 o[kDims / 2];
+#pragma unroll
+    for (int k = 0; k < kDims / 2; ++k)
         o[k] = __floats2half2_rn(num[2 * k] / den, num[2 * k + 1] / den);
-    out_row[c] = *reinterpret_cast<const uint4 *>(o);
+#pragma unroll
+    for (int k = 0; k < kDims / 8; ++k)
+        out_row[(kDims / 8) * c + k] = reinterpret_cast<const uint4 *>(o)[k];
 }
 
-template <int D, int NW, int S>
+template <int D, bool kInt8, int NW, int S>
 __global__ void __launch_bounds__(NW * 32) paged_decode_kernel(const DecodeParams p)
 {
-    using Sh = DecodeShape<D>;
-    using Sm = DecodeSmem<D, NW, S>;
+    using Sh = DecodeShape<D, kInt8>;
+    using Sm = DecodeSmem<D, kInt8, NW, S>;
     constexpr int T = Sh::kTokens;
     constexpr int kThreads = Sm::kThreads;
     constexpr int kWarps = NW;
+    constexpr int kDims = Sh::kDims;
 
     extern __shared__ __align__(128) unsigned char smem[];
     __shared__ long long s_warp_sum[kWarps];
@@ -528,7 +642,7 @@ __global__ void __launch_bounds__(NW * 32) paged_decode_kernel(const DecodeParam
             if (s < lane)
                 mc.template advance<T>(p);
         if (lane < first)
-            load_tile_ids<D>(p, mc, ids);
+            load_tile_ids<Sh>(p, mc, ids);
         __syncwarp();
         for (int s = 0; s < first; ++s) {
             TileCursor cs;
@@ -543,9 +657,9 @@ __global__ void __launch_bounds__(NW * 32) paged_decode_kernel(const DecodeParam
             for (int e = 0; e < Sh::kMaxIds; ++e)
                 ids_s[e] = __shfl_sync(kFullMask, ids[e], s);
             if (lane == 0)
-                issue_tile<D>(p, cs, ids_s, cs.i == 0 || cs.k == lo,
-                              my_buf + size_t(s) * Sm::kStageBytes, my_bar + 8 * s, my_meta + s,
-                              policy);
+                issue_tile<D, kInt8, Sm>(p, cs, ids_s, cs.i == 0 || cs.k == lo,
+                                         my_buf + size_t(s) * Sm::kStageBytes, my_bar + 8 * s,
+                                         my_meta + s, policy);
             if (s == first - 1)
                 prod = cs;
         }
@@ -553,15 +667,19 @@ __global__ void __launch_bounds__(NW * 32) paged_decode_kernel(const DecodeParam
     int issued = first;
     if (issued < ntiles) {
         prod.template advance<T>(p);
-        load_tile_ids<D>(p, prod, ids);
+        load_tile_ids<Sh>(p, prod, ids);
     }
 
     // ---- 5. stream --------------------------------------------------------
-    uint4 qh = make_uint4(0, 0, 0, 0);
-    float m = -INFINITY, l_part = 0.f;
-    float acc[8];
+    uint4 qh[Sh::kQWords];
 #pragma unroll
-    for (int k = 0; k < 8; ++k)
+    for (int k = 0; k < Sh::kQWords; ++k)
+        qh[k] = make_uint4(0, 0, 0, 0);
+    float qsum = 0.f;
+    float m = -INFINITY, l_part = 0.f, corr = 0.f;
+    float acc[kDims];
+#pragma unroll
+    for (int k = 0; k < kDims; ++k)
         acc[k] = 0.f;
     int seg_i0 = 0;
     for (int j = 0; j < ntiles; ++j) {
@@ -581,31 +699,55 @@ __global__ void __launch_bounds__(NW * 32) paged_decode_kernel(const DecodeParam
         const int nv = min(T, mt.len - mt.i * T);
         const unsigned char *buf = my_buf + size_t(stage) * Sm::kStageBytes;
         if (mt.i == 0 || mt.k == lo) {  // first tile of a segment: fresh state, new q
-            qh = reinterpret_cast<const uint4 *>(buf + 2 * kTileBytes)[c];
+            const uint4 *qs = reinterpret_cast<const uint4 *>(buf + Sm::kOffQ);
 #pragma unroll
-            for (int k = 0; k < 8; ++k)
+            for (int k = 0; k < Sh::kQWords; ++k)
+                qh[k] = qs[Sh::kQWords * c + k];
+            if constexpr (kInt8) {
+                float part = 0.f;
+#pragma unroll
+                for (int k = 0; k < Sh::kQWords; ++k) {
+                    const uint32_t w4[4] = {qh[k].x, qh[k].y, qh[k].z, qh[k].w};
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) {
+                        const float2 f = h2f(w4[e]);
+                        part += f.x + f.y;
+                    }
+                }
+#pragma unroll
+                for (int off = Sh::kChunks >> 1; off >= 1; off >>= 1)
+                    part += __shfl_xor_sync(kFullMask, part, off);
+                qsum = part;
+            }
+#pragma unroll
+            for (int k = 0; k < kDims; ++k)
                 acc[k] = 0.f;
             m = -INFINITY;
             l_part = 0.f;
+            corr = 0.f;
             seg_i0 = mt.i;
         }
         const uint4 *ks = reinterpret_cast<const uint4 *>(buf);
-        const uint4 *vs = ks + kTileBytes / 16;
+        const uint4 *vs = reinterpret_cast<const uint4 *>(buf + Sm::kOffV);
+        const float2 *kp = reinterpret_cast<const float2 *>(buf + Sm::kOffKP);
+        const float2 *vp = reinterpret_cast<const float2 *>(buf + Sm::kOffVP);
         if (nv == T)
-            consume_tile<D, true>(ks, vs, nv, r, c, qh, p.qk_scale_log2, m, l_part, acc);
+            consume_tile<D, kInt8, true>(ks, vs, kp, vp, nv, r, c, qh, qsum, p.qk_scale_log2, m,
+                                         l_part, acc, corr);
         else
-            consume_tile<D, false>(ks, vs, nv, r, c, qh, p.qk_scale_log2, m, l_part, acc);
+            consume_tile<D, kInt8, false>(ks, vs, kp, vp, nv, r, c, qh, qsum, p.qk_scale_log2, m,
+                                          l_part, acc, corr);
         __syncwarp();
         if (issued < ntiles) {  // refill the stage just consumed
             if (lane == 0) {
                 fence_proxy_async_smem();
-                issue_tile<D>(p, prod, ids, prod.i == 0 || prod.k == lo,
-                              my_buf + size_t(stage) * Sm::kStageBytes, my_bar + 8 * stage,
-                              my_meta + stage, policy);
+                issue_tile<D, kInt8, Sm>(p, prod, ids, prod.i == 0 || prod.k == lo,
+                                         my_buf + size_t(stage) * Sm::kStageBytes,
+                                         my_bar + 8 * stage, my_meta + stage, policy);
             }
             if (++issued < ntiles) {
                 prod.template advance<T>(p);
-                load_tile_ids<D>(p, prod, ids);
+                load_tile_ids<Sh>(p, prod, ids);
             }
         }
         if (!(mt.i == nt - 1 || mt.k == hi - 1))
@@ -617,19 +759,29 @@ __global__ void __launch_bounds__(NW * 32) paged_decode_kernel(const DecodeParam
         for (int off = 16; off >= 1; off >>= 1)
             l += __shfl_xor_sync(kFullMask, l, off);
 #pragma unroll
-        for (int off = Sh::kChunks; off < 32; off <<= 1)
+        for (int off = Sh::kChunks; off < 32; off <<= 1) {
 #pragma unroll
-            for (int k = 0; k < 8; ++k)
+            for (int k = 0; k < kDims; ++k)
                 acc[k] += __shfl_xor_sync(kFullMask, acc[k], off);
+            if constexpr (kInt8)
+                corr += __shfl_xor_sync(kFullMask, corr, off);
+        }
+        if constexpr (kInt8) {
+#pragma unroll
+            for (int k = 0; k < kDims; ++k)
+                acc[k] -= corr;
+        }
         const size_t unit = size_t(mt.b) * H + mt.h;
         uint4 *out_row = reinterpret_cast<uint4 *>(p.out + unit * D);
         if (seg_i0 == 0 && mt.i == nt - 1) {
             if (r == 0) {
-                __half2 o[4];
+                __half2 o[kDims / 2];
 #pragma unroll
-                for (int k = 0; k < 4; ++k)
+                for (int k = 0; k < kDims / 2; ++k)
                     o[k] = __floats2half2_rn(acc[2 * k] / l, acc[2 * k + 1] / l);
-                out_row[c] = *reinterpret_cast<const uint4 *>(o);
+#pragma unroll
+                for (int k = 0; k < kDims / 8; ++k)
+                    out_row[(kDims / 8) * c + k] = reinterpret_cast<const uint4 *>(o)[k];
             }
             continue;
         }
@@ -637,9 +789,10 @@ __global__ void __launch_bounds__(NW * 32) paged_decode_kernel(const DecodeParam
         const int slot = u_start <= lo ? 0 : 1;     // first or last segment of this worker
         const size_t pidx = size_t(gw) * 2 + slot;
         if (r == 0) {
-            float4 *po = reinterpret_cast<float4 *>(p.ws_o + pidx * D + 8 * c);
-            po[0] = make_float4(acc[0], acc[1], acc[2], acc[3]);
-            po[1] = make_float4(acc[4], acc[5], acc[6], acc[7]);
+            float4 *po = reinterpret_cast<float4 *>(p.ws_o + pidx * D + kDims * c);
+#pragma unroll
+            for (int k = 0; k < kDims / 4; ++k)
+                po[k] = make_float4(acc[4 * k], acc[4 * k + 1], acc[4 * k + 2], acc[4 * k + 3]);
         }
         if (lane == 0) {
             p.ws_ml[pidx * 2 + 0] = m;
@@ -658,7 +811,7 @@ __global__ void __launch_bounds__(NW * 32) paged_decode_kernel(const DecodeParam
             continue;
         __threadfence();
         if (r == 0)
-            merge_partials<D>(p, out_row, c, u_start, w_first, w_last, total, workers);
+            merge_partials<D, kDims>(p, out_row, c, u_start, w_first, w_last, total, workers);
     }
 }
 

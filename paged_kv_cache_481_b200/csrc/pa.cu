@@ -75,32 +75,32 @@ WorkspaceLayout workspace_layout(int num_seqs, int num_heads, int head_dim)
     return w;
 }
 
-template <int D, int NW, int S>
+template <int D, bool kInt8, int NW, int S>
 pa_status launch_decode(const pa::DecodeParams &p, cudaStream_t stream)
 {
-    using Sm = pa::DecodeSmem<D, NW, S>;
+    using Sm = pa::DecodeSmem<D, kInt8, NW, S>;
     static std::atomic<int> grid_for[kMaxDevices];  // 0 = not configured yet
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices)
         return PA_ERR_CUDA;
     int grid = grid_for[dev].load(std::memory_order_acquire);
     if (grid == 0) {
-        if (cudaFuncSetAttribute(pa::paged_decode_kernel<D, NW, S>,
+        if (cudaFuncSetAttribute(pa::paged_decode_kernel<D, kInt8, NW, S>,
                                  cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  int(Sm::kBytes)) != cudaSuccess)
             return PA_ERR_CUDA;
         int sms = 0, per_sm = 0;
         if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess ||
-            cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, pa::paged_decode_kernel<D, NW, S>,
-                                                          pa::DecodeSmem<D, NW, S>::kThreads,
-                                                          Sm::kBytes) != cudaSuccess)
+            cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm,
+                                                          pa::paged_decode_kernel<D, kInt8, NW, S>,
+                                                          Sm::kThreads, Sm::kBytes) != cudaSuccess)
             return PA_ERR_CUDA;
         grid = sms * (per_sm > 0 ? per_sm : 1);
         if (grid * NW > pa::kMaxWorkers)
             grid = pa::kMaxWorkers / NW;
         grid_for[dev].store(grid, std::memory_order_release);
     }
-    return launch_pdl(pa::paged_decode_kernel<D, NW, S>, dim3(grid), dim3(Sm::kThreads),
+    return launch_pdl(pa::paged_decode_kernel<D, kInt8, NW, S>, dim3(grid), dim3(Sm::kThreads),
                       Sm::kBytes, stream, p) == cudaSuccess
                ? PA_OK
                : PA_ERR_CUDA;
@@ -230,11 +230,16 @@ pa_status pa_decode_workspace_init(void *workspace, size_t workspace_bytes, pa_s
                : PA_ERR_CUDA;
 }
 
-pa_status pa_decode(void *out, const void *q, const void *k_cache, const void *v_cache,
-                    const int32_t *block_tables, int max_blocks_per_seq, const int32_t *context_lens,
-                    int max_context_len, int num_seqs, int num_heads, int head_dim, int block_size,
-                    int num_blocks, float scale, void *workspace, size_t workspace_bytes,
-                    pa_stream_t stream)
+} // extern "C"
+
+namespace {
+
+pa_status decode_common(void *out, const void *q, const void *k_cache, const void *v_cache,
+                        const void *k_params, const void *v_params, bool int8,
+                        const int32_t *block_tables, int max_blocks_per_seq,
+                        const int32_t *context_lens, int max_context_len, int num_seqs,
+                        int num_heads, int head_dim, int block_size, int num_blocks, float scale,
+                        void *workspace, size_t workspace_bytes, pa_stream_t stream)
 {
     if (num_seqs < 0 || num_heads <= 0 || num_blocks <= 0 || max_context_len < 0 ||
         max_blocks_per_seq < 0)
@@ -249,6 +254,8 @@ pa_status pa_decode(void *out, const void *q, const void *k_cache, const void *v
         return PA_OK;
     if (!out || !q || !k_cache || !v_cache || !block_tables || !context_lens)
         return PA_ERR_INVALID_ARG;
+    if (int8 && (!k_params || !v_params || !aligned16(k_params) || !aligned16(v_params)))
+        return PA_ERR_INVALID_ARG;
     if (!aligned16(out) || !aligned16(q) || !aligned16(k_cache) || !aligned16(v_cache) ||
         (reinterpret_cast<uintptr_t>(block_tables) & 3u) ||
         (reinterpret_cast<uintptr_t>(context_lens) & 3u))
@@ -261,8 +268,10 @@ pa_status pa_decode(void *out, const void *q, const void *k_cache, const void *v
     pa::DecodeParams p{};
     p.out = static_cast<__half *>(out);
     p.q = static_cast<const __half *>(q);
-    p.k_cache = static_cast<const __half *>(k_cache);
-    p.v_cache = static_cast<const __half *>(v_cache);
+    p.k_cache = k_cache;
+    p.v_cache = v_cache;
+    p.k_params = static_cast<const float *>(k_params);
+    p.v_params = static_cast<const float *>(v_params);
     p.block_tables = block_tables;
     p.context_lens = context_lens;
     p.ws_o = reinterpret_cast<float *>(ws + w.o_off);
@@ -277,9 +286,100 @@ pa_status pa_decode(void *out, const void *q, const void *k_cache, const void *v
     p.qk_scale_log2 = float(double(scale) * 1.4426950408889634);  // scale * log2(e)
 
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    if (int8) {
+        if (head_dim == 128)
+            return launch_decode<128, true, kDecodeWarps, kDecodeStages>(p, s);
+        return launch_decode<64, true, kDecodeWarps, kDecodeStages>(p, s);
+    }
     if (head_dim == 128)
-        return launch_decode<128, kDecodeWarps, kDecodeStages>(p, s);
-    return launch_decode<64, kDecodeWarps, kDecodeStages>(p, s);
+        return launch_decode<128, false, kDecodeWarps, kDecodeStages>(p, s);
+    return launch_decode<64, false, kDecodeWarps, kDecodeStages>(p, s);
+}
+
+} // namespace
+
+extern "C" {
+
+pa_status pa_decode(void *out, const void *q, const void *k_cache, const void *v_cache,
+                    const int32_t *block_tables, int max_blocks_per_seq, const int32_t *context_lens,
+                    int max_context_len, int num_seqs, int num_heads, int head_dim, int block_size,
+                    int num_blocks, float scale, void *workspace, size_t workspace_bytes,
+                    pa_stream_t stream)
+{
+    return decode_common(out, q, k_cache, v_cache, nullptr, nullptr, false, block_tables,
+                         max_blocks_per_seq, context_lens, max_context_len, num_seqs, num_heads,
+                         head_dim, block_size, num_blocks, scale, workspace, workspace_bytes, stream);
+}
+
+pa_status pa_decode_int8(void *out, const void *q, const void *k_codes, const void *v_codes,
+                         const void *k_params, const void *v_params, const int32_t *block_tables,
+                         int max_blocks_per_seq, const int32_t *context_lens, int max_context_len,
+                         int num_seqs, int num_heads, int head_dim, int block_size, int num_blocks,
+                         float scale, void *workspace, size_t workspace_bytes, pa_stream_t stream)
+{
+    return decode_common(out, q, k_codes, v_codes, k_params, v_params, true, block_tables,
+                         max_blocks_per_seq, context_lens, max_context_len, num_seqs, num_heads,
+                         head_dim, block_size, num_blocks, scale, workspace, workspace_bytes, stream);
+}
+
+pa_status pa_reshape_and_cache_int8(const void *key, const void *value, void *k_codes,
+                                    void *v_codes, void *k_params, void *v_params,
+                                    const int64_t *slot_mapping, int num_tokens, int num_heads,
+                                    int head_dim, int block_size, int num_blocks, pa_stream_t stream)
+{
+    if (num_tokens < 0 || num_heads <= 0 || num_blocks <= 0)
+        return PA_ERR_INVALID_ARG;
+    if (!supported_head_dim(head_dim) || !supported_block_size(block_size))
+        return PA_ERR_UNSUPPORTED;
+    if (num_tokens == 0)
+        return PA_OK;
+    if (!key || !value || !k_codes || !v_codes || !k_params || !v_params || !slot_mapping)
+        return PA_ERR_INVALID_ARG;
+    if (!aligned16(key) || !aligned16(value) || !aligned16(k_codes) || !aligned16(v_codes) ||
+        !aligned16(k_params) || !aligned16(v_params) ||
+        (reinterpret_cast<uintptr_t>(slot_mapping) & 7u))
+        return PA_ERR_INVALID_ARG;
+    const dim3 grid(unsigned(num_tokens), unsigned((num_heads + 3) / 4), 2);
+    cudaError_t e;
+    if (head_dim == 128)
+        e = launch_pdl(pa::reshape_and_cache_int8_kernel<128>, grid, dim3(128), 0,
+                       reinterpret_cast<cudaStream_t>(stream), static_cast<const __half *>(key),
+                       static_cast<const __half *>(value), static_cast<uint8_t *>(k_codes),
+                       static_cast<uint8_t *>(v_codes), static_cast<float2 *>(k_params),
+                       static_cast<float2 *>(v_params), slot_mapping, num_heads, block_size,
+                       num_blocks);
+    else
+        e = launch_pdl(pa::reshape_and_cache_int8_kernel<64>, grid, dim3(128), 0,
+                       reinterpret_cast<cudaStream_t>(stream), static_cast<const __half *>(key),
+                       static_cast<const __half *>(value), static_cast<uint8_t *>(k_codes),
+                       static_cast<uint8_t *>(v_codes), static_cast<float2 *>(k_params),
+                       static_cast<float2 *>(v_params), slot_mapping, num_heads, block_size,
+                       num_blocks);
+    return e == cudaSuccess ? PA_OK : PA_ERR_CUDA;
+}
+
+pa_status pa_copy_blocks_raw(void *cache, size_t block_bytes, const int64_t *block_mapping,
+                             int num_pairs, int num_blocks, pa_stream_t stream)
+{
+    if (num_pairs < 0 || num_blocks <= 0 || block_bytes == 0 || (block_bytes & 15u))
+        return PA_ERR_INVALID_ARG;
+    if (num_pairs == 0)
+        return PA_OK;
+    if (!cache || !block_mapping || !aligned16(cache) ||
+        (reinterpret_cast<uintptr_t>(block_mapping) & 7u))
+        return PA_ERR_INVALID_ARG;
+    const int64_t block_vecs = int64_t(block_bytes / 16);
+    const int64_t per_cta = int64_t(pa::kCopyThreads) * pa::kCopyUnroll;
+    const int64_t chunks = (block_vecs + per_cta - 1) / per_cta;
+    if (chunks > 65535)
+        return PA_ERR_INVALID_ARG;
+    const dim3 grid(unsigned(num_pairs), 1, unsigned(chunks));
+    return launch_pdl(pa::copy_blocks_kernel, grid, dim3(pa::kCopyThreads), 0,
+                      reinterpret_cast<cudaStream_t>(stream), static_cast<uint4 *>(cache),
+                      static_cast<uint4 *>(cache), block_mapping, block_vecs,
+                      num_blocks) == cudaSuccess
+               ? PA_OK
+               : PA_ERR_CUDA;
 }
 
 } // extern "C"

@@ -75,6 +75,8 @@ class PagedWorkload:
     alias_block_tables: np.ndarray | None = None   # config 4: tables before the CoW copy
     logical_k: list | None = None     # per sequence [H, L, D] fp16 (small configs only)
     logical_v: list | None = None
+    device_k: list | None = None      # per sequence [H, L, D] fp16 on the device (on request)
+    device_v: list | None = None
 
     @property
     def num_seqs(self) -> int:
@@ -151,7 +153,7 @@ def _newest_token_slots(lens, tables, bs):
 
 def build_paged(name, seed, lens, num_heads, head_dim, block_size, num_blocks,
                 scale, device="cpu", rng=None, keep_logical=False,
-                logical_fn=None, placement="shuffled") -> PagedWorkload:
+                logical_fn=None, placement="shuffled", keep_tokens=False) -> PagedWorkload:
     """Generic builder: lengths -> placement -> values -> canary-marked pool.
 
     Every sequence must have L >= 1 (its newest token is written by the cache
@@ -172,6 +174,7 @@ def build_paged(name, seed, lens, num_heads, head_dim, block_size, num_blocks,
     new_key = torch.empty((len(lens), h, d), dtype=torch.float16, device=device)
     new_value = torch.empty_like(new_key)
     lk, lv = ([], []) if keep_logical else (None, None)
+    dk, dv = ([], []) if keep_tokens else (None, None)
     for b, length in enumerate(lens):
         if logical_fn is not None:
             kb, vb = logical_fn(b, gen)
@@ -186,12 +189,15 @@ def build_paged(name, seed, lens, num_heads, head_dim, block_size, num_blocks,
         if keep_logical:
             lk.append(kb.cpu())
             lv.append(vb.cpu())
+        if keep_tokens:
+            dk.append(kb)
+            dv.append(vb)
     slots = _newest_token_slots(lens, tables, bs)
     return PagedWorkload(name=name, seed=seed, num_heads=h, head_dim=d, block_size=bs,
                          num_blocks=num_blocks, scale=scale, context_lens=lens,
                          block_tables=tables, q=q, k_cache=k_cache, v_cache=v_cache,
                          new_key=new_key, new_value=new_value, slot_mapping=slots,
-                         logical_k=lk, logical_v=lv)
+                         logical_k=lk, logical_v=lv, device_k=dk, device_v=dv)
 
 
 def config_lengths(cfg: int, seed: int) -> np.ndarray:
@@ -210,7 +216,8 @@ def config_lengths(cfg: int, seed: int) -> np.ndarray:
 
 def make_workload(cfg: int, device="cpu", seed: int | None = None,
                   block_size: int | None = None, keep_logical: bool = False,
-                  num_seqs: int | None = None, placement: str = "shuffled") -> PagedWorkload:
+                  num_seqs: int | None = None, placement: str = "shuffled",
+                  keep_tokens: bool = False) -> PagedWorkload:
     """Build standard configuration ``cfg`` (1..5).  ``seed`` defaults to the
     config index (use cfg + 10 for the second draw).  ``num_seqs`` truncates
     the batch (smaller parity cases with the same length distribution);
@@ -239,7 +246,8 @@ def make_workload(cfg: int, device="cpu", seed: int | None = None,
     need = sum((int(x) + bs - 1) // bs for x in lens)
     nb = nb_fixed if nb_fixed is not None else int(math.ceil(factor * need))
     return build_paged(WORKLOAD_NAMES[cfg], seed, lens, h, d, bs, nb, 1.0 / math.sqrt(d),
-                       device=device, rng=rng, keep_logical=keep_logical, placement=placement)
+                       device=device, rng=rng, keep_logical=keep_logical, placement=placement,
+                       keep_tokens=keep_tokens)
 
 
 def make_shared_prefix(device="cpu", seed: int = 4, num_groups: int = 8,
@@ -320,11 +328,31 @@ def make_shared_prefix(device="cpu", seed: int = 4, num_groups: int = 8,
 
 def make_random(seed: int, lens, num_heads: int, head_dim: int, block_size: int,
                 pool_factor: float = 1.5, device="cpu", keep_logical=True,
-                scale: float | None = None) -> PagedWorkload:
+                scale: float | None = None, keep_tokens: bool = False) -> PagedWorkload:
     """Small ad-hoc workload for parity and edge-case tests."""
     lens = np.asarray(lens, dtype=np.int32)
     need = sum((int(x) + block_size - 1) // block_size for x in lens)
     nb = max(int(math.ceil(pool_factor * need)), 1)
     scale = 1.0 / math.sqrt(head_dim) if scale is None else scale
     return build_paged(f"random seed={seed}", seed, lens, num_heads, head_dim, block_size,
-                       nb, scale, device=device, keep_logical=keep_logical)
+                       nb, scale, device=device, keep_logical=keep_logical,
+                       keep_tokens=keep_tokens)
+
+
+def all_token_writes(wl: PagedWorkload, seqs=None):
+    """Every context token of the chosen sequences as one cache-write batch:
+    (keys [N, H, D], values [N, H, D], slots [N] int64), built from the kept
+    device tokens (``keep_tokens=True``) and the block tables."""
+    if wl.device_k is None:
+        raise ValueError("workload was built without keep_tokens")
+    seqs = range(wl.num_seqs) if seqs is None else seqs
+    bs = wl.block_size
+    keys, values, slots = [], [], []
+    for b in seqs:
+        length = int(wl.context_lens[b])
+        pos = np.arange(length)
+        slots.append(wl.block_tables[b, pos // bs].astype(np.int64) * bs + pos % bs)
+        keys.append(wl.device_k[b].permute(1, 0, 2))
+        values.append(wl.device_v[b].permute(1, 0, 2))
+    return (torch.cat(keys).contiguous(), torch.cat(values).contiguous(),
+            np.concatenate(slots))

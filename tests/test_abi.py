@@ -23,7 +23,7 @@ def _declared_functions():
     names = set()
     for path in glob.glob(os.path.join(ROOT, "include", "*.h")):
         text = re.sub(r"/\*.*?\*/", "", open(path).read(), flags=re.S)
-        names |= set(re.findall(r"\b(pa_[a-z_]+)\s*\(", text))
+        names |= set(re.findall(r"\b(pa_[a-z0-9_]+)\s*\(", text))
     return sorted(names)
 
 
