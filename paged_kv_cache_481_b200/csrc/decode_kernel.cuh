@@ -37,11 +37,11 @@
 //     lets its copies in flight land and stops.
 //   * Storage: fp16 rows, or int8 codes with one affine (s, z) per (token,
 //     head) row (brentwoodlivery.com 5.3.18: r_hat = s (q - z)).  For int8 a
-//     tile is 32 rows; the codes are widened exactly to fp16 as (q - 128)
-//     with a byte permute, the QK dot runs on them with the same
+//     tile is 32 rows; the QK dot runs on the widened codes with the same
 //     mixed-precision FMA, and the zero point enters once per row:
-//       q.K = s (sum_d q_d (c_d - 128) - (z - 128) sum_d q_d),
-//     sum_t w_t V_t = sum_t w_t s_t (c_t - 128) - sum_t w_t s_t (z_t - 128).
+//       q.K = s (sum_d q_d (1024 + c_d) - (1024 + z) sum_d q_d),
+//     sum_t w_t V_t = sum_t w_t s_t (1024 + c_t) - sum_t w_t s_t (1024 + z_t),
+//     the codes being widened exactly to fp16 as 1024 + c by a byte permute.
 #pragma once
 
 #include <cuda_fp16.h>
@@ -145,17 +145,18 @@ __device__ __forceinline__ float2 h2f(uint32_t bits)
     return __half22float2(h);
 }
 
-// Two int8 codes of a packed word, widened exactly to fp16 as (code - 128):
-// the byte permute builds halves 0x64cc = 1024 + code, then 1152 is removed.
+// Two int8 codes of a packed word, widened exactly to fp16 as 1024 + code:
+// the byte permute builds the halves 0x64cc (exponent of 1024, code in the
+// low mantissa bits).  The bias 1024 is removed once per row, through the
+// zero point, instead of once per code.
+constexpr float kCodeBias = 1024.f;
+
 __device__ __forceinline__ uint32_t codes_to_h2(uint32_t word, uint32_t selector)
 {
-    const uint32_t biased = __byte_perm(word, 0x64646464u, selector);
-    const __half2 h = __hsub2(*reinterpret_cast<const __half2 *>(&biased),
-                              __half2(__float2half_rn(1152.f), __float2half_rn(1152.f)));
-    return *reinterpret_cast<const uint32_t *>(&h);
+    return __byte_perm(word, 0x64646464u, selector);
 }
 
-// q . k over one 16-byte chunk: 8 fp16 of K, or 16 int8 codes (centred).
+// q . k over one 16-byte chunk: 8 fp16 of K, or 16 int8 codes (as 1024 + c).
 template <bool kInt8>
 __device__ __forceinline__ float dot_chunk(const uint4 (&q)[kInt8 ? 2 : 1], const uint4 &k)
 {
@@ -185,7 +186,7 @@ __device__ __forceinline__ void axpy_h2(float &a0, float &a1, float w, uint32_t 
     a1 = fmaf(w, v.y, a1);
 }
 
-// acc += w * chunk (8 fp16 values, or 16 centred int8 codes).
+// acc += w * chunk (8 fp16 values, or 16 int8 codes as 1024 + c).
 template <bool kInt8>
 __device__ __forceinline__ void axpy_chunk(float (&acc)[kInt8 ? 16 : 8], float w, const uint4 &u)
 {
@@ -209,7 +210,7 @@ __device__ __forceinline__ void axpy_chunk(float (&acc)[kInt8 ? 16 : 8], float w
 // Consume one staged tile: scores, online-softmax update and PV accumulate.
 // Lane (r, c) = (lane / kChunks, lane % kChunks) handles rows i*kRowsPerStep + r
 // and dims [kDims c, kDims (c + 1)).  For int8, kp / vp are the tile's (s, z)
-// rows, qsum = sum_d q_d, and corr accumulates sum_t w_t s_t (z_t - 128).
+// rows, qsum = sum_d q_d, and corr accumulates sum_t w_t s_t (1024 + z_t).
 template <int D, bool kInt8, bool kFull>
 __device__ __forceinline__ void consume_tile(const uint4 *__restrict__ ks, const uint4 *__restrict__ vs,
                                              const float2 *__restrict__ kp, const float2 *__restrict__ vp,
@@ -246,7 +247,7 @@ __device__ __forceinline__ void consume_tile(const uint4 *__restrict__ ks, const
     float s;
     if constexpr (kInt8) {
         const float2 pz = kp[my_row];  // (s, z) of this lane's row
-        s = pz.x * fmaf(-(pz.y - 128.f), qsum, v[0]) * qk_scale_log2;
+        s = pz.x * fmaf(-(pz.y + kCodeBias), qsum, v[0]) * qk_scale_log2;
     } else {
         s = v[0] * qk_scale_log2;
     }
@@ -275,7 +276,7 @@ __device__ __forceinline__ void consume_tile(const uint4 *__restrict__ ks, const
             if constexpr (kInt8) {
                 const float2 pz = vp[row];
                 const float ws = wi * pz.x;
-                corr = fmaf(ws, pz.y - 128.f, corr);
+                corr = fmaf(ws, pz.y + kCodeBias, corr);
                 axpy_chunk<true>(acc, ws, vs[row * S::kChunks + c]);
             } else {
                 axpy_chunk<false>(acc, wi, vs[row * S::kChunks + c]);
