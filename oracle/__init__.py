@@ -83,6 +83,9 @@ def _load():
         lib.oracle_paged_decode_int8.argtypes = [vp, vp, vp, vp, vp, vp, vp, i32, vp, i32, i32,
                                                  i32, i32, i32, ctypes.c_double]
         lib.oracle_paged_decode_int8.restype = i32
+        lib.oracle_paged_prefill.argtypes = [vp, vp, vp, vp, vp, i32, vp, vp, i32, i32, i32, i32,
+                                             i32, ctypes.c_double]
+        lib.oracle_paged_prefill.restype = i32
         lib.oracle_num_threads.argtypes = []
         lib.oracle_num_threads.restype = i32
         _lib = lib
@@ -235,5 +238,27 @@ def paged_decode_int8(q, k_codes, v_codes, k_params, v_params, block_tables, con
                                           _ptr(vp_), _ptr(tables), tables.shape[1], _ptr(lens),
                                           b, h, d, bs, nb, float(scale))
     _check(rc, "paged_decode_int8")
+    return out
+
+
+def paged_prefill(q, k_cache, v_cache, block_tables, context_lens, query_start_loc, scale):
+    """fp64 multi-query (chunked prefill) paged attention.  q [T, H, D] fp16
+    holds each sequence's new tokens (rows query_start_loc[b] ..
+    query_start_loc[b+1]); token i of sequence b is at position
+    context_lens[b] - n_b + i and attends to cached positions <= its own.
+    Returns out [T, H, D] float64."""
+    q = _bits(q)
+    kc, vc = _bits(k_cache), _bits(v_cache)
+    tables = np.ascontiguousarray(block_tables, dtype=np.int32)
+    lens = np.ascontiguousarray(context_lens, dtype=np.int32)
+    qsl = np.ascontiguousarray(query_start_loc, dtype=np.int32)
+    t, h, d = q.shape
+    nb, hk, bs, dk = kc.shape
+    assert (hk, dk) == (h, d) and vc.shape == kc.shape and qsl[-1] == t
+    out = np.zeros((t, h, d), dtype=np.float64)
+    rc = _load().oracle_paged_prefill(_ptr(out), _ptr(q), _ptr(kc), _ptr(vc), _ptr(tables),
+                                      tables.shape[1], _ptr(lens), _ptr(qsl), len(lens), h, d, bs,
+                                      nb, float(scale))
+    _check(rc, "paged_prefill")
     return out
 

@@ -249,6 +249,58 @@ int oracle_paged_decode(double *out, double *probs, int64_t probs_stride,
     return status;
 }
 
+/* Multi-query (prefill / chunked prefill) paged attention
+ * (brentwoodlivery.com 5.3.18: prefill processes all prompt tokens at once;
+ * polomodov.tech slide 11: the prompt's tokens are written into blocks, then
+ * decoding continues).  Sequence b holds L = context_lens[b] tokens in the
+ * cache, the last n = query_start_loc[b+1] - query_start_loc[b] of which are
+ * new.  Query token i of b (row query_start_loc[b] + i of q / out) sits at
+ * position p = L - n + i and attends causally to every cached t <= p:
+ * out = softmax_t(scale q.K_t) V over t in [0, p] -- the decode arithmetic
+ * with context length p + 1.  q, out [num_tokens, H, D]. */
+int oracle_paged_prefill(double *out, const uint16_t *q, const uint16_t *k_cache,
+                         const uint16_t *v_cache, const int32_t *block_tables,
+                         int max_blocks_per_seq, const int32_t *context_lens,
+                         const int32_t *query_start_loc, int num_seqs, int num_heads,
+                         int head_dim, int block_size, int num_blocks, double scale)
+{
+    if (num_seqs < 0 || num_heads <= 0 || head_dim <= 0 || block_size <= 0 ||
+        num_blocks <= 0 || max_blocks_per_seq < 0)
+        return ORACLE_ERR_ARG;
+    pthread_once(&half_table_once, fill_half_table);
+    const int64_t H = num_heads, D = head_dim, bs = block_size;
+    for (int b = 0; b < num_seqs; ++b) {
+        const int n = query_start_loc[b + 1] - query_start_loc[b];
+        const int len = context_lens[b];
+        if (n < 0 || n > len || (int64_t)len > (int64_t)max_blocks_per_seq * bs)
+            return ORACLE_ERR_ARG;
+    }
+    const int64_t tokens = query_start_loc[num_seqs];
+    int status = ORACLE_OK;
+#pragma omp parallel for schedule(dynamic, 1) reduction(max : status)
+    for (int64_t u = 0; u < tokens * H; ++u) {
+        const int64_t tok = u / H;
+        const int h = (int)(u % H);
+        int b = 0;
+        while (query_start_loc[b + 1] <= tok)
+            ++b;
+        const int n = query_start_loc[b + 1] - query_start_loc[b];
+        const int pos = context_lens[b] - n + (int)(tok - query_start_loc[b]);
+        double *scores = (double *)malloc(sizeof(double) * (size_t)(pos + 1));
+        if (!scores) {
+            status = status > ORACLE_ERR_ARG ? status : ORACLE_ERR_ARG;
+            continue;
+        }
+        const int rc = decode_one(out + u * D, NULL, scores, q + u * D, k_cache, v_cache,
+                                  block_tables + (int64_t)b * max_blocks_per_seq, pos + 1, h, H, D,
+                                  bs, num_blocks, scale);
+        free(scores);
+        if (rc > status)
+            status = rc;
+    }
+    return status;
+}
+
 /* ------------------------------------------------------------------------
  * Low-bit KV cache (brentwoodlivery.com "5.3.18 LLM serving, vLLM, quantized
  * inference": the KV cache can be kept in low-bit integer formats; affine

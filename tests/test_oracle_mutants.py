@@ -31,6 +31,10 @@ MUTANTS = {
     "quant_levels": ("const float qmax = (float)((1 << bits) - 1);",
                      "const float qmax = (float)(1 << bits);"),
     "quant_zero_point_unrounded": ("const float z = rintf(-rmin / s);", "const float z = -rmin / s;"),
+    "causal_off_by_one": ("block_tables + (int64_t)b * max_blocks_per_seq, pos + 1, h, H, D,",
+                          "block_tables + (int64_t)b * max_blocks_per_seq, pos, h, H, D,"),
+    "query_position": ("const int pos = context_lens[b] - n + (int)(tok - query_start_loc[b]);",
+                       "const int pos = context_lens[b] - n;"),
     "dequant_sign": ("dot += h2d(q[u * D + d]) * (s * ((double)k_codes[row * D + d] - z));",
                      "dot += h2d(q[u * D + d]) * (s * ((double)k_codes[row * D + d] + z));"),
 }
@@ -49,6 +53,7 @@ def test_pins_catch_planted_mistake(name, tmp_path):
     env = dict(os.environ, PA_ORACLE_LIB=str(lib))
     r = subprocess.run([sys.executable, "-m", "pytest", "-x", "-q", "-p", "no:cacheprovider",
                         os.path.join(ROOT, "tests", "test_oracle_pins.py"),
-                        os.path.join(ROOT, "tests", "test_quant_pins.py")],
+                        os.path.join(ROOT, "tests", "test_quant_pins.py"),
+                        os.path.join(ROOT, "tests", "test_prefill_pins.py")],
                        cwd=ROOT, env=env, capture_output=True, text=True, timeout=600)
     assert r.returncode == 1, f"pins did not catch {name}:\n{r.stdout[-2000:]}"
