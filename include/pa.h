@@ -211,6 +211,30 @@ PA_API pa_status pa_decode_int8(void *out, const void *q, const void *k_codes,
 PA_API pa_status pa_copy_blocks_raw(void *cache, size_t block_bytes, const int64_t *block_mapping,
                                     int num_pairs, int num_blocks, pa_stream_t stream);
 
+/*
+ * Multi-query paged attention: prefill and chunked prefill
+ * (brentwoodlivery.com "5.3.18 …": prefill processes all prompt tokens at
+ * once and is compute-bound; comfyai.app "6.4 PagedAttention", 6.4.3).
+ * Sequence b holds L = context_lens[b] tokens in the cache (already written
+ * with pa_reshape_and_cache), the last n_b = query_start_loc[b+1] -
+ * query_start_loc[b] of which are new.  New token i of b, at position
+ * p = L - n_b + i, attends causally to the cached tokens t <= p:
+ *     out[row] = softmax_t(scale q[row].K_t) V_t,  row = query_start_loc[b] + i.
+ *   q, out           [num_tokens, num_heads, head_dim] fp16 (device)
+ *   query_start_loc  [num_seqs + 1] int32 (device), query_start_loc[0] = 0
+ *   max_query_len    host-side bound on n_b (sizes the grid)
+ * Runs on the tensor cores (tcgen05, fp16 inputs, fp32 accumulation; the
+ * attention weights enter the P.V product rounded to fp16).  head_dim must
+ * be 128 (else PA_ERR_UNSUPPORTED).  n_b > L_b is reported in the device
+ * error word (PA_DEVERR_CONTEXT_LEN) and that sequence is skipped.
+ */
+PA_API pa_status pa_prefill(void *out, const void *q, const void *k_cache, const void *v_cache,
+                            const int32_t *block_tables, int max_blocks_per_seq,
+                            const int32_t *context_lens, int max_context_len,
+                            const int32_t *query_start_loc, int num_tokens, int max_query_len,
+                            int num_seqs, int num_heads, int head_dim, int block_size,
+                            int num_blocks, float scale, pa_stream_t stream);
+
 /* Static description of a status code. */
 PA_API const char *pa_status_string(pa_status status);
 

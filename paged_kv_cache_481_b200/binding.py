@@ -32,7 +32,7 @@ EXPORTED = ("pa_reshape_and_cache", "pa_decode_workspace_size", "pa_decode_works
             "pa_bm_create", "pa_bm_destroy", "pa_bm_num_free", "pa_bm_refcount",
             "pa_bm_add_sequence", "pa_bm_fork", "pa_bm_free_sequence", "pa_bm_append_slots",
             "pa_bm_block_tables", "pa_reshape_and_cache_int8", "pa_decode_int8",
-            "pa_copy_blocks_raw")
+            "pa_copy_blocks_raw", "pa_prefill")
 
 _lock = threading.Lock()
 _lib = None
@@ -97,6 +97,9 @@ def load(path: str | None = None):
         lib.pa_decode_int8.restype = i32
         lib.pa_copy_blocks_raw.argtypes = [vp, sz, vp, i32, i32, vp]
         lib.pa_copy_blocks_raw.restype = i32
+        lib.pa_prefill.argtypes = [vp, vp, vp, vp, vp, i32, vp, i32, vp, i32, i32, i32, i32, i32,
+                                   i32, i32, ctypes.c_float, vp]
+        lib.pa_prefill.restype = i32
         lib.pa_copy_blocks.argtypes = [vp, vp, vp, i32, i32, i32, i32, i32, vp]
         lib.pa_copy_blocks.restype = i32
         lib.pa_status_string.argtypes = [i32]
@@ -258,6 +261,24 @@ def pa_copy_blocks_raw(cache, block_mapping, stream=None):
                                      _ptr(block_mapping) if pairs else ctypes.c_void_p(None),
                                      pairs, nb, _stream(stream)),
            "pa_copy_blocks_raw")
+
+
+def pa_prefill(out, q, k_cache, v_cache, block_tables, context_lens, max_context_len,
+               query_start_loc, max_query_len, scale, stream=None):
+    """Causal multi-query attention of each sequence's new tokens (the last
+    n_b of its context) over its paged cache, on the tensor cores."""
+    t, h, d = q.shape
+    nb, hk, bs, dk = k_cache.shape
+    assert q.dtype == out.dtype == k_cache.dtype == v_cache.dtype == torch.float16
+    assert out.shape == q.shape and (hk, dk) == (h, d) and v_cache.shape == k_cache.shape
+    assert block_tables.dtype == context_lens.dtype == query_start_loc.dtype == torch.int32
+    b = context_lens.numel()
+    assert query_start_loc.numel() == b + 1
+    _check(load().pa_prefill(_ptr(out), _ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(block_tables),
+                             block_tables.shape[1], _ptr(context_lens), int(max_context_len),
+                             _ptr(query_start_loc), t, int(max_query_len), b, h, d, bs, nb,
+                             float(scale), _stream(stream)),
+           "pa_prefill")
 
 
 def pa_get_last_device_error() -> int:
