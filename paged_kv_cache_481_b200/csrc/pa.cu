@@ -9,55 +9,12 @@
 #include <cstdint>
 
 #include "../../include/pa.h"
-#include <cudaTypedefs.h>
 
 #include "cache_kernels.cuh"
 #include "decode_kernel.cuh"
-#include "prefill_kernel.cuh"
+#include "host_common.cuh"
 
 namespace {
-
-constexpr int kMaxDevices = 64;
-
-bool aligned16(const void *p)
-{
-    return (reinterpret_cast<uintptr_t>(p) & 15u) == 0;
-}
-
-bool supported_head_dim(int d)
-{
-    return d == 64 || d == 128;
-}
-
-bool supported_block_size(int bs)
-{
-    return bs == 8 || bs == 16 || bs == 32 || bs == 64 || bs == 128;
-}
-
-size_t align256(size_t x)
-{
-    return (x + 255) & ~size_t(255);
-}
-
-// Launch with programmatic stream serialisation: the grid may begin while the
-// previous kernel in the stream drains; every kernel here waits on
-// griddepcontrol.wait before it touches memory, so ordering is unchanged.
-template <typename... KArgs, typename... Args>
-cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem,
-                       cudaStream_t stream, Args... args)
-{
-    cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = grid;
-    cfg.blockDim = block;
-    cfg.dynamicSmemBytes = smem;
-    cfg.stream = stream;
-    cudaLaunchAttribute attr[1];
-    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-    attr[0].val.programmaticStreamSerializationAllowed = 1;
-    cfg.attrs = attr;
-    cfg.numAttrs = 1;
-    return cudaLaunchKernelEx(&cfg, kernel, static_cast<KArgs>(args)...);
-}
 
 // Workspace: for each worker (warp) two partial-result slots (its first and
 // its last (sequence, head), the only ones that can straddle workers), then
@@ -149,6 +106,25 @@ pa_status pa_get_last_device_error(unsigned int *code)
     *code = v;
     return PA_OK;
 }
+
+} // extern "C"
+
+unsigned int *pa_host::device_error_word()
+{
+    static std::atomic<void *> addr[kMaxDevices];
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices)
+        return nullptr;
+    void *a = addr[dev].load(std::memory_order_acquire);
+    if (!a) {
+        if (cudaGetSymbolAddress(&a, pa::g_device_error) != cudaSuccess)
+            return nullptr;
+        addr[dev].store(a, std::memory_order_release);
+    }
+    return static_cast<unsigned int *>(a);
+}
+
+extern "C" {
 
 pa_status pa_reshape_and_cache(const void *key, const void *value, void *k_cache, void *v_cache,
                                const int64_t *slot_mapping, int num_tokens, int num_heads,
@@ -386,111 +362,6 @@ pa_status pa_copy_blocks_raw(void *cache, size_t block_bytes, const int64_t *blo
 }
 
 } // extern "C"
-
-// ---------------------------------------------------------------------------
-// Multi-query (chunked prefill) attention on the tensor cores.
-
-namespace {
-
-PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder()
-{
-    static std::atomic<void *> fn{nullptr};
-    void *f = fn.load(std::memory_order_acquire);
-    if (!f) {
-        cudaDriverEntryPointQueryResult q;
-        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &f, cudaEnableDefault, &q) !=
-                cudaSuccess ||
-            q != cudaDriverEntryPointSuccess)
-            return nullptr;
-        fn.store(f, std::memory_order_release);
-    }
-    return reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(f);
-}
-
-// 2-D fp16 tensor map with 128-byte swizzle: `rows` rows of `cols` elements,
-// `row_bytes` apart, read in boxes of 64 x box_rows.
-bool make_map(CUtensorMap *map, const void *base, uint64_t cols, uint64_t rows, uint64_t row_bytes,
-              uint32_t box_rows)
-{
-    auto encode = tensor_map_encoder();
-    if (!encode)
-        return false;
-    const cuuint64_t dims[2] = {cols, rows};
-    const cuuint64_t strides[1] = {row_bytes};
-    const cuuint32_t box[2] = {64, box_rows};
-    const cuuint32_t elem[2] = {1, 1};
-    return encode(map, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, const_cast<void *>(base), dims, strides,
-                  box, elem, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
-                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
-}
-
-} // namespace
-
-extern "C" pa_status pa_prefill(void *out, const void *q, const void *k_cache, const void *v_cache,
-                                const int32_t *block_tables, int max_blocks_per_seq,
-                                const int32_t *context_lens, int max_context_len,
-                                const int32_t *query_start_loc, int num_tokens, int max_query_len,
-                                int num_seqs, int num_heads, int head_dim, int block_size,
-                                int num_blocks, float scale, pa_stream_t stream)
-{
-    if (num_seqs < 0 || num_tokens < 0 || max_query_len < 0 || num_heads <= 0 || num_blocks <= 0 ||
-        max_context_len < 0 || max_blocks_per_seq < 0)
-        return PA_ERR_INVALID_ARG;
-    if (head_dim != pa::kPD || !supported_block_size(block_size))
-        return PA_ERR_UNSUPPORTED;
-    if (int64_t(max_context_len) > int64_t(max_blocks_per_seq) * block_size ||
-        max_query_len > max_context_len || !std::isfinite(scale))
-        return PA_ERR_INVALID_ARG;
-    if (num_seqs == 0 || num_tokens == 0 || max_query_len == 0)
-        return PA_OK;
-    if (!out || !q || !k_cache || !v_cache || !block_tables || !context_lens || !query_start_loc)
-        return PA_ERR_INVALID_ARG;
-    if (!aligned16(out) || !aligned16(q) || !aligned16(k_cache) || !aligned16(v_cache) ||
-        (reinterpret_cast<uintptr_t>(block_tables) & 3u) ||
-        (reinterpret_cast<uintptr_t>(context_lens) & 3u) ||
-        (reinterpret_cast<uintptr_t>(query_start_loc) & 3u))
-        return PA_ERR_INVALID_ARG;
-    if (num_seqs > 65535 || num_heads > 65535 ||
-        int64_t(num_blocks) * num_heads * block_size > INT32_MAX)
-        return PA_ERR_INVALID_ARG;
-
-    CUtensorMap tm_q, tm_k, tm_v;
-    const uint64_t cache_rows = uint64_t(num_blocks) * num_heads * block_size;
-    const uint32_t box_rows = uint32_t(block_size < pa::kPN ? block_size : pa::kPN);
-    if (!make_map(&tm_q, q, uint64_t(num_heads) * head_dim, uint64_t(num_tokens),
-                  uint64_t(num_heads) * head_dim * 2, pa::kPM) ||
-        !make_map(&tm_k, k_cache, head_dim, cache_rows, uint64_t(head_dim) * 2, box_rows) ||
-        !make_map(&tm_v, v_cache, head_dim, cache_rows, uint64_t(head_dim) * 2, box_rows))
-        return PA_ERR_CUDA;
-
-    static std::atomic<bool> configured[kMaxDevices];
-    int dev = 0;
-    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices)
-        return PA_ERR_CUDA;
-    if (!configured[dev].load(std::memory_order_acquire)) {
-        if (cudaFuncSetAttribute(pa::paged_prefill_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 int(pa::kPrefillSmem)) != cudaSuccess)
-            return PA_ERR_CUDA;
-        configured[dev].store(true, std::memory_order_release);
-    }
-    pa::PrefillParams p{};
-    p.out = static_cast<__half *>(out);
-    p.block_tables = block_tables;
-    p.context_lens = context_lens;
-    p.query_start_loc = query_start_loc;
-    p.max_blocks_per_seq = max_blocks_per_seq;
-    p.max_context_len = max_context_len;
-    p.num_heads = num_heads;
-    p.block_size = block_size;
-    p.num_blocks = num_blocks;
-    p.qk_scale_log2 = float(double(scale) * 1.4426950408889634);
-    const dim3 grid(unsigned((max_query_len + pa::kPM - 1) / pa::kPM), unsigned(num_heads),
-                    unsigned(num_seqs));
-    return launch_pdl(pa::paged_prefill_kernel, grid, dim3(pa::kPrefillThreads), pa::kPrefillSmem,
-                      reinterpret_cast<cudaStream_t>(stream), tm_q, tm_k, tm_v, p) == cudaSuccess
-               ? PA_OK
-               : PA_ERR_CUDA;
-}
 
 // ---------------------------------------------------------------------------
 // Allocation-free variant of pa_decode.

@@ -28,7 +28,8 @@
 #include <cuda_fp16.h>
 #include <cstdint>
 
-#include "decode_kernel.cuh"
+#include "../../include/pa.h"
+#include "ptx.cuh"
 #include "tcgen05.cuh"
 
 namespace pa {
@@ -44,7 +45,13 @@ struct PrefillParams {
     int block_size;
     int num_blocks;
     float qk_scale_log2;              // softmax scale * log2(e)
+    unsigned int *error_word;         // PA_DEVERR_* bits
 };
+
+__device__ __forceinline__ void prefill_error(const PrefillParams &p, unsigned int bits)
+{
+    atomicOr(p.error_word, bits);
+}
 
 constexpr int kPM = 128;              // query rows per CTA (MMA M)
 constexpr int kPN = 128;              // context tokens per tile (MMA N of Q K^T)
@@ -77,14 +84,14 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
     int L = p.context_lens[b];
     if (L < 0 || L > p.max_context_len) {
         if (tid == 0 && qt == 0 && h == 0)
-            raise_device_error(kErrContextLen);
-        L = clamp_len(L, p.max_context_len);
+            prefill_error(p, PA_DEVERR_CONTEXT_LEN);
+        L = max(0, min(L, p.max_context_len));
     }
     if (n <= 0 || qt * kPM >= n)
         return;
     if (n > L) {  // more new tokens than the context holds: nothing sensible to do
         if (tid == 0 && qt == 0 && h == 0)
-            raise_device_error(kErrContextLen);
+            prefill_error(p, PA_DEVERR_CONTEXT_LEN);
         return;
     }
     const int row0 = qt * kPM;              // first new token of this tile
@@ -151,7 +158,7 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
                 const int tok = t0 + i * box_rows;
                 const int id = trow[tok / bsz];
                 if (unsigned(id) >= unsigned(p.num_blocks)) {
-                    raise_device_error(kErrBlockId);
+                    prefill_error(p, PA_DEVERR_BLOCK_ID);
                     continue;
                 }
                 const int y = (id * H + h) * bsz + tok % bsz;
@@ -163,7 +170,7 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
             }
             const bool ok = (j > 0 || mbar_wait_bounded(bq, 0u)) && mbar_wait_bounded(bkv, par);
             if (!ok) {
-                raise_device_error(kErrTimeout);
+                prefill_error(p, PA_DEVERR_TIMEOUT);
                 s_abort = 1;
             } else {
                 tc_fence_after_sync();
@@ -181,7 +188,7 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
         float alpha = 1.f;
         if (row_thread) {
             if (!mbar_wait_bounded(bs_, par)) {
-                raise_device_error(kErrTimeout);
+                prefill_error(p, PA_DEVERR_TIMEOUT);
                 s_abort = 1;
             } else {
                 tc_fence_after_sync();
@@ -264,7 +271,7 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
         }
         if (row_thread || ctrl) {
             if (!mbar_wait_bounded(bo, par)) {
-                raise_device_error(kErrTimeout);
+                prefill_error(p, PA_DEVERR_TIMEOUT);
                 s_abort = 1;
             } else if (row_thread) {
                 tc_fence_after_sync();
