@@ -212,6 +212,29 @@ PA_API pa_status pa_copy_blocks_raw(void *cache, size_t block_bytes, const int64
                                     int num_pairs, int num_blocks, pa_stream_t stream);
 
 /*
+ * Swap of whole blocks between two pools, typically the device pool and a
+ * pool in page-locked host memory (polomodov.tech "vLLM and PagedAttention",
+ * slide 15: a preempted request is brought back by swapping its blocks or by
+ * recomputing them).  For each pair i, block block_mapping[2i] of `src`
+ * (num_src_blocks blocks of block_bytes bytes) is copied to block
+ * block_mapping[2i+1] of `dst` (num_dst_blocks blocks).  Host pools must be
+ * device-addressable: allocated with cudaHostAlloc / cudaMallocHost or
+ * registered with cudaHostRegister (mapped at the same address, as under
+ * unified addressing); a pointer that is neither device memory nor such host
+ * memory is refused with PA_ERR_INVALID_ARG.  One call moves one pool array: call it
+ * for the K and the V cache (and, for int8 caches, their parameter arrays,
+ * with their own block_bytes).  block_mapping [num_pairs, 2] int64 lives in
+ * device-addressable memory and the pairs the host block manager's
+ * pa_bm_swap_out / pa_bm_swap_in emit fit it directly.  src and dst must be
+ * distinct arrays (PA_ERR_INVALID_ARG otherwise), 16-byte aligned, and
+ * block_bytes a multiple of 16.  A pair outside the pools is skipped and
+ * reported in the device error word (PA_DEVERR_COPY_PAIR).
+ */
+PA_API pa_status pa_swap_blocks(const void *src, void *dst, size_t block_bytes,
+                                const int64_t *block_mapping, int num_pairs, int num_src_blocks,
+                                int num_dst_blocks, pa_stream_t stream);
+
+/*
  * Multi-query paged attention: prefill and chunked prefill
  * (brentwoodlivery.com "5.3.18 …": prefill processes all prompt tokens at
  * once and is compute-bound; comfyai.app "6.4 PagedAttention", 6.4.3).

@@ -13,11 +13,22 @@
  *     the first write into a shared block copies it (copy-on-write): the
  *     writer gets a new block (reference count 1), the old block's count drops
  *     by one, and only that last block is copied.
+ *   - slide 15: preemption is all-or-nothing (the newest request is evicted)
+ *     and a preempted request comes back by swapping its blocks out to host
+ *     memory and in again, or by recomputation.  The manager keeps a second
+ *     pool for swapped blocks and moves whole sequence groups between the
+ *     pools; the data itself moves with pa_swap_blocks.
  *
  * Policy choices the pages leave open (fixed here, deterministic):
  *   - free blocks form a stack; a fresh manager hands out 0, 1, 2, ... and a
  *     freed block is the next one handed out;
- *   - sequence ids are caller-chosen 64-bit integers.
+ *   - sequence ids are caller-chosen 64-bit integers;
+ *   - a swap moves a group of sequences that holds every reference to its
+ *     blocks (e.g. a request and all its forked samples); each distinct block
+ *     gets one block of the other pool, in order of first appearance
+ *     (sequences in the given order, each table front to back), keeping its
+ *     reference count; the released blocks go back to their pool's stack in
+ *     that same order.
  *
  * Ownership: the manager is host memory owned by the caller (create/destroy).
  * Every pointer argument is a HOST pointer.  A manager is safe to use from
@@ -41,6 +52,9 @@ typedef struct pa_block_manager pa_block_manager;
 /* New manager over a pool of num_blocks blocks of block_size tokens.
  * Returns NULL on invalid sizes or host allocation failure. */
 PA_API pa_block_manager *pa_bm_create(int num_blocks, int block_size);
+/* Same, with a host (swap) pool of num_cpu_blocks blocks (>= 0). */
+PA_API pa_block_manager *pa_bm_create_with_swap(int num_blocks, int num_cpu_blocks,
+                                                int block_size);
 PA_API void pa_bm_destroy(pa_block_manager *bm);
 
 /* Blocks currently in the free pool. */
@@ -48,13 +62,43 @@ PA_API int pa_bm_num_free(const pa_block_manager *bm);
 /* Reference count of a physical block (0 = free); -1 for an invalid id. */
 PA_API int pa_bm_refcount(const pa_block_manager *bm, int block);
 
+/* Blocks free in the host (swap) pool; reference count of a host block
+ * (-1 for an invalid id). */
+PA_API int pa_bm_num_free_cpu(const pa_block_manager *bm);
+PA_API int pa_bm_cpu_refcount(const pa_block_manager *bm, int block);
+/* 1 if the sequence's blocks are in the host pool, 0 if on the device, -1 if
+ * unknown. */
+PA_API int pa_bm_is_swapped(const pa_block_manager *bm, int64_t seq);
+
+/*
+ * Swap-out: move the n sequences `seqs` (all on the device) to the host pool.
+ * pairs ([max_pairs, 2] int64) receives one (device block, host block) pair
+ * per distinct block, for pa_swap_blocks from the device pool to the host
+ * pool; *num_pairs is set to the number of distinct blocks even when the call
+ * fails for lack of room in `pairs`.  The device blocks return to the free
+ * pool.  PA_ERR_INVALID_ARG (nothing changed) for an unknown, repeated or
+ * already swapped sequence, a block also held by a sequence outside the
+ * group, or max_pairs < *num_pairs; PA_ERR_OUT_OF_BLOCKS if the host pool is
+ * short.  Swapped sequences cannot fork, append or appear in block tables
+ * until they are swapped in; they can be freed.
+ *
+ * Swap-in: the reverse, (host block, device block) pairs for pa_swap_blocks
+ * from the host pool to the device pool; PA_ERR_OUT_OF_BLOCKS if the device
+ * pool is short.
+ */
+PA_API pa_status pa_bm_swap_out(pa_block_manager *bm, const int64_t *seqs, int n, int64_t *pairs,
+                                int max_pairs, int *num_pairs);
+PA_API pa_status pa_bm_swap_in(pa_block_manager *bm, const int64_t *seqs, int n, int64_t *pairs,
+                               int max_pairs, int *num_pairs);
+
 /* Register sequence `seq` with `prompt_len` tokens already in the cache:
  * takes ceil(prompt_len / block_size) blocks.  PA_ERR_INVALID_ARG if seq
  * exists or prompt_len < 0; PA_ERR_OUT_OF_BLOCKS if the pool is short. */
 PA_API pa_status pa_bm_add_sequence(pa_block_manager *bm, int64_t seq, int prompt_len);
 
 /* Parallel sampling: `child` starts as a copy of `parent`'s table and length,
- * sharing every block (each block's reference count + 1). */
+ * sharing every block (each block's reference count + 1).  The parent must be
+ * on the device. */
 PA_API pa_status pa_bm_fork(pa_block_manager *bm, int64_t parent, int64_t child);
 
 /* Release a sequence: every block's reference count - 1; blocks reaching 0

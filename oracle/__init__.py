@@ -14,7 +14,7 @@ Passages followed (page title, section):
     (blocks, block table, sharing, copy-on-write);
   * brentwoodlivery.com "5.3.18 LLM serving, vLLM, quantized inference"
     (KV size formula 2*B*S*L*d_model*p; attention math unchanged by paging);
-  * polomodov.tech "vLLM and PagedAttention", slides 5, 9, 10, 11, 13.
+  * polomodov.tech "vLLM and PagedAttention", slides 5, 9, 10, 11, 13, 15.
 
 Every function is pinned by ``tests/test_oracle_pins.py`` to values the pages
 print, closed forms, library routines or invariants; no function here is
@@ -154,6 +154,21 @@ def copy_blocks(k_cache, v_cache, block_mapping):
                                     h, d, bs, nb)
     _check(rc, "copy_blocks")
     return kc.view(np.float16), vc.view(np.float16)
+
+
+def swap_blocks(src_pool, dst_pool, block_mapping):
+    """polomodov.tech slide 15 (a preempted request comes back by swapping):
+    return a copy of dst_pool in which block dst of each (src, dst) pair holds
+    src_pool's block src, byte for byte.  Pools are arrays whose first axis
+    indexes blocks."""
+    src = np.asarray(src_pool)
+    out = np.array(dst_pool, copy=True)
+    assert src.dtype == out.dtype and src.shape[1:] == out.shape[1:]
+    for s, d in np.asarray(block_mapping, dtype=np.int64).reshape(-1, 2):
+        if not (0 <= s < src.shape[0] and 0 <= d < out.shape[0]):
+            raise ValueError("swap pair outside the pools")
+        out[d] = src[s]
+    return out
 
 
 def paged_decode(q, k_cache, v_cache, block_tables, context_lens, scale,

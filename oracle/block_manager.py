@@ -11,6 +11,13 @@ Follows the pages step by step:
     sequences share blocks with reference counts; writing into a shared block
     first copies it: the writer gets a new block (count 1), the old block's
     count drops by one; only that last block is copied.
+  * slide 15: preemption is all-or-nothing and a preempted request comes
+    back by swapping (or recomputation).  A swap moves a group of sequences
+    that holds every reference to its blocks to a second (host) pool: each
+    distinct block, in order of first appearance (sequences in the given
+    order, tables front to back), takes one block of the other pool and
+    keeps its reference count; the released blocks go back to their pool's
+    stack in that same order.
 Slots are physical_block * block_size + offset.
 """
 from __future__ import annotations
@@ -21,12 +28,15 @@ class OutOfBlocks(Exception):
 
 
 class BlockManagerOracle:
-    def __init__(self, num_blocks: int, block_size: int):
+    def __init__(self, num_blocks: int, block_size: int, num_cpu_blocks: int = 0):
         self.block_size = block_size
         self.free = list(range(num_blocks - 1, -1, -1))   # pop() gives 0, 1, 2, ...
         self.ref = [0] * num_blocks
+        self.cpu_free = list(range(num_cpu_blocks - 1, -1, -1))
+        self.cpu_ref = [0] * num_cpu_blocks
         self.tables: dict[int, list[int]] = {}
         self.lens: dict[int, int] = {}
+        self.swapped: set[int] = set()
 
     def _take(self) -> int:
         b = self.free.pop()
@@ -46,7 +56,7 @@ class BlockManagerOracle:
         self.lens[seq] = prompt_len
 
     def fork(self, parent: int, child: int):
-        if parent not in self.tables or child in self.tables:
+        if parent not in self.tables or parent in self.swapped or child in self.tables:
             raise KeyError(child)
         self.tables[child] = list(self.tables[parent])
         self.lens[child] = self.lens[parent]
@@ -54,15 +64,61 @@ class BlockManagerOracle:
             self.ref[b] += 1
 
     def free_sequence(self, seq: int):
+        ref, free = (self.cpu_ref, self.cpu_free) if seq in self.swapped else (self.ref, self.free)
         for b in self.tables.pop(seq):
-            self.ref[b] -= 1
-            if self.ref[b] == 0:
-                self.free.append(b)
+            ref[b] -= 1
+            if ref[b] == 0:
+                free.append(b)
         del self.lens[seq]
+        self.swapped.discard(seq)
+
+    def _move(self, seqs, to_cpu: bool):
+        if len(set(seqs)) != len(seqs) or not seqs:
+            raise KeyError(seqs)
+        for s in seqs:
+            if s not in self.tables or (s in self.swapped) == to_cpu:
+                raise KeyError(s)
+        src_ref, src_free = (self.ref, self.free) if to_cpu else (self.cpu_ref, self.cpu_free)
+        dst_ref, dst_free = (self.cpu_ref, self.cpu_free) if to_cpu else (self.ref, self.free)
+        order, holders = [], {}
+        for s in seqs:
+            for b in self.tables[s]:
+                if b not in holders:
+                    order.append(b)
+                holders[b] = holders.get(b, 0) + 1
+        if any(src_ref[b] != n for b, n in holders.items()):
+            raise KeyError("group shares blocks with other sequences")
+        if len(order) > len(dst_free):
+            raise OutOfBlocks
+        moved, pairs = {}, []
+        for b in order:
+            nb = dst_free.pop()
+            dst_ref[nb] = src_ref[b]
+            moved[b] = nb
+            pairs.append((b, nb))
+        for b in order:
+            src_ref[b] = 0
+            src_free.append(b)
+        for s in seqs:
+            self.tables[s] = [moved[b] for b in self.tables[s]]
+            if to_cpu:
+                self.swapped.add(s)
+            else:
+                self.swapped.discard(s)
+        return pairs
+
+    def swap_out(self, seqs):
+        """(device block, host block) pairs; the group's blocks move to the host pool."""
+        return self._move(list(seqs), True)
+
+    def swap_in(self, seqs):
+        """(host block, device block) pairs; the group comes back to the device."""
+        return self._move(list(seqs), False)
 
     def append_slots(self, seqs):
         """Returns (slots, cow_pairs).  All-or-nothing on a short pool."""
-        if len(set(seqs)) != len(seqs) or any(s not in self.tables for s in seqs):
+        if len(set(seqs)) != len(seqs) or any(s not in self.tables or s in self.swapped
+                                               for s in seqs):
             raise KeyError(seqs)
         # count what the step needs, with reference counts as they will evolve
         refs = {}

@@ -32,7 +32,9 @@ EXPORTED = ("pa_reshape_and_cache", "pa_decode_workspace_size", "pa_decode_works
             "pa_bm_create", "pa_bm_destroy", "pa_bm_num_free", "pa_bm_refcount",
             "pa_bm_add_sequence", "pa_bm_fork", "pa_bm_free_sequence", "pa_bm_append_slots",
             "pa_bm_block_tables", "pa_reshape_and_cache_int8", "pa_decode_int8",
-            "pa_copy_blocks_raw", "pa_prefill")
+            "pa_copy_blocks_raw", "pa_prefill", "pa_swap_blocks", "pa_bm_create_with_swap",
+            "pa_bm_num_free_cpu", "pa_bm_cpu_refcount", "pa_bm_is_swapped", "pa_bm_swap_out",
+            "pa_bm_swap_in")
 
 _lock = threading.Lock()
 _lib = None
@@ -97,6 +99,19 @@ def load(path: str | None = None):
         lib.pa_decode_int8.restype = i32
         lib.pa_copy_blocks_raw.argtypes = [vp, sz, vp, i32, i32, vp]
         lib.pa_copy_blocks_raw.restype = i32
+        lib.pa_swap_blocks.argtypes = [vp, vp, sz, vp, i32, i32, i32, vp]
+        lib.pa_swap_blocks.restype = i32
+        lib.pa_bm_create_with_swap.argtypes = [i32, i32, i32]
+        lib.pa_bm_create_with_swap.restype = vp
+        lib.pa_bm_num_free_cpu.argtypes = [vp]
+        lib.pa_bm_num_free_cpu.restype = i32
+        lib.pa_bm_cpu_refcount.argtypes = [vp, i32]
+        lib.pa_bm_cpu_refcount.restype = i32
+        lib.pa_bm_is_swapped.argtypes = [vp, i64]
+        lib.pa_bm_is_swapped.restype = i32
+        for f in (lib.pa_bm_swap_out, lib.pa_bm_swap_in):
+            f.argtypes = [vp, vp, i32, vp, i32, ctypes.POINTER(ctypes.c_int)]
+            f.restype = i32
         lib.pa_prefill.argtypes = [vp, vp, vp, vp, vp, i32, vp, i32, vp, i32, i32, i32, i32, i32,
                                    i32, i32, ctypes.c_float, vp]
         lib.pa_prefill.restype = i32
@@ -263,6 +278,28 @@ def pa_copy_blocks_raw(cache, block_mapping, stream=None):
            "pa_copy_blocks_raw")
 
 
+def _ptr_addressable(t: torch.Tensor) -> ctypes.c_void_p:
+    """Device tensor, or page-locked host tensor the device can address."""
+    if not (t.is_cuda or t.is_pinned()):
+        raise ValueError("pa_swap_blocks takes device or pinned host tensors")
+    if not t.is_contiguous():
+        raise ValueError("libpa takes contiguous tensors")
+    return ctypes.c_void_p(t.data_ptr())
+
+
+def pa_swap_blocks(src, dst, block_mapping, stream=None):
+    """Copy whole blocks (dim 0) of pool `src` into pool `dst`, one of them
+    typically pinned host memory: block_mapping[i] = (src block, dst block)."""
+    assert src.dtype == dst.dtype and src.shape[1:] == dst.shape[1:]
+    assert block_mapping.dtype == torch.int64
+    block_bytes = src[0].numel() * src.element_size()
+    pairs = block_mapping.numel() // 2
+    _check(load().pa_swap_blocks(_ptr_addressable(src), _ptr_addressable(dst), block_bytes,
+                                 _ptr_addressable(block_mapping) if pairs else ctypes.c_void_p(None),
+                                 pairs, src.shape[0], dst.shape[0], _stream(stream)),
+           "pa_swap_blocks")
+
+
 def pa_prefill(out, q, k_cache, v_cache, block_tables, context_lens, max_context_len,
                query_start_loc, max_query_len, scale, stream=None):
     """Causal multi-query attention of each sequence's new tokens (the last
@@ -289,14 +326,16 @@ def pa_get_last_device_error() -> int:
 
 class BlockManager:
     """Host KV block manager (C++ in libpa): shared free pool, reference
-    counts, slot allocation per decode step and copy-on-write decisions."""
+    counts, slot allocation per decode step, copy-on-write decisions and
+    swapping of sequence groups to a host pool of num_cpu_blocks blocks."""
 
-    def __init__(self, num_blocks: int, block_size: int):
+    def __init__(self, num_blocks: int, block_size: int, num_cpu_blocks: int = 0):
         self._lib = load()
-        self._h = self._lib.pa_bm_create(num_blocks, block_size)
+        self._h = self._lib.pa_bm_create_with_swap(num_blocks, num_cpu_blocks, block_size)
         if not self._h:
-            raise PAError(PA_ERR_INVALID_ARG, "pa_bm_create")
+            raise PAError(PA_ERR_INVALID_ARG, "pa_bm_create_with_swap")
         self.num_blocks, self.block_size = num_blocks, block_size
+        self.num_cpu_blocks = num_cpu_blocks
 
     def close(self):
         if self._h:
@@ -314,6 +353,33 @@ class BlockManager:
 
     def refcount(self, block: int) -> int:
         return int(self._lib.pa_bm_refcount(self._h, int(block)))
+
+    def num_free_cpu(self) -> int:
+        return int(self._lib.pa_bm_num_free_cpu(self._h))
+
+    def cpu_refcount(self, block: int) -> int:
+        return int(self._lib.pa_bm_cpu_refcount(self._h, int(block)))
+
+    def is_swapped(self, seq: int) -> int:
+        return int(self._lib.pa_bm_is_swapped(self._h, int(seq)))
+
+    def _move(self, fn, name, seqs):
+        import numpy as np
+        ids = np.ascontiguousarray(seqs, dtype=np.int64)
+        cap = max(1, self.num_blocks + self.num_cpu_blocks)
+        pairs = np.empty((cap, 2), dtype=np.int64)
+        npairs = ctypes.c_int(0)
+        _check(fn(self._h, ids.ctypes.data, ids.shape[0], pairs.ctypes.data, cap,
+                  ctypes.byref(npairs)), name)
+        return pairs[:npairs.value].copy()
+
+    def swap_out(self, seqs):
+        """Move a sequence group to the host pool; (device, host) block pairs."""
+        return self._move(self._lib.pa_bm_swap_out, "pa_bm_swap_out", seqs)
+
+    def swap_in(self, seqs):
+        """Move a swapped group back to the device; (host, device) block pairs."""
+        return self._move(self._lib.pa_bm_swap_in, "pa_bm_swap_in", seqs)
 
     def add_sequence(self, seq: int, prompt_len: int):
         _check(self._lib.pa_bm_add_sequence(self._h, int(seq), int(prompt_len)), "pa_bm_add_sequence")

@@ -106,28 +106,32 @@ __global__ void __launch_bounds__(128) reshape_and_cache_int8_kernel(
         (is_v ? v_params : k_params)[row] = make_float2(sc, z);
 }
 
-// comfyai.app "6.4 PagedAttention", 6.4.2-6.4.3 / polomodov.tech slide 13:
-// copy-on-write duplicates a shared block before a divergent write.  Grid
-// (num_pairs, 2, chunks): y selects K or V, z a 16 KB chunk of the block.
+// Whole-block copies.  comfyai.app "6.4 PagedAttention", 6.4.2-6.4.3 /
+// polomodov.tech slide 13: copy-on-write duplicates a shared block inside a
+// pool before a divergent write; slide 15: a preempted request's blocks are
+// swapped between the device pool and a pool in host memory.  Pair i copies
+// block map[2i] of the source pool to block map[2i+1] of the destination pool.
+// Grid (num_pairs, pools, chunks): y selects the (src, dst) pool pair (K or
+// V), z a 16 KB chunk of the block.
 constexpr int kCopyThreads = 256;
 constexpr int kCopyUnroll = 4;
 
 __global__ void __launch_bounds__(kCopyThreads) copy_blocks_kernel(
-    uint4 *__restrict__ k_cache, uint4 *__restrict__ v_cache, const int64_t *__restrict__ block_mapping,
-    int64_t block_vecs, int num_blocks)
+    const uint4 *src0, uint4 *dst0, const uint4 *src1, uint4 *dst1,
+    const int64_t *__restrict__ block_mapping, int64_t block_vecs, int num_src_blocks,
+    int num_dst_blocks)
 {
     grid_dependency_wait();
     allow_dependent_launch();
     const int pair = blockIdx.x;
     const int64_t src = block_mapping[2 * pair], dst = block_mapping[2 * pair + 1];
-    if (src < 0 || src >= num_blocks || dst < 0 || dst >= num_blocks) {
+    if (src < 0 || src >= num_src_blocks || dst < 0 || dst >= num_dst_blocks) {
         if (threadIdx.x == 0 && blockIdx.y == 0 && blockIdx.z == 0)
             raise_device_error(1u << 3);
         return;
     }
-    uint4 *cache = blockIdx.y == 0 ? k_cache : v_cache;
-    const uint4 *s = cache + src * block_vecs;
-    uint4 *d = cache + dst * block_vecs;
+    const uint4 *s = (blockIdx.y == 0 ? src0 : src1) + src * block_vecs;
+    uint4 *d = (blockIdx.y == 0 ? dst0 : dst1) + dst * block_vecs;
     const int64_t base = int64_t(blockIdx.z) * kCopyThreads * kCopyUnroll + threadIdx.x;
     uint4 tmp[kCopyUnroll];
 #pragma unroll

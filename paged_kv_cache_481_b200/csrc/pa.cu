@@ -181,10 +181,10 @@ pa_status pa_copy_blocks(void *k_cache, void *v_cache, const int64_t *block_mapp
     if (chunks > 65535)
         return PA_ERR_INVALID_ARG;
     const dim3 grid(unsigned(num_pairs), 2, unsigned(chunks));
+    uint4 *k = static_cast<uint4 *>(k_cache), *v = static_cast<uint4 *>(v_cache);
     return launch_pdl(pa::copy_blocks_kernel, grid, dim3(pa::kCopyThreads), 0,
-                      reinterpret_cast<cudaStream_t>(stream), static_cast<uint4 *>(k_cache),
-                      static_cast<uint4 *>(v_cache), block_mapping, block_vecs,
-                      num_blocks) == cudaSuccess
+                      reinterpret_cast<cudaStream_t>(stream), k, k, v, v, block_mapping, block_vecs,
+                      num_blocks, num_blocks) == cudaSuccess
                ? PA_OK
                : PA_ERR_CUDA;
 }
@@ -337,14 +337,43 @@ pa_status pa_reshape_and_cache_int8(const void *key, const void *value, void *k_
     return e == cudaSuccess ? PA_OK : PA_ERR_CUDA;
 }
 
-pa_status pa_copy_blocks_raw(void *cache, size_t block_bytes, const int64_t *block_mapping,
-                             int num_pairs, int num_blocks, pa_stream_t stream)
+namespace {
+
+// True if a kernel on the current device may dereference `p` as is: device
+// or managed memory, or page-locked host memory mapped at the same address.
+// Pageable host memory (which a kernel cannot touch) is refused here.
+bool device_addressable(const void *p)
 {
-    if (num_pairs < 0 || num_blocks <= 0 || block_bytes == 0 || (block_bytes & 15u))
+    if (!p)
+        return false;
+    cudaPointerAttributes a{};
+    if (cudaPointerGetAttributes(&a, p) != cudaSuccess) {
+        cudaGetLastError();  // clear the sticky-free error of the query
+        return false;
+    }
+    switch (a.type) {
+    case cudaMemoryTypeDevice:
+    case cudaMemoryTypeManaged:
+        return true;
+    case cudaMemoryTypeHost:
+        return a.devicePointer == p;
+    default:
+        return false;
+    }
+}
+
+// One pool array's blocks from `src` to `dst` (the same array for
+// copy-on-write, or a device and a host pool for swapping).
+pa_status launch_block_copies(const void *src, void *dst, size_t block_bytes,
+                              const int64_t *block_mapping, int num_pairs, int num_src_blocks,
+                              int num_dst_blocks, pa_stream_t stream)
+{
+    if (num_pairs < 0 || num_src_blocks <= 0 || num_dst_blocks <= 0 || block_bytes == 0 ||
+        (block_bytes & 15u))
         return PA_ERR_INVALID_ARG;
     if (num_pairs == 0)
         return PA_OK;
-    if (!cache || !block_mapping || !aligned16(cache) ||
+    if (!src || !dst || !block_mapping || !aligned16(src) || !aligned16(dst) ||
         (reinterpret_cast<uintptr_t>(block_mapping) & 7u))
         return PA_ERR_INVALID_ARG;
     const int64_t block_vecs = int64_t(block_bytes / 16);
@@ -353,12 +382,35 @@ pa_status pa_copy_blocks_raw(void *cache, size_t block_bytes, const int64_t *blo
     if (chunks > 65535)
         return PA_ERR_INVALID_ARG;
     const dim3 grid(unsigned(num_pairs), 1, unsigned(chunks));
+    const uint4 *s = static_cast<const uint4 *>(src);
+    uint4 *d = static_cast<uint4 *>(dst);
     return launch_pdl(pa::copy_blocks_kernel, grid, dim3(pa::kCopyThreads), 0,
-                      reinterpret_cast<cudaStream_t>(stream), static_cast<uint4 *>(cache),
-                      static_cast<uint4 *>(cache), block_mapping, block_vecs,
-                      num_blocks) == cudaSuccess
+                      reinterpret_cast<cudaStream_t>(stream), s, d, s, d, block_mapping,
+                      block_vecs, num_src_blocks, num_dst_blocks) == cudaSuccess
                ? PA_OK
                : PA_ERR_CUDA;
+}
+
+} // namespace
+
+pa_status pa_copy_blocks_raw(void *cache, size_t block_bytes, const int64_t *block_mapping,
+                             int num_pairs, int num_blocks, pa_stream_t stream)
+{
+    return launch_block_copies(cache, cache, block_bytes, block_mapping, num_pairs, num_blocks,
+                               num_blocks, stream);
+}
+
+pa_status pa_swap_blocks(const void *src, void *dst, size_t block_bytes,
+                         const int64_t *block_mapping, int num_pairs, int num_src_blocks,
+                         int num_dst_blocks, pa_stream_t stream)
+{
+    if (src == dst && src != nullptr)
+        return PA_ERR_INVALID_ARG;  // within one pool: pa_copy_blocks_raw
+    if (num_pairs > 0 && (!device_addressable(src) || !device_addressable(dst) ||
+                          !device_addressable(block_mapping)))
+        return PA_ERR_INVALID_ARG;
+    return launch_block_copies(src, dst, block_bytes, block_mapping, num_pairs, num_src_blocks,
+                               num_dst_blocks, stream);
 }
 
 } // extern "C"
