@@ -48,7 +48,8 @@ def _decode_kernel_hash():
     h = hashlib.sha256()
     for rel in ("paged_kv_cache_481_b200/csrc/decode_kernel.cuh",
                 "paged_kv_cache_481_b200/csrc/ptx.cuh",
-                "paged_kv_cache_481_b200/csrc/pa.cu"):
+                "paged_kv_cache_481_b200/csrc/host_common.cuh",
+                "paged_kv_cache_481_b200/csrc/decode.cu"):
         with open(os.path.join(ROOT, rel), "rb") as f:
             h.update(f.read())
     return h.hexdigest()

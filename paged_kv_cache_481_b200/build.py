@@ -2,8 +2,8 @@
 
     python -m paged_kv_cache_481_b200.build [--force] [--verbose-ptxas]
 
-The library is compiled from csrc/pa.cu and csrc/prefill.cu (which include
-the kernel headers) and csrc/block_manager.cpp (host code) for ``arch=compute_100a,code=sm_100a`` only, with the CUDA runtime linked
+The library is compiled from csrc/decode.cu, csrc/cache.cu and csrc/prefill.cu
+(which include the kernel headers) and csrc/block_manager.cpp (host code) for ``arch=compute_100a,code=sm_100a`` only, with the CUDA runtime linked
 statically so the .so does not depend on the toolkit's libcudart at run time.
 """
 from __future__ import annotations
@@ -49,7 +49,8 @@ def build(force: bool = False, verbose_ptxas: bool = False) -> str:
     cmd = [_nvcc(), *ARCH_FLAGS, "-O3", "-lineinfo", "-std=c++17", "-shared",
            "-Xcompiler", "-fPIC", "-Xcompiler", "-fvisibility=hidden",
            "-cudart", "static", "-I", os.path.join(ROOT, "include"),
-           "-o", tmp, os.path.join(CSRC, "pa.cu"), os.path.join(CSRC, "prefill.cu"),
+           "-o", tmp, os.path.join(CSRC, "decode.cu"), os.path.join(CSRC, "cache.cu"),
+           os.path.join(CSRC, "prefill.cu"),
            os.path.join(CSRC, "block_manager.cpp")]
     if verbose_ptxas:
         cmd.insert(1, "-Xptxas=-v")

@@ -1,10 +1,14 @@
-// Cache write (slot scatter) and copy-on-write block copy for sm_100a.
-// Both are pure data movement with 16-byte vector accesses; bit-exact.
+// Cache writes (slot scatter, fp16 and int8), whole-block copies and the
+// bounded-wait self-test for sm_100a.  Errors are OR-ed into the device error
+// word `err` (PA_DEVERR_* bits).
 #pragma once
+
+#include <cuda_fp16.h>
 
 #include <cstdint>
 
-#include "decode_kernel.cuh"  // g_device_error / raise_device_error
+#include "../../include/pa.h"
+#include "ptx.cuh"
 
 namespace pa {
 
@@ -15,7 +19,7 @@ namespace pa {
 __global__ void __launch_bounds__(256) reshape_and_cache_kernel(
     const uint4 *__restrict__ key, const uint4 *__restrict__ value, uint4 *__restrict__ k_cache,
     uint4 *__restrict__ v_cache, const int64_t *__restrict__ slot_mapping, int num_heads,
-    int head_chunks, int block_size, int num_blocks)
+    int head_chunks, int block_size, int num_blocks, unsigned int *err)
 {
     grid_dependency_wait();
     allow_dependent_launch();
@@ -25,7 +29,7 @@ __global__ void __launch_bounds__(256) reshape_and_cache_kernel(
         return;
     if (slot >= int64_t(num_blocks) * block_size) {
         if (threadIdx.x == 0 && blockIdx.y == 0)
-            raise_device_error(1u << 2);
+            atomicOr(err, PA_DEVERR_SLOT);
         return;
     }
     const int64_t block = slot / block_size, offset = slot % block_size;
@@ -51,7 +55,8 @@ template <int D>
 __global__ void __launch_bounds__(128) reshape_and_cache_int8_kernel(
     const __half *__restrict__ key, const __half *__restrict__ value, uint8_t *__restrict__ k_codes,
     uint8_t *__restrict__ v_codes, float2 *__restrict__ k_params, float2 *__restrict__ v_params,
-    const int64_t *__restrict__ slot_mapping, int num_heads, int block_size, int num_blocks)
+    const int64_t *__restrict__ slot_mapping, int num_heads, int block_size, int num_blocks,
+    unsigned int *err)
 {
     grid_dependency_wait();
     allow_dependent_launch();
@@ -65,7 +70,7 @@ __global__ void __launch_bounds__(128) reshape_and_cache_int8_kernel(
         return;
     if (slot >= int64_t(num_blocks) * block_size) {
         if (lane == 0 && h == 0 && blockIdx.z == 0)
-            raise_device_error(1u << 2);
+            atomicOr(err, PA_DEVERR_SLOT);
         return;
     }
     const bool is_v = blockIdx.z == 1;
@@ -119,7 +124,7 @@ constexpr int kCopyUnroll = 4;
 __global__ void __launch_bounds__(kCopyThreads) copy_blocks_kernel(
     const uint4 *src0, uint4 *dst0, const uint4 *src1, uint4 *dst1,
     const int64_t *__restrict__ block_mapping, int64_t block_vecs, int num_src_blocks,
-    int num_dst_blocks)
+    int num_dst_blocks, unsigned int *err)
 {
     grid_dependency_wait();
     allow_dependent_launch();
@@ -127,7 +132,7 @@ __global__ void __launch_bounds__(kCopyThreads) copy_blocks_kernel(
     const int64_t src = block_mapping[2 * pair], dst = block_mapping[2 * pair + 1];
     if (src < 0 || src >= num_src_blocks || dst < 0 || dst >= num_dst_blocks) {
         if (threadIdx.x == 0 && blockIdx.y == 0 && blockIdx.z == 0)
-            raise_device_error(1u << 3);
+            atomicOr(err, PA_DEVERR_COPY_PAIR);
         return;
     }
     const uint4 *s = (blockIdx.y == 0 ? src0 : src1) + src * block_vecs;
@@ -151,7 +156,7 @@ __global__ void __launch_bounds__(kCopyThreads) copy_blocks_kernel(
 // Self-test of the bounded wait every kernel here relies on: one warp waits
 // on an mbarrier that nothing ever arrives at; the wait must give up after
 // limit_ns and record PA_DEVERR_TIMEOUT, leaving the context usable.
-__global__ void __launch_bounds__(32) bounded_wait_selftest_kernel(uint64_t limit_ns)
+__global__ void __launch_bounds__(32) bounded_wait_selftest_kernel(uint64_t limit_ns, unsigned int *err)
 {
     __shared__ __align__(8) uint64_t bar;
     if (threadIdx.x == 0) {
@@ -161,7 +166,7 @@ __global__ void __launch_bounds__(32) bounded_wait_selftest_kernel(uint64_t limi
     __syncwarp();
     const bool ok = mbar_wait_bounded(smem_u32(&bar), 0u, limit_ns);
     if (!__all_sync(kFullMask, ok) && threadIdx.x == 0)
-        raise_device_error(kErrTimeout);
+        atomicOr(err, PA_DEVERR_TIMEOUT);
 }
 
 } // namespace pa
