@@ -111,7 +111,8 @@ extern "C" pa_status pa_prefill(void *out, const void *q, const void *k_cache, c
     if (!p.error_word)
         return PA_ERR_CUDA;
     p.qk_scale_log2 = float(double(scale) * 1.4426950408889634);
-    const dim3 grid(unsigned((max_query_len + pa::kPM - 1) / pa::kPM), unsigned(num_heads),
+    constexpr int kRowsPerCta = pa::kQTiles * pa::kPM;
+    const dim3 grid(unsigned((max_query_len + kRowsPerCta - 1) / kRowsPerCta), unsigned(num_heads),
                     unsigned(num_seqs));
     return launch_pdl(pa::paged_prefill_kernel, grid, dim3(pa::kPrefillThreads), pa::kPrefillSmem,
                       reinterpret_cast<cudaStream_t>(stream), tm_q, tm_k, tm_v, p) == cudaSuccess

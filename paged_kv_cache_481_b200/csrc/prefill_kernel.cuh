@@ -8,20 +8,30 @@
 // (position p = L - n + i) attends causally to the cached tokens t <= p:
 //   out = softmax_t(scale q.K_t) V_t, K_t / V_t read through the block table.
 //
-// How: one CTA per (128 new tokens, head, sequence).  Warps 0-3 own one
-// query row each per thread (TMEM lane = row); warp 4 drives the copies and
-// the matrix multiplies.  For each 128-token tile of the context:
-//   * TMA tensor loads bring K and V rows, (block, head) run by run, into
-//     128-byte-swizzled shared-memory tiles (two 64-column halves each);
-//   * tcgen05.mma computes S = Q K^T (both operands K-major) into TMEM;
-//   * the row threads read S back (tcgen05.ld), apply the causal mask and the
-//     online softmax in the log2 domain, and write P as fp16 into a swizzled
-//     shared tile (rows of V past the context end are zeroed so 0 * garbage
-//     cannot reach the output);
-//   * tcgen05.mma computes P V (V as an N-major operand) into TMEM, and the
-//     row threads fold it into their fp32 output row: o = o * alpha + P V.
-// Every mbarrier wait is bounded; a wait that runs out records
-// PA_DEVERR_TIMEOUT and the CTA stops after the current tile.
+// How: one CTA per (256 new tokens = two 128-row query tiles, head,
+// sequence); warp-specialised, with the two query tiles in ping-pong so the
+// tensor core works on one tile while the other tile's softmax runs.
+//   * warp 8 (loads): TMA tensor loads of Q, then of each 128-token K and V
+//     tile, (block, head) run by run through the block table, into a ring of
+//     four 128-byte-swizzled shared-memory tiles;
+//   * warp 9 (matrix unit, one thread): S_t = Q_t K^T into TMEM, and, once
+//     the softmax of tile t has written P_t, O_t += P_t V with P_t read
+//     straight from TMEM (P overwrites S in place) and V from shared memory;
+//     the order S_0 PV_0 S_0' PV_1 S_1' keeps one tile's matrix work in
+//     flight while the other tile's softmax runs;
+//   * warps 0-3 / 4-7 (softmax of query tile 0 / 1, one query row per
+//     thread = TMEM lane): read S back, causal mask, online softmax in the
+//     log2 domain, P as fp16 into TMEM.  The running max is only moved when
+//     it grows by more than 2^8 (in base-2 exponent units); then the warp
+//     rescales its O rows and l in TMEM.  Otherwise P is taken against the
+//     stale max (P <= 2^8, exact up to fp16 rounding, no overflow).  The
+//     result is the same softmax: O and l always share one reference max.
+//   * epilogue: O / l to fp16, written straight to global memory.
+// TMEM: S0 / S1 at columns 0 / 128, O0 / O1 at 256 / 384 (all 512 columns;
+// one CTA per SM).  Every wait is bounded: a wait that runs out records
+// PA_DEVERR_TIMEOUT and raises an abort flag that ends every role's loop,
+// after which in-flight copies and matrix operations are drained (bounded)
+// before TMEM is released.
 #pragma once
 
 #include <cuda.h>
@@ -48,33 +58,66 @@ struct PrefillParams {
     unsigned int *error_word;         // PA_DEVERR_* bits
 };
 
+constexpr int kPM = 128;              // query rows per tile (MMA M)
+constexpr int kPN = 128;              // context tokens per tile (MMA N of Q K^T)
+constexpr int kPD = 128;              // head dim handled here
+constexpr int kQTiles = 2;            // query tiles per CTA
+constexpr int kRing = 4;              // K / V tile slots
+constexpr uint32_t kSub = 128 * 128;  // bytes of one [128 rows x 64 fp16] swizzled half tile
+constexpr uint32_t kTileBytes = 2 * kSub;
+constexpr uint32_t kOffRing = kQTiles * kTileBytes;
+constexpr uint32_t kPrefillSmem = kOffRing + kRing * kTileBytes + 1024;  // + 1024-B alignment slack
+constexpr int kLoadWarp = 8, kMmaWarp = 9;
+constexpr int kPrefillThreads = 10 * 32;
+constexpr uint32_t kTmemCols = 512;
+constexpr float kRescaleLog2 = 8.0f;  // move the reference max only past this growth
+
 __device__ __forceinline__ void prefill_error(const PrefillParams &p, unsigned int bits)
 {
     atomicOr(p.error_word, bits);
 }
 
-constexpr int kPM = 128;              // query rows per CTA (MMA M)
-constexpr int kPN = 128;              // context tokens per tile (MMA N of Q K^T)
-constexpr int kPD = 128;              // head dim handled here
-constexpr uint32_t kSub = 128 * 128;  // bytes of one [128 rows x 64 fp16] swizzled half tile
-constexpr uint32_t kOffK = 2 * kSub, kOffV = 4 * kSub, kOffP = 6 * kSub;
-constexpr uint32_t kPrefillSmem = 8 * kSub + 1024;  // + slack to align to 1024
-constexpr int kPrefillThreads = 160;
-constexpr uint32_t kTmemCols = 256;   // S at column 0, P V at column 128
+// Bounded wait that also gives up as soon as another role raised the abort
+// flag; a wait that runs out raises it (and records the timeout).
+__device__ __forceinline__ bool wait_or_abort(uint32_t bar, uint32_t parity, volatile int *abort,
+                                              const PrefillParams &p)
+{
+    if (mbar_try_wait(bar, parity))
+        return true;
+    const uint64_t t0 = global_timer_ns();
+    while (!mbar_try_wait(bar, parity)) {
+        if (*abort)
+            return false;
+        if (global_timer_ns() - t0 > kWaitLimitNs) {
+            prefill_error(p, PA_DEVERR_TIMEOUT);
+            *abort = 1;
+            return false;
+        }
+    }
+    return true;
+}
+
+struct PrefillTiles {
+    int rows[kQTiles];   // new tokens in query tile t (0 = tile absent)
+    int pos0[kQTiles];   // position of row 0 of tile t
+    int nt[kQTiles];     // context tiles tile t attends to
+    int ntiles;          // context tiles the CTA walks
+};
 
 __global__ void __launch_bounds__(kPrefillThreads, 1)
     paged_prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                          const __grid_constant__ CUtensorMap tm_v, const PrefillParams p)
 {
     extern __shared__ unsigned char smem_raw[];
-    __shared__ __align__(8) uint64_t bar_q, bar_kv, bar_s, bar_o;
+    __shared__ __align__(8) uint64_t bar_q, bar_drain, kv_full[kRing], kv_empty[kRing],
+        s_full[kQTiles], p_full[kQTiles], o_full[kQTiles];
     __shared__ uint32_t s_tmem;
-    __shared__ int s_abort;
+    __shared__ volatile int s_abort;
 
-    const int qt = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
-    const int tid = threadIdx.x, warp = tid >> 5;
-    const bool ctrl = tid == 4 * 32;
-    const bool row_thread = tid < kPM;
+    // heavier (later) query tiles of each (head, sequence) first
+    const int pair = int(gridDim.x) - 1 - int(blockIdx.x);
+    const int h = blockIdx.y, b = blockIdx.z;
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
 
     grid_dependency_wait();
     allow_dependent_launch();
@@ -83,230 +126,359 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
     const int n = p.query_start_loc[b + 1] - q_first;
     int L = p.context_lens[b];
     if (L < 0 || L > p.max_context_len) {
-        if (tid == 0 && qt == 0 && h == 0)
+        if (tid == 0 && pair == 0 && h == 0)
             prefill_error(p, PA_DEVERR_CONTEXT_LEN);
         L = max(0, min(L, p.max_context_len));
     }
-    if (n <= 0 || qt * kPM >= n)
+    const int row0 = pair * kQTiles * kPM;
+    if (n <= 0 || row0 >= n)
         return;
     if (n > L) {  // more new tokens than the context holds: nothing sensible to do
-        if (tid == 0 && qt == 0 && h == 0)
+        if (tid == 0 && pair == 0 && h == 0)
             prefill_error(p, PA_DEVERR_CONTEXT_LEN);
         return;
     }
-    const int row0 = qt * kPM;              // first new token of this tile
-    const int rows = min(kPM, n - row0);    // new tokens in this tile
-    const int pos0 = L - n + row0;          // position of row 0
-    const int ntiles = (pos0 + rows - 1) / kPN + 1;
+    PrefillTiles T;
+    T.ntiles = 0;
+#pragma unroll
+    for (int t = 0; t < kQTiles; ++t) {
+        const int r0 = row0 + t * kPM;
+        T.rows[t] = max(0, min(kPM, n - r0));
+        T.pos0[t] = L - n + r0;
+        T.nt[t] = T.rows[t] > 0 ? (T.pos0[t] + T.rows[t] - 1) / kPN + 1 : 0;
+        T.ntiles = max(T.ntiles, T.nt[t]);
+    }
 
     const uint32_t raw = smem_u32(smem_raw);
-    const uint32_t sQ = (raw + 1023u) & ~1023u;
-    unsigned char *smem = smem_raw + (sQ - raw);
-    const uint32_t bq = smem_u32(&bar_q), bkv = smem_u32(&bar_kv), bs_ = smem_u32(&bar_s),
-                   bo = smem_u32(&bar_o);
+    const uint32_t sbase = (raw + 1023u) & ~1023u;
+    unsigned char *smem = smem_raw + (sbase - raw);
     if (tid == 0) {
-        mbar_init(bq, 1);
-        mbar_init(bkv, 1);
-        mbar_init(bs_, 1);
-        mbar_init(bo, 1);
+        mbar_init(smem_u32(&bar_q), 1);
+        mbar_init(smem_u32(&bar_drain), 1);
+        for (int i = 0; i < kRing; ++i) {
+            mbar_init(smem_u32(&kv_full[i]), 1);
+            mbar_init(smem_u32(&kv_empty[i]), 1);
+        }
+        for (int t = 0; t < kQTiles; ++t) {
+            mbar_init(smem_u32(&s_full[t]), 1);
+            mbar_init(smem_u32(&p_full[t]), 4);  // one arrival per softmax warp
+            mbar_init(smem_u32(&o_full[t]), 1);
+        }
         s_abort = 0;
         fence_mbar_init();
     }
-    if (warp == 4)
+    if (warp == kMmaWarp)
         tmem_alloc(smem_u32(&s_tmem), kTmemCols);
     tc_fence_before_sync();
     __syncthreads();
     tc_fence_after_sync();
     const uint32_t tmem = s_tmem;
-    const uint32_t tS = tmem, tO = tmem + kPN;
 
     const int H = p.num_heads, bsz = p.block_size;
-    const int box_rows = bsz < kPN ? bsz : kPN;
-    const int32_t *trow = p.block_tables + size_t(b) * p.max_blocks_per_seq;
-    constexpr uint32_t kIdescS = idesc_f16_f32(kPM, kPN, false);
-    constexpr uint32_t kIdescO = idesc_f16_f32(kPM, kPD, true);
 
-    if (ctrl) {
-        mbar_arrive_expect_tx(bq, 2 * kSub);
-        tma_load_2d(sQ, &tm_q, h * kPD, q_first + row0, bq);
-        tma_load_2d(sQ + kSub, &tm_q, h * kPD + 64, q_first + row0, bq);
-    }
-
-    float o[kPD];
+    if (warp == kLoadWarp) {
+        // ------------------------------------------------------------ loads
+        const int box_rows = bsz < kPN ? bsz : kPN;
+        const int32_t *trow = p.block_tables + size_t(b) * p.max_blocks_per_seq;
+        int last_use[kRing];
 #pragma unroll
-    for (int d = 0; d < kPD; ++d)
-        o[d] = 0.f;
-    float m = -INFINITY, l = 0.f;
-    const int my_pos = pos0 + tid;
-    const uint32_t lane_base = uint32_t(warp * 32) << 16;  // this warp's TMEM lanes
-
-    for (int j = 0; j < ntiles; ++j) {
-        const int t0 = j * kPN;
-        const int valid = min(kPN, L - t0);   // context tokens in this tile
-        const uint32_t par = uint32_t(j) & 1u;
-
-        // ---- K, V of tile j, then S = Q K^T --------------------------------
-        if (ctrl) {
-            uint32_t bytes = 0;
-            for (int i = 0; i * box_rows < valid; ++i) {
-                const int tok = t0 + i * box_rows;
-                if (unsigned(trow[tok / bsz]) < unsigned(p.num_blocks))
-                    bytes += 4u * uint32_t(box_rows) * 128u;
-            }
-            mbar_arrive_expect_tx(bkv, bytes);
-            for (int i = 0; i * box_rows < valid; ++i) {
-                const int tok = t0 + i * box_rows;
-                const int id = trow[tok / bsz];
-                if (unsigned(id) >= unsigned(p.num_blocks)) {
-                    prefill_error(p, PA_DEVERR_BLOCK_ID);
+        for (int i = 0; i < kRing; ++i)
+            last_use[i] = -1;
+        if (lane == 0) {
+            uint32_t qbytes = 0;
+            for (int t = 0; t < kQTiles; ++t)
+                qbytes += T.rows[t] > 0 ? kTileBytes : 0u;
+            mbar_arrive_expect_tx(smem_u32(&bar_q), qbytes);
+            for (int t = 0; t < kQTiles; ++t) {
+                if (T.rows[t] <= 0)
                     continue;
-                }
-                const int y = (id * H + h) * bsz + tok % bsz;
-                const uint32_t off = uint32_t(i * box_rows) * 128u;
-                tma_load_2d(sQ + kOffK + off, &tm_k, 0, y, bkv);
-                tma_load_2d(sQ + kOffK + kSub + off, &tm_k, 64, y, bkv);
-                tma_load_2d(sQ + kOffV + off, &tm_v, 0, y, bkv);
-                tma_load_2d(sQ + kOffV + kSub + off, &tm_v, 64, y, bkv);
+                const int y = q_first + row0 + t * kPM;
+                tma_load_2d(sbase + t * kTileBytes, &tm_q, h * kPD, y, smem_u32(&bar_q));
+                tma_load_2d(sbase + t * kTileBytes + kSub, &tm_q, h * kPD + 64, y, smem_u32(&bar_q));
             }
-            const bool ok = (j > 0 || mbar_wait_bounded(bq, 0u)) && mbar_wait_bounded(bkv, par);
-            if (!ok) {
-                prefill_error(p, PA_DEVERR_TIMEOUT);
-                s_abort = 1;
-            } else {
+        }
+        for (int j = 0; j < T.ntiles; ++j) {
+            const int t0 = j * kPN;
+            const int valid = min(kPN, L - t0);
+            const int runs = (valid + box_rows - 1) / box_rows;
+            int y = 0;
+            bool ok_id = false;
+            if (lane < runs) {
+                const int tok = t0 + lane * box_rows;
+                const int id = trow[tok / bsz];
+                ok_id = unsigned(id) < unsigned(p.num_blocks);
+                if (!ok_id)
+                    prefill_error(p, PA_DEVERR_BLOCK_ID);
+                y = (id * H + h) * bsz + tok % bsz;
+            }
+            const uint32_t bytes = uint32_t(__popc(__ballot_sync(kFullMask, ok_id))) *
+                                   uint32_t(box_rows) * 256u;
+            bool go = true;
+            for (int kind = 0; kind < 2 && go; ++kind) {  // K, then V
+                const int i = 2 * j + kind, slot = i % kRing, use = i / kRing;
+                const uint32_t full = smem_u32(&kv_full[slot]);
+                if (use > 0) {
+                    bool ok = lane == 0 ? wait_or_abort(smem_u32(&kv_empty[slot]),
+                                                        uint32_t(use - 1) & 1u, &s_abort, p)
+                                        : true;
+                    go = __shfl_sync(kFullMask, int(ok), 0) != 0;
+                    if (!go)
+                        break;
+                }
+                if (lane == 0)
+                    mbar_arrive_expect_tx(full, bytes);
+                last_use[slot] = use;
+                __syncwarp();
+                if (ok_id) {
+                    const CUtensorMap *map = kind == 0 ? &tm_k : &tm_v;
+                    const uint32_t dst = sbase + kOffRing + uint32_t(slot) * kTileBytes +
+                                         uint32_t(lane * box_rows) * 128u;
+                    tma_load_2d(dst, map, 0, y, full);
+                    tma_load_2d(dst + kSub, map, 64, y, full);
+                }
+            }
+            if (!go)
+                break;
+        }
+        // After an abort, let the copies already issued land before the CTA
+        // (and its shared memory) goes away.
+        if (s_abort && lane == 0) {
+            for (int i = 0; i < kRing; ++i)
+                if (last_use[i] >= 0)
+                    mbar_wait_bounded(smem_u32(&kv_full[i]), uint32_t(last_use[i]) & 1u);
+            mbar_wait_bounded(smem_u32(&bar_q), 0u);
+        }
+    } else if (warp == kMmaWarp) {
+        // ------------------------------------------------- matrix unit
+        if (lane == 0) {
+            constexpr uint32_t kIdescS = idesc_f16_f32(kPM, kPN, false);
+            constexpr uint32_t kIdescO = idesc_f16_f32(kPM, kPD, true);
+            volatile int *abort = &s_abort;
+            const bool act0 = T.rows[0] > 0, act1 = T.rows[1] > 0;
+            auto slot_addr = [&](int i) { return sbase + kOffRing + uint32_t(i % kRing) * kTileBytes; };
+            auto wait_full = [&](int i) {
+                const bool ok = wait_or_abort(smem_u32(&kv_full[i % kRing]), uint32_t(i / kRing) & 1u,
+                                              abort, p);
                 tc_fence_after_sync();
+                return ok;
+            };
+            auto issue_s = [&](int t, uint32_t k_addr) {
+                const uint32_t q_addr = sbase + uint32_t(t) * kTileBytes;
 #pragma unroll
                 for (int k = 0; k < kPD / 16; ++k) {
                     const uint32_t kb = uint32_t(k >> 2) * kSub, kk = uint32_t(k & 3) * 32u;
-                    umma_f16(tS, smem_desc_sw128(sQ + kb + kk, 16, 1024),
-                             smem_desc_sw128(sQ + kOffK + kb + kk, 16, 1024), kIdescS, k > 0);
+                    umma_f16(tmem + uint32_t(t) * kPN, smem_desc_sw128(q_addr + kb + kk, 16, 1024),
+                             smem_desc_sw128(k_addr + kb + kk, 16, 1024), kIdescS, k > 0);
                 }
-                umma_commit(bs_);
-            }
-        }
-
-        // ---- softmax of S, P to shared memory ------------------------------
-        float alpha = 1.f;
-        if (row_thread) {
-            if (!mbar_wait_bounded(bs_, par)) {
-                prefill_error(p, PA_DEVERR_TIMEOUT);
-                s_abort = 1;
-            } else {
+                umma_commit(smem_u32(&s_full[t]));
+            };
+            auto issue_pv = [&](int t, uint32_t v_addr, bool accumulate) {
+                const uint32_t p_tmem = tmem + uint32_t(t) * kPN;          // P aliases S
+                const uint32_t o_tmem = tmem + 2u * kPN + uint32_t(t) * kPD;
+#pragma unroll
+                for (int k = 0; k < kPN / 16; ++k)
+                    umma_f16_ts(o_tmem, p_tmem + uint32_t(k) * 8u,
+                                smem_desc_sw128(v_addr + uint32_t(k) * 2048u, kSub, 1024), kIdescO,
+                                accumulate || k > 0);
+                umma_commit(smem_u32(&o_full[t]));
+            };
+            auto wait_p = [&](int t, int j) {
+                const bool ok = wait_or_abort(smem_u32(&p_full[t]), uint32_t(j) & 1u, abort, p);
                 tc_fence_after_sync();
+                return ok;
+            };
+
+            bool ok = wait_or_abort(smem_u32(&bar_q), 0u, abort, p) && wait_full(0);
+            if (ok) {
+                if (act0 && T.nt[0] > 0)
+                    issue_s(0, slot_addr(0));
+                if (act1 && T.nt[1] > 0)
+                    issue_s(1, slot_addr(0));
+                umma_commit(smem_u32(&kv_empty[0]));
+            }
+            for (int j = 0; ok && j < T.ntiles; ++j) {
+                const int iv = 2 * j + 1, ik = 2 * j + 2;
+                const bool next = j + 1 < T.ntiles;
+                if (!(ok = wait_full(iv)))
+                    break;
+                if (act0 && j < T.nt[0]) {
+                    if (!(ok = wait_p(0, j)))
+                        break;
+                    issue_pv(0, slot_addr(iv), j > 0);
+                }
+                if (next) {
+                    if (!(ok = wait_full(ik)))
+                        break;
+                    if (act0 && j + 1 < T.nt[0])
+                        issue_s(0, slot_addr(ik));
+                }
+                if (act1 && j < T.nt[1]) {
+                    if (!(ok = wait_p(1, j)))
+                        break;
+                    issue_pv(1, slot_addr(iv), j > 0);
+                }
+                umma_commit(smem_u32(&kv_empty[iv % kRing]));
+                if (next) {
+                    if (act1 && j + 1 < T.nt[1])
+                        issue_s(1, slot_addr(ik));
+                    umma_commit(smem_u32(&kv_empty[ik % kRing]));
+                }
+            }
+            // every matrix operation issued has finished before TMEM and the
+            // shared tiles are released
+            umma_commit(smem_u32(&bar_drain));
+            mbar_wait_bounded(smem_u32(&bar_drain), 0u);
+        }
+        __syncwarp();
+    } else {
+        // ------------------------------------------------------- softmax
+        const int t = warp >> 2;
+        const int r = tid & 127;
+        if (T.rows[t] > 0) {
+            const uint32_t lane_base = uint32_t((warp & 3) * 32) << 16;
+            const uint32_t tS = tmem + uint32_t(t) * kPN + lane_base;
+            const uint32_t tO = tmem + 2u * kPN + uint32_t(t) * kPD + lane_base;
+            const int my_pos = T.pos0[t] + r;
+            const float c = p.qk_scale_log2;
+            float m_ref = -INFINITY, l = 0.f;
+            bool ok = true;
+            for (int j = 0; j < T.nt[t]; ++j) {
+                ok = __all_sync(kFullMask, wait_or_abort(smem_u32(&s_full[t]), uint32_t(j) & 1u,
+                                                          &s_abort, p));
+                if (!ok)
+                    break;
+                tc_fence_after_sync();
+                const int t0 = j * kPN;
+                const bool masked = (t0 + kPN - 1 > my_pos) || (t0 + kPN > L);
+                // pass 1: row max of the scaled, masked scores
                 float mx = -INFINITY;
 #pragma unroll
-                for (int c = 0; c < kPN / 32; ++c) {
-                    float s[32];
-                    tmem_load32(tS + lane_base + uint32_t(c * 32), s);
+                for (int cc = 0; cc < kPN / 32; ++cc) {
+                    uint32_t s[32];
+                    tmem_load32_async(tS + uint32_t(cc * 32), s);
+                    tmem_wait_ld();
 #pragma unroll
                     for (int i = 0; i < 32; ++i) {
-                        const int t = t0 + c * 32 + i;
-                        const float v = (t > my_pos || t >= L) ? -INFINITY : s[i] * p.qk_scale_log2;
+                        const int tok = t0 + cc * 32 + i;
+                        float v = __uint_as_float(s[i]) * c;
+                        if (masked && (tok > my_pos || tok >= L))
+                            v = -INFINITY;
                         mx = fmaxf(mx, v);
                     }
                 }
-                const float m_new = fmaxf(m, mx);
-                alpha = exp2f(m - m_new);
+                const float m_new = fmaxf(m_ref, mx);
+                if (j == 0) {
+                    m_ref = m_new;
+                } else if (__any_sync(kFullMask, m_new > m_ref + kRescaleLog2)) {
+                    // move this warp's reference max: rescale O and l
+                    ok = __all_sync(kFullMask, wait_or_abort(smem_u32(&o_full[t]),
+                                                              uint32_t(j - 1) & 1u, &s_abort, p));
+                    if (!ok)
+                        break;
+                    tc_fence_after_sync();
+                    const float alpha = exp2f(m_ref - m_new);
+#pragma unroll
+                    for (int cc = 0; cc < kPD / 32; ++cc) {
+                        uint32_t o[32];
+                        tmem_load32_async(tO + uint32_t(cc * 32), o);
+                        tmem_wait_ld();
+#pragma unroll
+                        for (int i = 0; i < 32; ++i)
+                            o[i] = __float_as_uint(__uint_as_float(o[i]) * alpha);
+                        tmem_store32(tO + uint32_t(cc * 32), o);
+                    }
+                    l *= alpha;
+                    m_ref = m_new;
+                }
+                // pass 2: P = 2^(scaled score - m_ref) as fp16 into TMEM over S
                 float lsum = 0.f;
 #pragma unroll
-                for (int c = 0; c < kPN / 32; ++c) {
-                    float s[32];
-                    tmem_load32(tS + lane_base + uint32_t(c * 32), s);
+                for (int cc = 0; cc < kPN / 32; ++cc) {
+                    uint32_t s[32], pk[16];
+                    tmem_load32_async(tS + uint32_t(cc * 32), s);
+                    tmem_wait_ld();
 #pragma unroll
-                    for (int g = 0; g < 4; ++g) {  // 8 tokens -> one 16-byte chunk of P
-                        __half2 ph[4];
+                    for (int e = 0; e < 16; ++e) {
+                        float pr[2];
 #pragma unroll
-                        for (int e = 0; e < 4; ++e) {
-                            float pr[2];
-#pragma unroll
-                            for (int u = 0; u < 2; ++u) {
-                                const int i = g * 8 + e * 2 + u;
-                                const int t = t0 + c * 32 + i;
-                                pr[u] = (t > my_pos || t >= L) ? 0.f
-                                                               : exp2f(s[i] * p.qk_scale_log2 - m_new);
-                            }
-                            ph[e] = __floats2half2_rn(pr[0], pr[1]);
-                            const float2 back = __half22float2(ph[e]);
-                            lsum += back.x + back.y;
+                        for (int u = 0; u < 2; ++u) {
+                            const int i = 2 * e + u, tok = t0 + cc * 32 + i;
+                            pr[u] = exp2f(fmaf(__uint_as_float(s[i]), c, -m_ref));
+                            if (masked && (tok > my_pos || tok >= L))
+                                pr[u] = 0.f;
                         }
-                        const int tok = c * 32 + g * 8;           // first token of the chunk
-                        const uint32_t half = uint32_t(tok >> 6) * kSub;
-                        const uint32_t chunk = uint32_t((tok & 63) >> 3);
-                        *reinterpret_cast<uint4 *>(smem + kOffP + half + uint32_t(tid) * 128u +
-                                                   ((chunk ^ (uint32_t(tid) & 7u)) << 4)) =
-                            *reinterpret_cast<const uint4 *>(ph);
+                        const __half2 ph = __floats2half2_rn(pr[0], pr[1]);
+                        const float2 back = __half22float2(ph);
+                        lsum += back.x + back.y;
+                        pk[e] = *reinterpret_cast<const uint32_t *>(&ph);
+                    }
+                    tmem_store16(tS + uint32_t(cc * 16), pk);
+                }
+                tmem_wait_st();
+                l += lsum;
+                // V rows past the context end (the tail of the last block, or
+                // stale ring contents) are zeroed, so 0 * garbage cannot reach
+                // O.  Done by the first query tile that uses this context tile.
+                const int valid = L - t0;
+                const int tz = (T.rows[0] > 0 && j < T.nt[0]) ? 0 : 1;
+                if (valid < kPN && t == tz) {
+                    const int iv = 2 * j + 1;
+                    ok = __all_sync(kFullMask,
+                                    wait_or_abort(smem_u32(&kv_full[iv % kRing]),
+                                                  uint32_t(iv / kRing) & 1u, &s_abort, p));
+                    if (!ok)
+                        break;
+                    if (r >= valid) {
+                        unsigned char *row = smem + kOffRing + uint32_t(iv % kRing) * kTileBytes +
+                                             uint32_t(r) * 128u;
+#pragma unroll
+                        for (int q16 = 0; q16 < 8; ++q16) {
+                            *reinterpret_cast<uint4 *>(row + q16 * 16) = make_uint4(0, 0, 0, 0);
+                            *reinterpret_cast<uint4 *>(row + kSub + q16 * 16) = make_uint4(0, 0, 0, 0);
+                        }
+                    }
+                    fence_proxy_async_smem();
+                }
+                tc_fence_before_sync();
+                __syncwarp();
+                if (lane == 0)
+                    mbar_arrive(smem_u32(&p_full[t]));
+            }
+            // epilogue: out = O / l
+            if (ok) {
+                ok = __all_sync(kFullMask, wait_or_abort(smem_u32(&o_full[t]),
+                                                          uint32_t(T.nt[t] - 1) & 1u, &s_abort, p));
+            }
+            if (ok) {
+                tc_fence_after_sync();
+                const float inv = 1.f / l;
+                uint4 *dst = reinterpret_cast<uint4 *>(
+                    p.out + (size_t(q_first + row0 + t * kPM + r) * H + h) * kPD);
+                const bool store = r < T.rows[t];
+#pragma unroll
+                for (int cc = 0; cc < kPD / 32; ++cc) {
+                    uint32_t o[32];
+                    tmem_load32_async(tO + uint32_t(cc * 32), o);
+                    tmem_wait_ld();
+                    if (store) {
+#pragma unroll
+                        for (int g = 0; g < 4; ++g) {
+                            __half2 v[4];
+#pragma unroll
+                            for (int e = 0; e < 4; ++e)
+                                v[e] = __floats2half2_rn(__uint_as_float(o[g * 8 + 2 * e]) * inv,
+                                                         __uint_as_float(o[g * 8 + 2 * e + 1]) * inv);
+                            dst[cc * 4 + g] = *reinterpret_cast<const uint4 *>(v);
+                        }
                     }
                 }
-                l = l * alpha + lsum;
-                m = m_new;
-            }
-            // V rows past the context end (loaded with the last block, or stale)
-            // are zeroed; S having completed, the tile's loads have landed.
-            if (!s_abort && tid >= valid) {
-#pragma unroll
-                for (int c = 0; c < 8; ++c) {
-                    *reinterpret_cast<uint4 *>(smem + kOffV + uint32_t(tid) * 128u + c * 16u) =
-                        make_uint4(0, 0, 0, 0);
-                    *reinterpret_cast<uint4 *>(smem + kOffV + kSub + uint32_t(tid) * 128u + c * 16u) =
-                        make_uint4(0, 0, 0, 0);
-                }
-            }
-            fence_proxy_async_smem();
-        }
-        tc_fence_before_sync();
-        __syncthreads();
-        if (s_abort)
-            break;
-
-        // ---- P V -------------------------------------------------------------
-        if (ctrl) {
-            tc_fence_after_sync();
-#pragma unroll
-            for (int k = 0; k < kPN / 16; ++k) {
-                const uint32_t kb = uint32_t(k >> 2) * kSub, kk = uint32_t(k & 3) * 32u;
-                umma_f16(tO, smem_desc_sw128(sQ + kOffP + kb + kk, 16, 1024),
-                         smem_desc_sw128(sQ + kOffV + uint32_t(k) * 2048u, kSub, 1024), kIdescO,
-                         k > 0);
-            }
-            umma_commit(bo);
-        }
-        if (row_thread || ctrl) {
-            if (!mbar_wait_bounded(bo, par)) {
-                prefill_error(p, PA_DEVERR_TIMEOUT);
-                s_abort = 1;
-            } else if (row_thread) {
-                tc_fence_after_sync();
-#pragma unroll
-                for (int c = 0; c < kPD / 32; ++c) {
-                    float ov[32];
-                    tmem_load32(tO + lane_base + uint32_t(c * 32), ov);
-#pragma unroll
-                    for (int i = 0; i < 32; ++i)
-                        o[c * 32 + i] = fmaf(o[c * 32 + i], alpha, ov[i]);
-                }
             }
         }
-        tc_fence_before_sync();
-        __syncthreads();
-        if (s_abort)
-            break;
     }
 
-    // ---- epilogue ----------------------------------------------------------
-    if (row_thread && !s_abort && tid < rows) {
-        const float inv = 1.f / l;
-        uint4 *dst = reinterpret_cast<uint4 *>(p.out + (size_t(q_first + row0 + tid) * H + h) * kPD);
-#pragma unroll
-        for (int c = 0; c < kPD / 8; ++c) {
-            __half2 v[4];
-#pragma unroll
-            for (int e = 0; e < 4; ++e)
-                v[e] = __floats2half2_rn(o[c * 8 + 2 * e] * inv, o[c * 8 + 2 * e + 1] * inv);
-            dst[c] = *reinterpret_cast<const uint4 *>(v);
-        }
-    }
     tc_fence_before_sync();
     __syncthreads();
-    if (warp == 4) {
+    if (warp == kMmaWarp) {
         tc_fence_after_sync();
         tmem_free(tmem, kTmemCols);
     }

@@ -20,9 +20,14 @@ def _lib():
     torch.cuda.init()
 
 
-def _run(seed, lens, n_new, bs, h=4, d=128):
+def _run(seed, lens, n_new, bs, h=4, d=128, growth=0.0):
     wl = workloads.make_random(seed, lens, num_heads=h, head_dim=d, block_size=bs,
                                keep_logical=False, pool_factor=2.0)
+    if growth:  # later keys larger: the running max grows from tile to tile
+        for b, length in enumerate(wl.context_lens):
+            for t in range(int(length) - 1):
+                blk, row = int(wl.block_tables[b, t // bs]), t % bs
+                wl.k_cache[blk, :, row, :] *= 1.0 + growth * t / length
     kc, vc = wl.k_cache.cuda(), wl.v_cache.cuda()
     binding.pa_reshape_and_cache(wl.new_key.cuda(), wl.new_value.cuda(), kc, vc,
                                  torch.from_numpy(wl.slot_mapping).cuda())
@@ -69,3 +74,11 @@ def test_prefill_rejects_other_head_dims():
         binding.pa_prefill(z, z, c, c, i, torch.ones(1, dtype=torch.int32, device="cuda"), 1,
                            torch.tensor([0, 1], dtype=torch.int32, device="cuda"), 1, 1.0)
     assert e.value.status == binding.PA_ERR_UNSUPPORTED
+
+
+def test_prefill_running_max_grows_across_tiles():
+    """Scores grow with the key position, so the row max rises by more than
+    2^8 between context tiles and the output accumulator is rescaled."""
+    out, ref = _run(311, [1000, 600], [700, 600], 16, growth=10.0)
+    assert max_abs_err(out, ref) <= ATOL
+    assert binding.pa_get_last_device_error() == 0
