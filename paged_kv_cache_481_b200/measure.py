@@ -64,12 +64,14 @@ PREFILL_CASES = [
 ]
 
 
-def measure_prefill(iters: int, block_size: int = 16, seed: int = 0):
+def measure_prefill(iters: int, block_size: int = 16, seed: int = 0, case: str | None = None):
     h, d, bs = 40, 128, block_size
     peak, peak_sus, kind = _peaks()
     g = torch.Generator(device="cuda").manual_seed(seed)
     out_lines = []
     for name, b, length, n in PREFILL_CASES:
+        if case is not None and case != name:
+            continue
         per_seq = -(-length // bs)
         nb = b * per_seq
         kc = torch.randn((nb, h, bs, d), generator=g, device="cuda").half()
@@ -123,11 +125,12 @@ def main(argv=None):
     ap.add_argument("what", choices=["prefill", "swap"])
     ap.add_argument("--iters", type=int, default=10)
     ap.add_argument("--block-size", type=int, default=16)
+    ap.add_argument("--case", default=None, help="only the prefill case of this name")
     args = ap.parse_args(argv)
     build.build()
     binding.load()
     if args.what == "prefill":
-        measure_prefill(args.iters, args.block_size)
+        measure_prefill(args.iters, args.block_size, case=args.case)
     else:
         measure_swap(args.iters)
 
