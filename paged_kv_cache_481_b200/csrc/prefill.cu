@@ -63,7 +63,7 @@ extern "C" pa_status pa_prefill(void *out, const void *q, const void *k_cache, c
     if (head_dim != pa::kPD || !supported_block_size(block_size))
         return PA_ERR_UNSUPPORTED;
     if (int64_t(max_context_len) > int64_t(max_blocks_per_seq) * block_size ||
-        max_query_len > max_context_len || !std::isfinite(scale))
+        max_query_len > max_context_len || !std::isfinite(scale) || !(scale > 0.f))
         return PA_ERR_INVALID_ARG;
     if (num_seqs == 0 || num_tokens == 0 || max_query_len == 0)
         return PA_OK;

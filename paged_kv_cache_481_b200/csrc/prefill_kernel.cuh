@@ -21,7 +21,9 @@
 //     flight while the other tile's softmax runs;
 //   * warps 0-3 / 4-7 (softmax of query tile 0 / 1, one query row per
 //     thread = TMEM lane): read S back, causal mask, online softmax in the
-//     log2 domain, P as fp16 into TMEM.  The running max is only moved when
+//     log2 domain, P as fp16 into TMEM (the row sum l is taken from P before
+//     its fp16 rounding).  Only warps holding a diagonal or context-end tile
+//     pay for the mask.  The running max is only moved when
 //     it grows by more than 2^8 (in base-2 exponent units); then the warp
 //     rescales its O rows and l in TMEM.  Otherwise P is taken against the
 //     stale max (P <= 2^8, exact up to fp16 rounding, no overflow).  The
@@ -54,7 +56,7 @@ struct PrefillParams {
     int num_heads;
     int block_size;
     int num_blocks;
-    float qk_scale_log2;              // softmax scale * log2(e)
+    float qk_scale_log2;              // softmax scale * log2(e), > 0
     unsigned int *error_word;         // PA_DEVERR_* bits
 };
 
@@ -95,6 +97,114 @@ __device__ __forceinline__ bool wait_or_abort(uint32_t bar, uint32_t parity, vol
         }
     }
     return true;
+}
+
+// ---- softmax arithmetic helpers (inline PTX of documented sm_100 forms) ----
+
+__device__ __forceinline__ float max3f(float a, float b, float c)
+{
+    float d;
+    asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+    return d;
+}
+
+// 2^x on the special-function unit (approximate, subnormal results flushed).
+__device__ __forceinline__ float ex2_approx(float x)
+{
+    float y;
+    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
+}
+
+__device__ __forceinline__ uint64_t pack2(float lo, float hi)
+{
+    uint64_t d;
+    asm("mov.b64 %0, {%1, %2};" : "=l"(d) : "f"(lo), "f"(hi));
+    return d;
+}
+
+__device__ __forceinline__ void unpack2(uint64_t v, float &lo, float &hi)
+{
+    asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(v));
+}
+
+// two fp32 lanes at once: a * b + c, a + b
+__device__ __forceinline__ uint64_t fma2(uint64_t a, uint64_t b, uint64_t c)
+{
+    uint64_t d;
+    asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
+    return d;
+}
+
+__device__ __forceinline__ uint64_t add2(uint64_t a, uint64_t b)
+{
+    uint64_t d;
+    asm("add.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+    return d;
+}
+
+// Row max of the raw scores of one 128-column S tile (this thread's TMEM
+// lane); with kMasked, only the first `lim` columns count.
+template <bool kMasked>
+__device__ __forceinline__ float tile_row_max(uint32_t tS, int lim)
+{
+    float m0 = -INFINITY, m1 = -INFINITY;
+#pragma unroll
+    for (int cc = 0; cc < kPN / 32; ++cc) {
+        uint32_t s[32];
+        tmem_load32_async(tS + uint32_t(cc * 32), s);
+        tmem_wait_ld();
+#pragma unroll
+        for (int i = 0; i < 32; i += 4) {
+            float a = __uint_as_float(s[i]), b = __uint_as_float(s[i + 1]);
+            float c = __uint_as_float(s[i + 2]), d = __uint_as_float(s[i + 3]);
+            if (kMasked) {
+                const int col = cc * 32 + i;
+                a = col < lim ? a : -INFINITY;
+                b = col + 1 < lim ? b : -INFINITY;
+                c = col + 2 < lim ? c : -INFINITY;
+                d = col + 3 < lim ? d : -INFINITY;
+            }
+            m0 = max3f(m0, a, b);
+            m1 = max3f(m1, c, d);
+        }
+    }
+    return fmaxf(m0, m1);
+}
+
+// P = 2^(c * s - m) of one S tile, as fp16 pairs written back into TMEM over
+// the first 64 columns of S; returns the row sum of P (fp32, before the fp16
+// rounding).  With kMasked, columns >= lim give P = 0.
+template <bool kMasked>
+__device__ __forceinline__ float tile_write_p(uint32_t tS, int lim, float c, float m)
+{
+    const uint64_t c2 = pack2(c, c), nm2 = pack2(-m, -m);
+    uint64_t sum2 = pack2(0.f, 0.f);
+#pragma unroll
+    for (int cc = 0; cc < kPN / 32; ++cc) {
+        uint32_t s[32], pk[16];
+        tmem_load32_async(tS + uint32_t(cc * 32), s);
+        tmem_wait_ld();
+#pragma unroll
+        for (int e = 0; e < 16; ++e) {
+            float x0, x1;
+            unpack2(fma2(pack2(__uint_as_float(s[2 * e]), __uint_as_float(s[2 * e + 1])), c2, nm2),
+                    x0, x1);
+            float p0 = ex2_approx(x0), p1 = ex2_approx(x1);
+            if (kMasked) {
+                const int col = cc * 32 + 2 * e;
+                p0 = col < lim ? p0 : 0.f;
+                p1 = col + 1 < lim ? p1 : 0.f;
+            }
+            sum2 = add2(sum2, pack2(p0, p1));
+            const __half2 ph = __floats2half2_rn(p0, p1);
+            pk[e] = *reinterpret_cast<const uint32_t *>(&ph);
+        }
+        tmem_store16(tS + uint32_t(cc * 16), pk);
+    }
+    float lo, hi;
+    unpack2(sum2, lo, hi);
+    return lo + hi;
 }
 
 struct PrefillTiles {
@@ -349,23 +459,10 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
                     break;
                 tc_fence_after_sync();
                 const int t0 = j * kPN;
-                const bool masked = (t0 + kPN - 1 > my_pos) || (t0 + kPN > L);
-                // pass 1: row max of the scaled, masked scores
-                float mx = -INFINITY;
-#pragma unroll
-                for (int cc = 0; cc < kPN / 32; ++cc) {
-                    uint32_t s[32];
-                    tmem_load32_async(tS + uint32_t(cc * 32), s);
-                    tmem_wait_ld();
-#pragma unroll
-                    for (int i = 0; i < 32; ++i) {
-                        const int tok = t0 + cc * 32 + i;
-                        float v = __uint_as_float(s[i]) * c;
-                        if (masked && (tok > my_pos || tok >= L))
-                            v = -INFINITY;
-                        mx = fmaxf(mx, v);
-                    }
-                }
+                // columns of this tile this row may see: t <= my_pos and t < L
+                const int lim = min(my_pos, L - 1) - t0 + 1;
+                const bool masked = __any_sync(kFullMask, lim < kPN);
+                const float mx = (masked ? tile_row_max<true>(tS, lim) : tile_row_max<false>(tS, lim)) * c;
                 const float m_new = fmaxf(m_ref, mx);
                 if (j == 0) {
                     m_ref = m_new;
@@ -376,8 +473,8 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
                     if (!ok)
                         break;
                     tc_fence_after_sync();
-                    const float alpha = exp2f(m_ref - m_new);
-#pragma unroll
+                    const float alpha = ex2_approx(m_ref - m_new);
+#pragma unroll 1
                     for (int cc = 0; cc < kPD / 32; ++cc) {
                         uint32_t o[32];
                         tmem_load32_async(tO + uint32_t(cc * 32), o);
@@ -390,32 +487,9 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
                     l *= alpha;
                     m_ref = m_new;
                 }
-                // pass 2: P = 2^(scaled score - m_ref) as fp16 into TMEM over S
-                float lsum = 0.f;
-#pragma unroll
-                for (int cc = 0; cc < kPN / 32; ++cc) {
-                    uint32_t s[32], pk[16];
-                    tmem_load32_async(tS + uint32_t(cc * 32), s);
-                    tmem_wait_ld();
-#pragma unroll
-                    for (int e = 0; e < 16; ++e) {
-                        float pr[2];
-#pragma unroll
-                        for (int u = 0; u < 2; ++u) {
-                            const int i = 2 * e + u, tok = t0 + cc * 32 + i;
-                            pr[u] = exp2f(fmaf(__uint_as_float(s[i]), c, -m_ref));
-                            if (masked && (tok > my_pos || tok >= L))
-                                pr[u] = 0.f;
-                        }
-                        const __half2 ph = __floats2half2_rn(pr[0], pr[1]);
-                        const float2 back = __half22float2(ph);
-                        lsum += back.x + back.y;
-                        pk[e] = *reinterpret_cast<const uint32_t *>(&ph);
-                    }
-                    tmem_store16(tS + uint32_t(cc * 16), pk);
-                }
+                // P = 2^(scaled score - m_ref) as fp16 into TMEM over S
+                l += masked ? tile_write_p<true>(tS, lim, c, m_ref) : tile_write_p<false>(tS, lim, c, m_ref);
                 tmem_wait_st();
-                l += lsum;
                 // V rows past the context end (the tail of the last block, or
                 // stale ring contents) are zeroed, so 0 * garbage cannot reach
                 // O.  Done by the first query tile that uses this context tile.
