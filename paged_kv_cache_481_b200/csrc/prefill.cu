@@ -87,15 +87,18 @@ extern "C" pa_status pa_prefill(void *out, const void *q, const void *k_cache, c
         !make_map(&tm_v, v_cache, head_dim, cache_rows, uint64_t(head_dim) * 2, box_rows))
         return PA_ERR_CUDA;
 
-    static std::atomic<bool> configured[kMaxDevices];
+    static std::atomic<int> sm_count[kMaxDevices];  // 0 = not configured yet
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices)
         return PA_ERR_CUDA;
-    if (!configured[dev].load(std::memory_order_acquire)) {
+    int sms = sm_count[dev].load(std::memory_order_acquire);
+    if (sms == 0) {
         if (cudaFuncSetAttribute(pa::paged_prefill_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 int(pa::kPrefillSmem)) != cudaSuccess)
+                                 int(pa::kPrefillSmem)) != cudaSuccess ||
+            cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess ||
+            sms <= 0)
             return PA_ERR_CUDA;
-        configured[dev].store(true, std::memory_order_release);
+        sm_count[dev].store(sms, std::memory_order_release);
     }
     pa::PrefillParams p{};
     p.out = static_cast<__half *>(out);
@@ -111,9 +114,15 @@ extern "C" pa_status pa_prefill(void *out, const void *q, const void *k_cache, c
     if (!p.error_word)
         return PA_ERR_CUDA;
     p.qk_scale_log2 = float(double(scale) * 1.4426950408889634);
-    constexpr int kRowsPerCta = pa::kQTiles * pa::kPM;
-    const dim3 grid(unsigned((max_query_len + kRowsPerCta - 1) / kRowsPerCta), unsigned(num_heads),
-                    unsigned(num_seqs));
+    // persistent: one CTA per SM (the shared-memory footprint allows one),
+    // never more CTAs than items
+    constexpr int kRowsPerItem = pa::kQTiles * pa::kPM;
+    p.num_seqs = num_seqs;
+    p.num_pairs = (max_query_len + kRowsPerItem - 1) / kRowsPerItem;
+    const int64_t items = int64_t(p.num_pairs) * num_heads * num_seqs;
+    if (items > INT32_MAX)
+        return PA_ERR_INVALID_ARG;
+    const dim3 grid(unsigned(items < sms ? items : sms));
     return launch_pdl(pa::paged_prefill_kernel, grid, dim3(pa::kPrefillThreads), pa::kPrefillSmem,
                       reinterpret_cast<cudaStream_t>(stream), tm_q, tm_k, tm_v, p) == cudaSuccess
                ? PA_OK

@@ -8,9 +8,11 @@
 // (position p = L - n + i) attends causally to the cached tokens t <= p:
 //   out = softmax_t(scale q.K_t) V_t, K_t / V_t read through the block table.
 //
-// How: one CTA per (256 new tokens = two 128-row query tiles, head,
-// sequence); warp-specialised, with the two query tiles in ping-pong so the
-// tensor core works on one tile while the other tile's softmax runs.
+// How: persistent CTAs (one per SM) walk a list of items (256 new tokens =
+// two 128-row query tiles, head, sequence); each CTA is
+// warp-specialised, with the two query tiles in ping-pong so the tensor core
+// works on one tile while the other tile's softmax runs, and one item's
+// epilogue overlaps the next item's loads and score products.
 //   * warp 8 (loads): TMA tensor loads of Q, then of each 128-token K and V
 //     tile, (block, head) run by run through the block table, into a ring of
 //     four 128-byte-swizzled shared-memory tiles;
@@ -28,7 +30,9 @@
 //     rescales its O rows and l in TMEM.  Otherwise P is taken against the
 //     stale max (P <= 2^8, exact up to fp16 rounding, no overflow).  The
 //     result is the same softmax: O and l always share one reference max.
-//   * epilogue: O / l to fp16, written straight to global memory.
+//   * epilogue: O / l to fp16, written straight to global memory; O_t is
+//     then released to the next item (o_empty), Q once the item's last score
+//     product is done (q_empty).
 // TMEM: S0 / S1 at columns 0 / 128, O0 / O1 at 256 / 384 (all 512 columns;
 // one CTA per SM).  Every wait is bounded: a wait that runs out records
 // PA_DEVERR_TIMEOUT and raises an abort flag that ends every role's loop,
@@ -58,6 +62,8 @@ struct PrefillParams {
     int num_blocks;
     float qk_scale_log2;              // softmax scale * log2(e), > 0
     unsigned int *error_word;         // PA_DEVERR_* bits
+    int num_seqs;
+    int num_pairs;                    // query-tile pairs per sequence: ceil(max_query_len / 256)
 };
 
 constexpr int kPM = 128;              // query rows per tile (MMA M)
@@ -207,109 +213,114 @@ __device__ __forceinline__ float tile_write_p(uint32_t tS, int lim, float c, flo
     return lo + hi;
 }
 
-struct PrefillTiles {
+// One unit of work: two query tiles (256 new tokens) of one (head, sequence).
+struct PrefillItem {
+    int b, h, row0, q_first, L;
     int rows[kQTiles];   // new tokens in query tile t (0 = tile absent)
     int pos0[kQTiles];   // position of row 0 of tile t
     int nt[kQTiles];     // context tiles tile t attends to
-    int ntiles;          // context tiles the CTA walks
+    int ntiles;          // context tiles the item walks
 };
 
-__global__ void __launch_bounds__(kPrefillThreads, 1)
-    paged_prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
-                         const __grid_constant__ CUtensorMap tm_v, const PrefillParams p)
+// Items are numbered (head, sequence)-major, the pairs of one (head,
+// sequence) heaviest (latest) first: k -> hb = k / P, pair = P - 1 - k % P.
+// CTA c of G takes items c, c + G, c + 2G, ...: the items running at the
+// same time then belong to few (head, sequence), whose K / V stay in L2,
+// and since G is rarely a multiple of P each CTA samples every pair level.
+// Every role walks the same list; empty items (past a sequence's new tokens,
+// or with more new tokens than context) are skipped by all of them alike.
+// `report` lets exactly one thread record per-sequence argument errors.
+__device__ __forceinline__ bool prefill_item(const PrefillParams &p, int k, PrefillItem &it,
+                                             bool report)
 {
-    extern __shared__ unsigned char smem_raw[];
-    __shared__ __align__(8) uint64_t bar_q, bar_drain, kv_full[kRing], kv_empty[kRing],
-        s_full[kQTiles], p_full[kQTiles], o_full[kQTiles];
-    __shared__ uint32_t s_tmem;
-    __shared__ volatile int s_abort;
-
-    // heavier (later) query tiles of each (head, sequence) first
-    const int pair = int(gridDim.x) - 1 - int(blockIdx.x);
-    const int h = blockIdx.y, b = blockIdx.z;
-    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-
-    grid_dependency_wait();
-    allow_dependent_launch();
-
-    const int q_first = p.query_start_loc[b];
-    const int n = p.query_start_loc[b + 1] - q_first;
-    int L = p.context_lens[b];
+    const int hb = k / p.num_pairs;
+    const int pair = p.num_pairs - 1 - k % p.num_pairs;
+    it.h = hb % p.num_heads;
+    it.b = hb / p.num_heads;
+    it.q_first = p.query_start_loc[it.b];
+    const int n = p.query_start_loc[it.b + 1] - it.q_first;
+    int L = p.context_lens[it.b];
+    const bool first = report && pair == 0 && it.h == 0;
     if (L < 0 || L > p.max_context_len) {
-        if (tid == 0 && pair == 0 && h == 0)
+        if (first)
             prefill_error(p, PA_DEVERR_CONTEXT_LEN);
         L = max(0, min(L, p.max_context_len));
     }
-    const int row0 = pair * kQTiles * kPM;
-    if (n <= 0 || row0 >= n)
-        return;
+    it.L = L;
+    it.row0 = pair * kQTiles * kPM;
+    if (n <= 0 || it.row0 >= n)
+        return false;
     if (n > L) {  // more new tokens than the context holds: nothing sensible to do
-        if (tid == 0 && pair == 0 && h == 0)
+        if (first)
             prefill_error(p, PA_DEVERR_CONTEXT_LEN);
-        return;
+        return false;
     }
-    PrefillTiles T;
-    T.ntiles = 0;
+    it.ntiles = 0;
 #pragma unroll
     for (int t = 0; t < kQTiles; ++t) {
-        const int r0 = row0 + t * kPM;
-        T.rows[t] = max(0, min(kPM, n - r0));
-        T.pos0[t] = L - n + r0;
-        T.nt[t] = T.rows[t] > 0 ? (T.pos0[t] + T.rows[t] - 1) / kPN + 1 : 0;
-        T.ntiles = max(T.ntiles, T.nt[t]);
+        const int r0 = it.row0 + t * kPM;
+        it.rows[t] = max(0, min(kPM, n - r0));
+        it.pos0[t] = L - n + r0;
+        it.nt[t] = it.rows[t] > 0 ? (it.pos0[t] + it.rows[t] - 1) / kPN + 1 : 0;
+        it.ntiles = max(it.ntiles, it.nt[t]);
     }
+    return true;
+}
 
-    const uint32_t raw = smem_u32(smem_raw);
-    const uint32_t sbase = (raw + 1023u) & ~1023u;
-    unsigned char *smem = smem_raw + (sbase - raw);
-    if (tid == 0) {
-        mbar_init(smem_u32(&bar_q), 1);
-        mbar_init(smem_u32(&bar_drain), 1);
-        for (int i = 0; i < kRing; ++i) {
-            mbar_init(smem_u32(&kv_full[i]), 1);
-            mbar_init(smem_u32(&kv_empty[i]), 1);
-        }
-        for (int t = 0; t < kQTiles; ++t) {
-            mbar_init(smem_u32(&s_full[t]), 1);
-            mbar_init(smem_u32(&p_full[t]), 4);  // one arrival per softmax warp
-            mbar_init(smem_u32(&o_full[t]), 1);
-        }
-        s_abort = 0;
-        fence_mbar_init();
-    }
-    if (warp == kMmaWarp)
-        tmem_alloc(smem_u32(&s_tmem), kTmemCols);
-    tc_fence_before_sync();
-    __syncthreads();
-    tc_fence_after_sync();
-    const uint32_t tmem = s_tmem;
+struct PrefillShared {
+    uint64_t q_full, q_empty, drain;
+    uint64_t kv_full[kRing], kv_empty[kRing];
+    uint64_t s_full[kQTiles], p_full[kQTiles], o_full[kQTiles], o_empty[kQTiles];
+    uint32_t tmem;
+    int abort;
+};
 
+// ---------------------------------------------------------------- loads
+__device__ __forceinline__ void prefill_load_role(const CUtensorMap *tm_q, const CUtensorMap *tm_k,
+                                                  const CUtensorMap *tm_v, const PrefillParams &p,
+                                                  PrefillShared &sh, uint32_t sbase, int lane)
+{
+    volatile int *abort = &sh.abort;
     const int H = p.num_heads, bsz = p.block_size;
-
-    if (warp == kLoadWarp) {
-        // ------------------------------------------------------------ loads
-        const int box_rows = bsz < kPN ? bsz : kPN;
-        const int32_t *trow = p.block_tables + size_t(b) * p.max_blocks_per_seq;
-        int last_use[kRing];
+    const int box_rows = bsz < kPN ? bsz : kPN;
+    const int total = p.num_pairs * H * p.num_seqs;
+    int last_use[kRing];
 #pragma unroll
-        for (int i = 0; i < kRing; ++i)
-            last_use[i] = -1;
+    for (int i = 0; i < kRing; ++i)
+        last_use[i] = -1;
+    int ring = 0, items = 0;
+    bool go = true;
+    for (int k = blockIdx.x; go && k < total; k += gridDim.x) {
+        PrefillItem it;
+        if (!prefill_item(p, k, it, lane == 0))
+            continue;
+        // Q of this item once the previous item's score products are done
+        if (items > 0) {
+            const bool ok = lane == 0 ? wait_or_abort(smem_u32(&sh.q_empty), uint32_t(items - 1) & 1u,
+                                                      abort, p)
+                                      : true;
+            if (!(go = __shfl_sync(kFullMask, int(ok), 0) != 0))
+                break;
+        }
         if (lane == 0) {
             uint32_t qbytes = 0;
             for (int t = 0; t < kQTiles; ++t)
-                qbytes += T.rows[t] > 0 ? kTileBytes : 0u;
-            mbar_arrive_expect_tx(smem_u32(&bar_q), qbytes);
+                qbytes += it.rows[t] > 0 ? kTileBytes : 0u;
+            mbar_arrive_expect_tx(smem_u32(&sh.q_full), qbytes);
             for (int t = 0; t < kQTiles; ++t) {
-                if (T.rows[t] <= 0)
+                if (it.rows[t] <= 0)
                     continue;
-                const int y = q_first + row0 + t * kPM;
-                tma_load_2d(sbase + t * kTileBytes, &tm_q, h * kPD, y, smem_u32(&bar_q));
-                tma_load_2d(sbase + t * kTileBytes + kSub, &tm_q, h * kPD + 64, y, smem_u32(&bar_q));
+                const int y = it.q_first + it.row0 + t * kPM;
+                tma_load_2d(sbase + t * kTileBytes, tm_q, it.h * kPD, y, smem_u32(&sh.q_full));
+                tma_load_2d(sbase + t * kTileBytes + kSub, tm_q, it.h * kPD + 64, y,
+                            smem_u32(&sh.q_full));
             }
         }
-        for (int j = 0; j < T.ntiles; ++j) {
+        ++items;
+        const int32_t *trow = p.block_tables + size_t(it.b) * p.max_blocks_per_seq;
+        for (int j = 0; go && j < it.ntiles; ++j) {
             const int t0 = j * kPN;
-            const int valid = min(kPN, L - t0);
+            const int valid = min(kPN, it.L - t0);
             const int runs = (valid + box_rows - 1) / box_rows;
             int y = 0;
             bool ok_id = false;
@@ -319,20 +330,18 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
                 ok_id = unsigned(id) < unsigned(p.num_blocks);
                 if (!ok_id)
                     prefill_error(p, PA_DEVERR_BLOCK_ID);
-                y = (id * H + h) * bsz + tok % bsz;
+                y = (id * H + it.h) * bsz + tok % bsz;
             }
             const uint32_t bytes = uint32_t(__popc(__ballot_sync(kFullMask, ok_id))) *
                                    uint32_t(box_rows) * 256u;
-            bool go = true;
-            for (int kind = 0; kind < 2 && go; ++kind) {  // K, then V
-                const int i = 2 * j + kind, slot = i % kRing, use = i / kRing;
-                const uint32_t full = smem_u32(&kv_full[slot]);
+            for (int kind = 0; kind < 2; ++kind) {  // K, then V
+                const int i = ring + 2 * j + kind, slot = i % kRing, use = i / kRing;
+                const uint32_t full = smem_u32(&sh.kv_full[slot]);
                 if (use > 0) {
-                    bool ok = lane == 0 ? wait_or_abort(smem_u32(&kv_empty[slot]),
-                                                        uint32_t(use - 1) & 1u, &s_abort, p)
-                                        : true;
-                    go = __shfl_sync(kFullMask, int(ok), 0) != 0;
-                    if (!go)
+                    const bool ok = lane == 0 ? wait_or_abort(smem_u32(&sh.kv_empty[slot]),
+                                                              uint32_t(use - 1) & 1u, abort, p)
+                                              : true;
+                    if (!(go = __shfl_sync(kFullMask, int(ok), 0) != 0))
                         break;
                 }
                 if (lane == 0)
@@ -340,221 +349,312 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
                 last_use[slot] = use;
                 __syncwarp();
                 if (ok_id) {
-                    const CUtensorMap *map = kind == 0 ? &tm_k : &tm_v;
+                    const CUtensorMap *map = kind == 0 ? tm_k : tm_v;
                     const uint32_t dst = sbase + kOffRing + uint32_t(slot) * kTileBytes +
                                          uint32_t(lane * box_rows) * 128u;
                     tma_load_2d(dst, map, 0, y, full);
                     tma_load_2d(dst + kSub, map, 64, y, full);
                 }
             }
-            if (!go)
-                break;
         }
-        // After an abort, let the copies already issued land before the CTA
-        // (and its shared memory) goes away.
-        if (s_abort && lane == 0) {
-            for (int i = 0; i < kRing; ++i)
-                if (last_use[i] >= 0)
-                    mbar_wait_bounded(smem_u32(&kv_full[i]), uint32_t(last_use[i]) & 1u);
-            mbar_wait_bounded(smem_u32(&bar_q), 0u);
-        }
-    } else if (warp == kMmaWarp) {
-        // ------------------------------------------------- matrix unit
-        if (lane == 0) {
-            constexpr uint32_t kIdescS = idesc_f16_f32(kPM, kPN, false);
-            constexpr uint32_t kIdescO = idesc_f16_f32(kPM, kPD, true);
-            volatile int *abort = &s_abort;
-            const bool act0 = T.rows[0] > 0, act1 = T.rows[1] > 0;
-            auto slot_addr = [&](int i) { return sbase + kOffRing + uint32_t(i % kRing) * kTileBytes; };
-            auto wait_full = [&](int i) {
-                const bool ok = wait_or_abort(smem_u32(&kv_full[i % kRing]), uint32_t(i / kRing) & 1u,
-                                              abort, p);
-                tc_fence_after_sync();
-                return ok;
-            };
-            auto issue_s = [&](int t, uint32_t k_addr) {
-                const uint32_t q_addr = sbase + uint32_t(t) * kTileBytes;
-#pragma unroll
-                for (int k = 0; k < kPD / 16; ++k) {
-                    const uint32_t kb = uint32_t(k >> 2) * kSub, kk = uint32_t(k & 3) * 32u;
-                    umma_f16(tmem + uint32_t(t) * kPN, smem_desc_sw128(q_addr + kb + kk, 16, 1024),
-                             smem_desc_sw128(k_addr + kb + kk, 16, 1024), kIdescS, k > 0);
-                }
-                umma_commit(smem_u32(&s_full[t]));
-            };
-            auto issue_pv = [&](int t, uint32_t v_addr, bool accumulate) {
-                const uint32_t p_tmem = tmem + uint32_t(t) * kPN;          // P aliases S
-                const uint32_t o_tmem = tmem + 2u * kPN + uint32_t(t) * kPD;
-#pragma unroll
-                for (int k = 0; k < kPN / 16; ++k)
-                    umma_f16_ts(o_tmem, p_tmem + uint32_t(k) * 8u,
-                                smem_desc_sw128(v_addr + uint32_t(k) * 2048u, kSub, 1024), kIdescO,
-                                accumulate || k > 0);
-                umma_commit(smem_u32(&o_full[t]));
-            };
-            auto wait_p = [&](int t, int j) {
-                const bool ok = wait_or_abort(smem_u32(&p_full[t]), uint32_t(j) & 1u, abort, p);
-                tc_fence_after_sync();
-                return ok;
-            };
+        ring += 2 * it.ntiles;
+    }
+    // After an abort, let the copies already issued land before the CTA (and
+    // its shared memory) goes away.
+    if (*abort && lane == 0) {
+        for (int i = 0; i < kRing; ++i)
+            if (last_use[i] >= 0)
+                mbar_wait_bounded(smem_u32(&sh.kv_full[i]), uint32_t(last_use[i]) & 1u);
+        if (items > 0)
+            mbar_wait_bounded(smem_u32(&sh.q_full), uint32_t(items - 1) & 1u);
+    }
+}
 
-            bool ok = wait_or_abort(smem_u32(&bar_q), 0u, abort, p) && wait_full(0);
-            if (ok) {
-                if (act0 && T.nt[0] > 0)
-                    issue_s(0, slot_addr(0));
-                if (act1 && T.nt[1] > 0)
-                    issue_s(1, slot_addr(0));
-                umma_commit(smem_u32(&kv_empty[0]));
-            }
-            for (int j = 0; ok && j < T.ntiles; ++j) {
-                const int iv = 2 * j + 1, ik = 2 * j + 2;
-                const bool next = j + 1 < T.ntiles;
-                if (!(ok = wait_full(iv)))
-                    break;
-                if (act0 && j < T.nt[0]) {
-                    if (!(ok = wait_p(0, j)))
-                        break;
-                    issue_pv(0, slot_addr(iv), j > 0);
-                }
-                if (next) {
-                    if (!(ok = wait_full(ik)))
-                        break;
-                    if (act0 && j + 1 < T.nt[0])
-                        issue_s(0, slot_addr(ik));
-                }
-                if (act1 && j < T.nt[1]) {
-                    if (!(ok = wait_p(1, j)))
-                        break;
-                    issue_pv(1, slot_addr(iv), j > 0);
-                }
-                umma_commit(smem_u32(&kv_empty[iv % kRing]));
-                if (next) {
-                    if (act1 && j + 1 < T.nt[1])
-                        issue_s(1, slot_addr(ik));
-                    umma_commit(smem_u32(&kv_empty[ik % kRing]));
-                }
-            }
-            // every matrix operation issued has finished before TMEM and the
-            // shared tiles are released
-            umma_commit(smem_u32(&bar_drain));
-            mbar_wait_bounded(smem_u32(&bar_drain), 0u);
+// ------------------------------------------------------------ matrix unit
+__device__ __forceinline__ void prefill_mma_role(const PrefillParams &p, PrefillShared &sh,
+                                                 uint32_t sbase)
+{
+    constexpr uint32_t kIdescS = idesc_f16_f32(kPM, kPN, false);
+    constexpr uint32_t kIdescO = idesc_f16_f32(kPM, kPD, true);
+    volatile int *abort = &sh.abort;
+    const uint32_t tmem = sh.tmem;
+    const int total = p.num_pairs * p.num_heads * p.num_seqs;
+    auto slot_addr = [&](int i) { return sbase + kOffRing + uint32_t(i % kRing) * kTileBytes; };
+    auto wait_full = [&](int i) {
+        const bool ok = wait_or_abort(smem_u32(&sh.kv_full[i % kRing]), uint32_t(i / kRing) & 1u,
+                                      abort, p);
+        tc_fence_after_sync();
+        return ok;
+    };
+    auto issue_s = [&](int t, uint32_t k_addr) {
+        const uint32_t q_addr = sbase + uint32_t(t) * kTileBytes;
+#pragma unroll
+        for (int k = 0; k < kPD / 16; ++k) {
+            const uint32_t kb = uint32_t(k >> 2) * kSub, kk = uint32_t(k & 3) * 32u;
+            umma_f16(tmem + uint32_t(t) * kPN, smem_desc_sw128(q_addr + kb + kk, 16, 1024),
+                     smem_desc_sw128(k_addr + kb + kk, 16, 1024), kIdescS, k > 0);
         }
-        __syncwarp();
-    } else {
-        // ------------------------------------------------------- softmax
-        const int t = warp >> 2;
-        const int r = tid & 127;
-        if (T.rows[t] > 0) {
-            const uint32_t lane_base = uint32_t((warp & 3) * 32) << 16;
-            const uint32_t tS = tmem + uint32_t(t) * kPN + lane_base;
-            const uint32_t tO = tmem + 2u * kPN + uint32_t(t) * kPD + lane_base;
-            const int my_pos = T.pos0[t] + r;
-            const float c = p.qk_scale_log2;
-            float m_ref = -INFINITY, l = 0.f;
-            bool ok = true;
-            for (int j = 0; j < T.nt[t]; ++j) {
-                ok = __all_sync(kFullMask, wait_or_abort(smem_u32(&s_full[t]), uint32_t(j) & 1u,
-                                                          &s_abort, p));
+        umma_commit(smem_u32(&sh.s_full[t]));
+    };
+    auto issue_pv = [&](int t, uint32_t v_addr, bool accumulate) {
+        const uint32_t p_tmem = tmem + uint32_t(t) * kPN;  // P aliases S
+        const uint32_t o_tmem = tmem + 2u * kPN + uint32_t(t) * kPD;
+#pragma unroll
+        for (int k = 0; k < kPN / 16; ++k)
+            umma_f16_ts(o_tmem, p_tmem + uint32_t(k) * 8u,
+                        smem_desc_sw128(v_addr + uint32_t(k) * 2048u, kSub, 1024), kIdescO,
+                        accumulate || k > 0);
+        umma_commit(smem_u32(&sh.o_full[t]));
+    };
+
+    int ring = 0, items = 0;
+    int cnt[kQTiles] = {0, 0};       // context tiles processed per query tile (all items)
+    int t_items[kQTiles] = {0, 0};   // items in which query tile t took part
+    bool ok = true;
+    for (int k = blockIdx.x; ok && k < total; k += gridDim.x) {
+        PrefillItem it;
+        if (!prefill_item(p, k, it, false))
+            continue;
+        const bool act[kQTiles] = {it.rows[0] > 0, it.rows[1] > 0};
+        // P V of tile t at context tile j: the softmax has written P_t, and,
+        // for an item's first tile, the previous item's epilogue has read O_t
+        auto pv = [&](int t, int j, uint32_t v_addr) {
+            if (j == 0 && t_items[t] > 0 &&
+                !wait_or_abort(smem_u32(&sh.o_empty[t]), uint32_t(t_items[t] - 1) & 1u, abort, p))
+                return false;
+            if (!wait_or_abort(smem_u32(&sh.p_full[t]), uint32_t(cnt[t] + j) & 1u, abort, p))
+                return false;
+            tc_fence_after_sync();
+            issue_pv(t, v_addr, j > 0);
+            return true;
+        };
+        if (!(ok = wait_or_abort(smem_u32(&sh.q_full), uint32_t(items) & 1u, abort, p) &&
+                   wait_full(ring)))
+            break;
+        ++items;
+        for (int t = 0; t < kQTiles; ++t)
+            if (act[t] && it.nt[t] > 0)
+                issue_s(t, slot_addr(ring));
+        umma_commit(smem_u32(&sh.kv_empty[ring % kRing]));
+        if (it.ntiles == 1)
+            umma_commit(smem_u32(&sh.q_empty));  // last score product of the item issued
+        for (int j = 0; j < it.ntiles; ++j) {
+            const int iv = ring + 2 * j + 1, ik = ring + 2 * j + 2;
+            const bool next = j + 1 < it.ntiles;
+            if (!(ok = wait_full(iv)))
+                break;
+            if (act[0] && j < it.nt[0] && !(ok = pv(0, j, slot_addr(iv))))
+                break;
+            if (next) {
+                if (!(ok = wait_full(ik)))
+                    break;
+                if (act[0] && j + 1 < it.nt[0])
+                    issue_s(0, slot_addr(ik));
+            }
+            if (act[1] && j < it.nt[1] && !(ok = pv(1, j, slot_addr(iv))))
+                break;
+            umma_commit(smem_u32(&sh.kv_empty[iv % kRing]));
+            if (next) {
+                if (act[1] && j + 1 < it.nt[1])
+                    issue_s(1, slot_addr(ik));
+                umma_commit(smem_u32(&sh.kv_empty[ik % kRing]));
+                if (j + 2 == it.ntiles)
+                    umma_commit(smem_u32(&sh.q_empty));
+            }
+        }
+        for (int t = 0; t < kQTiles; ++t)
+            if (act[t]) {
+                cnt[t] += it.nt[t];
+                ++t_items[t];
+            }
+        ring += 2 * it.ntiles;
+    }
+    // every matrix operation issued has finished before TMEM and the shared
+    // tiles are released
+    umma_commit(smem_u32(&sh.drain));
+    mbar_wait_bounded(smem_u32(&sh.drain), 0u);
+}
+
+// ---------------------------------------------------------------- softmax
+__device__ __forceinline__ void prefill_softmax_role(const PrefillParams &p, PrefillShared &sh,
+                                                     unsigned char *smem, int warp, int lane)
+{
+    volatile int *abort = &sh.abort;
+    const int t = warp >> 2;
+    const int r = (warp & 3) * 32 + lane;
+    const uint32_t lane_base = uint32_t((warp & 3) * 32) << 16;
+    const uint32_t tS = sh.tmem + uint32_t(t) * kPN + lane_base;
+    const uint32_t tO = sh.tmem + 2u * kPN + uint32_t(t) * kPD + lane_base;
+    const float c = p.qk_scale_log2;
+    const int H = p.num_heads;
+    const int total = p.num_pairs * H * p.num_seqs;
+    int ring = 0, cnt = 0;
+    for (int k = blockIdx.x; k < total; k += gridDim.x) {
+        PrefillItem it;
+        if (!prefill_item(p, k, it, false))
+            continue;
+        const int item_ring = ring;
+        ring += 2 * it.ntiles;
+        if (it.rows[t] <= 0)
+            continue;
+        const int my_pos = it.pos0[t] + r;
+        const int L = it.L;
+        float m_ref = -INFINITY, l = 0.f;
+        bool ok = true;
+        for (int j = 0; j < it.nt[t]; ++j) {
+            ok = __all_sync(kFullMask,
+                            wait_or_abort(smem_u32(&sh.s_full[t]), uint32_t(cnt + j) & 1u, abort, p));
+            if (!ok)
+                break;
+            tc_fence_after_sync();
+            const int t0 = j * kPN;
+            // columns of this tile this row may see: t <= my_pos and t < L
+            const int lim = min(my_pos, L - 1) - t0 + 1;
+            const bool masked = __any_sync(kFullMask, lim < kPN);
+            const float mx = (masked ? tile_row_max<true>(tS, lim) : tile_row_max<false>(tS, lim)) * c;
+            const float m_new = fmaxf(m_ref, mx);
+            if (j == 0) {
+                m_ref = m_new;
+            } else if (__any_sync(kFullMask, m_new > m_ref + kRescaleLog2)) {
+                // move this warp's reference max: rescale O and l
+                ok = __all_sync(kFullMask, wait_or_abort(smem_u32(&sh.o_full[t]),
+                                                          uint32_t(cnt + j - 1) & 1u, abort, p));
                 if (!ok)
                     break;
                 tc_fence_after_sync();
-                const int t0 = j * kPN;
-                // columns of this tile this row may see: t <= my_pos and t < L
-                const int lim = min(my_pos, L - 1) - t0 + 1;
-                const bool masked = __any_sync(kFullMask, lim < kPN);
-                const float mx = (masked ? tile_row_max<true>(tS, lim) : tile_row_max<false>(tS, lim)) * c;
-                const float m_new = fmaxf(m_ref, mx);
-                if (j == 0) {
-                    m_ref = m_new;
-                } else if (__any_sync(kFullMask, m_new > m_ref + kRescaleLog2)) {
-                    // move this warp's reference max: rescale O and l
-                    ok = __all_sync(kFullMask, wait_or_abort(smem_u32(&o_full[t]),
-                                                              uint32_t(j - 1) & 1u, &s_abort, p));
-                    if (!ok)
-                        break;
-                    tc_fence_after_sync();
-                    const float alpha = ex2_approx(m_ref - m_new);
+                const float alpha = ex2_approx(m_ref - m_new);
 #pragma unroll 1
-                    for (int cc = 0; cc < kPD / 32; ++cc) {
-                        uint32_t o[32];
-                        tmem_load32_async(tO + uint32_t(cc * 32), o);
-                        tmem_wait_ld();
-#pragma unroll
-                        for (int i = 0; i < 32; ++i)
-                            o[i] = __float_as_uint(__uint_as_float(o[i]) * alpha);
-                        tmem_store32(tO + uint32_t(cc * 32), o);
-                    }
-                    l *= alpha;
-                    m_ref = m_new;
-                }
-                // P = 2^(scaled score - m_ref) as fp16 into TMEM over S
-                l += masked ? tile_write_p<true>(tS, lim, c, m_ref) : tile_write_p<false>(tS, lim, c, m_ref);
-                tmem_wait_st();
-                // V rows past the context end (the tail of the last block, or
-                // stale ring contents) are zeroed, so 0 * garbage cannot reach
-                // O.  Done by the first query tile that uses this context tile.
-                const int valid = L - t0;
-                const int tz = (T.rows[0] > 0 && j < T.nt[0]) ? 0 : 1;
-                if (valid < kPN && t == tz) {
-                    const int iv = 2 * j + 1;
-                    ok = __all_sync(kFullMask,
-                                    wait_or_abort(smem_u32(&kv_full[iv % kRing]),
-                                                  uint32_t(iv / kRing) & 1u, &s_abort, p));
-                    if (!ok)
-                        break;
-                    if (r >= valid) {
-                        unsigned char *row = smem + kOffRing + uint32_t(iv % kRing) * kTileBytes +
-                                             uint32_t(r) * 128u;
-#pragma unroll
-                        for (int q16 = 0; q16 < 8; ++q16) {
-                            *reinterpret_cast<uint4 *>(row + q16 * 16) = make_uint4(0, 0, 0, 0);
-                            *reinterpret_cast<uint4 *>(row + kSub + q16 * 16) = make_uint4(0, 0, 0, 0);
-                        }
-                    }
-                    fence_proxy_async_smem();
-                }
-                tc_fence_before_sync();
-                __syncwarp();
-                if (lane == 0)
-                    mbar_arrive(smem_u32(&p_full[t]));
-            }
-            // epilogue: out = O / l
-            if (ok) {
-                ok = __all_sync(kFullMask, wait_or_abort(smem_u32(&o_full[t]),
-                                                          uint32_t(T.nt[t] - 1) & 1u, &s_abort, p));
-            }
-            if (ok) {
-                tc_fence_after_sync();
-                const float inv = 1.f / l;
-                uint4 *dst = reinterpret_cast<uint4 *>(
-                    p.out + (size_t(q_first + row0 + t * kPM + r) * H + h) * kPD);
-                const bool store = r < T.rows[t];
-#pragma unroll
                 for (int cc = 0; cc < kPD / 32; ++cc) {
                     uint32_t o[32];
                     tmem_load32_async(tO + uint32_t(cc * 32), o);
                     tmem_wait_ld();
-                    if (store) {
 #pragma unroll
-                        for (int g = 0; g < 4; ++g) {
-                            __half2 v[4];
+                    for (int i = 0; i < 32; ++i)
+                        o[i] = __float_as_uint(__uint_as_float(o[i]) * alpha);
+                    tmem_store32(tO + uint32_t(cc * 32), o);
+                }
+                l *= alpha;
+                m_ref = m_new;
+            }
+            // P = 2^(scaled score - m_ref) as fp16 into TMEM over S
+            l += masked ? tile_write_p<true>(tS, lim, c, m_ref) : tile_write_p<false>(tS, lim, c, m_ref);
+            tmem_wait_st();
+            // V rows past the context end (the tail of the last block, or
+            // stale ring contents) are zeroed, so 0 * garbage cannot reach O.
+            // Done by the first query tile that uses this context tile.
+            const int valid = L - t0;
+            const int tz = (it.rows[0] > 0 && j < it.nt[0]) ? 0 : 1;
+            if (valid < kPN && t == tz) {
+                const int iv = item_ring + 2 * j + 1;
+                ok = __all_sync(kFullMask, wait_or_abort(smem_u32(&sh.kv_full[iv % kRing]),
+                                                          uint32_t(iv / kRing) & 1u, abort, p));
+                if (!ok)
+                    break;
+                if (r >= valid) {
+                    unsigned char *row =
+                        smem + kOffRing + uint32_t(iv % kRing) * kTileBytes + uint32_t(r) * 128u;
 #pragma unroll
-                            for (int e = 0; e < 4; ++e)
-                                v[e] = __floats2half2_rn(__uint_as_float(o[g * 8 + 2 * e]) * inv,
-                                                         __uint_as_float(o[g * 8 + 2 * e + 1]) * inv);
-                            dst[cc * 4 + g] = *reinterpret_cast<const uint4 *>(v);
-                        }
+                    for (int q16 = 0; q16 < 8; ++q16) {
+                        *reinterpret_cast<uint4 *>(row + q16 * 16) = make_uint4(0, 0, 0, 0);
+                        *reinterpret_cast<uint4 *>(row + kSub + q16 * 16) = make_uint4(0, 0, 0, 0);
                     }
+                }
+                fence_proxy_async_smem();
+            }
+            tc_fence_before_sync();
+            __syncwarp();
+            if (lane == 0)
+                mbar_arrive(smem_u32(&sh.p_full[t]));
+        }
+        if (!ok)
+            break;
+        // epilogue: out = O / l, then O_t is free for the next item
+        ok = __all_sync(kFullMask, wait_or_abort(smem_u32(&sh.o_full[t]),
+                                                  uint32_t(cnt + it.nt[t] - 1) & 1u, abort, p));
+        if (!ok)
+            break;
+        cnt += it.nt[t];
+        tc_fence_after_sync();
+        const float inv = 1.f / l;
+        uint4 *dst = reinterpret_cast<uint4 *>(
+            p.out + (size_t(it.q_first + it.row0 + t * kPM + r) * H + it.h) * kPD);
+        const bool store = r < it.rows[t];
+#pragma unroll 1
+        for (int cc = 0; cc < kPD / 32; ++cc) {
+            uint32_t o[32];
+            tmem_load32_async(tO + uint32_t(cc * 32), o);
+            tmem_wait_ld();
+            if (store) {
+#pragma unroll
+                for (int g = 0; g < 4; ++g) {
+                    __half2 v[4];
+#pragma unroll
+                    for (int e = 0; e < 4; ++e)
+                        v[e] = __floats2half2_rn(__uint_as_float(o[g * 8 + 2 * e]) * inv,
+                                                 __uint_as_float(o[g * 8 + 2 * e + 1]) * inv);
+                    dst[cc * 4 + g] = *reinterpret_cast<const uint4 *>(v);
                 }
             }
         }
+        tc_fence_before_sync();
+        __syncwarp();
+        if (lane == 0)
+            mbar_arrive(smem_u32(&sh.o_empty[t]));
+    }
+}
+
+__global__ void __launch_bounds__(kPrefillThreads, 1)
+    paged_prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+                         const __grid_constant__ CUtensorMap tm_v, const PrefillParams p)
+{
+    extern __shared__ unsigned char smem_raw[];
+    __shared__ __align__(8) PrefillShared sh;
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+
+    grid_dependency_wait();
+    allow_dependent_launch();
+
+    const uint32_t raw = smem_u32(smem_raw);
+    const uint32_t sbase = (raw + 1023u) & ~1023u;
+    unsigned char *smem = smem_raw + (sbase - raw);
+    if (tid == 0) {
+        mbar_init(smem_u32(&sh.q_full), 1);
+        mbar_init(smem_u32(&sh.q_empty), 1);
+        mbar_init(smem_u32(&sh.drain), 1);
+        for (int i = 0; i < kRing; ++i) {
+            mbar_init(smem_u32(&sh.kv_full[i]), 1);
+            mbar_init(smem_u32(&sh.kv_empty[i]), 1);
+        }
+        for (int t = 0; t < kQTiles; ++t) {
+            mbar_init(smem_u32(&sh.s_full[t]), 1);
+            mbar_init(smem_u32(&sh.p_full[t]), 4);   // one arrival per softmax warp
+            mbar_init(smem_u32(&sh.o_full[t]), 1);
+            mbar_init(smem_u32(&sh.o_empty[t]), 4);  // one arrival per softmax warp
+        }
+        sh.abort = 0;
+        fence_mbar_init();
+    }
+    if (warp == kMmaWarp)
+        tmem_alloc(smem_u32(&sh.tmem), kTmemCols);
+    tc_fence_before_sync();
+    __syncthreads();
+    tc_fence_after_sync();
+
+    if (warp == kLoadWarp) {
+        prefill_load_role(&tm_q, &tm_k, &tm_v, p, sh, sbase, lane);
+    } else if (warp == kMmaWarp) {
+        if (lane == 0)
+            prefill_mma_role(p, sh, sbase);
+        __syncwarp();
+    } else {
+        prefill_softmax_role(p, sh, smem, warp, lane);
     }
 
     tc_fence_before_sync();
     __syncthreads();
     if (warp == kMmaWarp) {
         tc_fence_after_sync();
-        tmem_free(tmem, kTmemCols);
+        tmem_free(sh.tmem, kTmemCols);
     }
 }
 

@@ -82,3 +82,16 @@ def test_prefill_running_max_grows_across_tiles():
     out, ref = _run(311, [1000, 600], [700, 600], 16, growth=10.0)
     assert max_abs_err(out, ref) <= ATOL
     assert binding.pa_get_last_device_error() == 0
+
+
+def test_prefill_many_items_per_persistent_cta():
+    """More (query-tile pair, head, sequence) items than SMs, so every
+    persistent CTA walks several items back to back (reusing its Q buffers,
+    TMEM accumulators and K/V ring), with empty items mixed in."""
+    rng = np.random.default_rng(312)
+    lens = rng.integers(1, 700, size=24)
+    n_new = [int(rng.integers(0, min(int(x), 600) + 1)) for x in lens]
+    n_new[3] = int(lens[3])           # one whole prompt
+    out, ref = _run(312, lens.tolist(), n_new, 16, h=8)
+    assert max_abs_err(out, ref) <= ATOL
+    assert binding.pa_get_last_device_error() == 0
