@@ -249,7 +249,10 @@ PA_API pa_status pa_swap_blocks(const void *src, void *dst, size_t block_bytes,
  * Runs on the tensor cores (tcgen05, fp16 inputs, fp32 accumulation; the
  * attention weights enter the P.V product rounded to fp16).  head_dim must
  * be 128 (else PA_ERR_UNSUPPORTED); scale must be finite and > 0 (else
- * PA_ERR_INVALID_ARG).  n_b > L_b is reported in the device
+ * PA_ERR_INVALID_ARG).  The kernel hands out its work through one of 64
+ * per-device counters taken in turn, so at most 64 pa_prefill launches may be
+ * in flight on one device at a time (for example on different streams).
+ * n_b > L_b is reported in the device
  * error word (PA_DEVERR_CONTEXT_LEN) and that sequence is skipped.
  */
 PA_API pa_status pa_prefill(void *out, const void *q, const void *k_cache, const void *v_cache,

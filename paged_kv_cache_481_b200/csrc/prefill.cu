@@ -48,6 +48,28 @@ bool make_map(CUtensorMap *map, const void *base, uint64_t cols, uint64_t rows, 
                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// Work counters of the persistent prefill kernel: each launch takes the next
+// of kSchedSlots (next item, CTAs finished) pairs, which start at zero (module
+// load) and are reset by the launch's last CTA.  Slots rotate per device, so
+// launches on different streams get different counters as long as fewer than
+// kSchedSlots prefill launches are in flight on a device at once.
+constexpr int kSchedSlots = 64;
+__device__ unsigned int g_prefill_sched[kSchedSlots][2];
+
+unsigned int *next_sched_slot(int dev)
+{
+    static std::atomic<void *> base[kMaxDevices];
+    static std::atomic<unsigned> turn[kMaxDevices];
+    void *b = base[dev].load(std::memory_order_acquire);
+    if (!b) {
+        if (cudaGetSymbolAddress(&b, g_prefill_sched) != cudaSuccess || !b)
+            return nullptr;
+        base[dev].store(b, std::memory_order_release);
+    }
+    const unsigned slot = turn[dev].fetch_add(1u, std::memory_order_relaxed) % kSchedSlots;
+    return static_cast<unsigned int *>(b) + 2 * slot;
+}
+
 } // namespace
 
 extern "C" pa_status pa_prefill(void *out, const void *q, const void *k_cache, const void *v_cache,
@@ -120,8 +142,11 @@ extern "C" pa_status pa_prefill(void *out, const void *q, const void *k_cache, c
     p.num_seqs = num_seqs;
     p.num_pairs = (max_query_len + kRowsPerItem - 1) / kRowsPerItem;
     const int64_t items = int64_t(p.num_pairs) * num_heads * num_seqs;
-    if (items > INT32_MAX)
+    if (items > (int64_t(1) << 30))
         return PA_ERR_INVALID_ARG;
+    p.sched = next_sched_slot(dev);
+    if (!p.sched)
+        return PA_ERR_CUDA;
     const dim3 grid(unsigned(items < sms ? items : sms));
     return launch_pdl(pa::paged_prefill_kernel, grid, dim3(pa::kPrefillThreads), pa::kPrefillSmem,
                       reinterpret_cast<cudaStream_t>(stream), tm_q, tm_k, tm_v, p) == cudaSuccess

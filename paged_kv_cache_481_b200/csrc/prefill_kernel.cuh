@@ -8,12 +8,14 @@
 // (position p = L - n + i) attends causally to the cached tokens t <= p:
 //   out = softmax_t(scale q.K_t) V_t, K_t / V_t read through the block table.
 //
-// How: persistent CTAs (one per SM) walk a list of items (256 new tokens =
-// two 128-row query tiles, head, sequence); each CTA is
+// How: persistent CTAs (one per SM) claim items (256 new tokens = two
+// 128-row query tiles, head, sequence) from a global counter; each CTA is
 // warp-specialised, with the two query tiles in ping-pong so the tensor core
 // works on one tile while the other tile's softmax runs, and one item's
 // epilogue overlaps the next item's loads and score products.
-//   * warp 8 (loads): TMA tensor loads of Q, then of each 128-token K and V
+//   * warp 8 (loads): claims the next item and passes its index to the other
+//     roles through a two-deep shared-memory queue; TMA tensor loads of Q,
+//     then of each 128-token K and V
 //     tile, (block, head) run by run through the block table, into a ring of
 //     four 128-byte-swizzled shared-memory tiles;
 //   * warp 9 (matrix unit, one thread): S_t = Q_t K^T into TMEM, and, once
@@ -64,6 +66,7 @@ struct PrefillParams {
     unsigned int *error_word;         // PA_DEVERR_* bits
     int num_seqs;
     int num_pairs;                    // query-tile pairs per sequence: ceil(max_query_len / 256)
+    unsigned int *sched;              // [2]: next item to hand out, CTAs finished (both 0 at launch)
 };
 
 constexpr int kPM = 128;              // query rows per tile (MMA M)
@@ -79,6 +82,9 @@ constexpr int kLoadWarp = 8, kMmaWarp = 9;
 constexpr int kPrefillThreads = 10 * 32;
 constexpr uint32_t kTmemCols = 512;
 constexpr float kRescaleLog2 = 8.0f;  // move the reference max only past this growth
+constexpr int kItemRing = 2;          // items handed from the load warp to the other roles
+constexpr int kItemConsumers = 1 + 8; // the MMA thread and the eight softmax warps
+constexpr int kGroupHB = 32;          // (head, sequence) units per scheduling group
 
 __device__ __forceinline__ void prefill_error(const PrefillParams &p, unsigned int bits)
 {
@@ -222,19 +228,26 @@ struct PrefillItem {
     int ntiles;          // context tiles the item walks
 };
 
-// Items are numbered (head, sequence)-major, the pairs of one (head,
-// sequence) heaviest (latest) first: k -> hb = k / P, pair = P - 1 - k % P.
-// CTA c of G takes items c, c + G, c + 2G, ...: the items running at the
-// same time then belong to few (head, sequence), whose K / V stay in L2,
-// and since G is rarely a multiple of P each CTA samples every pair level.
-// Every role walks the same list; empty items (past a sequence's new tokens,
-// or with more new tokens than context) are skipped by all of them alike.
+// Item numbering.  The (head, sequence) units are cut into groups of
+// kGroupHB; within a group the items run pair-major, the latest (heaviest)
+// pair of every unit first: k -> group g = k / (kGroupHB P), then
+// pair = P - 1 - r / n_g and unit = g kGroupHB + r % n_g for r = k mod
+// (kGroupHB P) and n_g units in the group.  CTAs take the next item from a
+// global counter when their load warp is ready, so the work balances itself;
+// the items in flight at one time belong to about one group, whose K / V
+// (kGroupHB units) stay in L2; and each group ends with its lightest items.
+// Empty items (past a sequence's new tokens, or with more new tokens than
+// context) are skipped by the load warp and never reach the other roles.
 // `report` lets exactly one thread record per-sequence argument errors.
 __device__ __forceinline__ bool prefill_item(const PrefillParams &p, int k, PrefillItem &it,
                                              bool report)
 {
-    const int hb = k / p.num_pairs;
-    const int pair = p.num_pairs - 1 - k % p.num_pairs;
+    const int units = p.num_heads * p.num_seqs;
+    const int per_group = kGroupHB * p.num_pairs;
+    const int g = k / per_group, r = k % per_group;
+    const int n_g = min(kGroupHB, units - g * kGroupHB);
+    const int pair = p.num_pairs - 1 - r / n_g;
+    const int hb = g * kGroupHB + r % n_g;
     it.h = hb % p.num_heads;
     it.b = hb / p.num_heads;
     it.q_first = p.query_start_loc[it.b];
@@ -268,12 +281,29 @@ __device__ __forceinline__ bool prefill_item(const PrefillParams &p, int k, Pref
 }
 
 struct PrefillShared {
+    uint64_t item_full[kItemRing], item_empty[kItemRing];
     uint64_t q_full, q_empty, drain;
     uint64_t kv_full[kRing], kv_empty[kRing];
     uint64_t s_full[kQTiles], p_full[kQTiles], o_full[kQTiles], o_empty[kQTiles];
+    int item[kItemRing];   // item index, or -1 = no more items
     uint32_t tmem;
     int abort;
 };
+
+// Next item for the MMA / softmax roles: the load warp's choice, in order.
+// Returns -1 when there are no more items (or on abort).  The caller
+// releases the slot right away (it copies the index).
+__device__ __forceinline__ int prefill_pop_item(const PrefillParams &p, PrefillShared &sh, int u,
+                                                bool arrive)
+{
+    const int slot = u % kItemRing;
+    if (!wait_or_abort(smem_u32(&sh.item_full[slot]), uint32_t(u / kItemRing) & 1u, &sh.abort, p))
+        return -1;
+    const int k = *reinterpret_cast<volatile int *>(&sh.item[slot]);
+    if (arrive)
+        mbar_arrive(smem_u32(&sh.item_empty[slot]));
+    return k;
+}
 
 // ---------------------------------------------------------------- loads
 __device__ __forceinline__ void prefill_load_role(const CUtensorMap *tm_q, const CUtensorMap *tm_k,
@@ -290,10 +320,37 @@ __device__ __forceinline__ void prefill_load_role(const CUtensorMap *tm_q, const
         last_use[i] = -1;
     int ring = 0, items = 0;
     bool go = true;
-    for (int k = blockIdx.x; go && k < total; k += gridDim.x) {
+    for (;;) {
+        // claim the next non-empty item and hand it to the other roles
+        int k = -1;
         PrefillItem it;
-        if (!prefill_item(p, k, it, lane == 0))
-            continue;
+        for (;;) {
+            int kk = 0;
+            if (lane == 0)
+                kk = *abort ? total : int(atomicAdd(p.sched, 1u));
+            kk = __shfl_sync(kFullMask, kk, 0);
+            if (kk >= total)
+                break;
+            if (prefill_item(p, kk, it, lane == 0)) {
+                k = kk;
+                break;
+            }
+        }
+        {
+            const int slot = items % kItemRing, use = items / kItemRing;
+            bool ok = true;
+            if (use > 0 && lane == 0)
+                ok = wait_or_abort(smem_u32(&sh.item_empty[slot]), uint32_t(use - 1) & 1u, abort, p);
+            if (!__shfl_sync(kFullMask, int(ok), 0))
+                break;
+            if (lane == 0) {
+                sh.item[slot] = k;
+                mbar_arrive(smem_u32(&sh.item_full[slot]));  // release: the index is visible
+            }
+            __syncwarp();
+        }
+        if (k < 0)
+            break;
         // Q of this item once the previous item's score products are done
         if (items > 0) {
             const bool ok = lane == 0 ? wait_or_abort(smem_u32(&sh.q_empty), uint32_t(items - 1) & 1u,
@@ -358,6 +415,8 @@ __device__ __forceinline__ void prefill_load_role(const CUtensorMap *tm_q, const
             }
         }
         ring += 2 * it.ntiles;
+        if (!go)
+            break;
     }
     // After an abort, let the copies already issued land before the CTA (and
     // its shared memory) goes away.
@@ -378,7 +437,6 @@ __device__ __forceinline__ void prefill_mma_role(const PrefillParams &p, Prefill
     constexpr uint32_t kIdescO = idesc_f16_f32(kPM, kPD, true);
     volatile int *abort = &sh.abort;
     const uint32_t tmem = sh.tmem;
-    const int total = p.num_pairs * p.num_heads * p.num_seqs;
     auto slot_addr = [&](int i) { return sbase + kOffRing + uint32_t(i % kRing) * kTileBytes; };
     auto wait_full = [&](int i) {
         const bool ok = wait_or_abort(smem_u32(&sh.kv_full[i % kRing]), uint32_t(i / kRing) & 1u,
@@ -411,10 +469,12 @@ __device__ __forceinline__ void prefill_mma_role(const PrefillParams &p, Prefill
     int cnt[kQTiles] = {0, 0};       // context tiles processed per query tile (all items)
     int t_items[kQTiles] = {0, 0};   // items in which query tile t took part
     bool ok = true;
-    for (int k = blockIdx.x; ok && k < total; k += gridDim.x) {
+    for (int u = 0; ok; ++u) {
+        const int k = prefill_pop_item(p, sh, u, true);
+        if (k < 0)
+            break;
         PrefillItem it;
-        if (!prefill_item(p, k, it, false))
-            continue;
+        prefill_item(p, k, it, false);
         const bool act[kQTiles] = {it.rows[0] > 0, it.rows[1] > 0};
         // P V of tile t at context tile j: the softmax has written P_t, and,
         // for an item's first tile, the previous item's epilogue has read O_t
@@ -487,12 +547,16 @@ __device__ __forceinline__ void prefill_softmax_role(const PrefillParams &p, Pre
     const uint32_t tO = sh.tmem + 2u * kPN + uint32_t(t) * kPD + lane_base;
     const float c = p.qk_scale_log2;
     const int H = p.num_heads;
-    const int total = p.num_pairs * H * p.num_seqs;
     int ring = 0, cnt = 0;
-    for (int k = blockIdx.x; k < total; k += gridDim.x) {
+    for (int u = 0;; ++u) {
+        const int k = __shfl_sync(kFullMask, lane == 0 ? prefill_pop_item(p, sh, u, false) : 0, 0);
+        __syncwarp();
+        if (lane == 0 && k >= 0)
+            mbar_arrive(smem_u32(&sh.item_empty[u % kItemRing]));
+        if (k < 0)
+            break;
         PrefillItem it;
-        if (!prefill_item(p, k, it, false))
-            continue;
+        prefill_item(p, k, it, false);
         const int item_ring = ring;
         ring += 2 * it.ntiles;
         if (it.rows[t] <= 0)
@@ -618,6 +682,10 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
     const uint32_t sbase = (raw + 1023u) & ~1023u;
     unsigned char *smem = smem_raw + (sbase - raw);
     if (tid == 0) {
+        for (int i = 0; i < kItemRing; ++i) {
+            mbar_init(smem_u32(&sh.item_full[i]), 1);
+            mbar_init(smem_u32(&sh.item_empty[i]), kItemConsumers);
+        }
         mbar_init(smem_u32(&sh.q_full), 1);
         mbar_init(smem_u32(&sh.q_empty), 1);
         mbar_init(smem_u32(&sh.drain), 1);
@@ -655,6 +723,16 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
     if (warp == kMmaWarp) {
         tc_fence_after_sync();
         tmem_free(sh.tmem, kTmemCols);
+    }
+    // The last CTA to finish resets the item counter for the launch that
+    // next uses this scheduling slot (every CTA has stopped claiming items).
+    if (tid == 0) {
+        __threadfence();
+        if (atomicAdd(p.sched + 1, 1u) == gridDim.x - 1) {
+            atomicExch(p.sched, 0u);
+            atomicExch(p.sched + 1, 0u);
+            __threadfence();
+        }
     }
 }
 
