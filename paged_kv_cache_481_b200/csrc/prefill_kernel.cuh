@@ -26,7 +26,8 @@
 //   * warps 0-3 / 4-7 (softmax of query tile 0 / 1, one query row per
 //     thread = TMEM lane): read S back, causal mask, online softmax in the
 //     log2 domain, P as fp16 into TMEM (the row sum l is taken from P before
-//     its fp16 rounding).  Only warps holding a diagonal or context-end tile
+//     its fp16 rounding); a share of the exp2 can run as a polynomial on the
+//     FMA pipes instead of the special-function unit (kExp2FmaPairsPer8).  Only warps holding a diagonal or context-end tile
 //     pay for the mask.  The running max is only moved when
 //     it grows by more than 2^8 (in base-2 exponent units); then the warp
 //     rescales its O rows and l in TMEM.  Otherwise P is taken against the
@@ -155,6 +156,54 @@ __device__ __forceinline__ uint64_t add2(uint64_t a, uint64_t b)
     return d;
 }
 
+// 2^x for a pair of scores on the FMA pipes, relieving the special-function
+// unit (which alone would need as many cycles per tile as the tensor core).
+// Cody-Waite range reduction x = j + f, j = floor(x) exact in fp32 (adding
+// 1.5 * 2^23 with round-down leaves floor(x) in the low mantissa bits), and a
+// degree-3 minimax polynomial p(f) ~ 2^f on [0, 1) (max relative error
+// 7.5e-5, fitted by Remez exchange in paged_kv_cache_481_b200/exp2_poly.py);
+// 2^j is added to p's exponent field.  x is clamped below at -126 (the
+// result is then ~2^-126, which the fp16 weight rounds to 0; at -127 the
+// exponent field of p(0) < 1 would wrap).
+constexpr float kExp2C0 = 0.99992521856271543f;
+constexpr float kExp2C1 = 0.69583354049475277f;
+constexpr float kExp2C2 = 0.22606715542748301f;
+constexpr float kExp2C3 = 0.07802452264047964f;
+constexpr float kExp2Magic = 12582912.0f;  // 1.5 * 2^23
+
+__device__ __forceinline__ uint64_t add2_rm(uint64_t a, uint64_t b)
+{
+    uint64_t d;
+    asm("add.rm.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+    return d;
+}
+
+__device__ __forceinline__ void ex2_poly2(float x0, float x1, float &y0, float &y1)
+{
+    const uint64_t xx = pack2(fmaxf(x0, -126.f), fmaxf(x1, -126.f));
+    const uint64_t t = add2_rm(xx, pack2(kExp2Magic, kExp2Magic));      // magic + floor(x)
+    const uint64_t j = add2(t, pack2(-kExp2Magic, -kExp2Magic));          // floor(x), exact
+    const uint64_t f = fma2(j, pack2(-1.f, -1.f), xx);                    // x - floor(x) in [0, 1)
+    uint64_t q = fma2(pack2(kExp2C3, kExp2C3), f, pack2(kExp2C2, kExp2C2));
+    q = fma2(q, f, pack2(kExp2C1, kExp2C1));
+    q = fma2(q, f, pack2(kExp2C0, kExp2C0));
+    float q0, q1, t0, t1;
+    unpack2(q, q0, q1);
+    unpack2(t, t0, t1);
+    // (magic + j) << 23 keeps exactly j << 23 (mod 2^32): 2^j into the exponent
+    y0 = __uint_as_float(__float_as_uint(q0) + (__float_as_uint(t0) << 23));
+    y1 = __uint_as_float(__float_as_uint(q1) + (__float_as_uint(t1) << 23));
+}
+
+// Pairs out of every 8 whose exp2 goes to the FMA pipes.  Measured on the
+// 13B prefill cases: 3 of 8 was 2-6 % slower than 0 (the special-function
+// unit is not yet the limit there), so the polynomial stays off for now.
+constexpr int kExp2FmaPairsPer8 = 0;
+__host__ __device__ constexpr bool exp2_on_fma(int e)
+{
+    return (e & 7) < kExp2FmaPairsPer8;
+}
+
 // Row max of the raw scores of one 128-column S tile (this thread's TMEM
 // lane); with kMasked, only the first `lim` columns count.
 template <bool kMasked>
@@ -202,7 +251,13 @@ __device__ __forceinline__ float tile_write_p(uint32_t tS, int lim, float c, flo
             float x0, x1;
             unpack2(fma2(pack2(__uint_as_float(s[2 * e]), __uint_as_float(s[2 * e + 1])), c2, nm2),
                     x0, x1);
-            float p0 = ex2_approx(x0), p1 = ex2_approx(x1);
+            float p0, p1;
+            if (exp2_on_fma(e)) {
+                ex2_poly2(x0, x1, p0, p1);
+            } else {
+                p0 = ex2_approx(x0);
+                p1 = ex2_approx(x1);
+            }
             if (kMasked) {
                 const int col = cc * 32 + 2 * e;
                 p0 = col < lim ? p0 : 0.f;
