@@ -24,7 +24,8 @@
 //     the order S_0 PV_0 S_0' PV_1 S_1' keeps one tile's matrix work in
 //     flight while the other tile's softmax runs;
 //   * warps 0-3 / 4-7 (softmax of query tile 0 / 1, one query row per
-//     thread = TMEM lane): read S back, causal mask, online softmax in the
+//     thread = TMEM lane): read the S row back (all 128 columns, one wait),
+//     causal mask, online softmax in the
 //     log2 domain, P as fp16 into TMEM (the row sum l is taken from P before
 //     its fp16 rounding); a share of the exp2 can run as a polynomial on the
 //     FMA pipes instead of the special-function unit (kExp2FmaPairsPer8).  Only warps holding a diagonal or context-end tile
@@ -204,53 +205,57 @@ __host__ __device__ constexpr bool exp2_on_fma(int e)
     return (e & 7) < kExp2FmaPairsPer8;
 }
 
-// Row max of the raw scores of one 128-column S tile (this thread's TMEM
-// lane); with kMasked, only the first `lim` columns count.
-template <bool kMasked>
-__device__ __forceinline__ float tile_row_max(uint32_t tS, int lim)
+// One S tile row in registers: all 128 scores of this thread's TMEM lane,
+// loaded with one wait.
+struct ScoreRow {
+    uint32_t s[kPN];
+};
+
+__device__ __forceinline__ void load_score_row(uint32_t tS, ScoreRow &r)
 {
-    float m0 = -INFINITY, m1 = -INFINITY;
 #pragma unroll
-    for (int cc = 0; cc < kPN / 32; ++cc) {
-        uint32_t s[32];
-        tmem_load32_async(tS + uint32_t(cc * 32), s);
-        tmem_wait_ld();
-#pragma unroll
-        for (int i = 0; i < 32; i += 4) {
-            float a = __uint_as_float(s[i]), b = __uint_as_float(s[i + 1]);
-            float c = __uint_as_float(s[i + 2]), d = __uint_as_float(s[i + 3]);
-            if (kMasked) {
-                const int col = cc * 32 + i;
-                a = col < lim ? a : -INFINITY;
-                b = col + 1 < lim ? b : -INFINITY;
-                c = col + 2 < lim ? c : -INFINITY;
-                d = col + 3 < lim ? d : -INFINITY;
-            }
-            m0 = max3f(m0, a, b);
-            m1 = max3f(m1, c, d);
-        }
-    }
-    return fmaxf(m0, m1);
+    for (int cc = 0; cc < kPN / 32; ++cc)
+        tmem_load32_into(tS + uint32_t(cc * 32), r.s + cc * 32);
+    tmem_wait_ld();
 }
 
-// P = 2^(c * s - m) of one S tile, as fp16 pairs written back into TMEM over
-// the first 64 columns of S; returns the row sum of P (fp32, before the fp16
+// Row max of the raw scores; with kMasked only the first `lim` columns count.
+template <bool kMasked>
+__device__ __forceinline__ float score_row_max(const ScoreRow &r, int lim)
+{
+    float m[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+#pragma unroll
+    for (int i = 0; i < kPN; i += 8) {
+#pragma unroll
+        for (int a = 0; a < 4; ++a) {
+            float x = __uint_as_float(r.s[i + 2 * a]), y = __uint_as_float(r.s[i + 2 * a + 1]);
+            if (kMasked) {
+                x = i + 2 * a < lim ? x : -INFINITY;
+                y = i + 2 * a + 1 < lim ? y : -INFINITY;
+            }
+            m[a] = max3f(m[a], x, y);
+        }
+    }
+    return fmaxf(fmaxf(m[0], m[1]), fmaxf(m[2], m[3]));
+}
+
+// P = 2^(c * s - m) of the row, as fp16 pairs written into TMEM over the
+// first 64 columns of S; returns the row sum of P (fp32, before the fp16
 // rounding).  With kMasked, columns >= lim give P = 0.
 template <bool kMasked>
-__device__ __forceinline__ float tile_write_p(uint32_t tS, int lim, float c, float m)
+__device__ __forceinline__ float write_p_row(uint32_t tS, const ScoreRow &r, int lim, float c,
+                                             float m)
 {
     const uint64_t c2 = pack2(c, c), nm2 = pack2(-m, -m);
-    uint64_t sum2 = pack2(0.f, 0.f);
+    uint64_t sum2[2] = {pack2(0.f, 0.f), pack2(0.f, 0.f)};
 #pragma unroll
     for (int cc = 0; cc < kPN / 32; ++cc) {
-        uint32_t s[32], pk[16];
-        tmem_load32_async(tS + uint32_t(cc * 32), s);
-        tmem_wait_ld();
+        uint32_t pk[16];
 #pragma unroll
         for (int e = 0; e < 16; ++e) {
+            const int i = cc * 32 + 2 * e;
             float x0, x1;
-            unpack2(fma2(pack2(__uint_as_float(s[2 * e]), __uint_as_float(s[2 * e + 1])), c2, nm2),
-                    x0, x1);
+            unpack2(fma2(pack2(__uint_as_float(r.s[i]), __uint_as_float(r.s[i + 1])), c2, nm2), x0, x1);
             float p0, p1;
             if (exp2_on_fma(e)) {
                 ex2_poly2(x0, x1, p0, p1);
@@ -259,19 +264,19 @@ __device__ __forceinline__ float tile_write_p(uint32_t tS, int lim, float c, flo
                 p1 = ex2_approx(x1);
             }
             if (kMasked) {
-                const int col = cc * 32 + 2 * e;
-                p0 = col < lim ? p0 : 0.f;
-                p1 = col + 1 < lim ? p1 : 0.f;
+                p0 = i < lim ? p0 : 0.f;
+                p1 = i + 1 < lim ? p1 : 0.f;
             }
-            sum2 = add2(sum2, pack2(p0, p1));
+            sum2[e & 1] = add2(sum2[e & 1], pack2(p0, p1));
             const __half2 ph = __floats2half2_rn(p0, p1);
             pk[e] = *reinterpret_cast<const uint32_t *>(&ph);
         }
         tmem_store16(tS + uint32_t(cc * 16), pk);
     }
-    float lo, hi;
-    unpack2(sum2, lo, hi);
-    return lo + hi;
+    float a0, a1, b0, b1;
+    unpack2(sum2[0], a0, a1);
+    unpack2(sum2[1], b0, b1);
+    return (a0 + a1) + (b0 + b1);
 }
 
 // One unit of work: two query tiles (256 new tokens) of one (head, sequence).
@@ -630,7 +635,9 @@ __device__ __forceinline__ void prefill_softmax_role(const PrefillParams &p, Pre
             // columns of this tile this row may see: t <= my_pos and t < L
             const int lim = min(my_pos, L - 1) - t0 + 1;
             const bool masked = __any_sync(kFullMask, lim < kPN);
-            const float mx = (masked ? tile_row_max<true>(tS, lim) : tile_row_max<false>(tS, lim)) * c;
+            ScoreRow row;
+            load_score_row(tS, row);
+            const float mx = (masked ? score_row_max<true>(row, lim) : score_row_max<false>(row, lim)) * c;
             const float m_new = fmaxf(m_ref, mx);
             if (j == 0) {
                 m_ref = m_new;
@@ -643,20 +650,21 @@ __device__ __forceinline__ void prefill_softmax_role(const PrefillParams &p, Pre
                 tc_fence_after_sync();
                 const float alpha = ex2_approx(m_ref - m_new);
 #pragma unroll 1
-                for (int cc = 0; cc < kPD / 32; ++cc) {
-                    uint32_t o[32];
-                    tmem_load32_async(tO + uint32_t(cc * 32), o);
+                for (int cc = 0; cc < kPD / 16; ++cc) {  // 16 columns at a time: the score row is live
+                    uint32_t o[16];
+                    tmem_load16_async(tO + uint32_t(cc * 16), o);
                     tmem_wait_ld();
 #pragma unroll
-                    for (int i = 0; i < 32; ++i)
+                    for (int i = 0; i < 16; ++i)
                         o[i] = __float_as_uint(__uint_as_float(o[i]) * alpha);
-                    tmem_store32(tO + uint32_t(cc * 32), o);
+                    tmem_store16(tO + uint32_t(cc * 16), o);
                 }
                 l *= alpha;
                 m_ref = m_new;
             }
             // P = 2^(scaled score - m_ref) as fp16 into TMEM over S
-            l += masked ? tile_write_p<true>(tS, lim, c, m_ref) : tile_write_p<false>(tS, lim, c, m_ref);
+            l += masked ? write_p_row<true>(tS, row, lim, c, m_ref)
+                        : write_p_row<false>(tS, row, lim, c, m_ref);
             tmem_wait_st();
             // V rows past the context end (the tail of the last block, or
             // stale ring contents) are zeroed, so 0 * garbage cannot reach O.
