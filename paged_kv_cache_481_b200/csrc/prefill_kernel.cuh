@@ -84,6 +84,9 @@ constexpr int kLoadWarp = 8, kMmaWarp = 9;
 constexpr int kPrefillThreads = 10 * 32;
 constexpr uint32_t kTmemCols = 512;
 constexpr float kRescaleLog2 = 8.0f;  // move the reference max only past this growth
+#ifndef PA_PREFILL_SCALAR_P
+#define PA_PREFILL_SCALAR_P 1
+#endif
 constexpr int kItemRing = 2;          // items handed from the load warp to the other roles
 constexpr int kItemConsumers = 1 + 8; // the MMA thread and the eight softmax warps
 constexpr int kGroupHB = 32;          // (head, sequence) units per scheduling group
@@ -246,8 +249,12 @@ template <bool kMasked>
 __device__ __forceinline__ float write_p_row(uint32_t tS, const ScoreRow &r, int lim, float c,
                                              float m)
 {
+#if PA_PREFILL_SCALAR_P
+    float sum[4] = {0.f, 0.f, 0.f, 0.f};
+#else
     const uint64_t c2 = pack2(c, c), nm2 = pack2(-m, -m);
     uint64_t sum2[2] = {pack2(0.f, 0.f), pack2(0.f, 0.f)};
+#endif
 #pragma unroll
     for (int cc = 0; cc < kPN / 32; ++cc) {
         uint32_t pk[16];
@@ -255,7 +262,12 @@ __device__ __forceinline__ float write_p_row(uint32_t tS, const ScoreRow &r, int
         for (int e = 0; e < 16; ++e) {
             const int i = cc * 32 + 2 * e;
             float x0, x1;
+#if PA_PREFILL_SCALAR_P
+            x0 = fmaf(__uint_as_float(r.s[i]), c, -m);
+            x1 = fmaf(__uint_as_float(r.s[i + 1]), c, -m);
+#else
             unpack2(fma2(pack2(__uint_as_float(r.s[i]), __uint_as_float(r.s[i + 1])), c2, nm2), x0, x1);
+#endif
             float p0, p1;
             if (exp2_on_fma(e)) {
                 ex2_poly2(x0, x1, p0, p1);
@@ -267,16 +279,25 @@ __device__ __forceinline__ float write_p_row(uint32_t tS, const ScoreRow &r, int
                 p0 = i < lim ? p0 : 0.f;
                 p1 = i + 1 < lim ? p1 : 0.f;
             }
+#if PA_PREFILL_SCALAR_P
+            sum[(e & 1) * 2] += p0;
+            sum[(e & 1) * 2 + 1] += p1;
+#else
             sum2[e & 1] = add2(sum2[e & 1], pack2(p0, p1));
+#endif
             const __half2 ph = __floats2half2_rn(p0, p1);
             pk[e] = *reinterpret_cast<const uint32_t *>(&ph);
         }
         tmem_store16(tS + uint32_t(cc * 16), pk);
     }
+#if PA_PREFILL_SCALAR_P
+    return (sum[0] + sum[1]) + (sum[2] + sum[3]);
+#else
     float a0, a1, b0, b1;
     unpack2(sum2[0], a0, a1);
     unpack2(sum2[1], b0, b1);
     return (a0 + a1) + (b0 + b1);
+#endif
 }
 
 // One unit of work: two query tiles (256 new tokens) of one (head, sequence).
