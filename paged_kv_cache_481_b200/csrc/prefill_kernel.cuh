@@ -83,10 +83,14 @@ constexpr uint32_t kPrefillSmem = kOffRing + kRing * kTileBytes + 1024;  // + 10
 constexpr int kLoadWarp = 8, kMmaWarp = 9;
 constexpr int kPrefillThreads = 10 * 32;
 constexpr uint32_t kTmemCols = 512;
-constexpr float kRescaleLog2 = 8.0f;  // move the reference max only past this growth
-#ifndef PA_PREFILL_SCALAR_P
-#define PA_PREFILL_SCALAR_P 1
+#ifndef PA_PREFILL_EXP2_HALF
+#define PA_PREFILL_EXP2_HALF 0
 #endif
+// exp2 of the scores on fp16 pairs (one special-function instruction per
+// pair) instead of fp32 singles
+constexpr bool kExp2Half = PA_PREFILL_EXP2_HALF != 0;
+// move the reference max only past this growth (base-2 units)
+constexpr float kRescaleLog2 = kExp2Half ? 2.0f : 8.0f;
 constexpr int kItemRing = 2;          // items handed from the load warp to the other roles
 constexpr int kItemConsumers = 1 + 8; // the MMA thread and the eight softmax warps
 constexpr int kGroupHB = 32;          // (head, sequence) units per scheduling group
@@ -242,62 +246,75 @@ __device__ __forceinline__ float score_row_max(const ScoreRow &r, int lim)
     return fmaxf(fmaxf(m[0], m[1]), fmaxf(m[2], m[3]));
 }
 
+// 2^x of two fp32 arguments in one special-function instruction at half
+// precision: the arguments are rounded to fp16 (with the reference max moved
+// by at most 2^2, |x| <= 2 for the weights that matter, so the argument
+// rounding costs at most 2^-10 relative) and the result is the fp16 pair P
+// that the tensor core takes anyway.
+__device__ __forceinline__ uint32_t ex2_half2(float x0, float x1)
+{
+    uint32_t in, out;
+    asm("cvt.rn.f16x2.f32 %0, %1, %2;" : "=r"(in) : "f"(x1), "f"(x0));
+    asm("ex2.approx.f16x2 %0, %1;" : "=r"(out) : "r"(in));
+    return out;
+}
+
+// acc += the two fp16 halves of v (exact products with 1.0, fp32 adds)
+__device__ __forceinline__ void add_half2_f32(uint32_t v, float &acc0, float &acc1)
+{
+    asm("{\n\t.reg .f16 lo, hi, one;\n\t"
+        "mov.b16 one, 0x3C00;\n\t"
+        "mov.b32 {lo, hi}, %2;\n\t"
+        "fma.rn.f32.f16 %0, lo, one, %0;\n\t"
+        "fma.rn.f32.f16 %1, hi, one, %1;\n\t}"
+        : "+f"(acc0), "+f"(acc1)
+        : "r"(v));
+}
+
 // P = 2^(c * s - m) of the row, as fp16 pairs written into TMEM over the
-// first 64 columns of S; returns the row sum of P (fp32, before the fp16
-// rounding).  With kMasked, columns >= lim give P = 0.
+// first 64 columns of S; returns the row sum of P (fp32; of the fp16 values
+// with the half-precision exponential, else before the fp16 rounding).
+// With kMasked, columns >= lim give P = 0.
 template <bool kMasked>
 __device__ __forceinline__ float write_p_row(uint32_t tS, const ScoreRow &r, int lim, float c,
                                              float m)
 {
-#if PA_PREFILL_SCALAR_P
     float sum[4] = {0.f, 0.f, 0.f, 0.f};
-#else
-    const uint64_t c2 = pack2(c, c), nm2 = pack2(-m, -m);
-    uint64_t sum2[2] = {pack2(0.f, 0.f), pack2(0.f, 0.f)};
-#endif
 #pragma unroll
     for (int cc = 0; cc < kPN / 32; ++cc) {
         uint32_t pk[16];
 #pragma unroll
         for (int e = 0; e < 16; ++e) {
             const int i = cc * 32 + 2 * e;
-            float x0, x1;
-#if PA_PREFILL_SCALAR_P
-            x0 = fmaf(__uint_as_float(r.s[i]), c, -m);
-            x1 = fmaf(__uint_as_float(r.s[i + 1]), c, -m);
-#else
-            unpack2(fma2(pack2(__uint_as_float(r.s[i]), __uint_as_float(r.s[i + 1])), c2, nm2), x0, x1);
-#endif
-            float p0, p1;
-            if (exp2_on_fma(e)) {
-                ex2_poly2(x0, x1, p0, p1);
+            const float x0 = fmaf(__uint_as_float(r.s[i]), c, -m);
+            const float x1 = fmaf(__uint_as_float(r.s[i + 1]), c, -m);
+            if (kExp2Half) {
+                uint32_t ph = ex2_half2(x0, x1);
+                if (kMasked)
+                    ph &= (i < lim ? 0x0000FFFFu : 0u) | (i + 1 < lim ? 0xFFFF0000u : 0u);
+                add_half2_f32(ph, sum[(e & 1) * 2], sum[(e & 1) * 2 + 1]);
+                pk[e] = ph;
             } else {
-                p0 = ex2_approx(x0);
-                p1 = ex2_approx(x1);
+                float p0, p1;
+                if (exp2_on_fma(e)) {
+                    ex2_poly2(x0, x1, p0, p1);
+                } else {
+                    p0 = ex2_approx(x0);
+                    p1 = ex2_approx(x1);
+                }
+                if (kMasked) {
+                    p0 = i < lim ? p0 : 0.f;
+                    p1 = i + 1 < lim ? p1 : 0.f;
+                }
+                sum[(e & 1) * 2] += p0;
+                sum[(e & 1) * 2 + 1] += p1;
+                const __half2 ph = __floats2half2_rn(p0, p1);
+                pk[e] = *reinterpret_cast<const uint32_t *>(&ph);
             }
-            if (kMasked) {
-                p0 = i < lim ? p0 : 0.f;
-                p1 = i + 1 < lim ? p1 : 0.f;
-            }
-#if PA_PREFILL_SCALAR_P
-            sum[(e & 1) * 2] += p0;
-            sum[(e & 1) * 2 + 1] += p1;
-#else
-            sum2[e & 1] = add2(sum2[e & 1], pack2(p0, p1));
-#endif
-            const __half2 ph = __floats2half2_rn(p0, p1);
-            pk[e] = *reinterpret_cast<const uint32_t *>(&ph);
         }
         tmem_store16(tS + uint32_t(cc * 16), pk);
     }
-#if PA_PREFILL_SCALAR_P
     return (sum[0] + sum[1]) + (sum[2] + sum[3]);
-#else
-    float a0, a1, b0, b1;
-    unpack2(sum2[0], a0, a1);
-    unpack2(sum2[1], b0, b1);
-    return (a0 + a1) + (b0 + b1);
-#endif
 }
 
 // One unit of work: two query tiles (256 new tokens) of one (head, sequence).
