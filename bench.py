@@ -3,10 +3,12 @@
     python bench.py [--gpus N] [--steps K] [--warmup W] [--workload C] [--block-size BS]
     python bench.py --impl reference ...     # the fp64 CPU oracle, same metric
 
-One step = one decode iteration of the whole hot path over one batch:
-pa_reshape_and_cache of each sequence's newest token, then pa_decode over all
-(sequence, head) pairs (and, for the shared-prefix workload, the copy-on-write
-pa_copy_blocks before them).  The default workload is the LLaMA-13B-shaped
+One step = one decode iteration of the whole hot path over one batch: the
+cache write of each sequence's newest token and the decode over all
+(sequence, head) pairs -- fused into one pa_decode_append launch for fp16
+caches (--unfused: pa_reshape_and_cache, then pa_decode; int8 caches always
+take the two calls) -- and, for the shared-prefix workload, the
+copy-on-write pa_copy_blocks before them.  The default workload is the LLaMA-13B-shaped
 single-layer decode batch (B=32, H=40, D=128, bs=16, context U[256, 2048]).
 
 Under torchrun each rank runs its own batch (a different seed) on its own GPU:
@@ -55,7 +57,7 @@ def _decode_kernel_hash():
     return h.hexdigest()
 
 
-def _recorded_traffic(workload: str):
+def _recorded_traffic(workload: str, launch: str = "pa_decode"):
     """DRAM bytes per decode launch from the committed ncu summary, only if
     it was taken on the current kernel source and this workload."""
     path = os.path.join(ROOT, "profiles", "decode_traffic.json")
@@ -64,7 +66,8 @@ def _recorded_traffic(workload: str):
             rec = json.load(f)
     except Exception:
         return None
-    if rec.get("kernel_sha256") != _decode_kernel_hash() or rec.get("workload") != workload:
+    if (rec.get("kernel_sha256") != _decode_kernel_hash() or rec.get("workload") != workload
+            or rec.get("launch", "pa_decode") != launch):
         return None
     return rec.get("dram_bytes_per_launch")
 
@@ -370,17 +373,24 @@ def run_gpu(args):
         else:
             binding.pa_copy_blocks(kc, vc, pairs, stream=stream)
 
+    fused = not int8 and not args.unfused
+
     def step(ev_pair=None):
         if pairs is not None:
             copy_step()
-        write_step(key, value, slots)
+        if not fused:
+            write_step(key, value, slots)
         if ev_pair is not None:
             ev_pair[0].record(stream)
-        decode_step(out, q, tables, lens)
+        if fused:
+            binding.pa_decode_append(out, q, key, value, kc, vc, slots, tables, lens, mcl,
+                                     wl.scale, ws, stream=stream)
+        else:
+            decode_step(out, q, tables, lens)
         if ev_pair is not None:
             ev_pair[1].record(stream)
 
-    launches_per_step = 2 + ((4 if int8 else 1) if pairs is not None else 0)
+    launches_per_step = (1 if fused else 2) + ((4 if int8 else 1) if pairs is not None else 0)
     with torch.cuda.stream(stream):
         for _ in range(args.warmup):
             step()
@@ -433,8 +443,12 @@ def run_gpu(args):
         d_stage.copy_(h_stage, non_blocking=True)
         if pairs is not None:
             copy_step()
-        write_step(d_key, d_value, d_slots)
-        decode_step(out, d_q, d_tables, d_lens)
+        if fused:
+            binding.pa_decode_append(out, d_q, d_key, d_value, kc, vc, d_slots, d_tables, d_lens,
+                                     mcl, wl.scale, ws, stream=stream)
+        else:
+            write_step(d_key, d_value, d_slots)
+            decode_step(out, d_q, d_tables, d_lens)
         h_out.copy_(out, non_blocking=True)
 
     with torch.cuda.stream(stream):
@@ -462,6 +476,8 @@ def run_gpu(args):
     if wl.alias_block_tables is not None and not int8:
         roof_bytes = accounting.decode_unique_bytes(wl.block_tables, wl.context_lens, h, d,
                                                     wl.block_size)
+    if fused:  # the fused launch also writes each new K and V row to the cache
+        roof_bytes += 2 * b * h * d * 2
     step_bytes = dec_bytes + (b * h * (2 * d * 2 + 2 * (d + 8)) if int8
                               else accounting.cache_write_bytes(b, h, d))
     if pairs is not None:
@@ -481,7 +497,8 @@ def run_gpu(args):
         kv_bytes = dec_bytes
         desc.update({
             "step": ("pa_copy_blocks + " if pairs is not None else "")
-                    + f"pa_reshape_and_cache({b} tokens) + pa_decode",
+                    + (f"pa_decode_append (cache write of {b} tokens fused into the decode)"
+                       if fused else f"pa_reshape_and_cache({b} tokens) + pa_decode"),
             "l2": f"inputs larger than L2: {kv_bytes / 1e9:.2f} GB of K/V read per step "
                   f"vs {L2_BYTES / 2**20:.0f} MiB L2 (no flush)",
             "parallelism": f"dp{world} (independent batches per GPU)",
@@ -507,7 +524,7 @@ def run_gpu(args):
                 "kernel": "paged_decode_kernel" + ("<int8>" if int8 else ""), "bound": "hbm",
                 "achieved": achieved,
                 "peak": peak, "peak_kind": f"{peak_kind} (hbm_gbs)", "unit": "GB/s",
-                "frac": achieved / peak, "traffic": _recorded_traffic(desc["workload"]),
+                "frac": achieved / peak, "traffic": _recorded_traffic(desc["workload"], "pa_decode_append" if fused else "pa_decode"),
                 "algorithmic_bytes_per_launch": roof_bytes,
                 "logical_bytes_per_launch": dec_bytes,
             },
@@ -541,6 +558,8 @@ def main(argv=None):
                     help="KV cache storage (int8 = 8-bit affine codes per row)")
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--unfused", action="store_true",
+                    help="time the cache write and the decode as two launches")
     args = ap.parse_args(argv)
     if args.warmup < 3:
         raise SystemExit("--warmup must be >= 3")

@@ -68,7 +68,7 @@ typedef enum pa_status {
 /* Bits of the device error word (pa_get_last_device_error). */
 #define PA_DEVERR_BLOCK_ID    1u   /* decode: block table entry outside [0, num_blocks) */
 #define PA_DEVERR_CONTEXT_LEN 2u   /* decode: context_lens[b] < 0 or > max_context_len */
-#define PA_DEVERR_SLOT        4u   /* cache write: slot >= num_blocks * block_size */
+#define PA_DEVERR_SLOT        4u   /* cache write: slot >= num_blocks * block_size (decode_append: or not the slot of position L - 1) */
 #define PA_DEVERR_COPY_PAIR   8u   /* copy: src or dst outside [0, num_blocks) */
 #define PA_DEVERR_TIMEOUT     16u  /* decode: a shared-memory transfer did not arrive in ~1 s */
 
@@ -127,6 +127,27 @@ PA_API pa_status pa_decode(void *out, const void *q, const void *k_cache, const 
                     int num_heads, int head_dim, int block_size, int num_blocks,
                     float scale, void *workspace, size_t workspace_bytes,
                     pa_stream_t stream);
+
+/*
+ * pa_reshape_and_cache of each sequence's newest token followed by pa_decode,
+ * in ONE launch (the cache write of a decode step, polomodov.tech "vLLM and
+ * PagedAttention" slide 11, fused into the attention that reads it).  For a
+ * sequence b with slot_mapping[b] >= 0, position context_lens[b] - 1 is its
+ * new token: key[b] / value[b] ([num_seqs, H, D] fp16, device) are written
+ * to the cache at slot_mapping[b], which must be the slot the block table
+ * gives that position (else PA_DEVERR_SLOT; a slot outside the pool is not
+ * written), and the attention uses them for that position.  slot_mapping[b]
+ * < 0: no new token, plain decode of the cached context.  Outputs and cache
+ * contents are those of the two separate calls.  fp16 caches only; other
+ * arguments, layouts and errors as pa_decode.
+ */
+PA_API pa_status pa_decode_append(void *out, const void *q, const void *key, const void *value,
+                                  void *k_cache, void *v_cache, const int64_t *slot_mapping,
+                                  const int32_t *block_tables, int max_blocks_per_seq,
+                                  const int32_t *context_lens, int max_context_len, int num_seqs,
+                                  int num_heads, int head_dim, int block_size, int num_blocks,
+                                  float scale, void *workspace, size_t workspace_bytes,
+                                  pa_stream_t stream);
 
 /*
  * Copy-on-write block copy (comfyai.app 6.4.2-6.4.3; polomodov.tech slide

@@ -34,7 +34,7 @@ EXPORTED = ("pa_reshape_and_cache", "pa_decode_workspace_size", "pa_decode_works
             "pa_bm_block_tables", "pa_reshape_and_cache_int8", "pa_decode_int8",
             "pa_copy_blocks_raw", "pa_prefill", "pa_swap_blocks", "pa_bm_create_with_swap",
             "pa_bm_num_free_cpu", "pa_bm_cpu_refcount", "pa_bm_is_swapped", "pa_bm_swap_out",
-            "pa_bm_swap_in")
+            "pa_bm_swap_in", "pa_decode_append")
 
 _lock = threading.Lock()
 _lib = None
@@ -99,6 +99,9 @@ def load(path: str | None = None):
         lib.pa_decode_int8.restype = i32
         lib.pa_copy_blocks_raw.argtypes = [vp, sz, vp, i32, i32, vp]
         lib.pa_copy_blocks_raw.restype = i32
+        lib.pa_decode_append.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, i32, vp, i32, i32, i32, i32,
+                                         i32, i32, ctypes.c_float, vp, sz, vp]
+        lib.pa_decode_append.restype = i32
         lib.pa_swap_blocks.argtypes = [vp, vp, sz, vp, i32, i32, i32, vp]
         lib.pa_swap_blocks.restype = i32
         lib.pa_bm_create_with_swap.argtypes = [i32, i32, i32]
@@ -198,6 +201,28 @@ def pa_decode(out, q, k_cache, v_cache, block_tables, context_lens, max_context_
                             _ptr(workspace), workspace.numel() * workspace.element_size(),
                             _stream(stream)),
            "pa_decode")
+
+
+def pa_decode_append(out, q, key, value, k_cache, v_cache, slot_mapping, block_tables,
+                     context_lens, max_context_len, scale, workspace, stream=None):
+    """The decode step's cache write and the paged decode in one launch: for
+    each sequence b with slot_mapping[b] >= 0, key[b] / value[b] are its new
+    token (position context_lens[b] - 1), written to that slot and used by
+    the attention."""
+    b, h, d = q.shape
+    nb, hk, bs, dk = k_cache.shape
+    assert q.dtype == out.dtype == key.dtype == value.dtype == k_cache.dtype == torch.float16
+    assert out.shape == q.shape == key.shape == value.shape and (hk, dk) == (h, d)
+    assert v_cache.shape == k_cache.shape
+    assert slot_mapping.dtype == torch.int64 and slot_mapping.numel() == b
+    assert block_tables.dtype == torch.int32 and block_tables.dim() == 2
+    assert context_lens.dtype == torch.int32 and context_lens.numel() == b
+    _check(load().pa_decode_append(_ptr(out), _ptr(q), _ptr(key), _ptr(value), _ptr(k_cache),
+                                   _ptr(v_cache), _ptr(slot_mapping), _ptr(block_tables),
+                                   block_tables.shape[1], _ptr(context_lens), int(max_context_len),
+                                   b, h, d, bs, nb, float(scale), _ptr(workspace),
+                                   workspace.numel() * workspace.element_size(), _stream(stream)),
+           "pa_decode_append")
 
 
 def pa_decode_no_alloc(out, q, k_cache, v_cache, block_tables, context_lens, max_context_len,

@@ -141,7 +141,9 @@ pa_status decode_common(void *out, const void *q, const void *k_cache, const voi
                         const int32_t *block_tables, int max_blocks_per_seq,
                         const int32_t *context_lens, int max_context_len, int num_seqs,
                         int num_heads, int head_dim, int block_size, int num_blocks, float scale,
-                        void *workspace, size_t workspace_bytes, pa_stream_t stream)
+                        void *workspace, size_t workspace_bytes, pa_stream_t stream,
+                        const void *new_k = nullptr, const void *new_v = nullptr,
+                        const int64_t *new_slots = nullptr)
 {
     if (num_seqs < 0 || num_heads <= 0 || num_blocks <= 0 || max_context_len < 0 ||
         max_blocks_per_seq < 0)
@@ -186,6 +188,9 @@ pa_status decode_common(void *out, const void *q, const void *k_cache, const voi
     p.block_size = block_size;
     p.num_blocks = num_blocks;
     p.qk_scale_log2 = float(double(scale) * 1.4426950408889634);  // scale * log2(e)
+    p.new_k = static_cast<const __half *>(new_k);
+    p.new_v = static_cast<const __half *>(new_v);
+    p.new_slots = new_slots;
 
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
     if (int8) {
@@ -211,6 +216,22 @@ pa_status pa_decode(void *out, const void *q, const void *k_cache, const void *v
     return decode_common(out, q, k_cache, v_cache, nullptr, nullptr, false, block_tables,
                          max_blocks_per_seq, context_lens, max_context_len, num_seqs, num_heads,
                          head_dim, block_size, num_blocks, scale, workspace, workspace_bytes, stream);
+}
+
+pa_status pa_decode_append(void *out, const void *q, const void *key, const void *value,
+                           void *k_cache, void *v_cache, const int64_t *slot_mapping,
+                           const int32_t *block_tables, int max_blocks_per_seq,
+                           const int32_t *context_lens, int max_context_len, int num_seqs,
+                           int num_heads, int head_dim, int block_size, int num_blocks, float scale,
+                           void *workspace, size_t workspace_bytes, pa_stream_t stream)
+{
+    if (num_seqs > 0 && (!key || !value || !slot_mapping || !aligned16(key) || !aligned16(value) ||
+                         (reinterpret_cast<uintptr_t>(slot_mapping) & 7u)))
+        return PA_ERR_INVALID_ARG;
+    return decode_common(out, q, k_cache, v_cache, nullptr, nullptr, false, block_tables,
+                         max_blocks_per_seq, context_lens, max_context_len, num_seqs, num_heads,
+                         head_dim, block_size, num_blocks, scale, workspace, workspace_bytes, stream,
+                         key, value, slot_mapping);
 }
 
 pa_status pa_decode_int8(void *out, const void *q, const void *k_codes, const void *v_codes,

@@ -60,6 +60,7 @@ __device__ __forceinline__ void raise_device_error(unsigned int bits)
 
 constexpr unsigned kErrBlockId = 1u << 0;
 constexpr unsigned kErrContextLen = 1u << 1;
+constexpr unsigned kErrSlot = 1u << 2;
 constexpr unsigned kErrTimeout = 1u << 4;
 
 constexpr int kTileBytes = 4096;  // one fp16 K (or V) tile in shared memory
@@ -84,6 +85,13 @@ struct DecodeParams {
     int block_size;
     int num_blocks;
     float qk_scale_log2; // softmax scale * log2(e)
+    // Fused append (fp16 cache only; new_slots == nullptr: plain decode).  For
+    // a sequence b with new_slots[b] >= 0, position context_lens[b] - 1 is a
+    // new token: its K / V rows come from new_k / new_v [B, H, D] (not from
+    // the cache) and are also written to the cache at slot new_slots[b].
+    const __half *new_k;
+    const __half *new_v;
+    const int64_t *new_slots;
 };
 
 constexpr int ilog2(int x)
@@ -397,6 +405,12 @@ __device__ __forceinline__ void issue_tile(const DecodeParams &p, const TileCurs
     meta->k = cur.k;
 
     const uint32_t dst = smem_u32(stage_buf);
+    // the last tile of a unit whose sequence appends a token: its last row
+    // comes from the new-token input instead (append_new_row)
+    int nf = nv;
+    if constexpr (!kInt8)
+        if (p.new_slots && cur.i == cur.nt - 1 && p.new_slots[cur.b] >= 0)
+            nf = nv - 1;
     // an id outside the pool is recorded and its rows are not fetched
     bool ok[Sh::kMaxIds];
 #pragma unroll
@@ -405,17 +419,17 @@ __device__ __forceinline__ void issue_tile(const DecodeParams &p, const TileCurs
     uint32_t total = with_q ? uint32_t(D * 2) : 0u;
     bool bad = false;
     if (bs >= Sh::kTokens) {
-        if (ok[0])
-            total += rows_tx_bytes<D, kInt8>(nv);
-        else
+        if (!ok[0])
             bad = true;
+        else if (nf > 0)
+            total += rows_tx_bytes<D, kInt8>(nf);
     } else {
 #pragma unroll
         for (int s = 0; s < Sh::kMaxIds; ++s) {
-            if (s * bs >= nv)
+            if (s * bs >= nf)
                 break;
             if (ok[s])
-                total += rows_tx_bytes<D, kInt8>(min(bs, nv - s * bs));
+                total += rows_tx_bytes<D, kInt8>(min(bs, nf - s * bs));
             else
                 bad = true;
         }
@@ -426,20 +440,64 @@ __device__ __forceinline__ void issue_tile(const DecodeParams &p, const TileCurs
     if (with_q)
         bulk_copy_g2s(dst + Sm::kOffQ, p.q + (size_t(cur.b) * p.num_heads + cur.h) * D, D * 2, bar);
     if (bs >= Sh::kTokens) {
-        if (ok[0])
+        if (ok[0] && nf > 0)
             copy_rows<D, kInt8, Sm>(p, (size_t(ids[0]) * p.num_heads + cur.h) * bs + size_t(t0 % bs),
-                                    nv, dst, 0, bar, stream_policy);
+                                    nf, dst, 0, bar, stream_policy);
     } else {
 #pragma unroll
         for (int s = 0; s < Sh::kMaxIds; ++s) {
-            if (s * bs >= nv)
+            if (s * bs >= nf)
                 break;
             if (!ok[s])
                 continue;
             copy_rows<D, kInt8, Sm>(p, (size_t(ids[s]) * p.num_heads + cur.h) * bs,
-                                    min(bs, nv - s * bs), dst, uint32_t(s * bs), bar, stream_policy);
+                                    min(bs, nf - s * bs), dst, uint32_t(s * bs), bar, stream_policy);
         }
     }
+}
+
+// Fused append, whole warp, right after the tile under the cursor was issued:
+// if it is the last tile of its unit and the sequence appends a token, put
+// the new K / V rows (position len - 1) into the stage from the new-token
+// input and write them to the cache slot (polomodov.tech "vLLM and
+// PagedAttention", slide 11: the new token goes into the next free slot).
+// The slot must be the one the block table gives that position; otherwise
+// PA_DEVERR_SLOT is recorded (and a slot outside the pool is not written).
+template <int D, class Sm>
+__device__ __forceinline__ void append_new_row(const DecodeParams &p, const TileCursor &cur,
+                                               unsigned char *stage_buf, int lane)
+{
+    using Sh = DecodeShape<D, false>;
+    if (cur.i != cur.nt - 1)
+        return;
+    const int64_t slot = p.new_slots[cur.b];
+    if (slot < 0)
+        return;
+    constexpr int kChunks = D * 2 / 16;  // 16-byte chunks of one row
+    const int bs = p.block_size;
+    const int pos = cur.len - 1;
+    const int r = pos - cur.i * Sh::kTokens;  // the row's place in the stage
+    const bool in_pool = slot < int64_t(p.num_blocks) * bs;
+    if (lane == 0) {
+        const int id = p.block_tables[size_t(cur.b) * p.max_blocks_per_seq + pos / bs];
+        if (!in_pool || slot != int64_t(id) * bs + pos % bs)
+            raise_device_error(kErrSlot);
+    }
+    if (lane < 2 * kChunks) {
+        const bool is_v = lane >= kChunks;
+        const int c = lane % kChunks;
+        const size_t src_row = size_t(cur.b) * p.num_heads + cur.h;
+        const uint4 val = __ldg(reinterpret_cast<const uint4 *>((is_v ? p.new_v : p.new_k) + src_row * D) + c);
+        *reinterpret_cast<uint4 *>(stage_buf + (is_v ? Sm::kOffV : 0u) + uint32_t(r) * Sh::kRowBytes +
+                                   uint32_t(c) * 16u) = val;
+        if (in_pool) {
+            const size_t row = (size_t(slot / bs) * p.num_heads + cur.h) * bs + size_t(slot % bs);
+            uint4 *cache = reinterpret_cast<uint4 *>(const_cast<void *>(is_v ? p.v_cache : p.k_cache));
+            cache[row * kChunks + c] = val;
+        }
+    }
+    fence_proxy_async_smem();  // before a later bulk copy overwrites the stage
+    __syncwarp();
 }
 
 // Merge the partial results of a (sequence, head) whose tiles were split
@@ -661,6 +719,9 @@ __global__ void __launch_bounds__(NW * 32) paged_decode_kernel(const DecodeParam
                 issue_tile<D, kInt8, Sm>(p, cs, ids_s, cs.i == 0 || cs.k == lo,
                                          my_buf + size_t(s) * Sm::kStageBytes, my_bar + 8 * s,
                                          my_meta + s, policy);
+            if constexpr (!kInt8)
+                if (p.new_slots)
+                    append_new_row<D, Sm>(p, cs, my_buf + size_t(s) * Sm::kStageBytes, lane);
             if (s == first - 1)
                 prod = cs;
         }
@@ -746,6 +807,9 @@ __global__ void __launch_bounds__(NW * 32) paged_decode_kernel(const DecodeParam
                                          my_buf + size_t(stage) * Sm::kStageBytes,
                                          my_bar + 8 * stage, my_meta + stage, policy);
             }
+            if constexpr (!kInt8)
+                if (p.new_slots)
+                    append_new_row<D, Sm>(p, prod, my_buf + size_t(stage) * Sm::kStageBytes, lane);
             if (++issued < ntiles) {
                 prod.template advance<T>(p);
                 load_tile_ids<Sh>(p, prod, ids);
