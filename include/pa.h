@@ -283,6 +283,42 @@ PA_API pa_status pa_prefill(void *out, const void *q, const void *k_cache, const
                             int num_seqs, int num_heads, int head_dim, int block_size,
                             int num_blocks, float scale, pa_stream_t stream);
 
+/*
+ * Decode of groups of sequences that share the first blocks of their context
+ * -- parallel samples of one prompt, beam candidates (comfyai.app "6.4
+ * PagedAttention", 6.4.2; polomodov.tech "vLLM and PagedAttention", slides
+ * 13-14: candidates share a prefix of blocks like processes after fork).
+ * Same result as pa_decode over the same arguments, but each shared prefix
+ * is read once per (group, head): its scores are a small matrix product on
+ * the tensor cores (the members' queries against the prefix), each member's
+ * own tail goes through the decode kernel, and the two parts are merged by
+ * their softmax normalisers.  Three more launches than pa_decode, so it pays
+ * when prefixes are long against the tails.
+ *   group_start [num_groups + 1] int32 (device): group g = sequences
+ *     group_start[g] .. group_start[g+1] - 1; group_start[0] = 0 and
+ *     group_start[num_groups] = num_seqs, nondecreasing.
+ *   prefix_lens [num_groups] int32 (device): tokens shared by group g, a
+ *     multiple of block_size, at most every member's context length; the
+ *     members' block tables must agree on those blocks (0 = nothing shared).
+ *   max_group_size: host bound on group sizes (sizes the grid).
+ *   workspace: pa_decode_grouped_workspace_size(num_seqs, num_heads,
+ *     head_dim, max_blocks_per_seq) bytes, 16-byte aligned, zeroed once with
+ *     pa_decode_workspace_init before first use (like pa_decode's).
+ * head_dim must be 128, scale > 0.  A prefix that breaks these rules is
+ * recorded (PA_DEVERR_CONTEXT_LEN) and that group decodes with no shared
+ * prefix; group bounds outside the batch are recorded and skipped.
+ */
+PA_API size_t pa_decode_grouped_workspace_size(int num_seqs, int num_heads, int head_dim,
+                                               int max_blocks_per_seq);
+PA_API pa_status pa_decode_grouped(void *out, const void *q, const void *k_cache,
+                                   const void *v_cache, const int32_t *block_tables,
+                                   int max_blocks_per_seq, const int32_t *context_lens,
+                                   int max_context_len, const int32_t *group_start,
+                                   const int32_t *prefix_lens, int num_groups, int max_group_size,
+                                   int num_seqs, int num_heads, int head_dim, int block_size,
+                                   int num_blocks, float scale, void *workspace,
+                                   size_t workspace_bytes, pa_stream_t stream);
+
 /* Static description of a status code. */
 PA_API const char *pa_status_string(pa_status status);
 

@@ -34,7 +34,8 @@ EXPORTED = ("pa_reshape_and_cache", "pa_decode_workspace_size", "pa_decode_works
             "pa_bm_block_tables", "pa_reshape_and_cache_int8", "pa_decode_int8",
             "pa_copy_blocks_raw", "pa_prefill", "pa_swap_blocks", "pa_bm_create_with_swap",
             "pa_bm_num_free_cpu", "pa_bm_cpu_refcount", "pa_bm_is_swapped", "pa_bm_swap_out",
-            "pa_bm_swap_in", "pa_decode_append")
+            "pa_bm_swap_in", "pa_decode_append", "pa_decode_grouped_workspace_size",
+            "pa_decode_grouped")
 
 _lock = threading.Lock()
 _lib = None
@@ -99,6 +100,11 @@ def load(path: str | None = None):
         lib.pa_decode_int8.restype = i32
         lib.pa_copy_blocks_raw.argtypes = [vp, sz, vp, i32, i32, vp]
         lib.pa_copy_blocks_raw.restype = i32
+        lib.pa_decode_grouped_workspace_size.argtypes = [i32, i32, i32, i32]
+        lib.pa_decode_grouped_workspace_size.restype = sz
+        lib.pa_decode_grouped.argtypes = [vp, vp, vp, vp, vp, i32, vp, i32, vp, vp, i32, i32, i32,
+                                          i32, i32, i32, i32, ctypes.c_float, vp, sz, vp]
+        lib.pa_decode_grouped.restype = i32
         lib.pa_decode_append.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, i32, vp, i32, i32, i32, i32,
                                          i32, i32, ctypes.c_float, vp, sz, vp]
         lib.pa_decode_append.restype = i32
@@ -223,6 +229,34 @@ def pa_decode_append(out, q, key, value, k_cache, v_cache, slot_mapping, block_t
                                    b, h, d, bs, nb, float(scale), _ptr(workspace),
                                    workspace.numel() * workspace.element_size(), _stream(stream)),
            "pa_decode_append")
+
+
+def new_grouped_workspace(num_seqs, num_heads, head_dim, max_blocks_per_seq, device="cuda"):
+    """Zeroed workspace for pa_decode_grouped."""
+    n = load().pa_decode_grouped_workspace_size(num_seqs, num_heads, head_dim, max_blocks_per_seq)
+    return torch.zeros(max(int(n), 16), dtype=torch.uint8, device=device)
+
+
+def pa_decode_grouped(out, q, k_cache, v_cache, block_tables, context_lens, max_context_len,
+                      group_start, prefix_lens, max_group_size, scale, workspace, stream=None):
+    """Decode of sequence groups sharing a block prefix: the prefix read once
+    per (group, head) on the tensor cores, tails by the decode kernel, merged.
+    Same result as pa_decode."""
+    b, h, d = q.shape
+    nb, hk, bs, dk = k_cache.shape
+    assert q.dtype == out.dtype == k_cache.dtype == v_cache.dtype == torch.float16
+    assert out.shape == q.shape and (hk, dk) == (h, d) and v_cache.shape == k_cache.shape
+    assert block_tables.dtype == context_lens.dtype == group_start.dtype == torch.int32
+    assert prefix_lens.dtype == torch.int32
+    g = prefix_lens.numel()
+    assert group_start.numel() == g + 1
+    _check(load().pa_decode_grouped(_ptr(out), _ptr(q), _ptr(k_cache), _ptr(v_cache),
+                                    _ptr(block_tables), block_tables.shape[1], _ptr(context_lens),
+                                    int(max_context_len), _ptr(group_start), _ptr(prefix_lens), g,
+                                    int(max_group_size), b, h, d, bs, nb, float(scale),
+                                    _ptr(workspace), workspace.numel() * workspace.element_size(),
+                                    _stream(stream)),
+           "pa_decode_grouped")
 
 
 def pa_decode_no_alloc(out, q, k_cache, v_cache, block_tables, context_lens, max_context_len,

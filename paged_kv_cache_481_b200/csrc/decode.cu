@@ -143,7 +143,7 @@ pa_status decode_common(void *out, const void *q, const void *k_cache, const voi
                         int num_heads, int head_dim, int block_size, int num_blocks, float scale,
                         void *workspace, size_t workspace_bytes, pa_stream_t stream,
                         const void *new_k = nullptr, const void *new_v = nullptr,
-                        const int64_t *new_slots = nullptr)
+                        const int64_t *new_slots = nullptr, float *lse = nullptr)
 {
     if (num_seqs < 0 || num_heads <= 0 || num_blocks <= 0 || max_context_len < 0 ||
         max_blocks_per_seq < 0)
@@ -191,6 +191,7 @@ pa_status decode_common(void *out, const void *q, const void *k_cache, const voi
     p.new_k = static_cast<const __half *>(new_k);
     p.new_v = static_cast<const __half *>(new_v);
     p.new_slots = new_slots;
+    p.lse = lse;
 
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
     if (int8) {
@@ -315,4 +316,17 @@ extern "C" pa_status pa_decode_no_alloc(void *out, const void *q, const void *k_
     return pa_decode(out, q, k_cache, v_cache, block_tables, max_blocks_per_seq, context_lens,
                      max_context_len, num_seqs, num_heads, head_dim, block_size, num_blocks, scale,
                      scratch, kNoAllocScratchBytes, stream);
+}
+
+pa_status pa_host::decode_with_lse(void *out, const void *q, const void *k_cache,
+                                   const void *v_cache, const int32_t *block_tables,
+                                   int max_blocks_per_seq, const int32_t *context_lens,
+                                   int max_context_len, int num_seqs, int num_heads, int head_dim,
+                                   int block_size, int num_blocks, float scale, void *workspace,
+                                   size_t workspace_bytes, float *lse, pa_stream_t stream)
+{
+    return decode_common(out, q, k_cache, v_cache, nullptr, nullptr, false, block_tables,
+                         max_blocks_per_seq, context_lens, max_context_len, num_seqs, num_heads,
+                         head_dim, block_size, num_blocks, scale, workspace, workspace_bytes, stream,
+                         nullptr, nullptr, nullptr, lse);
 }

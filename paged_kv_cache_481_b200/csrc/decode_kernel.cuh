@@ -92,6 +92,9 @@ struct DecodeParams {
     const __half *new_k;
     const __half *new_v;
     const int64_t *new_slots;
+    // optional [B, H]: log2 of each unit's softmax denominator relative to
+    // 2^0, i.e. max + log2(sum) in base-2 units (to merge with other parts)
+    float *lse;
 };
 
 constexpr int ilog2(int x)
@@ -539,6 +542,8 @@ __device__ __forceinline__ void merge_partials(const DecodeParams &p, uint4 *out
 #pragma unroll
     for (int k = 0; k < kDims / 8; ++k)
         out_row[(kDims / 8) * c + k] = reinterpret_cast<const uint4 *>(o)[k];
+    if (p.lse && c == 0)
+        p.lse[(reinterpret_cast<const __half *>(out_row) - p.out) / D] = gmax + log2f(den);
 }
 
 template <int D, bool kInt8, int NW, int S>
@@ -848,6 +853,8 @@ __global__ void __launch_bounds__(NW * 32) paged_decode_kernel(const DecodeParam
                 for (int k = 0; k < kDims / 8; ++k)
                     out_row[(kDims / 8) * c + k] = reinterpret_cast<const uint4 *>(o)[k];
             }
+            if (p.lse && lane == 0)
+                p.lse[unit] = m + log2f(l);
             continue;
         }
         const long long u_start = mt.k - mt.i;      // global index of the unit's tile 0

@@ -5,6 +5,8 @@
 
 #include <cuda_runtime.h>
 
+#include "../../include/pa.h"
+
 #include <cstddef>
 #include <cstdint>
 
@@ -13,6 +15,15 @@ namespace pa_host {
 // Device address of the library's device error word (the PA_DEVERR_* bits)
 // on the current device; nullptr if it cannot be looked up.
 unsigned int *device_error_word();
+
+// pa_decode that also writes each (sequence, head)'s softmax log-normaliser
+// lse = max + log2(sum) in base-2 units ([num_seqs, num_heads] fp32), so the
+// result can be merged with attention over other parts of the context.
+pa_status decode_with_lse(void *out, const void *q, const void *k_cache, const void *v_cache,
+                          const int32_t *block_tables, int max_blocks_per_seq,
+                          const int32_t *context_lens, int max_context_len, int num_seqs,
+                          int num_heads, int head_dim, int block_size, int num_blocks, float scale,
+                          void *workspace, size_t workspace_bytes, float *lse, pa_stream_t stream);
 
 } // namespace pa_host
 

@@ -2,6 +2,7 @@
 
     python -m paged_kv_cache_481_b200.measure prefill [--iters N]
     python -m paged_kv_cache_481_b200.measure swap [--iters N]
+    python -m paged_kv_cache_481_b200.measure grouped [--iters N]
 
 Each prints one JSON line per case.  Times are CUDA events on the launching
 stream around N back-to-back calls after warm-up; inputs are synthetic
@@ -13,6 +14,11 @@ paged cache.  Algorithmic FLOPs count only the unmasked scores: a new token
 at position p does 2*D*(p+1) multiply-adds for q.K and the same for P.V per
 head, i.e. 4*D*(p+1) FLOPs.  The roofline peak is the measured dense bf16
 tensor rate (fp16 runs at the same rate on this architecture).
+
+grouped: decode of the shared-prefix batch (8 groups of 8 sequences, a
+1024-token prefix, private tails of 1-256 tokens, H=40, D=128, bs=16) with
+pa_decode and with pa_decode_grouped (the prefix read once per group and
+head); bytes = what DRAM must deliver, each physical row once.
 
 swap: pa_swap_blocks between the device pool and a page-locked host pool, in
 both directions, against a plain copy of the same number of contiguous bytes
@@ -120,9 +126,46 @@ def measure_swap(iters: int, num_blocks: int = 1024, seed: int = 0):
     return lines
 
 
+def measure_grouped(iters: int):
+    from . import accounting, workloads
+    wl = workloads.make_shared_prefix(device="cuda")
+    h, d, bs = wl.num_heads, wl.head_dim, wl.block_size
+    dev = torch.device("cuda")
+    kc, vc = wl.k_cache, wl.v_cache
+    binding.pa_reshape_and_cache(wl.new_key, wl.new_value, kc, vc,
+                                 torch.from_numpy(wl.slot_mapping).to(dev))
+    binding.pa_copy_blocks(kc, vc, torch.from_numpy(wl.copy_pairs).to(dev))
+    q = wl.q
+    lens = torch.from_numpy(wl.context_lens).to(dev)
+    out = torch.empty_like(q)
+    lines = []
+    for name, tables, prefix in (("aliased prefix (64 shared blocks)", wl.alias_block_tables, 1024),
+                                 ("copy-on-write prefix (63 shared blocks)", wl.block_tables, 1008)):
+        t = torch.from_numpy(np.ascontiguousarray(tables)).to(dev)
+        nbytes = accounting.decode_unique_bytes(tables, wl.context_lens, h, d, bs)
+        ws = binding.new_workspace(wl.num_seqs, h, d, wl.max_context_len)
+        ms_plain = _time_ms(lambda: binding.pa_decode(out, q, kc, vc, t, lens, wl.max_context_len,
+                                                      wl.scale, ws), iters)
+        gws = binding.new_grouped_workspace(wl.num_seqs, h, d, tables.shape[1])
+        gs = torch.arange(0, wl.num_seqs + 1, 8, dtype=torch.int32, device=dev)
+        pl = torch.full((wl.num_seqs // 8,), prefix, dtype=torch.int32, device=dev)
+        ms_grp = _time_ms(lambda: binding.pa_decode_grouped(out, q, kc, vc, t, lens,
+                                                            wl.max_context_len, gs, pl, 8,
+                                                            wl.scale, gws), iters)
+        line = {"what": "pa_decode_grouped", "case": name, "num_seqs": wl.num_seqs,
+                "groups": wl.num_seqs // 8, "prefix_len": prefix, "num_heads": h,
+                "unique_bytes": nbytes, "plain_us": ms_plain * 1e3, "grouped_us": ms_grp * 1e3,
+                "plain_gbs": nbytes / (ms_plain * 1e-3) / 1e9,
+                "grouped_gbs": nbytes / (ms_grp * 1e-3) / 1e9, "speedup": ms_plain / ms_grp,
+                "device_error": binding.pa_get_last_device_error()}
+        print(json.dumps(line), flush=True)
+        lines.append(line)
+    return lines
+
+
 def main(argv=None):
     ap = argparse.ArgumentParser(description=__doc__.split("\n\n")[0])
-    ap.add_argument("what", choices=["prefill", "swap"])
+    ap.add_argument("what", choices=["prefill", "swap", "grouped"])
     ap.add_argument("--iters", type=int, default=10)
     ap.add_argument("--block-size", type=int, default=16)
     ap.add_argument("--case", default=None, help="only the prefill case of this name")
@@ -131,6 +174,8 @@ def main(argv=None):
     binding.load()
     if args.what == "prefill":
         measure_prefill(args.iters, args.block_size, case=args.case)
+    elif args.what == "grouped":
+        measure_grouped(args.iters)
     else:
         measure_swap(args.iters)
 

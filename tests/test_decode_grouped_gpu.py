@@ -1,0 +1,122 @@
+"""pa_decode_grouped (shared prefix once per group and head on the tensor
+cores, tails by the decode kernel, merged by their softmax normalisers)
+against the oracle's plain paged decode of every member over its full block
+table -- the same mathematics (comfyai.app "6.4 PagedAttention", 6.4.2;
+polomodov.tech slides 13-14)."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from paged_kv_cache_481_b200 import binding, build, workloads
+
+from gpu_helpers import ATOL, max_abs_err, to_dev
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _lib():
+    build.build()
+    binding.load()
+    torch.cuda.init()
+
+
+def _groups(seed, sizes, prefix_blocks, max_tail, bs, h=4, d=128):
+    """Groups of sequences sharing prefix blocks, each member with a private
+    tail (0..max_tail tokens); random pool placement and values."""
+    rng = np.random.default_rng(seed)
+    tails = [[int(rng.integers(0, max_tail + 1)) for _ in range(n)] for n in sizes]
+    need = sum(prefix_blocks) + sum(-(-t // bs) for ts in tails for t in ts) + 4
+    nb = need * 2
+    perm = rng.permutation(nb).astype(np.int32)
+    off = 0
+    lens, rows = [], []
+    for pbk, ts in zip(prefix_blocks, tails):
+        shared = perm[off:off + pbk]
+        off += pbk
+        for t in ts:
+            own = perm[off:off + -(-t // bs)]
+            off += len(own)
+            rows.append(np.concatenate([shared, own]))
+            lens.append(pbk * bs + t)
+    mb = max(1, max(len(r) for r in rows))
+    tables = np.full((len(rows), mb), -1, np.int32)
+    for i, r in enumerate(rows):
+        tables[i, :len(r)] = r
+    g = torch.Generator().manual_seed(seed)
+    kc = torch.randn((nb, h, bs, d), generator=g).half()
+    vc = torch.randn((nb, h, bs, d), generator=g).half()
+    q = torch.randn((len(rows), h, d), generator=g).half()
+    gs = np.concatenate([[0], np.cumsum(sizes)]).astype(np.int32)
+    pl = (np.asarray(prefix_blocks) * bs).astype(np.int32)
+    return dict(kc=kc, vc=vc, q=q, tables=tables, lens=np.asarray(lens, np.int32), gs=gs, pl=pl,
+                scale=d ** -0.5, max_group=max(sizes))
+
+
+def _run(c, prefix_lens=None):
+    dev = "cuda"
+    b, h, d = c["q"].shape
+    out = torch.full((b, h, d), float("nan"), dtype=torch.float16, device=dev)
+    ws = binding.new_grouped_workspace(b, h, d, c["tables"].shape[1])
+    pl = c["pl"] if prefix_lens is None else prefix_lens
+    binding.pa_decode_grouped(out, c["q"].to(dev), c["kc"].to(dev), c["vc"].to(dev),
+                              torch.from_numpy(c["tables"]).to(dev), torch.from_numpy(c["lens"]).to(dev),
+                              int(c["lens"].max()), torch.from_numpy(c["gs"]).to(dev),
+                              torch.from_numpy(np.ascontiguousarray(pl, np.int32)).to(dev),
+                              c["max_group"], c["scale"], ws)
+    torch.cuda.synchronize()
+    ref = oracle.paged_decode(c["q"].numpy(), c["kc"].numpy(), c["vc"].numpy(), c["tables"],
+                              c["lens"], c["scale"])
+    return out, ref
+
+
+@pytest.mark.parametrize("seed,sizes,prefix_blocks,max_tail,bs", [
+    (501, [3, 1, 5, 2], [4, 0, 2, 7], 40, 16),        # a group with nothing shared
+    (502, [8, 8], [64, 30], 256, 16),                 # long prefixes, several context tiles
+    (503, [6, 4, 9], [9, 20, 3], 0, 16),              # no tails at all: prefix is everything
+    (504, [4, 4], [33, 17], 100, 8),
+    (505, [2, 3], [5, 3], 300, 64),
+    (506, [130, 3], [4, 2], 20, 16),                  # a group larger than one query tile
+])
+def test_grouped_equals_plain_decode(seed, sizes, prefix_blocks, max_tail, bs):
+    c = _groups(seed, sizes, prefix_blocks, max_tail, bs)
+    out, ref = _run(c)
+    assert not torch.isnan(out).any()
+    assert max_abs_err(out, ref) <= ATOL
+    assert binding.pa_get_last_device_error() == 0
+
+
+def test_grouped_prefix_breaking_the_rules_falls_back():
+    c = _groups(507, [3, 2], [4, 3], 30, 16)
+    bad = c["pl"].copy()
+    bad[0] += 5                                       # not a whole number of blocks
+    out, ref = _run(c, bad)
+    assert max_abs_err(out, ref) <= ATOL              # that group decodes without a shared prefix
+    assert binding.pa_get_last_device_error() == binding.PA_DEVERR_CONTEXT_LEN
+
+
+def test_grouped_on_the_shared_prefix_workload():
+    """The shared-prefix workload (8 groups of 8, prefix 1024 tokens), smaller
+    heads: through the aliased tables (all 64 prefix blocks shared) and the
+    copy-on-write tables (the prefix's last block copied per member)."""
+    wl = workloads.make_shared_prefix(device="cuda", num_heads=8)
+    t = to_dev(wl)
+    binding.pa_reshape_and_cache(t["new_key"], t["new_value"], t["k_cache"], t["v_cache"], t["slots"])
+    binding.pa_copy_blocks(t["k_cache"], t["v_cache"], torch.from_numpy(wl.copy_pairs).cuda())
+    okc, ovc = oracle.reshape_and_cache(wl.new_key.cpu().numpy(), wl.new_value.cpu().numpy(),
+                                        wl.k_cache.cpu().numpy(), wl.v_cache.cpu().numpy(),
+                                        wl.slot_mapping, wl.block_size)
+    okc, ovc = oracle.copy_blocks(okc, ovc, wl.copy_pairs)
+    gs = torch.arange(0, 65, 8, dtype=torch.int32, device="cuda")
+    for tables, prefix in ((wl.alias_block_tables, 1024), (wl.block_tables, 1008)):
+        out = torch.empty_like(t["q"])
+        ws = binding.new_grouped_workspace(wl.num_seqs, wl.num_heads, wl.head_dim, tables.shape[1])
+        binding.pa_decode_grouped(out, t["q"], t["k_cache"], t["v_cache"],
+                                  torch.from_numpy(np.ascontiguousarray(tables)).cuda(), t["lens"],
+                                  wl.max_context_len, gs,
+                                  torch.full((8,), prefix, dtype=torch.int32, device="cuda"), 8,
+                                  wl.scale, ws)
+        ref = oracle.paged_decode(wl.q.cpu().numpy(), okc, ovc, tables, wl.context_lens, wl.scale)
+        assert max_abs_err(out, ref) <= ATOL
+    assert binding.pa_get_last_device_error() == 0
