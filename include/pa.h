@@ -304,9 +304,11 @@ PA_API pa_status pa_prefill(void *out, const void *q, const void *k_cache, const
  *   workspace: pa_decode_grouped_workspace_size(num_seqs, num_heads,
  *     head_dim, max_blocks_per_seq) bytes, 16-byte aligned, zeroed once with
  *     pa_decode_workspace_init before first use (like pa_decode's).
- * head_dim must be 128, scale > 0.  A prefix that breaks these rules is
- * recorded (PA_DEVERR_CONTEXT_LEN) and that group decodes with no shared
- * prefix; group bounds outside the batch are recorded and skipped.
+ * head_dim must be 128, scale > 0, max_group_size <= 65535.  A prefix that
+ * breaks these rules for a member is recorded (PA_DEVERR_CONTEXT_LEN, possibly
+ * with PA_DEVERR_BLOCK_ID from reading past its blocks) and that member
+ * decodes its whole context as its tail; group bounds outside the batch are
+ * recorded and skipped.
  */
 PA_API size_t pa_decode_grouped_workspace_size(int num_seqs, int num_heads, int head_dim,
                                                int max_blocks_per_seq);

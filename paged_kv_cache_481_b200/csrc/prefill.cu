@@ -139,11 +139,11 @@ pa_status launch_prefill(void *out, const void *q, const void *k_cache, const vo
 
 // ---- shared-prefix (grouped) decode ---------------------------------------
 
-// For every member b of group g: its tail table (its block-table row from the
-// first block past the shared prefix on, padded with -1), its tail length
-// L_b - P_g, and P_g.  A prefix that is not a whole number of blocks, or
-// longer than a member's context, is recorded (PA_DEVERR_CONTEXT_LEN) and
-// treated as empty for the group.
+// For member m of group g (block (g, m)): its tail table (its block-table row
+// from the first block past the shared prefix on, padded with -1), its tail
+// length L_b - P_g, and P_g.  A prefix that is not a whole number of blocks,
+// or longer than this member's context, is recorded (PA_DEVERR_CONTEXT_LEN)
+// and treated as empty for this member.
 __global__ void __launch_bounds__(128) grouped_tails_kernel(
     const int32_t *__restrict__ block_tables, int max_blocks, const int32_t *__restrict__ context_lens,
     int max_context_len, const int32_t *__restrict__ group_start,
@@ -154,33 +154,30 @@ __global__ void __launch_bounds__(128) grouped_tails_kernel(
     pa::grid_dependency_wait();
     pa::allow_dependent_launch();
     const int g = blockIdx.x;
-    int b0 = group_start[g], b1 = group_start[g + 1];
+    const int b0 = group_start[g], b1 = group_start[g + 1];
+    const int b = b0 + int(blockIdx.y);
     if (b0 < 0 || b1 < b0 || b1 > num_seqs) {  // group bounds outside the batch
-        if (threadIdx.x == 0)
+        if (threadIdx.x == 0 && blockIdx.y == 0)
             atomicOr(err, PA_DEVERR_CONTEXT_LEN);
-        b0 = b1 = 0;
+        return;
     }
+    if (b >= b1)
+        return;
+    const int L = max(0, min(context_lens[b], max_context_len));
     int P = prefix_lens[g];
-    bool bad = P < 0 || P % block_size != 0;
-    for (int b = b0; b < b1; ++b) {
-        const int L = max(0, min(context_lens[b], max_context_len));
-        bad = bad || P > L;
-    }
-    if (bad) {
+    if (P < 0 || P % block_size != 0 || P > L) {
         if (threadIdx.x == 0)
             atomicOr(err, PA_DEVERR_CONTEXT_LEN);
         P = 0;
     }
     const int pb = P / block_size;
-    for (int b = b0; b < b1; ++b) {
-        const int32_t *row = block_tables + size_t(b) * max_blocks;
-        int32_t *trow = tail_tables + size_t(b) * max_blocks;
-        for (int k = threadIdx.x; k < max_blocks; k += blockDim.x)
-            trow[k] = pb + k < max_blocks ? row[pb + k] : -1;
-        if (threadIdx.x == 0) {
-            tail_lens[b] = max(0, min(context_lens[b], max_context_len)) - P;
-            prefix_of[b] = P;
-        }
+    const int32_t *row = block_tables + size_t(b) * max_blocks;
+    int32_t *trow = tail_tables + size_t(b) * max_blocks;
+    for (int k = threadIdx.x; k < max_blocks; k += blockDim.x)
+        trow[k] = pb + k < max_blocks ? row[pb + k] : -1;
+    if (threadIdx.x == 0) {
+        tail_lens[b] = L - P;
+        prefix_of[b] = P;
     }
 }
 
@@ -337,7 +334,10 @@ extern "C" pa_status pa_decode_grouped(void *out, const void *q, const void *k_c
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
 
     // 1. each member's tail table and length
-    if (launch_pdl(grouped_tails_kernel, dim3(unsigned(num_groups)), dim3(128), 0, s, block_tables,
+    if (max_group_size > 65535)
+        return PA_ERR_INVALID_ARG;
+    if (launch_pdl(grouped_tails_kernel, dim3(unsigned(num_groups), unsigned(max_group_size)),
+                   dim3(128), 0, s, block_tables,
                    max_blocks_per_seq, context_lens, max_context_len, group_start, prefix_lens,
                    block_size, num_seqs, tail_tables, tail_lens, prefix_of, err) != cudaSuccess)
         return PA_ERR_CUDA;
