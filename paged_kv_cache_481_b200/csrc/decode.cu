@@ -35,7 +35,7 @@ WorkspaceLayout workspace_layout(int num_seqs, int num_heads, int head_dim)
 }
 
 template <int D, bool kInt8, int NW, int S>
-pa_status launch_decode(const pa::DecodeParams &p, cudaStream_t stream)
+pa_status launch_decode(const pa::DecodeParams &p, const pa::DecodeExtras &x, cudaStream_t stream)
 {
     using Sm = pa::DecodeSmem<D, kInt8, NW, S>;
     static std::atomic<int> grid_for[kMaxDevices];  // 0 = not configured yet
@@ -60,7 +60,7 @@ pa_status launch_decode(const pa::DecodeParams &p, cudaStream_t stream)
         grid_for[dev].store(grid, std::memory_order_release);
     }
     return launch_pdl(pa::paged_decode_kernel<D, kInt8, NW, S>, dim3(grid), dim3(Sm::kThreads),
-                      Sm::kBytes, stream, p) == cudaSuccess
+                      Sm::kBytes, stream, p, x) == cudaSuccess
                ? PA_OK
                : PA_ERR_CUDA;
 }
@@ -188,20 +188,21 @@ pa_status decode_common(void *out, const void *q, const void *k_cache, const voi
     p.block_size = block_size;
     p.num_blocks = num_blocks;
     p.qk_scale_log2 = float(double(scale) * 1.4426950408889634);  // scale * log2(e)
-    p.new_k = static_cast<const __half *>(new_k);
-    p.new_v = static_cast<const __half *>(new_v);
-    p.new_slots = new_slots;
-    p.lse = lse;
+    pa::DecodeExtras x{};
+    x.new_k = static_cast<const __half *>(new_k);
+    x.new_v = static_cast<const __half *>(new_v);
+    x.new_slots = new_slots;
+    x.lse = lse;
 
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
     if (int8) {
         if (head_dim == 128)
-            return launch_decode<128, true, kDecodeWarps, kDecodeStages>(p, s);
-        return launch_decode<64, true, kDecodeWarps, kDecodeStages>(p, s);
+            return launch_decode<128, true, kDecodeWarps, kDecodeStages>(p, x, s);
+        return launch_decode<64, true, kDecodeWarps, kDecodeStages>(p, x, s);
     }
     if (head_dim == 128)
-        return launch_decode<128, false, kDecodeWarps, kDecodeStages>(p, s);
-    return launch_decode<64, false, kDecodeWarps, kDecodeStages>(p, s);
+        return launch_decode<128, false, kDecodeWarps, kDecodeStages>(p, x, s);
+    return launch_decode<64, false, kDecodeWarps, kDecodeStages>(p, x, s);
 }
 
 } // namespace

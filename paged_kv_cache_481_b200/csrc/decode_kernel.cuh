@@ -85,6 +85,12 @@ struct DecodeParams {
     int block_size;
     int num_blocks;
     float qk_scale_log2; // softmax scale * log2(e)
+};
+
+// Optional extras, a separate kernel parameter: adding these fields to
+// DecodeParams itself made ptxas allocate the kernel with 80 instead of 117
+// registers and ~10 % more instructions.
+struct DecodeExtras {
     // Fused append (fp16 cache only; new_slots == nullptr: plain decode).  For
     // a sequence b with new_slots[b] >= 0, position context_lens[b] - 1 is a
     // new token: its K / V rows come from new_k / new_v [B, H, D] (not from
@@ -392,7 +398,8 @@ __device__ __forceinline__ uint32_t rows_tx_bytes(int rows)
 // evict-first policy that keeps the small reused data (block tables, q, split
 // partials) resident.
 template <int D, bool kInt8, class Sm>
-__device__ __forceinline__ void issue_tile(const DecodeParams &p, const TileCursor &cur,
+__device__ __forceinline__ void issue_tile(const DecodeParams &p, const DecodeExtras &x,
+                                           const TileCursor &cur,
                                            const int (&ids)[DecodeShape<D, kInt8>::kMaxIds],
                                            bool with_q, unsigned char *stage_buf, uint32_t bar,
                                            TileMeta *meta, uint64_t stream_policy)
@@ -412,7 +419,7 @@ __device__ __forceinline__ void issue_tile(const DecodeParams &p, const TileCurs
     // comes from the new-token input instead (append_new_row)
     int nf = nv;
     if constexpr (!kInt8)
-        if (p.new_slots && cur.i == cur.nt - 1 && p.new_slots[cur.b] >= 0)
+        if (x.new_slots && cur.i == cur.nt - 1 && x.new_slots[cur.b] >= 0)
             nf = nv - 1;
     // an id outside the pool is recorded and its rows are not fetched
     bool ok[Sh::kMaxIds];
@@ -467,13 +474,14 @@ __device__ __forceinline__ void issue_tile(const DecodeParams &p, const TileCurs
 // The slot must be the one the block table gives that position; otherwise
 // PA_DEVERR_SLOT is recorded (and a slot outside the pool is not written).
 template <int D, class Sm>
-__device__ __forceinline__ void append_new_row(const DecodeParams &p, const TileCursor &cur,
-                                               unsigned char *stage_buf, int lane)
+__device__ __forceinline__ void append_new_row(const DecodeParams &p, const DecodeExtras &x,
+                                               const TileCursor &cur, unsigned char *stage_buf,
+                                               int lane)
 {
     using Sh = DecodeShape<D, false>;
     if (cur.i != cur.nt - 1)
         return;
-    const int64_t slot = p.new_slots[cur.b];
+    const int64_t slot = x.new_slots[cur.b];
     if (slot < 0)
         return;
     constexpr int kChunks = D * 2 / 16;  // 16-byte chunks of one row
@@ -490,7 +498,7 @@ __device__ __forceinline__ void append_new_row(const DecodeParams &p, const Tile
         const bool is_v = lane >= kChunks;
         const int c = lane % kChunks;
         const size_t src_row = size_t(cur.b) * p.num_heads + cur.h;
-        const uint4 val = __ldg(reinterpret_cast<const uint4 *>((is_v ? p.new_v : p.new_k) + src_row * D) + c);
+        const uint4 val = __ldg(reinterpret_cast<const uint4 *>((is_v ? x.new_v : x.new_k) + src_row * D) + c);
         *reinterpret_cast<uint4 *>(stage_buf + (is_v ? Sm::kOffV : 0u) + uint32_t(r) * Sh::kRowBytes +
                                    uint32_t(c) * 16u) = val;
         if (in_pool) {
@@ -508,7 +516,8 @@ __device__ __forceinline__ void append_new_row(const DecodeParams &p, const Tile
 // each contribution rescales the running sums to the running maximum, so all
 // loads are independent.  Lanes with r == 0 each handle kDims dims.
 template <int D, int kDims>
-__device__ __forceinline__ void merge_partials(const DecodeParams &p, uint4 *out_row, int c,
+__device__ __forceinline__ void merge_partials(const DecodeParams &p, const DecodeExtras &x,
+                                               uint4 *out_row, int c,
                                                long long u_start, long long w_first,
                                                long long w_last, long long total,
                                                long long workers)
@@ -542,12 +551,12 @@ __device__ __forceinline__ void merge_partials(const DecodeParams &p, uint4 *out
 #pragma unroll
     for (int k = 0; k < kDims / 8; ++k)
         out_row[(kDims / 8) * c + k] = reinterpret_cast<const uint4 *>(o)[k];
-    if (p.lse && c == 0)
-        p.lse[(reinterpret_cast<const __half *>(out_row) - p.out) / D] = gmax + log2f(den);
+    if (x.lse && c == 0)
+        x.lse[(reinterpret_cast<const __half *>(out_row) - p.out) / D] = gmax + log2f(den);
 }
 
 template <int D, bool kInt8, int NW, int S>
-__global__ void __launch_bounds__(NW * 32) paged_decode_kernel(const DecodeParams p)
+__global__ void __launch_bounds__(NW * 32) paged_decode_kernel(const DecodeParams p, const DecodeExtras x)
 {
     using Sh = DecodeShape<D, kInt8>;
     using Sm = DecodeSmem<D, kInt8, NW, S>;
@@ -721,12 +730,12 @@ __global__ void __launch_bounds__(NW * 32) paged_decode_kernel(const DecodeParam
             for (int e = 0; e < Sh::kMaxIds; ++e)
                 ids_s[e] = __shfl_sync(kFullMask, ids[e], s);
             if (lane == 0)
-                issue_tile<D, kInt8, Sm>(p, cs, ids_s, cs.i == 0 || cs.k == lo,
+                issue_tile<D, kInt8, Sm>(p, x, cs, ids_s, cs.i == 0 || cs.k == lo,
                                          my_buf + size_t(s) * Sm::kStageBytes, my_bar + 8 * s,
                                          my_meta + s, policy);
             if constexpr (!kInt8)
-                if (p.new_slots)
-                    append_new_row<D, Sm>(p, cs, my_buf + size_t(s) * Sm::kStageBytes, lane);
+                if (x.new_slots)
+                    append_new_row<D, Sm>(p, x, cs, my_buf + size_t(s) * Sm::kStageBytes, lane);
             if (s == first - 1)
                 prod = cs;
         }
@@ -808,13 +817,13 @@ __global__ void __launch_bounds__(NW * 32) paged_decode_kernel(const DecodeParam
         if (issued < ntiles) {  // refill the stage just consumed
             if (lane == 0) {
                 fence_proxy_async_smem();
-                issue_tile<D, kInt8, Sm>(p, prod, ids, prod.i == 0 || prod.k == lo,
+                issue_tile<D, kInt8, Sm>(p, x, prod, ids, prod.i == 0 || prod.k == lo,
                                          my_buf + size_t(stage) * Sm::kStageBytes,
                                          my_bar + 8 * stage, my_meta + stage, policy);
             }
             if constexpr (!kInt8)
-                if (p.new_slots)
-                    append_new_row<D, Sm>(p, prod, my_buf + size_t(stage) * Sm::kStageBytes, lane);
+                if (x.new_slots)
+                    append_new_row<D, Sm>(p, x, prod, my_buf + size_t(stage) * Sm::kStageBytes, lane);
             if (++issued < ntiles) {
                 prod.template advance<T>(p);
                 load_tile_ids<Sh>(p, prod, ids);
@@ -853,8 +862,8 @@ __global__ void __launch_bounds__(NW * 32) paged_decode_kernel(const DecodeParam
                 for (int k = 0; k < kDims / 8; ++k)
                     out_row[(kDims / 8) * c + k] = reinterpret_cast<const uint4 *>(o)[k];
             }
-            if (p.lse && lane == 0)
-                p.lse[unit] = m + log2f(l);
+            if (x.lse && lane == 0)
+                x.lse[unit] = m + log2f(l);
             continue;
         }
         const long long u_start = mt.k - mt.i;      // global index of the unit's tile 0
@@ -883,7 +892,7 @@ __global__ void __launch_bounds__(NW * 32) paged_decode_kernel(const DecodeParam
             continue;
         __threadfence();
         if (r == 0)
-            merge_partials<D, kDims>(p, out_row, c, u_start, w_first, w_last, total, workers);
+            merge_partials<D, kDims>(p, x, out_row, c, u_start, w_first, w_last, total, workers);
     }
 }
 
