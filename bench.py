@@ -47,13 +47,20 @@ def _peak_hbm():
 
 
 def _decode_kernel_hash():
+    """Hash of the decode kernel's code (its sources with comments and
+    whitespace removed), so that a recorded ncu capture stays attached to
+    the code it measured."""
+    import re
     h = hashlib.sha256()
     for rel in ("paged_kv_cache_481_b200/csrc/decode_kernel.cuh",
                 "paged_kv_cache_481_b200/csrc/ptx.cuh",
                 "paged_kv_cache_481_b200/csrc/host_common.cuh",
                 "paged_kv_cache_481_b200/csrc/decode.cu"):
-        with open(os.path.join(ROOT, rel), "rb") as f:
-            h.update(f.read())
+        with open(os.path.join(ROOT, rel), encoding="utf-8") as f:
+            src = f.read()
+        src = re.sub(r"/\*.*?\*/", " ", src, flags=re.S)
+        src = re.sub(r"//[^\n]*", " ", src)
+        h.update("".join(src.split()).encode())
     return h.hexdigest()
 
 

@@ -42,6 +42,12 @@
 //       q.K = s (sum_d q_d (1024 + c_d) - (1024 + z) sum_d q_d),
 //     sum_t w_t V_t = sum_t w_t s_t (1024 + c_t) - sum_t w_t s_t (1024 + z_t),
 //     the codes being widened exactly to fp16 as 1024 + c by a byte permute.
+//   * Fused append (DecodeExtras, fp16): the worker that issues a unit's last
+//     tile fetches one row fewer and its warp copies the new token's K / V
+//     rows from the input into the stage and into the cache slot (the decode
+//     step's cache write, polomodov.tech slide 11, in the same launch).
+//   * Optional log-normaliser output (DecodeExtras::lse) so a caller can merge
+//     this attention with attention over other parts of the context.
 #pragma once
 
 #include <cuda_fp16.h>
