@@ -567,7 +567,12 @@ def main(argv=None):
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--unfused", action="store_true",
                     help="time the cache write and the decode as two launches")
+    ap.add_argument("--cpu-threads", type=int, default=None,
+                    help="host threads for the oracle (CPU baseline / reference arm); default all")
     args = ap.parse_args(argv)
+    if args.cpu_threads:
+        # read by the oracle's OpenMP runtime when the oracle library first loads
+        os.environ["OMP_NUM_THREADS"] = str(args.cpu_threads)
     if args.warmup < 3:
         raise SystemExit("--warmup must be >= 3")
     if args.impl == "reference":

@@ -3,6 +3,7 @@
     python -m paged_kv_cache_481_b200.measure prefill [--iters N]
     python -m paged_kv_cache_481_b200.measure swap [--iters N]
     python -m paged_kv_cache_481_b200.measure grouped [--iters N]
+    python -m paged_kv_cache_481_b200.measure cache [--iters N]
 
 Each prints one JSON line per case.  Times are CUDA events on the launching
 stream around N back-to-back calls after warm-up; inputs are synthetic
@@ -19,6 +20,10 @@ grouped: decode of the shared-prefix batch (8 groups of 8 sequences, a
 1024-token prefix, private tails of 1-256 tokens, H=40, D=128, bs=16) with
 pa_decode and with pa_decode_grouped (the prefix read once per group and
 head); bytes = what DRAM must deliver, each physical row once.
+
+cache: pa_reshape_and_cache of one decode step's new tokens (32 and 256
+sequences, H=40, D=128, bs=16) and pa_copy_blocks of 64 copy-on-write pairs,
+GB/s = (bytes read + bytes written) / t.
 
 swap: pa_swap_blocks between the device pool and a page-locked host pool, in
 both directions, against a plain copy of the same number of contiguous bytes
@@ -163,9 +168,40 @@ def measure_grouped(iters: int):
     return lines
 
 
+def measure_cache(iters: int, seed: int = 0):
+    from . import accounting
+    h, d, bs = 40, 128, 16
+    g = torch.Generator(device="cuda").manual_seed(seed)
+    nb = 8192
+    kc = torch.randn((nb, h, bs, d), generator=g, device="cuda").half()
+    vc = torch.randn_like(kc)
+    lines = []
+    for n in (32, 256):
+        key = torch.randn((n, h, d), generator=g, device="cuda").half()
+        value = torch.randn_like(key)
+        slots = (torch.randperm(nb, generator=g, device="cuda")[:n] * bs
+                 + torch.randint(0, bs, (n,), generator=g, device="cuda")).long()
+        ms = _time_ms(lambda: binding.pa_reshape_and_cache(key, value, kc, vc, slots), iters)
+        nbytes = accounting.cache_write_bytes(n, h, d)
+        line = {"what": "pa_reshape_and_cache", "tokens": n, "num_heads": h, "head_dim": d,
+                "bytes": nbytes, "us": ms * 1e3, "gbs": nbytes / (ms * 1e-3) / 1e9}
+        print(json.dumps(line), flush=True)
+        lines.append(line)
+    perm = torch.randperm(nb, generator=g, device="cuda")[:128]
+    pairs = torch.stack([perm[:64], perm[64:]], 1).contiguous().long()
+    ms = _time_ms(lambda: binding.pa_copy_blocks(kc, vc, pairs), iters)
+    nbytes = accounting.copy_blocks_bytes(64, h, d, bs)
+    line = {"what": "pa_copy_blocks", "pairs": 64, "num_heads": h, "block_size": bs,
+            "bytes": nbytes, "us": ms * 1e3, "gbs": nbytes / (ms * 1e-3) / 1e9,
+            "device_error": binding.pa_get_last_device_error()}
+    print(json.dumps(line), flush=True)
+    lines.append(line)
+    return lines
+
+
 def main(argv=None):
     ap = argparse.ArgumentParser(description=__doc__.split("\n\n")[0])
-    ap.add_argument("what", choices=["prefill", "swap", "grouped"])
+    ap.add_argument("what", choices=["prefill", "swap", "grouped", "cache"])
     ap.add_argument("--iters", type=int, default=10)
     ap.add_argument("--block-size", type=int, default=16)
     ap.add_argument("--case", default=None, help="only the prefill case of this name")
@@ -176,6 +212,8 @@ def main(argv=None):
         measure_prefill(args.iters, args.block_size, case=args.case)
     elif args.what == "grouped":
         measure_grouped(args.iters)
+    elif args.what == "cache":
+        measure_cache(args.iters)
     else:
         measure_swap(args.iters)
 
