@@ -23,7 +23,9 @@ head); bytes = what DRAM must deliver, each physical row once.
 
 cache: pa_reshape_and_cache of one decode step's new tokens (32 and 256
 sequences, H=40, D=128, bs=16) and pa_copy_blocks of 64 copy-on-write pairs,
-GB/s = (bytes read + bytes written) / t.
+GB/s = (bytes read + bytes written) / t; these kernels are a few
+microseconds, so they are timed as 20 launches replayed from a CUDA graph
+(host launch overhead excluded).
 
 swap: pa_swap_blocks between the device pool and a page-locked host pool, in
 both directions, against a plain copy of the same number of contiguous bytes
@@ -63,6 +65,30 @@ def _time_ms(fn, iters, warmup=3):
     e1.record()
     torch.cuda.synchronize()
     return e0.elapsed_time(e1) / iters
+
+
+def _time_graph_ms(fn, launches: int = 20, iters: int = 5):
+    """Per-launch device time of a short kernel: `launches` calls captured in
+    a CUDA graph and replayed, so host launch overhead does not show."""
+    side = torch.cuda.Stream()
+    side.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(side):
+        for _ in range(3):
+            fn()
+    torch.cuda.current_stream().wait_stream(side)
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph):
+        for _ in range(launches):
+            fn()
+    graph.replay()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(iters):
+        graph.replay()
+    e1.record()
+    torch.cuda.synchronize()
+    return e0.elapsed_time(e1) / (iters * launches)
 
 
 PREFILL_CASES = [
@@ -181,7 +207,7 @@ def measure_cache(iters: int, seed: int = 0):
         value = torch.randn_like(key)
         slots = (torch.randperm(nb, generator=g, device="cuda")[:n] * bs
                  + torch.randint(0, bs, (n,), generator=g, device="cuda")).long()
-        ms = _time_ms(lambda: binding.pa_reshape_and_cache(key, value, kc, vc, slots), iters)
+        ms = _time_graph_ms(lambda: binding.pa_reshape_and_cache(key, value, kc, vc, slots))
         nbytes = accounting.cache_write_bytes(n, h, d)
         line = {"what": "pa_reshape_and_cache", "tokens": n, "num_heads": h, "head_dim": d,
                 "bytes": nbytes, "us": ms * 1e3, "gbs": nbytes / (ms * 1e-3) / 1e9}
@@ -189,7 +215,7 @@ def measure_cache(iters: int, seed: int = 0):
         lines.append(line)
     perm = torch.randperm(nb, generator=g, device="cuda")[:128]
     pairs = torch.stack([perm[:64], perm[64:]], 1).contiguous().long()
-    ms = _time_ms(lambda: binding.pa_copy_blocks(kc, vc, pairs), iters)
+    ms = _time_graph_ms(lambda: binding.pa_copy_blocks(kc, vc, pairs))
     nbytes = accounting.copy_blocks_bytes(64, h, d, bs)
     line = {"what": "pa_copy_blocks", "pairs": 64, "num_heads": h, "block_size": bs,
             "bytes": nbytes, "us": ms * 1e3, "gbs": nbytes / (ms * 1e-3) / 1e9,
