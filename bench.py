@@ -405,7 +405,12 @@ def run_gpu(args):
     assert binding.pa_get_last_device_error() == 0
 
     sampler = ClockSampler(local).start()
-    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+    # a step of one launch is timed as K back-to-back launches between two
+    # events (the region's mean is that launch's mean duration, gaps included);
+    # a step of several launches brackets each decode with its own events
+    single_launch = launches_per_step == 1
+    evs = [None if single_launch else
+           (torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
            for _ in range(args.steps)]
     start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     if world > 1:
@@ -423,55 +428,93 @@ def run_gpu(args):
         dist.barrier()
     sampler.stop()
     ms = start.elapsed_time(end)
-    decode_ms = [a.elapsed_time(z) for a, z in evs]
+    decode_ms = ([ms / args.steps] * args.steps if single_launch
+                 else [a.elapsed_time(z) for a, z in evs])
     assert binding.pa_get_last_device_error() == 0
 
     # end to end: each step's inputs (q, the new tokens' K/V, slots, block
     # tables, context lengths) leave one pinned host buffer in one copy, and
-    # out comes back to pinned host memory; the KV pool stays resident.
+    # out comes back to pinned host memory; the KV pool stays resident.  As a
+    # serving loop would, the copies are pipelined with the decode: two
+    # device staging buffers and two outputs, the inputs of step i + 1 going
+    # up (copy stream) and the result of step i - 1 coming back (second copy
+    # stream) while step i decodes.  Every step's copies are inside the timed
+    # region, which ends when the last result is in host memory.
     parts = [q, key, value, slots, tables, lens]
     offs, total = [], 0
     for t in parts:
         offs.append(total)
         total += (t.numel() * t.element_size() + 255) // 256 * 256
     h_stage = torch.empty(total, dtype=torch.uint8, pin_memory=True)
-    d_stage = torch.empty(total, dtype=torch.uint8, device=dev)
-    views = []
+    d_stages = [torch.empty(total, dtype=torch.uint8, device=dev) for _ in range(2)]
+    stage_views = []
+    for d_stage in d_stages:
+        views = []
+        for t, o in zip(parts, offs):
+            n = t.numel() * t.element_size()
+            views.append(d_stage[o:o + n].view(t.dtype).view(t.shape))
+        stage_views.append(views)
     for t, o in zip(parts, offs):
         n = t.numel() * t.element_size()
         h_stage[o:o + n].copy_(t.reshape(-1).view(torch.uint8).cpu())
-        views.append(d_stage[o:o + n].view(t.dtype).view(t.shape))
-    d_q, d_key, d_value, d_slots, d_tables, d_lens = views
-    h_out = torch.empty(out.shape, dtype=out.dtype, pin_memory=True)
+    outs = [out, torch.empty_like(out)]
+    h_outs = [torch.empty(out.shape, dtype=out.dtype, pin_memory=True) for _ in range(2)]
     h2d = sum(t.numel() * t.element_size() for t in parts)
-    d2h = h_out.numel() * h_out.element_size()
+    d2h = h_outs[0].numel() * h_outs[0].element_size()
+    up, down = torch.cuda.Stream(device=dev), torch.cuda.Stream(device=dev)
 
-    def e2e_step():
-        d_stage.copy_(h_stage, non_blocking=True)
+    def decode_from(views, o):
+        d_q, d_key, d_value, d_slots, d_tables, d_lens = views
         if pairs is not None:
             copy_step()
         if fused:
-            binding.pa_decode_append(out, d_q, d_key, d_value, kc, vc, d_slots, d_tables, d_lens,
+            binding.pa_decode_append(o, d_q, d_key, d_value, kc, vc, d_slots, d_tables, d_lens,
                                      mcl, wl.scale, ws, stream=stream)
         else:
             write_step(d_key, d_value, d_slots)
-            decode_step(out, d_q, d_tables, d_lens)
-        h_out.copy_(out, non_blocking=True)
+            decode_step(o, d_q, d_tables, d_lens)
 
-    with torch.cuda.stream(stream):
-        for _ in range(max(3, args.warmup)):
-            e2e_step()
+    def run_e2e(n, start_event):
+        up_done = [torch.cuda.Event() for _ in range(2)]
+        dec_done = [torch.cuda.Event() for _ in range(2)]
+        down_done = [torch.cuda.Event() for _ in range(2)]
+        up.wait_event(start_event)
+        with torch.cuda.stream(up):
+            d_stages[0].copy_(h_stage, non_blocking=True)
+            up_done[0].record(up)
+        for i in range(n):
+            cur, nxt = i % 2, (i + 1) % 2
+            if i + 1 < n:  # inputs of the next step, once step i - 1 has used that buffer
+                with torch.cuda.stream(up):
+                    if i >= 1:
+                        up.wait_event(dec_done[nxt])
+                    d_stages[nxt].copy_(h_stage, non_blocking=True)
+                    up_done[nxt].record(up)
+            stream.wait_event(up_done[cur])
+            if i >= 2:  # step i - 2's result has left outs[cur]
+                stream.wait_event(down_done[cur])
+            with torch.cuda.stream(stream):
+                decode_from(stage_views[cur], outs[cur])
+                dec_done[cur].record(stream)
+            with torch.cuda.stream(down):
+                down.wait_event(dec_done[cur])
+                h_outs[cur].copy_(outs[cur], non_blocking=True)
+                down_done[cur].record(down)
+        stream.wait_event(down_done[(n - 1) % 2])
+
+    warm = torch.cuda.Event()
+    warm.record(stream)
+    run_e2e(max(3, args.warmup), warm)
     if world > 1:
         dist.barrier()
     torch.cuda.synchronize()
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     e0.record(stream)
-    with torch.cuda.stream(stream):
-        for _ in range(args.steps):
-            e2e_step()
+    run_e2e(args.steps, e0)
     e1.record(stream)
     torch.cuda.synchronize()
     e2e_ms = e0.elapsed_time(e1)
+    assert binding.pa_get_last_device_error() == 0
     if world > 1:
         dist.barrier()
 
@@ -524,9 +567,12 @@ def run_gpu(args):
             "seq_heads_per_s": total_units * args.steps / (ms * 1e-3),
             "hbm_frac": achieved / peak,
             "decode_us_mean": mean_dec_ms * 1e3,
-            "decode_us_median": statistics.median(decode_ms) * 1e3,
-            "decode_us_max": max(decode_ms) * 1e3,
-            "decode_us_argmax": int(np.argmax(decode_ms)),
+            "launch_timing": ("events around the K back-to-back launches of the timed region"
+                              if single_launch else "events around each decode launch"),
+            **({} if single_launch else {
+                "decode_us_median": statistics.median(decode_ms) * 1e3,
+                "decode_us_max": max(decode_ms) * 1e3,
+                "decode_us_argmax": int(np.argmax(decode_ms))}),
             "roofline": {
                 "kernel": "paged_decode_kernel" + ("<int8>" if int8 else ""), "bound": "hbm",
                 "achieved": achieved,
@@ -536,6 +582,8 @@ def run_gpu(args):
                 "logical_bytes_per_launch": dec_bytes,
             },
             "e2e": {"value": total_bytes * args.steps / (e2e_ms * 1e-3) / 1e9, "unit": "GB/s",
+                    "copies": "pinned host <-> device every step, pipelined with the decode "
+                              "(two staging buffers and outputs, separate copy streams)",
                     "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                     "ms_per_step": e2e_ms / args.steps},
             "gpu_launches": launches_per_step * args.steps,
