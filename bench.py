@@ -623,6 +623,9 @@ def main(argv=None):
         os.environ["OMP_NUM_THREADS"] = str(args.cpu_threads)
     if args.warmup < 3:
         raise SystemExit("--warmup must be >= 3")
+    if args.kv_dtype == "int8" and args.workload == 4:
+        raise SystemExit("--kv-dtype int8 is not built for the shared-prefix workload (4): "
+                         "its int8 pool would need every aliased block's tokens once")
     if args.impl == "reference":
         return run_reference(args)
     return run_gpu(args)
