@@ -8,7 +8,7 @@ import torch
 import oracle
 from paged_kv_cache_481_b200 import binding, build, workloads
 
-from gpu_helpers import ATOL, gpu_write_and_decode, max_abs_err, to_dev
+from gpu_helpers import ATOL, gpu_write_and_decode, max_abs_err, oracle_write_and_decode, to_dev
 
 pytestmark = pytest.mark.gpu
 
@@ -90,3 +90,22 @@ def test_fused_reports_a_slot_that_is_not_the_last_position():
     slots[1] = slots[1] - 1                 # the slot of position L - 2 instead of L - 1
     _fused(wl, t, slots)
     assert binding.pa_get_last_device_error() == binding.PA_DEVERR_SLOT
+
+
+@pytest.mark.slow
+@pytest.mark.parametrize("cfg", [2, 3])
+def test_fused_step_at_full_size(cfg):
+    """The benchmarked step itself: pa_decode_append on the 13B decode batch
+    (B=32, H=40, D=128, bs=16) and on the serving batch (B=256), against the
+    oracle's cache write then decode over every sequence, and bit for bit
+    against the two separate calls."""
+    wl = workloads.make_workload(cfg, device="cuda")
+    t = to_dev(wl)
+    out = _fused(wl, t)
+    ref, okc, ovc = oracle_write_and_decode(wl)
+    assert max_abs_err(out, ref) <= ATOL
+    assert np.array_equal(t["k_cache"].cpu().numpy().view(np.uint16), okc.view(np.uint16))
+    assert np.array_equal(t["v_cache"].cpu().numpy().view(np.uint16), ovc.view(np.uint16))
+    out2, _, _ = gpu_write_and_decode(wl)
+    assert torch.equal(out, out2)
+    assert binding.pa_get_last_device_error() == 0
