@@ -46,16 +46,26 @@ def _peak_hbm():
         return FALLBACK_HBM_GBS, "fallback"
 
 
-def _decode_kernel_hash():
-    """Hash of the decode kernel's code (its sources with comments and
-    whitespace removed), so that a recorded ncu capture stays attached to
-    the code it measured."""
-    import re
-    h = hashlib.sha256()
-    for rel in ("paged_kv_cache_481_b200/csrc/decode_kernel.cuh",
+KERNEL_SOURCES = {
+    "decode": ("paged_kv_cache_481_b200/csrc/decode_kernel.cuh",
+               "paged_kv_cache_481_b200/csrc/ptx.cuh",
+               "paged_kv_cache_481_b200/csrc/host_common.cuh",
+               "paged_kv_cache_481_b200/csrc/decode.cu"),
+    "prefill": ("paged_kv_cache_481_b200/csrc/prefill_kernel.cuh",
+                "paged_kv_cache_481_b200/csrc/tcgen05.cuh",
                 "paged_kv_cache_481_b200/csrc/ptx.cuh",
                 "paged_kv_cache_481_b200/csrc/host_common.cuh",
-                "paged_kv_cache_481_b200/csrc/decode.cu"):
+                "paged_kv_cache_481_b200/csrc/prefill.cu"),
+}
+
+
+def _decode_kernel_hash(kind: str = "decode"):
+    """Hash of a kernel's code (its sources with comments and whitespace
+    removed), so that a recorded ncu capture stays attached to the code it
+    measured."""
+    import re
+    h = hashlib.sha256()
+    for rel in KERNEL_SOURCES[kind]:
         with open(os.path.join(ROOT, rel), encoding="utf-8") as f:
             src = f.read()
         src = re.sub(r"/\*.*?\*/", " ", src, flags=re.S)
@@ -64,16 +74,16 @@ def _decode_kernel_hash():
     return h.hexdigest()
 
 
-def _recorded_traffic(workload: str, launch: str = "pa_decode"):
-    """DRAM bytes per decode launch from the committed ncu summary, only if
-    it was taken on the current kernel source and this workload."""
-    path = os.path.join(ROOT, "profiles", "decode_traffic.json")
+def _recorded_traffic(workload: str, launch: str = "pa_decode", kind: str = "decode"):
+    """DRAM bytes per launch from the committed ncu summary of that kernel,
+    only if it was taken on the current kernel source and this workload."""
+    path = os.path.join(ROOT, "profiles", f"{kind}_traffic.json")
     try:
         with open(path) as f:
             rec = json.load(f)
     except Exception:
         return None
-    if (rec.get("kernel_sha256") != _decode_kernel_hash() or rec.get("workload") != workload
+    if (rec.get("kernel_sha256") != _decode_kernel_hash(kind) or rec.get("workload") != workload
             or rec.get("launch", "pa_decode") != launch):
         return None
     return rec.get("dram_bytes_per_launch")
@@ -207,26 +217,50 @@ def _cpu_sample(wl, max_units: int, seqs=None):
                 lens=wl.context_lens[seqs].copy(), scale=wl.scale)
 
 
-def _time_oracle(sample, reps: int = 1):
+def _quantize_sample(sample):
+    """The int8 cache of a sample: every row of its fp16 pool quantized by the
+    oracle (the same decisions as the CUDA cache write, bit for bit)."""
     import oracle
+    out = dict(sample)
+    for name in ("kc", "vc"):
+        x = sample[name]
+        codes, params = oracle.quantize_rows(x.reshape(-1, x.shape[-1]))
+        out[name] = codes.reshape(x.shape)
+        out[name[0] + "p"] = params.reshape(x.shape[:-1] + (2,))
+    out["int8"] = True
+    return out
+
+
+def _oracle_decode(sample):
+    import oracle
+    if sample.get("int8"):
+        return oracle.paged_decode_int8(sample["q"], sample["kc"], sample["vc"], sample["kp"],
+                                        sample["vp"], sample["tables"], sample["lens"],
+                                        sample["scale"])
+    return oracle.paged_decode(sample["q"], sample["kc"], sample["vc"], sample["tables"],
+                               sample["lens"], sample["scale"])
+
+
+def _time_oracle(sample, reps: int = 1):
     t = []
     for _ in range(reps):
         t0 = time.perf_counter()
-        oracle.paged_decode(sample["q"], sample["kc"], sample["vc"], sample["tables"],
-                            sample["lens"], sample["scale"])
+        _oracle_decode(sample)
         t.append(time.perf_counter() - t0)
     return statistics.median(t)
 
 
-def cpu_baseline_sample(wl, target_s: float = 10.0):
+def cpu_baseline_sample(wl, target_s: float = 10.0, int8: bool = False):
     """Size and cut the CPU-baseline sample (call before any GPU work touches
     the pool): about target_s seconds of oracle decode -- the first sequences
     of the batch, or, when the whole batch takes less, the whole batch
-    decoded repeatedly."""
-    probe = _cpu_sample(wl, wl.num_heads)                       # one sequence
+    decoded repeatedly.  int8: over the oracle-quantized cache."""
+    cut = (lambda units: _quantize_sample(_cpu_sample(wl, units))) if int8 else \
+        (lambda units: _cpu_sample(wl, units))
+    probe = cut(wl.num_heads)                                   # one sequence
     per_seq = max(_time_oracle(probe), 1e-4)
     nseq = int(min(wl.num_seqs, max(1, target_s / per_seq)))
-    sample = _cpu_sample(wl, nseq * wl.num_heads)
+    sample = cut(nseq * wl.num_heads)
     reps = 1
     if nseq == wl.num_seqs:
         per_batch = max(_time_oracle(sample), 1e-4)
@@ -243,15 +277,17 @@ def cpu_baseline(wl, sample):
     reps = int(sample.get("reps", 1))
     t0 = time.perf_counter()
     for _ in range(reps):
-        oracle.paged_decode(sample["q"], sample["kc"], sample["vc"], sample["tables"],
-                            sample["lens"], sample["scale"])
+        _oracle_decode(sample)
     t = time.perf_counter() - t0
-    nbytes = accounting.decode_bytes(sample["lens"], wl.num_heads, wl.head_dim) * reps
+    int8 = bool(sample.get("int8"))
+    nbytes = (accounting.decode_bytes_int8 if int8 else accounting.decode_bytes)(
+        sample["lens"], wl.num_heads, wl.head_dim) * reps
     what = (f"first {len(sample['lens'])} of {wl.num_seqs} sequences" if reps == 1 else
             f"all {wl.num_seqs} sequences, {reps} times")
     return {"value": nbytes / t / 1e9, "unit": "GB/s", "cores": oracle.num_threads(),
             "kind": "oracle",
-            "sample": f"{what} x {wl.num_heads} heads (decode only, fp64), {t:.1f} s wall"}
+            "sample": f"{what} x {wl.num_heads} heads (decode only, fp64"
+                      f"{' over the int8 cache' if int8 else ''}), {t:.1f} s wall"}
 
 
 def run_reference(args):
@@ -303,6 +339,87 @@ def run_reference(args):
     return 0
 
 
+def pipelined_e2e(parts, out_like, step, stream, warmup, steps, world):
+    """End-to-end timing through the public API with host buffers: each
+    step's inputs (`parts`, packed in one pinned host buffer) are copied to
+    the device and its output back to pinned host memory.  As a serving loop
+    would, the copies are pipelined with the compute: two device staging
+    buffers and two outputs, the inputs of step i + 1 going up on one copy
+    stream and the result of step i - 1 coming back on another while step i
+    runs on `stream`.  The timed region (CUDA events on `stream`) ends when
+    the last result is in host memory, so every step's copies are inside it.
+    `step(views, out)` launches one step on `stream` from the staged inputs.
+    Returns (ms for `steps` steps, h2d bytes per step, d2h bytes per step)."""
+    import torch
+    import torch.distributed as dist
+    dev = out_like.device
+    offs, total = [], 0
+    for t in parts:
+        offs.append(total)
+        total += (t.numel() * t.element_size() + 255) // 256 * 256
+    h_stage = torch.empty(total, dtype=torch.uint8, pin_memory=True)
+    d_stages = [torch.empty(total, dtype=torch.uint8, device=dev) for _ in range(2)]
+    stage_views = []
+    for d_stage in d_stages:
+        views = []
+        for t, o in zip(parts, offs):
+            n = t.numel() * t.element_size()
+            views.append(d_stage[o:o + n].view(t.dtype).view(t.shape))
+        stage_views.append(views)
+    for t, o in zip(parts, offs):
+        n = t.numel() * t.element_size()
+        h_stage[o:o + n].copy_(t.reshape(-1).view(torch.uint8).cpu())
+    outs = [torch.empty_like(out_like) for _ in range(2)]
+    h_outs = [torch.empty(out_like.shape, dtype=out_like.dtype, pin_memory=True)
+              for _ in range(2)]
+    h2d = sum(t.numel() * t.element_size() for t in parts)
+    d2h = h_outs[0].numel() * h_outs[0].element_size()
+    up, down = torch.cuda.Stream(device=dev), torch.cuda.Stream(device=dev)
+
+    def run(n, start_event):
+        up_done = [torch.cuda.Event() for _ in range(2)]
+        done = [torch.cuda.Event() for _ in range(2)]
+        down_done = [torch.cuda.Event() for _ in range(2)]
+        up.wait_event(start_event)
+        with torch.cuda.stream(up):
+            d_stages[0].copy_(h_stage, non_blocking=True)
+            up_done[0].record(up)
+        for i in range(n):
+            cur, nxt = i % 2, (i + 1) % 2
+            if i + 1 < n:  # inputs of the next step, once step i - 1 has used that buffer
+                with torch.cuda.stream(up):
+                    if i >= 1:
+                        up.wait_event(done[nxt])
+                    d_stages[nxt].copy_(h_stage, non_blocking=True)
+                    up_done[nxt].record(up)
+            stream.wait_event(up_done[cur])
+            if i >= 2:  # step i - 2's result has left outs[cur]
+                stream.wait_event(down_done[cur])
+            with torch.cuda.stream(stream):
+                step(stage_views[cur], outs[cur])
+                done[cur].record(stream)
+            with torch.cuda.stream(down):
+                down.wait_event(done[cur])
+                h_outs[cur].copy_(outs[cur], non_blocking=True)
+                down_done[cur].record(down)
+        stream.wait_event(down_done[(n - 1) % 2])
+
+    warm = torch.cuda.Event()
+    warm.record(stream)
+    run(max(3, warmup), warm)
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    run(steps, e0)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    return e0.elapsed_time(e1), h2d, d2h
+
+
 def run_gpu(args):
     import torch
     import torch.distributed as dist
@@ -328,8 +445,8 @@ def run_gpu(args):
                                  keep_tokens=int8)
     dev = torch.device("cuda", local)
     cpu_sample = None
-    if rank == 0 and world == 1 and not args.no_cpu_baseline and not int8:
-        cpu_sample = cpu_baseline_sample(wl, target_s=args.cpu_seconds)
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        cpu_sample = cpu_baseline_sample(wl, target_s=args.cpu_seconds, int8=int8)
     stream = torch.cuda.Stream(device=dev)
     b, h, d = wl.num_seqs, wl.num_heads, wl.head_dim
     q = wl.q
@@ -433,36 +550,8 @@ def run_gpu(args):
     assert binding.pa_get_last_device_error() == 0
 
     # end to end: each step's inputs (q, the new tokens' K/V, slots, block
-    # tables, context lengths) leave one pinned host buffer in one copy, and
-    # out comes back to pinned host memory; the KV pool stays resident.  As a
-    # serving loop would, the copies are pipelined with the decode: two
-    # device staging buffers and two outputs, the inputs of step i + 1 going
-    # up (copy stream) and the result of step i - 1 coming back (second copy
-    # stream) while step i decodes.  Every step's copies are inside the timed
-    # region, which ends when the last result is in host memory.
-    parts = [q, key, value, slots, tables, lens]
-    offs, total = [], 0
-    for t in parts:
-        offs.append(total)
-        total += (t.numel() * t.element_size() + 255) // 256 * 256
-    h_stage = torch.empty(total, dtype=torch.uint8, pin_memory=True)
-    d_stages = [torch.empty(total, dtype=torch.uint8, device=dev) for _ in range(2)]
-    stage_views = []
-    for d_stage in d_stages:
-        views = []
-        for t, o in zip(parts, offs):
-            n = t.numel() * t.element_size()
-            views.append(d_stage[o:o + n].view(t.dtype).view(t.shape))
-        stage_views.append(views)
-    for t, o in zip(parts, offs):
-        n = t.numel() * t.element_size()
-        h_stage[o:o + n].copy_(t.reshape(-1).view(torch.uint8).cpu())
-    outs = [out, torch.empty_like(out)]
-    h_outs = [torch.empty(out.shape, dtype=out.dtype, pin_memory=True) for _ in range(2)]
-    h2d = sum(t.numel() * t.element_size() for t in parts)
-    d2h = h_outs[0].numel() * h_outs[0].element_size()
-    up, down = torch.cuda.Stream(device=dev), torch.cuda.Stream(device=dev)
-
+    # tables, context lengths) leave pinned host memory and out comes back to
+    # it, pipelined with the decode; the KV pool stays resident.
     def decode_from(views, o):
         d_q, d_key, d_value, d_slots, d_tables, d_lens = views
         if pairs is not None:
@@ -474,49 +563,9 @@ def run_gpu(args):
             write_step(d_key, d_value, d_slots)
             decode_step(o, d_q, d_tables, d_lens)
 
-    def run_e2e(n, start_event):
-        up_done = [torch.cuda.Event() for _ in range(2)]
-        dec_done = [torch.cuda.Event() for _ in range(2)]
-        down_done = [torch.cuda.Event() for _ in range(2)]
-        up.wait_event(start_event)
-        with torch.cuda.stream(up):
-            d_stages[0].copy_(h_stage, non_blocking=True)
-            up_done[0].record(up)
-        for i in range(n):
-            cur, nxt = i % 2, (i + 1) % 2
-            if i + 1 < n:  # inputs of the next step, once step i - 1 has used that buffer
-                with torch.cuda.stream(up):
-                    if i >= 1:
-                        up.wait_event(dec_done[nxt])
-                    d_stages[nxt].copy_(h_stage, non_blocking=True)
-                    up_done[nxt].record(up)
-            stream.wait_event(up_done[cur])
-            if i >= 2:  # step i - 2's result has left outs[cur]
-                stream.wait_event(down_done[cur])
-            with torch.cuda.stream(stream):
-                decode_from(stage_views[cur], outs[cur])
-                dec_done[cur].record(stream)
-            with torch.cuda.stream(down):
-                down.wait_event(dec_done[cur])
-                h_outs[cur].copy_(outs[cur], non_blocking=True)
-                down_done[cur].record(down)
-        stream.wait_event(down_done[(n - 1) % 2])
-
-    warm = torch.cuda.Event()
-    warm.record(stream)
-    run_e2e(max(3, args.warmup), warm)
-    if world > 1:
-        dist.barrier()
-    torch.cuda.synchronize()
-    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    e0.record(stream)
-    run_e2e(args.steps, e0)
-    e1.record(stream)
-    torch.cuda.synchronize()
-    e2e_ms = e0.elapsed_time(e1)
+    e2e_ms, h2d, d2h = pipelined_e2e([q, key, value, slots, tables, lens], out, decode_from,
+                                     stream, args.warmup, args.steps, world)
     assert binding.pa_get_last_device_error() == 0
-    if world > 1:
-        dist.barrier()
 
     dec_bytes = (accounting.decode_bytes_int8(wl.context_lens, h, d) if int8
                  else accounting.decode_bytes(wl.context_lens, h, d))
@@ -599,6 +648,202 @@ def run_gpu(args):
     return 0
 
 
+PREFILL_METRIC = "paged prefill attention: algorithmic TFLOP/s (causal; % of tensor peak)"
+
+
+def _prefill_flops(lens, n_new, num_heads, head_dim):
+    """Algorithmic FLOPs of causal multi-query attention: a new token at
+    position p attends to p + 1 cached tokens, 2 D multiply-adds each for
+    q . K and for P V."""
+    total = 0.0
+    for length, n in zip(lens, n_new):
+        pos = np.arange(length - n, length, dtype=np.float64)
+        total += float((pos + 1).sum())
+    return total * num_heads * 4 * head_dim
+
+
+def prefill_cpu_baseline(q, key, value, n, length, num_heads, head_dim, block_size, scale,
+                         target_s: float = 10.0):
+    """The oracle's paged prefill as it stands, on the host cores, on a bounded
+    sample of the same workload: the first prompt, its first heads (about
+    target_s seconds); TFLOP/s over the sample's algorithmic FLOPs."""
+    import oracle
+    nblk = length // block_size
+
+    def sample(heads):
+        k = key[:n, :heads].reshape(nblk, block_size, heads, head_dim).transpose(0, 2, 1, 3)
+        v = value[:n, :heads].reshape(nblk, block_size, heads, head_dim).transpose(0, 2, 1, 3)
+        return (np.ascontiguousarray(q[:n, :heads]), np.ascontiguousarray(k),
+                np.ascontiguousarray(v), np.arange(nblk, dtype=np.int32)[None],
+                np.array([length], np.int32), np.array([0, n], np.int32))
+
+    def run(heads):
+        a = sample(heads)
+        t0 = time.perf_counter()
+        oracle.paged_prefill(*a, scale)
+        return time.perf_counter() - t0
+
+    per_head = max(run(1), 1e-4)
+    heads = int(max(1, min(num_heads, target_s / per_head)))
+    t = run(heads)
+    flops = _prefill_flops([length], [n], heads, head_dim)
+    return {"value": flops / t / 1e12, "unit": "TFLOP/s", "cores": oracle.num_threads(),
+            "kind": "oracle",
+            "sample": f"prompt 0 of the batch ({n} new tokens), {heads} of {num_heads} heads "
+                      f"(attention only, fp64), {t:.1f} s wall"}
+
+
+def run_prefill(args):
+    """One step = the prefill of a batch of prompts through the paged cache:
+    pa_reshape_and_cache of every prompt token's K/V into its slot, then
+    pa_prefill (causal multi-query attention on the tensor cores)."""
+    import torch
+    import torch.distributed as dist
+    from paged_kv_cache_481_b200 import binding, build
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world != args.gpus:
+        raise SystemExit(f"--gpus {args.gpus} but WORLD_SIZE={world}")
+    torch.cuda.set_device(local)
+    if world > 1:
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+    build.build()
+    binding.load()
+    dev = torch.device("cuda", local)
+
+    b, length, h, d = args.prompts, args.prompt_len, 40, 128
+    bs = args.block_size or 16
+    n = length
+    if length % bs:
+        raise SystemExit("--prompt-len must be a multiple of the block size")
+    seed = 7 + 100 * rank
+    rng = np.random.default_rng(seed)
+    gen = torch.Generator().manual_seed(seed)
+    tokens = b * n
+    # inputs drawn on the host (seeded), as the oracle sample needs them there too
+    q_h = torch.randn((tokens, h, d), generator=gen).half()
+    key_h = torch.randn((tokens, h, d), generator=gen).half()
+    value_h = torch.randn((tokens, h, d), generator=gen).half()
+    per_seq = length // bs
+    nb = b * per_seq
+    tables_h = rng.permutation(nb).astype(np.int32).reshape(b, per_seq)
+    pos = np.arange(n)
+    slots_h = np.concatenate([tables_h[i, pos // bs].astype(np.int64) * bs + pos % bs
+                              for i in range(b)])
+    scale = d ** -0.5
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        cpu = prefill_cpu_baseline(q_h.numpy(), key_h.numpy(), value_h.numpy(), n, length, h, d,
+                                   bs, scale, target_s=args.cpu_seconds)
+
+    q, key, value = q_h.to(dev), key_h.to(dev), value_h.to(dev)
+    slots = torch.from_numpy(slots_h).to(dev)
+    tables = torch.from_numpy(tables_h).to(dev)
+    lens = torch.full((b,), length, dtype=torch.int32, device=dev)
+    qsl = torch.arange(b + 1, dtype=torch.int32, device=dev) * n
+    kc = torch.zeros((nb, h, bs, d), dtype=torch.float16, device=dev)
+    vc = torch.zeros_like(kc)
+    out = torch.empty_like(q)
+    stream = torch.cuda.Stream(device=dev)
+    flops = _prefill_flops([length] * b, [n] * b, h, d)
+
+    def step(views, o, ev=None):
+        d_q, d_key, d_value, d_slots, d_tables, d_lens, d_qsl = views
+        binding.pa_reshape_and_cache(d_key, d_value, kc, vc, d_slots, stream=stream)
+        if ev is not None:
+            ev[0].record(stream)
+        binding.pa_prefill(o, d_q, kc, vc, d_tables, d_lens, length, d_qsl, n, scale,
+                           stream=stream)
+        if ev is not None:
+            ev[1].record(stream)
+
+    views = [q, key, value, slots, tables, lens, qsl]
+    with torch.cuda.stream(stream):
+        for _ in range(args.warmup):
+            step(views, out)
+    torch.cuda.synchronize()
+    assert binding.pa_get_last_device_error() == 0
+    sampler = ClockSampler(local).start()
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+           for _ in range(args.steps)]
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    w0 = time.perf_counter()
+    start.record(stream)
+    with torch.cuda.stream(stream):
+        for i in range(args.steps):
+            step(views, out, evs[i])
+    end.record(stream)
+    torch.cuda.synchronize()
+    w1 = time.perf_counter()
+    if world > 1:
+        dist.barrier()
+    sampler.stop()
+    ms = start.elapsed_time(end)
+    launch_ms = [a.elapsed_time(z) for a, z in evs]
+    assert binding.pa_get_last_device_error() == 0
+
+    e2e_ms, h2d, d2h = pipelined_e2e(views, out, step, stream, args.warmup, args.steps, world)
+    assert binding.pa_get_last_device_error() == 0
+
+    (ms, e2e_ms), (total_flops,) = reduce_over_ranks([ms, e2e_ms], [flops], dev)
+    result = None
+    if rank == 0:
+        try:
+            with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+                pk = json.load(f)
+            peak, peak_sus, kind = float(pk["bf16_tflops"]), float(pk["bf16_tflops_sustained"]), "measured"
+        except Exception:
+            peak, peak_sus, kind = 1590.0, 1400.0, "fallback"
+        mean_ms = statistics.fmean(launch_ms)
+        achieved = flops / (mean_ms * 1e-3) / 1e12
+        workload = (f"13B prefill: {b} prompts x {length} tokens, H={h} D={d} bs={bs}, "
+                    f"shuffled blocks, causal")
+        result = {
+            "metric": PREFILL_METRIC, "value": total_flops * args.steps / (ms * 1e-3) / 1e12,
+            "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": ms / args.steps, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "f16", "data": "synthetic",
+            "config": {"workload": workload,
+                       "num_seqs": b, "prompt_len": length, "num_heads": h, "head_dim": d,
+                       "block_size": bs, "seed": seed,
+                       "step": f"pa_reshape_and_cache({tokens} tokens) + pa_prefill",
+                       "l2": f"K/V {2 * nb * h * bs * d * 2 / 1e9:.2f} GB and q/out "
+                             f"{2 * tokens * h * d * 2 / 1e9:.2f} GB per step vs "
+                             f"{L2_BYTES / 2**20:.0f} MiB L2 (no flush)",
+                       "parallelism": f"dp{world} (independent prompts per GPU)"},
+            "prefill_us_mean": mean_ms * 1e3,
+            "roofline": {"kernel": "paged_prefill_kernel", "bound": "tensor",
+                         "achieved": achieved, "peak": peak,
+                         "peak_kind": f"{kind} (bf16_tflops, burst; fp16 runs at the bf16 rate)",
+                         "peak_sustained": peak_sus, "unit": "TFLOP/s", "frac": achieved / peak,
+                         "traffic": _recorded_traffic(workload, "pa_prefill", "prefill"),
+                         "algorithmic_flops_per_launch": flops},
+            "e2e": {"value": total_flops * args.steps / (e2e_ms * 1e-3) / 1e12,
+                    "unit": "TFLOP/s",
+                    "copies": "pinned host <-> device every step (q, prompt K/V, slots, tables), "
+                              "pipelined with the step (two staging buffers and outputs)",
+                    "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+                    "ms_per_step": e2e_ms / args.steps},
+            "gpu_launches": 2 * args.steps,
+            "clocks": sampler.summary(w0, w1),
+        }
+        if cpu is not None:
+            result["cpu_baseline"] = cpu
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    if result is not None:
+        print(json.dumps(result), flush=True)
+    return 0
+
+
 def main(argv=None):
     ap = argparse.ArgumentParser(description=__doc__.splitlines()[0])
     ap.add_argument("--gpus", type=int, default=1)
@@ -615,6 +860,10 @@ def main(argv=None):
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--unfused", action="store_true",
                     help="time the cache write and the decode as two launches")
+    ap.add_argument("--path", choices=["decode", "prefill"], default="decode",
+                    help="prefill: the prompt cache write + pa_prefill step instead of decode")
+    ap.add_argument("--prompts", type=int, default=8, help="prefill: prompts per step")
+    ap.add_argument("--prompt-len", type=int, default=2048, help="prefill: tokens per prompt")
     ap.add_argument("--cpu-threads", type=int, default=None,
                     help="host threads for the oracle (CPU baseline / reference arm); default all")
     args = ap.parse_args(argv)
@@ -627,7 +876,11 @@ def main(argv=None):
         raise SystemExit("--kv-dtype int8 is not built for the shared-prefix workload (4): "
                          "its int8 pool would need every aliased block's tokens once")
     if args.impl == "reference":
+        if args.path != "decode":
+            raise SystemExit("--impl reference times the decode path")
         return run_reference(args)
+    if args.path == "prefill":
+        return run_prefill(args)
     return run_gpu(args)
 
 

@@ -83,3 +83,20 @@ def test_reference_arm_other_ranks_exit_quietly():
 def test_warmup_below_three_is_refused():
     r = _run_bench(["--impl", "reference", "--workload", "1", "--steps", "3", "--warmup", "2"])
     assert r.returncode != 0
+
+
+def test_cpu_baselines_of_the_other_paths():
+    """The oracle legs of `bench.py --kv-dtype int8` and `--path prefill` on
+    tiny inputs: a positive rate over the sample they describe."""
+    from paged_kv_cache_481_b200 import workloads
+    wl = workloads.make_workload(1, keep_tokens=True)
+    sample = bench.cpu_baseline_sample(wl, target_s=0.05, int8=True)
+    assert sample["int8"] and sample["kc"].dtype == np.uint8 and sample["kp"].shape[-1] == 2
+    line = bench.cpu_baseline(wl, sample)
+    assert line["kind"] == "oracle" and line["value"] > 0 and "int8" in line["sample"]
+    rng = np.random.default_rng(0)
+    n, h, d, bs = 64, 2, 128, 16
+    q, k, v = (rng.standard_normal((n, h, d)).astype(np.float16) for _ in range(3))
+    line = bench.prefill_cpu_baseline(q, k, v, n, n, h, d, bs, d ** -0.5, target_s=0.05)
+    assert line["unit"] == "TFLOP/s" and line["value"] > 0 and line["cores"] >= 1
+    assert bench._prefill_flops([n], [n], h, d) == 4 * d * h * n * (n + 1) / 2
