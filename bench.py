@@ -5,9 +5,9 @@
 
 One step = one decode iteration of the whole hot path over one batch: the
 cache write of each sequence's newest token and the decode over all
-(sequence, head) pairs -- fused into one pa_decode_append launch for fp16
-caches (--unfused: pa_reshape_and_cache, then pa_decode; int8 caches always
-take the two calls) -- and, for the shared-prefix workload, the
+(sequence, head) pairs -- fused into one pa_decode_append launch
+(pa_decode_append_int8 for the int8 cache; --unfused: the cache write, then
+the decode) -- and, for the shared-prefix workload, the
 copy-on-write pa_copy_blocks before them.  The default workload is the LLaMA-13B-shaped
 single-layer decode batch (B=32, H=40, D=128, bs=16, context U[256, 2048]).
 
@@ -48,6 +48,7 @@ def _peak_hbm():
 
 KERNEL_SOURCES = {
     "decode": ("paged_kv_cache_481_b200/csrc/decode_kernel.cuh",
+               "paged_kv_cache_481_b200/csrc/quant.cuh",
                "paged_kv_cache_481_b200/csrc/ptx.cuh",
                "paged_kv_cache_481_b200/csrc/host_common.cuh",
                "paged_kv_cache_481_b200/csrc/decode.cu"),
@@ -497,7 +498,15 @@ def run_gpu(args):
         else:
             binding.pa_copy_blocks(kc, vc, pairs, stream=stream)
 
-    fused = not int8 and not args.unfused
+    fused = not args.unfused
+
+    def append_step(o, q_, key_, value_, slots_, tables_, lens_):
+        if int8:
+            binding.pa_decode_append_int8(o, q_, key_, value_, kc, vc, kp, vp, slots_, tables_,
+                                          lens_, mcl, wl.scale, ws, stream=stream)
+        else:
+            binding.pa_decode_append(o, q_, key_, value_, kc, vc, slots_, tables_, lens_, mcl,
+                                     wl.scale, ws, stream=stream)
 
     def step(ev_pair=None):
         if pairs is not None:
@@ -507,8 +516,7 @@ def run_gpu(args):
         if ev_pair is not None:
             ev_pair[0].record(stream)
         if fused:
-            binding.pa_decode_append(out, q, key, value, kc, vc, slots, tables, lens, mcl,
-                                     wl.scale, ws, stream=stream)
+            append_step(out, q, key, value, slots, tables, lens)
         else:
             decode_step(out, q, tables, lens)
         if ev_pair is not None:
@@ -557,8 +565,7 @@ def run_gpu(args):
         if pairs is not None:
             copy_step()
         if fused:
-            binding.pa_decode_append(o, d_q, d_key, d_value, kc, vc, d_slots, d_tables, d_lens,
-                                     mcl, wl.scale, ws, stream=stream)
+            append_step(o, d_q, d_key, d_value, d_slots, d_tables, d_lens)
         else:
             write_step(d_key, d_value, d_slots)
             decode_step(o, d_q, d_tables, d_lens)
@@ -576,7 +583,7 @@ def run_gpu(args):
         roof_bytes = accounting.decode_unique_bytes(wl.block_tables, wl.context_lens, h, d,
                                                     wl.block_size)
     if fused:  # the fused launch also writes each new K and V row to the cache
-        roof_bytes += 2 * b * h * d * 2
+        roof_bytes += 2 * b * h * (d + 8) if int8 else 2 * b * h * d * 2
     step_bytes = dec_bytes + (b * h * (2 * d * 2 + 2 * (d + 8)) if int8
                               else accounting.cache_write_bytes(b, h, d))
     if pairs is not None:
@@ -596,7 +603,8 @@ def run_gpu(args):
         kv_bytes = dec_bytes
         desc.update({
             "step": ("pa_copy_blocks + " if pairs is not None else "")
-                    + (f"pa_decode_append (cache write of {b} tokens fused into the decode)"
+                    + (f"pa_decode_append{'_int8' if int8 else ''} (cache write of {b} tokens "
+                       f"fused into the decode)"
                        if fused else f"pa_reshape_and_cache({b} tokens) + pa_decode"),
             "l2": f"inputs larger than L2: {kv_bytes / 1e9:.2f} GB of K/V read per step "
                   f"vs {L2_BYTES / 2**20:.0f} MiB L2 (no flush)",
@@ -626,7 +634,7 @@ def run_gpu(args):
                 "kernel": "paged_decode_kernel" + ("<int8>" if int8 else ""), "bound": "hbm",
                 "achieved": achieved,
                 "peak": peak, "peak_kind": f"{peak_kind} (hbm_gbs)", "unit": "GB/s",
-                "frac": achieved / peak, "traffic": _recorded_traffic(desc["workload"], "pa_decode_append" if fused else "pa_decode"),
+                "frac": achieved / peak, "traffic": None if int8 else _recorded_traffic(desc["workload"], "pa_decode_append" if fused else "pa_decode"),
                 "algorithmic_bytes_per_launch": roof_bytes,
                 "logical_bytes_per_launch": dec_bytes,
             },

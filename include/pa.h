@@ -223,6 +223,28 @@ PA_API pa_status pa_decode_int8(void *out, const void *q, const void *k_codes,
                                 pa_stream_t stream);
 
 /*
+ * pa_decode_append over the int8 cache: one launch that quantizes each
+ * sequence's new K/V row (key, value [num_seqs, H, D] fp16, exactly as
+ * pa_reshape_and_cache_int8 does), writes its codes and (s, z) to
+ * slot_mapping[b] (int64, device; negative = nothing to append) and decodes
+ * the sequence over its context including that row.  The slot must be the
+ * one the block table gives position context_lens[b] - 1, else
+ * PA_DEVERR_SLOT is recorded (a slot outside the pool is not written).
+ * Outputs and cache contents equal those of pa_reshape_and_cache_int8
+ * followed by pa_decode_int8.  Other arguments, layouts, ownership and
+ * errors as pa_decode_int8.
+ */
+PA_API pa_status pa_decode_append_int8(void *out, const void *q, const void *key,
+                                       const void *value, void *k_codes, void *v_codes,
+                                       void *k_params, void *v_params,
+                                       const int64_t *slot_mapping, const int32_t *block_tables,
+                                       int max_blocks_per_seq, const int32_t *context_lens,
+                                       int max_context_len, int num_seqs, int num_heads,
+                                       int head_dim, int block_size, int num_blocks, float scale,
+                                       void *workspace, size_t workspace_bytes,
+                                       pa_stream_t stream);
+
+/*
  * Copy-on-write copy of whole blocks of any per-block byte size (use it for
  * the int8 codes and their parameter arrays): for each (src, dst) pair, the
  * block_bytes bytes of block src are copied to block dst of `cache`

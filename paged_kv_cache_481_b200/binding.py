@@ -32,6 +32,7 @@ EXPORTED = ("pa_reshape_and_cache", "pa_decode_workspace_size", "pa_decode_works
             "pa_bm_create", "pa_bm_destroy", "pa_bm_num_free", "pa_bm_refcount",
             "pa_bm_add_sequence", "pa_bm_fork", "pa_bm_free_sequence", "pa_bm_append_slots",
             "pa_bm_block_tables", "pa_reshape_and_cache_int8", "pa_decode_int8",
+            "pa_decode_append_int8",
             "pa_copy_blocks_raw", "pa_prefill", "pa_swap_blocks", "pa_bm_create_with_swap",
             "pa_bm_num_free_cpu", "pa_bm_cpu_refcount", "pa_bm_is_swapped", "pa_bm_swap_out",
             "pa_bm_swap_in", "pa_decode_append", "pa_decode_grouped_workspace_size",
@@ -108,6 +109,9 @@ def load(path: str | None = None):
         lib.pa_decode_append.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, i32, vp, i32, i32, i32, i32,
                                          i32, i32, ctypes.c_float, vp, sz, vp]
         lib.pa_decode_append.restype = i32
+        lib.pa_decode_append_int8.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, i32, vp, i32,
+                                              i32, i32, i32, i32, i32, ctypes.c_float, vp, sz, vp]
+        lib.pa_decode_append_int8.restype = i32
         lib.pa_swap_blocks.argtypes = [vp, vp, sz, vp, i32, i32, i32, vp]
         lib.pa_swap_blocks.restype = i32
         lib.pa_bm_create_with_swap.argtypes = [i32, i32, i32]
@@ -229,6 +233,32 @@ def pa_decode_append(out, q, key, value, k_cache, v_cache, slot_mapping, block_t
                                    b, h, d, bs, nb, float(scale), _ptr(workspace),
                                    workspace.numel() * workspace.element_size(), _stream(stream)),
            "pa_decode_append")
+
+
+def pa_decode_append_int8(out, q, key, value, k_codes, v_codes, k_params, v_params, slot_mapping,
+                          block_tables, context_lens, max_context_len, scale, workspace,
+                          stream=None):
+    """pa_decode_append over the int8 cache: each new K/V row is quantized
+    into its slot and the decode sees it, in one launch."""
+    b, h, d = q.shape
+    nb, hk, bs, dk = k_codes.shape
+    assert q.dtype == out.dtype == key.dtype == value.dtype == torch.float16
+    assert k_codes.dtype == v_codes.dtype == torch.uint8 and v_codes.shape == k_codes.shape
+    assert out.shape == q.shape == key.shape == value.shape and (hk, dk) == (h, d)
+    assert k_params.shape == v_params.shape == (nb, h, bs, 2)
+    assert k_params.dtype == v_params.dtype == torch.float32
+    assert slot_mapping.dtype == torch.int64 and slot_mapping.numel() == b
+    assert block_tables.dtype == torch.int32 and block_tables.dim() == 2
+    assert context_lens.dtype == torch.int32 and context_lens.numel() == b
+    _check(load().pa_decode_append_int8(_ptr(out), _ptr(q), _ptr(key), _ptr(value), _ptr(k_codes),
+                                        _ptr(v_codes), _ptr(k_params), _ptr(v_params),
+                                        _ptr(slot_mapping), _ptr(block_tables),
+                                        block_tables.shape[1], _ptr(context_lens),
+                                        int(max_context_len), b, h, d, bs, nb, float(scale),
+                                        _ptr(workspace),
+                                        workspace.numel() * workspace.element_size(),
+                                        _stream(stream)),
+           "pa_decode_append_int8")
 
 
 def new_grouped_workspace(num_seqs, num_heads, head_dim, max_blocks_per_seq, device="cuda"):

@@ -9,6 +9,7 @@
 
 #include "../../include/pa.h"
 #include "ptx.cuh"
+#include "quant.cuh"
 
 namespace pa {
 
@@ -46,11 +47,8 @@ __global__ void __launch_bounds__(256) reshape_and_cache_kernel(
 
 // Cache write into the int8 cache (brentwoodlivery.com 5.3.18: affine
 // quantization with one (s, z) per group, here per (token, head) row of D
-// values, b = 8): s = (r_max - r_min) / 255, z = round(-r_min / s),
-// q = clamp(round(r / s) + z, 0, 255), all decisions in fp32 with IEEE
-// division and round-half-to-even.  A row with no spread (all values c) uses
-// s = |c| (1 when c = 0) so it reconstructs exactly.  One warp per (token,
-// head) row; grid (num_tokens, ceil(H / 4), 2): z = 0 writes K, 1 writes V.
+// values, b = 8; quantize_row_warp).  One warp per (token, head) row; grid
+// (num_tokens, ceil(H / 4), 2): z = 0 writes K, 1 writes V.
 template <int D>
 __global__ void __launch_bounds__(128) reshape_and_cache_int8_kernel(
     const __half *__restrict__ key, const __half *__restrict__ value, uint8_t *__restrict__ k_codes,
@@ -79,27 +77,8 @@ __global__ void __launch_bounds__(128) reshape_and_cache_int8_kernel(
 #pragma unroll
     for (int e = 0; e < E; ++e)
         x[e] = __half2float(src[e]);
-    float rmin = x[0], rmax = x[0];
-#pragma unroll
-    for (int e = 1; e < E; ++e) {
-        rmin = fminf(rmin, x[e]);
-        rmax = fmaxf(rmax, x[e]);
-    }
-#pragma unroll
-    for (int off = 16; off >= 1; off >>= 1) {
-        rmin = fminf(rmin, __shfl_xor_sync(kFullMask, rmin, off));
-        rmax = fmaxf(rmax, __shfl_xor_sync(kFullMask, rmax, off));
-    }
-    float sc = (rmax - rmin) / 255.0f;
-    if (sc == 0.0f)
-        sc = rmax != 0.0f ? fabsf(rmax) : 1.0f;
-    const float z = rintf(-rmin / sc);
-    uint32_t packed = 0;
-#pragma unroll
-    for (int e = 0; e < E; ++e) {
-        const float q = fminf(fmaxf(rintf(x[e] / sc) + z, 0.0f), 255.0f);
-        packed |= uint32_t(q) << (8 * e);
-    }
+    float sc, z;
+    const uint32_t packed = quantize_row_warp<E>(x, sc, z);
     const int64_t row = (slot / block_size) * num_heads * block_size + int64_t(h) * block_size +
                         slot % block_size;
     uint8_t *dst = (is_v ? v_codes : k_codes) + row * D + lane * E;

@@ -236,6 +236,23 @@ pa_status pa_decode_append(void *out, const void *q, const void *key, const void
                          key, value, slot_mapping);
 }
 
+pa_status pa_decode_append_int8(void *out, const void *q, const void *key, const void *value,
+                                void *k_codes, void *v_codes, void *k_params, void *v_params,
+                                const int64_t *slot_mapping, const int32_t *block_tables,
+                                int max_blocks_per_seq, const int32_t *context_lens,
+                                int max_context_len, int num_seqs, int num_heads, int head_dim,
+                                int block_size, int num_blocks, float scale, void *workspace,
+                                size_t workspace_bytes, pa_stream_t stream)
+{
+    if (num_seqs > 0 && (!key || !value || !slot_mapping || !aligned16(key) || !aligned16(value) ||
+                         (reinterpret_cast<uintptr_t>(slot_mapping) & 7u)))
+        return PA_ERR_INVALID_ARG;
+    return decode_common(out, q, k_codes, v_codes, k_params, v_params, true, block_tables,
+                         max_blocks_per_seq, context_lens, max_context_len, num_seqs, num_heads,
+                         head_dim, block_size, num_blocks, scale, workspace, workspace_bytes, stream,
+                         key, value, slot_mapping);
+}
+
 pa_status pa_decode_int8(void *out, const void *q, const void *k_codes, const void *v_codes,
                          const void *k_params, const void *v_params, const int32_t *block_tables,
                          int max_blocks_per_seq, const int32_t *context_lens, int max_context_len,

@@ -54,6 +54,7 @@
 #include <cstdint>
 
 #include "ptx.cuh"
+#include "quant.cuh"
 
 namespace pa {
 
@@ -424,9 +425,8 @@ __device__ __forceinline__ void issue_tile(const DecodeParams &p, const DecodeEx
     // the last tile of a unit whose sequence appends a token: its last row
     // comes from the new-token input instead (append_new_row)
     int nf = nv;
-    if constexpr (!kInt8)
-        if (x.new_slots && cur.i == cur.nt - 1 && x.new_slots[cur.b] >= 0)
-            nf = nv - 1;
+    if (x.new_slots && cur.i == cur.nt - 1 && x.new_slots[cur.b] >= 0)
+        nf = nv - 1;
     // an id outside the pool is recorded and its rows are not fetched
     bool ok[Sh::kMaxIds];
 #pragma unroll
@@ -511,6 +511,67 @@ __device__ __forceinline__ void append_new_row(const DecodeParams &p, const Deco
             const size_t row = (size_t(slot / bs) * p.num_heads + cur.h) * bs + size_t(slot % bs);
             uint4 *cache = reinterpret_cast<uint4 *>(const_cast<void *>(is_v ? p.v_cache : p.k_cache));
             cache[row * kChunks + c] = val;
+        }
+    }
+    fence_proxy_async_smem();  // before a later bulk copy overwrites the stage
+    __syncwarp();
+}
+
+// The same for the int8 cache, whole warp, once the tile's copies have
+// landed (the (s, z) copy of the other rows is rounded up to an even row
+// count, so it may cover this row's place in the stage): the new K and V
+// rows are quantized exactly as the int8 cache write does
+// (quantize_row_warp), their codes and (s, z) put into the stage and written
+// to the cache slot.
+template <int D, class Sm>
+__device__ __forceinline__ void append_new_row_int8(const DecodeParams &p, const DecodeExtras &x,
+                                                    const TileMeta &mt, unsigned char *stage_buf,
+                                                    int lane)
+{
+    using Sh = DecodeShape<D, true>;
+    constexpr int E = D / 32;  // values per lane
+    const int64_t slot = x.new_slots[mt.b];
+    if (slot < 0)
+        return;
+    const int bs = p.block_size;
+    const int pos = mt.len - 1;
+    const int r = pos - mt.i * Sh::kTokens;  // the row's place in the stage
+    const bool in_pool = slot < int64_t(p.num_blocks) * bs;
+    if (lane == 0) {
+        const int id = p.block_tables[size_t(mt.b) * p.max_blocks_per_seq + pos / bs];
+        if (!in_pool || slot != int64_t(id) * bs + pos % bs)
+            raise_device_error(kErrSlot);
+    }
+    const size_t src_row = size_t(mt.b) * p.num_heads + mt.h;
+    const size_t row = in_pool ? (size_t(slot / bs) * p.num_heads + mt.h) * bs + size_t(slot % bs) : 0;
+#pragma unroll
+    for (int kv = 0; kv < 2; ++kv) {
+        const __half *src = (kv ? x.new_v : x.new_k) + src_row * D + lane * E;
+        float v[E];
+#pragma unroll
+        for (int e = 0; e < E; ++e)
+            v[e] = __half2float(src[e]);
+        float sc, z;
+        const uint32_t packed = quantize_row_warp<E>(v, sc, z);
+        unsigned char *codes = stage_buf + (kv ? Sm::kOffV : 0u) + uint32_t(r) * Sh::kRowBytes +
+                               uint32_t(lane * E);
+        uint8_t *cache = static_cast<uint8_t *>(const_cast<void *>(kv ? p.v_cache : p.k_cache)) +
+                         row * D + lane * E;
+        if constexpr (E == 4) {
+            *reinterpret_cast<uint32_t *>(codes) = packed;
+            if (in_pool)
+                *reinterpret_cast<uint32_t *>(cache) = packed;
+        } else {
+            *reinterpret_cast<uint16_t *>(codes) = uint16_t(packed);
+            if (in_pool)
+                *reinterpret_cast<uint16_t *>(cache) = uint16_t(packed);
+        }
+        if (lane == 0) {
+            *reinterpret_cast<float2 *>(stage_buf + (kv ? Sm::kOffVP : Sm::kOffKP) + uint32_t(r) * 8u) =
+                make_float2(sc, z);
+            if (in_pool)
+                reinterpret_cast<float2 *>(const_cast<float *>(kv ? p.v_params : p.k_params))[row] =
+                    make_float2(sc, z);
         }
     }
     fence_proxy_async_smem();  // before a later bulk copy overwrites the stage
@@ -779,6 +840,9 @@ __global__ void __launch_bounds__(NW * 32) paged_decode_kernel(const DecodeParam
         const TileMeta mt = my_meta[stage];
         const int nt = (mt.len + T - 1) / T;
         const int nv = min(T, mt.len - mt.i * T);
+        if constexpr (kInt8)
+            if (x.new_slots && mt.i == nt - 1)
+                append_new_row_int8<D, Sm>(p, x, mt, my_buf + size_t(stage) * Sm::kStageBytes, lane);
         const unsigned char *buf = my_buf + size_t(stage) * Sm::kStageBytes;
         if (mt.i == 0 || mt.k == lo) {  // first tile of a segment: fresh state, new q
             const uint4 *qs = reinterpret_cast<const uint4 *>(buf + Sm::kOffQ);

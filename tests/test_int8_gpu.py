@@ -165,3 +165,88 @@ def test_int8_llama13b_decode_config_full():
                                    wl.context_lens, wl.scale)
     assert max_abs_err(out, ref) <= ATOL
     assert binding.pa_get_last_device_error() == 0
+
+
+def _pool_without_newest(wl, skip_slots):
+    """int8 pool holding every context token except those written to
+    `skip_slots` (the rows the fused call appends)."""
+    keys, values, slots = workloads.all_token_writes(wl)
+    keep = torch.from_numpy(~np.isin(slots, skip_slots))
+    kc, vc, kp, vp = _empty_int8(wl)
+    binding.pa_reshape_and_cache_int8(keys[keep.to(keys.device)].cuda(),
+                                      values[keep.to(values.device)].cuda(), kc, vc, kp, vp,
+                                      torch.from_numpy(slots[keep.numpy()]).cuda())
+    return (kc, vc, kp, vp), (keys, values, slots)
+
+
+def _fused_int8(wl, pool, slots):
+    kc, vc, kp, vp = pool
+    q = wl.q.cuda()
+    out = torch.empty_like(q)
+    ws = binding.new_workspace(wl.num_seqs, wl.num_heads, wl.head_dim, wl.max_context_len)
+    binding.pa_decode_append_int8(out, q, wl.new_key.cuda(), wl.new_value.cuda(), kc, vc, kp, vp,
+                                  slots, torch.from_numpy(np.ascontiguousarray(wl.block_tables)).cuda(),
+                                  torch.from_numpy(wl.context_lens).cuda(), wl.max_context_len,
+                                  wl.scale, ws)
+    torch.cuda.synchronize()
+    return out
+
+
+def _same_bits(a, b):
+    return torch.equal(a.contiguous().view(torch.uint8), b.contiguous().view(torch.uint8))
+
+
+@pytest.mark.parametrize("seed,d,bs,lens", CASES)
+def test_int8_fused_append_equals_write_then_decode(seed, d, bs, lens):
+    """pa_decode_append_int8 quantizes each sequence's newest row into its
+    slot and decodes with it: the same cache bits and output bits as
+    pa_reshape_and_cache_int8 of every token followed by pa_decode_int8, and
+    the oracle's int8 write + decode within the tolerance."""
+    wl = workloads.make_random(seed, lens, num_heads=5, head_dim=d, block_size=bs,
+                               keep_logical=False, keep_tokens=True, pool_factor=2.0)
+    pool, (keys, values, slots) = _pool_without_newest(wl, wl.slot_mapping)
+    out = _fused_int8(wl, pool, torch.from_numpy(wl.slot_mapping).cuda())
+    assert binding.pa_get_last_device_error() == 0
+    full, _ = _gpu_int8_pool(wl)
+    out2 = _decode(wl, full)
+    assert _same_bits(out, out2)
+    for got, want in zip(pool, full):
+        assert _same_bits(got, want)
+    ref_pool = _oracle_int8_pool(wl, keys, values, slots)
+    ref = oracle.paged_decode_int8(wl.q.numpy(), *ref_pool, wl.block_tables, wl.context_lens,
+                                   wl.scale)
+    assert max_abs_err(out, ref) <= ATOL
+
+
+def test_int8_fused_append_mixed_batch_and_bad_slot():
+    """Half the sequences append nothing (slot -1; their newest row is in the
+    cache already); then a slot that is not position L - 1's is reported."""
+    wl = workloads.make_random(209, [40, 1, 95, 33, 64, 200], num_heads=3, head_dim=128,
+                               block_size=16, keep_logical=False, keep_tokens=True, pool_factor=2.0)
+    slots = wl.slot_mapping.copy()
+    slots[::2] = -1
+    pool, _ = _pool_without_newest(wl, wl.slot_mapping[1::2])
+    out = _fused_int8(wl, pool, torch.from_numpy(slots).cuda())
+    assert binding.pa_get_last_device_error() == 0
+    full, _ = _gpu_int8_pool(wl)
+    assert _same_bits(out, _decode(wl, full))
+    for got, want in zip(pool, full):
+        assert _same_bits(got, want)
+    bad = wl.slot_mapping.copy()
+    bad[2] -= 1                       # the slot of position L - 2
+    _fused_int8(wl, pool, torch.from_numpy(bad).cuda())
+    assert binding.pa_get_last_device_error() == binding.PA_DEVERR_SLOT
+
+
+@pytest.mark.slow
+def test_int8_fused_append_llama13b_full():
+    wl = workloads.make_workload(2, device="cuda", keep_tokens=True)
+    pool, (keys, values, slots) = _pool_without_newest(wl, wl.slot_mapping)
+    out = _fused_int8(wl, pool, torch.from_numpy(wl.slot_mapping).cuda())
+    assert binding.pa_get_last_device_error() == 0
+    ref_pool = _oracle_int8_pool(wl, keys, values, slots)
+    for got, want in zip(pool, ref_pool):
+        assert np.array_equal(got.cpu().numpy().view(np.uint8), np.asarray(want).view(np.uint8))
+    ref = oracle.paged_decode_int8(wl.q.cpu().numpy(), *ref_pool, wl.block_tables,
+                                   wl.context_lens, wl.scale)
+    assert max_abs_err(out, ref) <= ATOL
