@@ -1,6 +1,8 @@
 """Benchmark of the paged decode path on B200.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--workload C] [--block-size BS]
+    python bench.py --kv-dtype int8 ...      # the same step over the int8 cache
+    python bench.py --path prefill ...       # prompt cache write + pa_prefill, TFLOP/s
     python bench.py --impl reference ...     # the fp64 CPU oracle, same metric
 
 One step = one decode iteration of the whole hot path over one batch: the
