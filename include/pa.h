@@ -223,7 +223,10 @@ PA_API pa_status pa_decode_int8(void *out, const void *q, const void *k_codes,
                                 pa_stream_t stream);
 
 /*
- * pa_decode_append over the int8 cache: one launch that quantizes each
+ * pa_decode_append over the int8 cache (the new token goes into the next
+ * free slot: polomodov.tech "vLLM and PagedAttention", slide 11; low-bit
+ * KV cache with affine (s, z) per row: brentwoodlivery.com 5.3.18): one
+ * launch that quantizes each
  * sequence's new K/V row (key, value [num_seqs, H, D] fp16, exactly as
  * pa_reshape_and_cache_int8 does), writes its codes and (s, z) to
  * slot_mapping[b] (int64, device; negative = nothing to append) and decodes
