@@ -78,6 +78,8 @@ def _run(c, prefix_lens=None):
     (504, [4, 4], [33, 17], 100, 8),
     (505, [2, 3], [5, 3], 300, 64),
     (506, [130, 3], [4, 2], 20, 16),                  # a group larger than one query tile
+    (508, [3, 5], [3, 2], 150, 128),                  # blocks as large as a context tile
+    (509, [1, 1, 2], [6, 1, 3], 33, 32),              # single-member groups
 ])
 def test_grouped_equals_plain_decode(seed, sizes, prefix_blocks, max_tail, bs):
     c = _groups(seed, sizes, prefix_blocks, max_tail, bs)

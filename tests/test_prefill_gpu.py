@@ -53,6 +53,8 @@ def _run(seed, lens, n_new, bs, h=4, d=128, growth=0.0):
     (305, 64, [513, 70], [256, 3]),
     (306, 128, [384, 260], [384, 100]),
     (307, 16, [50, 1, 64, 9], [0, 1, 64, 0]),             # sequences with no new tokens
+    (308, 8, [700, 129, 256], [3, 128, 255]),            # chunks ending mid-block, bs 8
+    (309, 128, [1000, 385], [600, 257]),                  # several items, 128-token blocks
 ])
 def test_prefill_matches_oracle(seed, bs, lens, n_new):
     out, ref = _run(seed, lens, n_new, bs)
