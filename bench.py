@@ -342,6 +342,27 @@ def run_reference(args):
     return 0
 
 
+def _init_ranks(args):
+    """This process's rank on its GPU (one process per GPU; NCCL process group
+    with a short timeout when there are several), and the library loaded."""
+    import torch
+    import torch.distributed as dist
+    from paged_kv_cache_481_b200 import binding, build
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world != args.gpus:
+        raise SystemExit(f"--gpus {args.gpus} but WORLD_SIZE={world}")
+    torch.cuda.set_device(local)
+    if world > 1:
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+    build.build()
+    binding.load()
+    return world, rank, local
+
+
 def pipelined_e2e(parts, out_like, step, stream, warmup, steps, world):
     """End-to-end timing through the public API with host buffers: each
     step's inputs (`parts`, packed in one pinned host buffer) are copied to
@@ -426,20 +447,9 @@ def pipelined_e2e(parts, out_like, step, stream, warmup, steps, world):
 def run_gpu(args):
     import torch
     import torch.distributed as dist
-    from paged_kv_cache_481_b200 import accounting, binding, build, workloads
+    from paged_kv_cache_481_b200 import accounting, binding, workloads
 
-    world = int(os.environ.get("WORLD_SIZE", "1"))
-    rank = int(os.environ.get("RANK", "0"))
-    local = int(os.environ.get("LOCAL_RANK", "0"))
-    if world != args.gpus:
-        raise SystemExit(f"--gpus {args.gpus} but WORLD_SIZE={world}")
-    torch.cuda.set_device(local)
-    if world > 1:
-        import datetime
-        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
-                                device_id=torch.device("cuda", local))
-    build.build()
-    binding.load()
+    world, rank, local = _init_ranks(args)
 
     cfg = args.workload
     int8 = args.kv_dtype == "int8"
@@ -709,20 +719,9 @@ def run_prefill(args):
     pa_prefill (causal multi-query attention on the tensor cores)."""
     import torch
     import torch.distributed as dist
-    from paged_kv_cache_481_b200 import binding, build
+    from paged_kv_cache_481_b200 import binding
 
-    world = int(os.environ.get("WORLD_SIZE", "1"))
-    rank = int(os.environ.get("RANK", "0"))
-    local = int(os.environ.get("LOCAL_RANK", "0"))
-    if world != args.gpus:
-        raise SystemExit(f"--gpus {args.gpus} but WORLD_SIZE={world}")
-    torch.cuda.set_device(local)
-    if world > 1:
-        import datetime
-        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
-                                device_id=torch.device("cuda", local))
-    build.build()
-    binding.load()
+    world, rank, local = _init_ranks(args)
     dev = torch.device("cuda", local)
 
     b, length, h, d = args.prompts, args.prompt_len, 40, 128
