@@ -178,6 +178,9 @@ PA_API pa_status pa_copy_blocks(void *k_cache, void *v_cache, const int64_t *blo
  *     cudaMemsetAsync on `stream`.
  *   - All calls on a device share the one array: calls that overlap on the
  *     GPU (other streams, other host threads) race and give wrong results.
+ *   - The looked-up address is kept per device ordinal for the life of the
+ *     process: do not use the library across a cudaDeviceReset (the same
+ *     holds for the device error word and the prefill scheduling counters).
  */
 PA_API pa_status pa_decode_no_alloc(void *out, const void *q, const void *k_cache,
                                     const void *v_cache, const int32_t *block_tables,

@@ -160,9 +160,20 @@ def _ptr(t: torch.Tensor | None) -> ctypes.c_void_p:
         return ctypes.c_void_p(None)
     if not t.is_cuda:
         raise ValueError("libpa takes device tensors")
+    _on_current_device(t)
     if not t.is_contiguous():
         raise ValueError("libpa takes contiguous tensors")
     return ctypes.c_void_p(t.data_ptr())
+
+
+def _on_current_device(t: torch.Tensor):
+    """The library launches on the current device and keeps per-device state
+    (error word, static scratch, scheduling counters) for it, so a tensor that
+    lives on another GPU would hand its kernels a foreign pointer."""
+    cur = torch.cuda.current_device()
+    if t.device.index != cur:
+        raise ValueError(f"tensor on cuda:{t.device.index} but the current device is "
+                         f"cuda:{cur}; call under torch.cuda.device({t.device.index})")
 
 
 def pa_reshape_and_cache(key, value, k_cache, v_cache, slot_mapping, stream=None):
@@ -371,6 +382,8 @@ def _ptr_addressable(t: torch.Tensor) -> ctypes.c_void_p:
     """Device tensor, or page-locked host tensor the device can address."""
     if not (t.is_cuda or t.is_pinned()):
         raise ValueError("pa_swap_blocks takes device or pinned host tensors")
+    if t.is_cuda:
+        _on_current_device(t)
     if not t.is_contiguous():
         raise ValueError("libpa takes contiguous tensors")
     return ctypes.c_void_p(t.data_ptr())

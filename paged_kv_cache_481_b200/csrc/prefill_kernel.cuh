@@ -27,8 +27,7 @@
 //     thread = TMEM lane): read the S row back (all 128 columns, one wait),
 //     causal mask, online softmax in the
 //     log2 domain, P as fp16 into TMEM (the row sum l is taken from P before
-//     its fp16 rounding); a share of the exp2 can run as a polynomial on the
-//     FMA pipes instead of the special-function unit (kExp2FmaPairsPer8).  Only warps holding a diagonal or context-end tile
+//     its fp16 rounding).  Only warps holding a diagonal or context-end tile
 //     pay for the mask.  The running max is only moved when
 //     it grows by more than 2^8 (in base-2 exponent units); then the warp
 //     rescales its O rows and l in TMEM.  Otherwise P is taken against the
@@ -92,14 +91,8 @@ constexpr uint32_t kPrefillSmem = kOffRing + kRing * kTileBytes + 1024;  // + 10
 constexpr int kLoadWarp = 8, kMmaWarp = 9;
 constexpr int kPrefillThreads = 10 * 32;
 constexpr uint32_t kTmemCols = 512;
-#ifndef PA_PREFILL_EXP2_HALF
-#define PA_PREFILL_EXP2_HALF 0
-#endif
-// exp2 of the scores on fp16 pairs (one special-function instruction per
-// pair) instead of fp32 singles
-constexpr bool kExp2Half = PA_PREFILL_EXP2_HALF != 0;
 // move the reference max only past this growth (base-2 units)
-constexpr float kRescaleLog2 = kExp2Half ? 2.0f : 8.0f;
+constexpr float kRescaleLog2 = 8.0f;
 constexpr int kItemRing = 2;          // items handed from the load warp to the other roles
 constexpr int kItemConsumers = 1 + 8; // the MMA thread and the eight softmax warps
 constexpr int kGroupHB = 32;          // (head, sequence) units per scheduling group
@@ -146,81 +139,6 @@ __device__ __forceinline__ float ex2_approx(float x)
     return y;
 }
 
-__device__ __forceinline__ uint64_t pack2(float lo, float hi)
-{
-    uint64_t d;
-    asm("mov.b64 %0, {%1, %2};" : "=l"(d) : "f"(lo), "f"(hi));
-    return d;
-}
-
-__device__ __forceinline__ void unpack2(uint64_t v, float &lo, float &hi)
-{
-    asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(v));
-}
-
-// two fp32 lanes at once: a * b + c, a + b
-__device__ __forceinline__ uint64_t fma2(uint64_t a, uint64_t b, uint64_t c)
-{
-    uint64_t d;
-    asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
-    return d;
-}
-
-__device__ __forceinline__ uint64_t add2(uint64_t a, uint64_t b)
-{
-    uint64_t d;
-    asm("add.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
-    return d;
-}
-
-// 2^x for a pair of scores on the FMA pipes, relieving the special-function
-// unit (which alone would need as many cycles per tile as the tensor core).
-// Cody-Waite range reduction x = j + f, j = floor(x) exact in fp32 (adding
-// 1.5 * 2^23 with round-down leaves floor(x) in the low mantissa bits), and a
-// degree-3 minimax polynomial p(f) ~ 2^f on [0, 1) (max relative error
-// 7.5e-5, fitted by Remez exchange in paged_kv_cache_481_b200/exp2_poly.py);
-// 2^j is added to p's exponent field.  x is clamped below at -126 (the
-// result is then ~2^-126, which the fp16 weight rounds to 0; at -127 the
-// exponent field of p(0) < 1 would wrap).
-constexpr float kExp2C0 = 0.99992521856271543f;
-constexpr float kExp2C1 = 0.69583354049475277f;
-constexpr float kExp2C2 = 0.22606715542748301f;
-constexpr float kExp2C3 = 0.07802452264047964f;
-constexpr float kExp2Magic = 12582912.0f;  // 1.5 * 2^23
-
-__device__ __forceinline__ uint64_t add2_rm(uint64_t a, uint64_t b)
-{
-    uint64_t d;
-    asm("add.rm.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
-    return d;
-}
-
-__device__ __forceinline__ void ex2_poly2(float x0, float x1, float &y0, float &y1)
-{
-    const uint64_t xx = pack2(fmaxf(x0, -126.f), fmaxf(x1, -126.f));
-    const uint64_t t = add2_rm(xx, pack2(kExp2Magic, kExp2Magic));      // magic + floor(x)
-    const uint64_t j = add2(t, pack2(-kExp2Magic, -kExp2Magic));          // floor(x), exact
-    const uint64_t f = fma2(j, pack2(-1.f, -1.f), xx);                    // x - floor(x) in [0, 1)
-    uint64_t q = fma2(pack2(kExp2C3, kExp2C3), f, pack2(kExp2C2, kExp2C2));
-    q = fma2(q, f, pack2(kExp2C1, kExp2C1));
-    q = fma2(q, f, pack2(kExp2C0, kExp2C0));
-    float q0, q1, t0, t1;
-    unpack2(q, q0, q1);
-    unpack2(t, t0, t1);
-    // (magic + j) << 23 keeps exactly j << 23 (mod 2^32): 2^j into the exponent
-    y0 = __uint_as_float(__float_as_uint(q0) + (__float_as_uint(t0) << 23));
-    y1 = __uint_as_float(__float_as_uint(q1) + (__float_as_uint(t1) << 23));
-}
-
-// Pairs out of every 8 whose exp2 goes to the FMA pipes.  Measured on the
-// 13B prefill cases: 3 of 8 was 2-6 % slower than 0 (the special-function
-// unit is not yet the limit there), so the polynomial stays off for now.
-constexpr int kExp2FmaPairsPer8 = 0;
-__host__ __device__ constexpr bool exp2_on_fma(int e)
-{
-    return (e & 7) < kExp2FmaPairsPer8;
-}
-
 // One S tile row in registers: all 128 scores of this thread's TMEM lane,
 // loaded with one wait.
 struct ScoreRow {
@@ -255,35 +173,9 @@ __device__ __forceinline__ float score_row_max(const ScoreRow &r, int lim)
     return fmaxf(fmaxf(m[0], m[1]), fmaxf(m[2], m[3]));
 }
 
-// 2^x of two fp32 arguments in one special-function instruction at half
-// precision: the arguments are rounded to fp16 (with the reference max moved
-// by at most 2^2, |x| <= 2 for the weights that matter, so the argument
-// rounding costs at most 2^-10 relative) and the result is the fp16 pair P
-// that the tensor core takes anyway.
-__device__ __forceinline__ uint32_t ex2_half2(float x0, float x1)
-{
-    uint32_t in, out;
-    asm("cvt.rn.f16x2.f32 %0, %1, %2;" : "=r"(in) : "f"(x1), "f"(x0));
-    asm("ex2.approx.f16x2 %0, %1;" : "=r"(out) : "r"(in));
-    return out;
-}
-
-// acc += the two fp16 halves of v (exact products with 1.0, fp32 adds)
-__device__ __forceinline__ void add_half2_f32(uint32_t v, float &acc0, float &acc1)
-{
-    asm("{\n\t.reg .f16 lo, hi, one;\n\t"
-        "mov.b16 one, 0x3C00;\n\t"
-        "mov.b32 {lo, hi}, %2;\n\t"
-        "fma.rn.f32.f16 %0, lo, one, %0;\n\t"
-        "fma.rn.f32.f16 %1, hi, one, %1;\n\t}"
-        : "+f"(acc0), "+f"(acc1)
-        : "r"(v));
-}
-
 // P = 2^(c * s - m) of the row, as fp16 pairs written into TMEM over the
-// first 64 columns of S; returns the row sum of P (fp32; of the fp16 values
-// with the half-precision exponential, else before the fp16 rounding).
-// With kMasked, columns >= lim give P = 0.
+// first 64 columns of S; returns the row sum of P (fp32, before the fp16
+// rounding).  With kMasked, columns >= lim give P = 0.
 template <bool kMasked>
 __device__ __forceinline__ float write_p_row(uint32_t tS, const ScoreRow &r, int lim, float c,
                                              float m)
@@ -297,29 +189,16 @@ __device__ __forceinline__ float write_p_row(uint32_t tS, const ScoreRow &r, int
             const int i = cc * 32 + 2 * e;
             const float x0 = fmaf(__uint_as_float(r.s[i]), c, -m);
             const float x1 = fmaf(__uint_as_float(r.s[i + 1]), c, -m);
-            if (kExp2Half) {
-                uint32_t ph = ex2_half2(x0, x1);
-                if (kMasked)
-                    ph &= (i < lim ? 0x0000FFFFu : 0u) | (i + 1 < lim ? 0xFFFF0000u : 0u);
-                add_half2_f32(ph, sum[(e & 1) * 2], sum[(e & 1) * 2 + 1]);
-                pk[e] = ph;
-            } else {
-                float p0, p1;
-                if (exp2_on_fma(e)) {
-                    ex2_poly2(x0, x1, p0, p1);
-                } else {
-                    p0 = ex2_approx(x0);
-                    p1 = ex2_approx(x1);
-                }
-                if (kMasked) {
-                    p0 = i < lim ? p0 : 0.f;
-                    p1 = i + 1 < lim ? p1 : 0.f;
-                }
-                sum[(e & 1) * 2] += p0;
-                sum[(e & 1) * 2 + 1] += p1;
-                const __half2 ph = __floats2half2_rn(p0, p1);
-                pk[e] = *reinterpret_cast<const uint32_t *>(&ph);
+            float p0 = ex2_approx(x0);
+            float p1 = ex2_approx(x1);
+            if (kMasked) {
+                p0 = i < lim ? p0 : 0.f;
+                p1 = i + 1 < lim ? p1 : 0.f;
             }
+            sum[(e & 1) * 2] += p0;
+            sum[(e & 1) * 2 + 1] += p1;
+            const __half2 ph = __floats2half2_rn(p0, p1);
+            pk[e] = *reinterpret_cast<const uint32_t *>(&ph);
         }
         tmem_store16(tS + uint32_t(cc * 16), pk);
     }

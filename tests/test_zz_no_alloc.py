@@ -14,7 +14,7 @@ import torch
 
 from paged_kv_cache_481_b200 import binding, build, workloads
 
-from gpu_helpers import ATOL, gpu_decode, to_dev
+from gpu_helpers import ATOL, gpu_decode, max_abs_err, oracle_write_and_decode, to_dev
 
 pytestmark = pytest.mark.gpu
 
@@ -47,12 +47,15 @@ def test_matches_workspace_entry_point_on_two_calls_in_a_row():
                                block_size=16, keep_logical=False)
     t = _written(wl)
     ref = gpu_decode(wl, t)
+    exact, _, _ = oracle_write_and_decode(wl)
     for _ in range(2):
         out = _no_alloc(wl, t)
         torch.cuda.synchronize()
         err = float((out.float() - ref.float()).abs().max())
         assert err <= ATOL
         assert torch.equal(out.view(torch.int16), ref.view(torch.int16))
+        # and against the oracle, so a fault shared by both entry points shows
+        assert max_abs_err(out, exact) <= ATOL
     assert binding.pa_get_last_device_error() == 0
 
 
@@ -65,8 +68,15 @@ def test_second_call_with_other_sizes_and_the_13b_shape():
     t2 = _written(wl)
     b = _no_alloc(wl, t2)
     torch.cuda.synchronize()
-    assert float((a.float() - gpu_decode(first, t1).float()).abs().max()) <= ATOL
-    assert float((b.float() - gpu_decode(wl, t2).float()).abs().max()) <= ATOL
+    assert binding.pa_get_last_device_error() == 0
+    ref_a, ref_b = gpu_decode(first, t1), gpu_decode(wl, t2)
+    assert float((a.float() - ref_a.float()).abs().max()) <= ATOL
+    assert float((b.float() - ref_b.float()).abs().max()) <= ATOL
+    assert torch.equal(a.view(torch.int16), ref_a.view(torch.int16))
+    assert torch.equal(b.view(torch.int16), ref_b.view(torch.int16))
+    exact_a, _, _ = oracle_write_and_decode(first)
+    assert max_abs_err(a, exact_a) <= ATOL
+    assert binding.pa_get_last_device_error() == 0
 
 
 def test_sizes_past_the_static_scratch_are_rejected_before_any_launch():
