@@ -317,28 +317,30 @@ PA_API pa_status pa_prefill(void *out, const void *q, const void *k_cache, const
  * PagedAttention", 6.4.2; polomodov.tech "vLLM and PagedAttention", slides
  * 13-14: candidates share a prefix of blocks like processes after fork).
  * Same result as pa_decode over the same arguments, but each shared prefix
- * is read once per (group, head): its scores are a small matrix product on
- * the tensor cores (the members' queries against the prefix), each member's
- * own tail goes through the decode kernel, and the two parts are merged by
- * their softmax normalisers.  Three more launches than pa_decode, so it pays
- * when prefixes are long against the tails.
+ * is read from memory once per (group, head): the group's queries are scored
+ * against it together on the tensor cores, each member's own tail is scored
+ * alone, and the parts are merged by their softmax normalisers, all in one
+ * persistent kernel after a small set-up kernel.
  *   group_start [num_groups + 1] int32 (device): group g = sequences
  *     group_start[g] .. group_start[g+1] - 1; group_start[0] = 0 and
- *     group_start[num_groups] = num_seqs, nondecreasing.
+ *     group_start[num_groups] = num_seqs, nondecreasing (every sequence in
+ *     exactly one group).
  *   prefix_lens [num_groups] int32 (device): tokens shared by group g, a
  *     multiple of block_size, at most every member's context length; the
  *     members' block tables must agree on those blocks (0 = nothing shared).
- *   max_group_size: host bound on group sizes (sizes the grid).
- *   workspace: pa_decode_grouped_workspace_size(num_seqs, num_heads,
- *     head_dim, max_blocks_per_seq) bytes, 16-byte aligned, zeroed once with
- *     pa_decode_workspace_init before first use (like pa_decode's).
- * head_dim must be 128, scale > 0, max_group_size <= 65535.  A prefix that
- * breaks these rules for a member is recorded (PA_DEVERR_CONTEXT_LEN, possibly
- * with PA_DEVERR_BLOCK_ID from reading past its blocks) and that member
- * decodes its whole context as its tail; group bounds outside the batch are
- * recorded and skipped.
+ *   max_group_size: host bound on group sizes (<= 65535).
+ *   workspace: pa_decode_grouped_workspace_size(num_seqs, num_groups,
+ *     num_heads, head_dim, max_context_len) bytes, 16-byte aligned; no
+ *     initialisation needed (each call clears what it uses), and one
+ *     workspace serves any smaller problem too.  Calls that share a
+ *     workspace must not overlap on the GPU.
+ * head_dim must be 128 (else PA_ERR_UNSUPPORTED), scale > 0.  A prefix that
+ * breaks these rules is recorded (PA_DEVERR_CONTEXT_LEN) and its group is
+ * decoded without a shared prefix; group bounds outside the batch are
+ * recorded and that group is skipped.
  */
-PA_API size_t pa_decode_grouped_workspace_size(int num_seqs, int num_heads, int head_dim,
+PA_API size_t pa_decode_grouped_workspace_size(int num_seqs, int num_groups, int num_heads,
+                                               int head_dim, int max_context_len,
                                                int max_blocks_per_seq);
 PA_API pa_status pa_decode_grouped(void *out, const void *q, const void *k_cache,
                                    const void *v_cache, const int32_t *block_tables,

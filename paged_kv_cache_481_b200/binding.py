@@ -101,7 +101,7 @@ def load(path: str | None = None):
         lib.pa_decode_int8.restype = i32
         lib.pa_copy_blocks_raw.argtypes = [vp, sz, vp, i32, i32, vp]
         lib.pa_copy_blocks_raw.restype = i32
-        lib.pa_decode_grouped_workspace_size.argtypes = [i32, i32, i32, i32]
+        lib.pa_decode_grouped_workspace_size.argtypes = [i32, i32, i32, i32, i32, i32]
         lib.pa_decode_grouped_workspace_size.restype = sz
         lib.pa_decode_grouped.argtypes = [vp, vp, vp, vp, vp, i32, vp, i32, vp, vp, i32, i32, i32,
                                           i32, i32, i32, i32, ctypes.c_float, vp, sz, vp]
@@ -272,17 +272,20 @@ def pa_decode_append_int8(out, q, key, value, k_codes, v_codes, k_params, v_para
            "pa_decode_append_int8")
 
 
-def new_grouped_workspace(num_seqs, num_heads, head_dim, max_blocks_per_seq, device="cuda"):
-    """Zeroed workspace for pa_decode_grouped."""
-    n = load().pa_decode_grouped_workspace_size(num_seqs, num_heads, head_dim, max_blocks_per_seq)
+def new_grouped_workspace(num_seqs, num_groups, num_heads, head_dim, max_context_len,
+                          max_blocks_per_seq, device="cuda"):
+    """Workspace for pa_decode_grouped (needs no initialisation)."""
+    n = load().pa_decode_grouped_workspace_size(num_seqs, num_groups, num_heads, head_dim,
+                                                max_context_len, max_blocks_per_seq)
     return torch.zeros(max(int(n), 16), dtype=torch.uint8, device=device)
 
 
 def pa_decode_grouped(out, q, k_cache, v_cache, block_tables, context_lens, max_context_len,
                       group_start, prefix_lens, max_group_size, scale, workspace, stream=None):
     """Decode of sequence groups sharing a block prefix: the prefix read once
-    per (group, head) on the tensor cores, tails by the decode kernel, merged.
-    Same result as pa_decode."""
+    per (group, head) and scored for the whole group on the tensor cores,
+    each member's tail scored alone, the parts merged.  Same result as
+    pa_decode."""
     b, h, d = q.shape
     nb, hk, bs, dk = k_cache.shape
     assert q.dtype == out.dtype == k_cache.dtype == v_cache.dtype == torch.float16

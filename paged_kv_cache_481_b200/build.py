@@ -2,7 +2,7 @@
 
     python -m paged_kv_cache_481_b200.build [--force] [--verbose-ptxas]
 
-The library is compiled from csrc/decode.cu, csrc/cache.cu and csrc/prefill.cu
+The library is compiled from csrc/decode.cu, csrc/cache.cu, csrc/prefill.cu and csrc/grouped.cu
 (which include the kernel headers) and csrc/block_manager.cpp (host code) for ``arch=compute_100a,code=sm_100a`` only, with the CUDA runtime linked
 statically so the .so does not depend on the toolkit's libcudart at run time.
 """
@@ -50,7 +50,7 @@ def build(force: bool = False, verbose_ptxas: bool = False) -> str:
            "-Xcompiler", "-fPIC", "-Xcompiler", "-fvisibility=hidden",
            "-cudart", "static", "-I", os.path.join(ROOT, "include"),
            "-o", tmp, os.path.join(CSRC, "decode.cu"), os.path.join(CSRC, "cache.cu"),
-           os.path.join(CSRC, "prefill.cu"),
+           os.path.join(CSRC, "prefill.cu"), os.path.join(CSRC, "grouped.cu"),
            os.path.join(CSRC, "block_manager.cpp")]
     if verbose_ptxas:
         cmd.insert(1, "-Xptxas=-v")

@@ -336,6 +336,11 @@ extern "C" pa_status pa_decode_no_alloc(void *out, const void *q, const void *k_
                      scratch, kNoAllocScratchBytes, stream);
 }
 
+size_t pa_host::decode_ticket_offset(int num_seqs, int num_heads, int head_dim)
+{
+    return workspace_layout(num_seqs, num_heads, head_dim).count_off;
+}
+
 pa_status pa_host::decode_with_lse(void *out, const void *q, const void *k_cache,
                                    const void *v_cache, const int32_t *block_tables,
                                    int max_blocks_per_seq, const int32_t *context_lens,

@@ -1,0 +1,456 @@
+// libpa, shared-prefix decode: C ABI of pa_decode_grouped.  Host code here
+// validates arguments, lays out the workspace, encodes the TMA tensor maps
+// and launches four kernels on the caller's stream:
+//   1. a one-CTA set-up kernel: the prefix work list (chunks), each member's
+//      tail table (its block-table row from the first block past the shared
+//      prefix) and tail length, zero outputs for empty contexts;
+//   2. the persistent tensor-core kernel of grouped_kernel.cuh over the
+//      prefix chunks, leaving (m, l, o) per member, head and chunk;
+//   3. the paged decode kernel over the tails, with each (member, head)'s
+//      base-2 log-normaliser;
+//   4. a merge kernel: the prefix partials and the tail result combined by
+//      their softmax normalisers.
+// Nothing here allocates device memory.
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <atomic>
+#include <climits>
+#include <cmath>
+#include <cstdint>
+
+#include "../../include/pa.h"
+#include "grouped_kernel.cuh"
+#include "host_common.cuh"
+#include "tma_host.cuh"
+
+namespace {
+
+using pa::grp::Chunk;
+using pa::grp::Group;
+using pa::grp::kChunk;
+using pa::grp::kD;
+using pa::grp::Member;
+using pa::grp::Meta;
+
+struct SetupParams {
+    const int32_t *group_start;   // [G + 1]
+    const int32_t *prefix_lens;   // [G]
+    const int32_t *context_lens;  // [B]
+    const int32_t *block_tables;  // [B, MB]
+    int num_groups, num_seqs, max_context_len, block_size, num_heads, max_blocks;
+    int max_chunks;               // capacity of `chunks` and of the partial columns
+    __half *out;                  // rows of empty contexts are zeroed here
+    Meta *meta;
+    Group *groups;
+    Member *members;
+    Chunk *chunks;
+    int32_t *tail_tables;         // [B, MB]
+    int32_t *tail_lens;           // [B]
+    unsigned int *dec_tickets;    // [B, H] merge tickets of the tail decode, cleared here
+    unsigned int *err;
+};
+
+constexpr int kSetupThreads = 1024;
+
+__device__ __forceinline__ int clamped_len(const SetupParams &p, int b)
+{
+    const int raw = p.context_lens[b];
+    if (raw < 0 || raw > p.max_context_len) {
+        atomicOr(p.err, PA_DEVERR_CONTEXT_LEN);
+        return raw < 0 ? 0 : p.max_context_len;
+    }
+    return raw;
+}
+
+// Exclusive scan of get(i), i < n, over the whole CTA; put(i, prefix).
+// Returns the total.  All threads of the CTA must call it.
+template <class Get, class Put>
+__device__ int block_exclusive_scan(int n, Get get, Put put, int *s_warp)
+{
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    int carry = 0;
+    for (int base = 0; base < n; base += kSetupThreads) {
+        const int i = base + tid;
+        const int v = i < n ? get(i) : 0;
+        int x = v;
+#pragma unroll
+        for (int off = 1; off < 32; off <<= 1) {
+            const int y = __shfl_up_sync(pa::kFullMask, x, off);
+            if (lane >= off)
+                x += y;
+        }
+        if (lane == 31)
+            s_warp[warp] = x;
+        __syncthreads();
+        if (warp == 0) {
+            int w = s_warp[lane];
+#pragma unroll
+            for (int off = 1; off < 32; off <<= 1) {
+                const int y = __shfl_up_sync(pa::kFullMask, w, off);
+                if (lane >= off)
+                    w += y;
+            }
+            s_warp[lane] = w;
+        }
+        __syncthreads();
+        const int before = carry + (warp > 0 ? s_warp[warp - 1] : 0);
+        if (i < n)
+            put(i, before + x - v);
+        carry += s_warp[31];
+        __syncthreads();
+    }
+    return carry;
+}
+
+// Group g with members g0 .. g0+n-1 and a valid prefix P (a multiple of the
+// block size, at most every member's context) gets ceil(P / 512) prefix
+// chunks per slice of up to 16 members, read through the first member's
+// table.  A prefix that breaks the rules is recorded (PA_DEVERR_CONTEXT_LEN)
+// and the group decodes without one.  Member b's tail is tokens P .. L_b - 1
+// of its own table: its tail table is that row from block P / bs on.
+__global__ void __launch_bounds__(kSetupThreads) grouped_setup_kernel(const SetupParams p)
+{
+    __shared__ int s_warp[32];
+    pa::grid_dependency_wait();
+    pa::allow_dependent_launch();
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int B = p.num_seqs, G = p.num_groups, bs = p.block_size, H = p.num_heads;
+    for (int b = tid; b < B; b += kSetupThreads) {
+        p.members[b] = Member{-1, 0, 0, 0};
+        p.tail_lens[b] = 0;
+    }
+    for (int i = tid; i < B * H; i += kSetupThreads)
+        p.dec_tickets[i] = 0u;
+    __syncthreads();
+
+    // A: per group (a warp each): bounds, prefix, tails
+    for (int g = warp; g < G; g += kSetupThreads / 32) {
+        int g0 = p.group_start[g];
+        const int g1 = p.group_start[g + 1];
+        const bool okg = 0 <= g0 && g0 <= g1 && g1 <= B;
+        if (!okg && lane == 0)
+            atomicOr(p.err, PA_DEVERR_CONTEXT_LEN);
+        const int n = okg ? g1 - g0 : 0;
+        if (!okg)
+            g0 = 0;
+        int P = p.prefix_lens[g];
+        int min_len = INT_MAX;
+        for (int b = g0 + lane; b < g0 + n; b += 32)
+            min_len = min(min_len, clamped_len(p, b));
+        min_len = __reduce_min_sync(pa::kFullMask, min_len);
+        if (n == 0 || P < 0 || P % bs != 0 || P > min_len) {
+            if (n > 0 && P != 0 && lane == 0)
+                atomicOr(p.err, PA_DEVERR_CONTEXT_LEN);
+            P = 0;
+        }
+        const int cp = (P + kChunk - 1) / kChunk;
+        const int slices = (n + 15) / 16;
+        for (int b = g0 + lane; b < g0 + n; b += 32) {
+            const int L = clamped_len(p, b);
+            p.members[b] = Member{g, L - P, 0, 0};
+            p.tail_lens[b] = L - P;
+            if (L == 0) {  // nothing to attend to: the output is zero
+                uint4 *o = reinterpret_cast<uint4 *>(p.out + size_t(b) * H * kD);
+                for (int e = 0; e < H * kD / 8; ++e)
+                    o[e] = make_uint4(0, 0, 0, 0);
+            }
+        }
+        if (lane == 0)  // colbase and pstart hold counts until the scans turn them into offsets
+            p.groups[g] = Group{g0, n, cp, P, n * cp, slices * cp, 0, 0};
+    }
+    __syncthreads();
+
+    // B: offsets of every group's chunks and partial columns
+    Group *gr = p.groups;
+    const int nchunks = block_exclusive_scan(
+        G, [&](int i) { return gr[i].pstart; }, [&](int i, int x) { gr[i].pstart = x; }, s_warp);
+    const int ncols = block_exclusive_scan(
+        G, [&](int i) { return gr[i].colbase; }, [&](int i, int x) { gr[i].colbase = x; }, s_warp);
+    const bool fits = nchunks <= p.max_chunks && ncols <= p.max_chunks;
+    if (!fits) {  // cannot happen with the host's bound; refuse rather than overrun
+        if (tid == 0) {
+            atomicOr(p.err, PA_DEVERR_CONTEXT_LEN);
+            *p.meta = Meta{0, 0, 0, 0};
+        }
+        return;
+    }
+
+    // C: the chunk descriptors, and the tail tables
+    for (int g = warp; g < G; g += kSetupThreads / 32) {
+        const Group gg = gr[g];
+        const int slices = (gg.n + 15) / 16;
+        for (int idx = lane; idx < slices * gg.cp; idx += 32) {
+            const int j = idx / slices, s = idx % slices;
+            p.chunks[gg.pstart + idx] =
+                Chunk{gg.g0, gg.g0 + 16 * s, min(16, gg.n - 16 * s), j * kChunk,
+                      min((j + 1) * kChunk, gg.P), g, gg.colbase + j * gg.n + 16 * s, 0};
+        }
+    }
+    const int MB = p.max_blocks;
+    for (size_t i = tid; i < size_t(B) * MB; i += kSetupThreads) {
+        const int b = int(i / MB), k = int(i % MB);
+        const int g = p.members[b].group;
+        const int pb = g >= 0 ? gr[g].P / bs : 0;
+        p.tail_tables[i] = pb + k < MB ? p.block_tables[size_t(b) * MB + pb + k] : -1;
+    }
+    if (tid == 0)
+        *p.meta = Meta{nchunks, ncols, 0, 0};
+}
+
+// out[b, h] = (sum_j 2^(m_j - M) o_j + 2^(lse_t - M) o_t) /
+//             (sum_j 2^(m_j - M) l_j + 2^(lse_t - M)),  M the largest exponent:
+// the prefix chunks' partials (m_j, l_j, o_j unnormalised, fp32) and the
+// tail's normalised fp16 result with its log-normaliser lse_t.  An empty
+// part has weight 0.  One warp per (member, head), four dims per lane.
+__global__ void __launch_bounds__(256) grouped_merge_kernel(
+    __half *__restrict__ out, const Group *__restrict__ groups, const Member *__restrict__ members,
+    const float *__restrict__ part_ml, const float *__restrict__ part_o,
+    const __half *__restrict__ o_t, const float *__restrict__ lse_t, int num_heads, int units)
+{
+    pa::grid_dependency_wait();
+    pa::allow_dependent_launch();
+    const int unit = blockIdx.x * 8 + (threadIdx.x >> 5), lane = threadIdx.x & 31;
+    if (unit >= units)
+        return;
+    const int b = unit / num_heads, h = unit % num_heads;
+    const Member mb = members[b];
+    if (mb.group < 0)
+        return;
+    const Group G = groups[mb.group];
+    if (G.P + mb.tail == 0)
+        return;  // empty context: zeroed by the set-up kernel
+    constexpr int kBatch = 4;
+    float M = -INFINITY, den = 0.f, num[4] = {0.f, 0.f, 0.f, 0.f};
+    auto add = [&](float m, float l, const float (&x)[4]) {
+        const float mn = fmaxf(M, m);
+        const float a = exp2f(M - mn), f = exp2f(m - mn);
+        M = mn;
+        den = fmaf(den, a, f * l);
+#pragma unroll
+        for (int e = 0; e < 4; ++e)
+            num[e] = fmaf(num[e], a, f * x[e]);
+    };
+    for (int j0 = 0; j0 < G.cp; j0 += kBatch) {
+        float2 v[kBatch];
+        float4 o[kBatch];
+#pragma unroll
+        for (int c = 0; c < kBatch; ++c) {
+            if (j0 + c < G.cp) {
+                const size_t ix = size_t(G.colbase + (j0 + c) * G.n + (b - G.g0)) * num_heads + h;
+                v[c] = reinterpret_cast<const float2 *>(part_ml)[ix];
+                o[c] = reinterpret_cast<const float4 *>(part_o + ix * kD)[lane];
+            }
+        }
+#pragma unroll
+        for (int c = 0; c < kBatch; ++c) {
+            if (j0 + c < G.cp) {
+                const float x[4] = {o[c].x, o[c].y, o[c].z, o[c].w};
+                add(v[c].x, v[c].y, x);
+            }
+        }
+    }
+    if (mb.tail > 0) {
+        const uint2 raw = reinterpret_cast<const uint2 *>(o_t + size_t(unit) * kD)[lane];
+        const float2 t01 = __half22float2(*reinterpret_cast<const __half2 *>(&raw.x));
+        const float2 t23 = __half22float2(*reinterpret_cast<const __half2 *>(&raw.y));
+        const float x[4] = {t01.x, t01.y, t23.x, t23.y};
+        add(lse_t[unit], 1.f, x);
+    }
+    const float inv = 1.f / den;
+    const __half2 r01 = __floats2half2_rn(num[0] * inv, num[1] * inv);
+    const __half2 r23 = __floats2half2_rn(num[2] * inv, num[3] * inv);
+    uint2 res;
+    res.x = *reinterpret_cast<const uint32_t *>(&r01);
+    res.y = *reinterpret_cast<const uint32_t *>(&r23);
+    reinterpret_cast<uint2 *>(out + size_t(unit) * kD)[lane] = res;
+}
+
+// Workspace of pa_decode_grouped: work-list header, group and member
+// records, prefix chunk descriptors, the prefix partials (reference max and
+// sum, and the fp32 output, per column and head), the tail tables and
+// lengths, the tail decode's own workspace, and its outputs and
+// log-normalisers.  Prefix chunks and columns are each at most
+// B ceil(max_context_len / 512): at most one column per member per 512
+// prefix tokens.
+struct Layout {
+    size_t meta, groups, members, chunks, part_ml, part_o, tail_tables, tail_lens, dec, o_t,
+        lse_t, total;
+    int max_chunks;
+};
+
+Layout layout(int num_seqs, int num_groups, int num_heads, int max_context_len, int max_blocks)
+{
+    Layout w{};
+    const size_t per_member = size_t((max_context_len + kChunk - 1) / kChunk);
+    const size_t cap = size_t(num_seqs) * (per_member > 0 ? per_member : 1);
+    const size_t units = size_t(num_seqs) * size_t(num_heads);
+    w.max_chunks = cap > size_t(INT_MAX) ? INT_MAX : int(cap);
+    w.meta = 0;
+    w.groups = align256(sizeof(Meta));
+    w.members = w.groups + align256(size_t(num_groups) * sizeof(Group));
+    w.chunks = w.members + align256(size_t(num_seqs) * sizeof(Member));
+    w.part_ml = w.chunks + align256(cap * sizeof(Chunk));
+    w.part_o = w.part_ml + align256(cap * num_heads * 2 * sizeof(float));
+    w.tail_tables = w.part_o + align256(cap * num_heads * kD * sizeof(float));
+    w.tail_lens = w.tail_tables + align256(size_t(num_seqs) * size_t(max_blocks) * sizeof(int32_t));
+    w.dec = w.tail_lens + align256(size_t(num_seqs) * sizeof(int32_t));
+    w.o_t = w.dec + align256(pa_decode_workspace_size(num_seqs, num_heads, kD, max_context_len));
+    w.lse_t = w.o_t + align256(units * kD * 2);
+    w.total = w.lse_t + align256(units * sizeof(float));
+    return w;
+}
+
+} // namespace
+
+extern "C" size_t pa_decode_grouped_workspace_size(int num_seqs, int num_groups, int num_heads,
+                                                   int head_dim, int max_context_len,
+                                                   int max_blocks_per_seq)
+{
+    if (num_seqs < 0 || num_groups < 0 || num_heads < 0 || head_dim < 0 || max_context_len < 0 ||
+        max_blocks_per_seq < 0)
+        return 0;
+    return layout(num_seqs, num_groups, num_heads, max_context_len, max_blocks_per_seq).total;
+}
+
+extern "C" pa_status pa_decode_grouped(void *out, const void *q, const void *k_cache,
+                                       const void *v_cache, const int32_t *block_tables,
+                                       int max_blocks_per_seq, const int32_t *context_lens,
+                                       int max_context_len, const int32_t *group_start,
+                                       const int32_t *prefix_lens, int num_groups,
+                                       int max_group_size, int num_seqs, int num_heads,
+                                       int head_dim, int block_size, int num_blocks, float scale,
+                                       void *workspace, size_t workspace_bytes, pa_stream_t stream)
+{
+    if (num_seqs < 0 || num_groups < 0 || max_group_size < 0 || num_heads <= 0 ||
+        num_blocks <= 0 || max_context_len < 0 || max_blocks_per_seq < 0)
+        return PA_ERR_INVALID_ARG;
+    if (head_dim != kD || !supported_block_size(block_size))
+        return PA_ERR_UNSUPPORTED;
+    if (int64_t(max_context_len) > int64_t(max_blocks_per_seq) * block_size ||
+        !std::isfinite(scale) || !(scale > 0.f) || (num_seqs > 0 && num_groups == 0) ||
+        num_groups > num_seqs)
+        return PA_ERR_INVALID_ARG;
+    if (num_seqs == 0)
+        return PA_OK;
+    if (!out || !q || !k_cache || !v_cache || !block_tables || !context_lens || !group_start ||
+        !prefix_lens || max_group_size == 0)
+        return PA_ERR_INVALID_ARG;
+    if (!aligned16(out) || !aligned16(q) || !aligned16(k_cache) || !aligned16(v_cache) ||
+        (reinterpret_cast<uintptr_t>(block_tables) & 3u) ||
+        (reinterpret_cast<uintptr_t>(context_lens) & 3u) ||
+        (reinterpret_cast<uintptr_t>(group_start) & 3u) ||
+        (reinterpret_cast<uintptr_t>(prefix_lens) & 3u))
+        return PA_ERR_INVALID_ARG;
+    if (num_seqs > 65535 || num_heads > 65535 || max_group_size > 65535 ||
+        int64_t(num_blocks) * num_heads * block_size > INT32_MAX ||
+        int64_t(num_heads) * ((max_context_len + kChunk - 1) / kChunk + 1) * num_seqs > INT32_MAX ||
+        int64_t(num_seqs) * max_blocks_per_seq > INT32_MAX)
+        return PA_ERR_INVALID_ARG;
+    const Layout w = layout(num_seqs, num_groups, num_heads, max_context_len, max_blocks_per_seq);
+    if (!workspace || workspace_bytes < w.total || !aligned16(workspace))
+        return PA_ERR_WORKSPACE;
+    unsigned char *ws = static_cast<unsigned char *>(workspace);
+    unsigned int *err = device_error_word();
+    if (!err)
+        return PA_ERR_CUDA;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices)
+        return PA_ERR_CUDA;
+    static std::atomic<int> sm_count[kMaxDevices];  // 0 = not configured yet
+    int sms = sm_count[dev].load(std::memory_order_acquire);
+    if (sms == 0) {
+        if (cudaFuncSetAttribute(pa::grp::grouped_decode_kernel,
+                                 cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 int(pa::grp::kSmem)) != cudaSuccess ||
+            cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess ||
+            sms <= 0)
+            return PA_ERR_CUDA;
+        sm_count[dev].store(sms, std::memory_order_release);
+    }
+
+    CUtensorMap tm_q, tm_k, tm_v;
+    const uint64_t cache_rows = uint64_t(num_blocks) * num_heads * block_size;
+    const uint32_t box_rows = uint32_t(block_size < pa::grp::kT ? block_size : pa::grp::kT);
+    if (!make_map(&tm_q, q, uint64_t(num_heads) * head_dim, uint64_t(num_seqs),
+                  uint64_t(num_heads) * head_dim * 2, pa::grp::kNQ) ||
+        !make_kv_map(&tm_k, k_cache, cache_rows, box_rows) ||
+        !make_kv_map(&tm_v, v_cache, cache_rows, box_rows))
+        return PA_ERR_CUDA;
+
+    Meta *meta = reinterpret_cast<Meta *>(ws + w.meta);
+    Group *groups = reinterpret_cast<Group *>(ws + w.groups);
+    Member *members = reinterpret_cast<Member *>(ws + w.members);
+    float *part_ml = reinterpret_cast<float *>(ws + w.part_ml);
+    float *part_o = reinterpret_cast<float *>(ws + w.part_o);
+    int32_t *tail_tables = reinterpret_cast<int32_t *>(ws + w.tail_tables);
+    int32_t *tail_lens = reinterpret_cast<int32_t *>(ws + w.tail_lens);
+    __half *o_t = reinterpret_cast<__half *>(ws + w.o_t);
+    float *lse_t = reinterpret_cast<float *>(ws + w.lse_t);
+
+    // 1. the prefix work list and the tails
+    SetupParams sp{};
+    sp.group_start = group_start;
+    sp.prefix_lens = prefix_lens;
+    sp.context_lens = context_lens;
+    sp.block_tables = block_tables;
+    sp.num_groups = num_groups;
+    sp.num_seqs = num_seqs;
+    sp.max_context_len = max_context_len;
+    sp.block_size = block_size;
+    sp.num_heads = num_heads;
+    sp.max_blocks = max_blocks_per_seq;
+    sp.max_chunks = w.max_chunks;
+    sp.out = static_cast<__half *>(out);
+    sp.meta = meta;
+    sp.groups = groups;
+    sp.members = members;
+    sp.chunks = reinterpret_cast<Chunk *>(ws + w.chunks);
+    sp.tail_tables = tail_tables;
+    sp.tail_lens = tail_lens;
+    sp.dec_tickets = reinterpret_cast<unsigned int *>(
+        ws + w.dec + pa_host::decode_ticket_offset(num_seqs, num_heads, kD));
+    sp.err = err;
+    if (launch_pdl(grouped_setup_kernel, dim3(1), dim3(kSetupThreads), 0, s, sp) != cudaSuccess)
+        return PA_ERR_CUDA;
+
+    // 2. the shared prefixes, once per (group, head), on the tensor cores
+    pa::grp::Params p{};
+    p.out = static_cast<__half *>(out);
+    p.block_tables = block_tables;
+    p.chunks = sp.chunks;
+    p.groups = groups;
+    p.members = members;
+    p.meta = meta;
+    p.part_ml = part_ml;
+    p.part_o = part_o;
+    p.max_blocks_per_seq = max_blocks_per_seq;
+    p.num_heads = num_heads;
+    p.block_size = block_size;
+    p.num_blocks = num_blocks;
+    p.qk_scale_log2 = float(double(scale) * 1.4426950408889634);
+    p.error_word = err;
+    if (launch_pdl(pa::grp::grouped_decode_kernel, dim3(unsigned(sms)), dim3(pa::grp::kThreads),
+                   pa::grp::kSmem, s, tm_q, tm_k, tm_v, p) != cudaSuccess)
+        return PA_ERR_CUDA;
+
+    // 3. each member's own tail
+    const pa_status st = pa_host::decode_with_lse(
+        o_t, q, k_cache, v_cache, tail_tables, max_blocks_per_seq, tail_lens, max_context_len,
+        num_seqs, num_heads, head_dim, block_size, num_blocks, scale, ws + w.dec, w.o_t - w.dec, lse_t,
+        stream);
+    if (st != PA_OK)
+        return st;
+
+    // 4. merge the parts
+    const int units = num_seqs * num_heads;
+    return launch_pdl(grouped_merge_kernel, dim3(unsigned((units + 7) / 8)), dim3(256), 0, s,
+                      static_cast<__half *>(out), static_cast<const Group *>(groups),
+                      static_cast<const Member *>(members), static_cast<const float *>(part_ml),
+                      static_cast<const float *>(part_o), static_cast<const __half *>(o_t),
+                      static_cast<const float *>(lse_t), num_heads, units) == cudaSuccess
+               ? PA_OK
+               : PA_ERR_CUDA;
+}

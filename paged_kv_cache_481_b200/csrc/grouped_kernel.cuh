@@ -1,0 +1,879 @@
+// The shared-prefix part of the decode of sequence groups (beam candidates,
+// parallel samples of one prompt) on the sm_100a tensor cores.
+//
+// What it computes (comfyai.app "6.4 PagedAttention", 6.4.2: the samples of
+// one prompt share its KV blocks; polomodov.tech "vLLM and PagedAttention",
+// slides 13-14): the members of group g share the physical blocks of their
+// first P_g tokens, so for every member b and head h the attention over those
+// tokens, softmax_t(scale q[b, h] . K_t) V_t for t < P_g, can be computed
+// with K and V read once per (group, head) and all the group's queries scored
+// against each K tile together.  This kernel leaves, per member, head and
+// 512-token chunk of the prefix, the unnormalised partial result (reference
+// max m in base-2 units, sum l, o = sum_t 2^(s_t - m) V_t); the members'
+// private tails are decoded by the paged decode kernel and the two parts are
+// merged by their softmax normalisers (grouped.cu).
+//
+// How: the score product is computed transposed, S^T = K Q^T, so the MMA's
+// M dimension is 128 context tokens and N is 16 query columns (up to 16
+// members); O^T = V^T P^T accumulates in TMEM with the head dimension as M.
+// A softmax thread then owns one token (one TMEM lane) and handles its <= 16
+// scores, so the per-tile softmax stays short.
+//   * Work items ("chunks", built by a set-up kernel): up to 512 tokens of a
+//     group's prefix for a slice of up to 16 members, read through the first
+//     member's table.  Items are (chunk, head) pairs; persistent CTAs (one per
+//     SM) take every gridDim-th item.
+//   * warp 8 (loads): walks the CTA's items, passes each to the other roles
+//     through a small shared-memory ring, and issues the TMA loads: the 16 Q
+//     rows of the next item, and per 128-token tile K and V through the block
+//     table, one 4-D box per (block, head) run, into six 32 KB slots.
+//   * warp 9 (one thread): S^T(n) = K_n Q^T into one of two TMEM score
+//     buffers and O^T += V_n^T P_n^T (V as an M-major operand, P^T from shared
+//     memory), each issued as soon as its inputs are ready; a K slot is
+//     released when its score product completes, a V slot when its P.V does.
+//   * warps 0-3 (softmax, thread = token): the tile maximum per query column
+//     (warp reduction, then the four warps' maxima through shared memory
+//     behind one named barrier), exp2 against a reference max per column that
+//     only moves when a tile's max exceeds it by more than 2^8 (then the
+//     column of O and the partial sums are rescaled), P^T as fp16 into a
+//     shared-memory operand tile; rows past the prefix end get P = 0 and
+//     their V rows are zeroed (by the MMA thread) so garbage never meets a
+//     zero weight.
+//   * warps 4-7 (epilogue, thread = head dimension): O^T columns and the
+//     per-column sums are written to the workspace as (m, l, o).
+// Every wait is bounded (1 s); the first to run out records PA_DEVERR_TIMEOUT
+// and raises an abort flag that ends every role; copies and matrix
+// operations in flight are drained (bounded) before TMEM is released.
+#pragma once
+
+#include <cuda.h>
+#include <cuda_fp16.h>
+#include <cstdint>
+
+#include "../../include/pa.h"
+#include "ptx.cuh"
+#include "tcgen05.cuh"
+
+namespace pa {
+namespace grp {
+
+constexpr int kD = 128;                     // head dim handled here
+constexpr int kT = 128;                     // context tokens per tile (M of S^T)
+constexpr int kNQ = 16;                     // query columns per item (N of both products)
+constexpr int kChunk = 512;                 // context tokens per work item
+constexpr int kSlots = 6;                   // K / V tile slots
+constexpr int kItemRing = 4;
+// A K or V tile in shared memory: [16 row groups][2 halves][8 rows][64 fp16]
+// with 128-byte swizzle, so every (row group, half) is one 1 KB swizzle atom.
+constexpr uint32_t kTile = 128u * 256u;     // one K or V tile (32 KB)
+constexpr uint32_t kAtom = 1024u;           // 8 rows x 128 bytes
+constexpr uint32_t kGroupStride = 2048u;    // between 8-row groups
+constexpr uint32_t kQHalf = kNQ * 128u;     // [16 rows x 64 fp16]
+constexpr uint32_t kQTile = 2 * kQHalf;     // Q rows of an item, or P^T of a tile (4 KB)
+constexpr int kQSlots = 4;                  // Q rows of the items in flight
+constexpr int kPBufs = 2;                   // P^T operand tiles
+constexpr uint32_t kOffQ = kSlots * kTile;
+constexpr uint32_t kOffP = kOffQ + kQSlots * kQTile;
+constexpr uint32_t kSmem = kOffP + kPBufs * kQTile + 1024;  // + 1024-byte alignment slack
+constexpr int kLoadWarps = 1;               // 2: K tiles and V tiles from separate warps
+constexpr int kLoadWarp = 8, kMmaWarp = 9, kLoadWarpV = 10;
+constexpr int kThreads = (kLoadWarps == 2 ? 11 : 10) * 32;
+// The loads are issued K(m), V(m - kVLag), K(m + 1), ...: a V tile is only
+// needed by its P.V, after the tile's score product and softmax, so issuing
+// it later lets it land about when it is used and keeps the shared-memory
+// slots holding data in flight rather than data waiting to be used.
+constexpr int kVLag = 0;
+constexpr uint32_t kTmemCols = 64;          // S0, S1, O0, O1: 16 columns each
+constexpr uint32_t kTmemO = 32;
+constexpr float kRescaleLog2 = 8.f;         // move a reference max only past this growth
+
+// One work item's context part (head-independent): tokens [t0, t1) of
+// block-table row `table_row`, scored for query rows q_row0 .. q_row0+nq-1.
+struct Chunk {
+    int table_row, q_row0, nq, t0, t1;
+    int group;     // the sequence group whose members it contributes to
+    int col;       // first partial-result column (column col + q: query row q_row0 + q)
+    int pad;
+};
+
+// A group as the set-up kernel found it: members g0 .. g0+n-1, prefix chunks
+// per 16-member slice (cp), the prefix length used (P), the first partial
+// column of its prefix chunks (prefix chunk j of member b uses column
+// colbase + j*n + (b - g0)), and the index of its first chunk in the work
+// list.
+struct Group {
+    int g0, n, cp, P, colbase, pstart, pad0, pad1;
+};
+
+// A member: its group (-1: in none) and its tail length L_b - P.
+struct Member {
+    int group, tail, pad0, pad1;
+};
+
+struct Meta {
+    int nchunks;      // prefix chunks of all groups
+    int ncols;        // partial columns they use
+    int pad0, pad1;
+};
+
+struct Params {
+    __half *out;                      // [B, H, D]
+    const int32_t *block_tables;      // [B, MB]
+    const Chunk *chunks;
+    const Group *groups;
+    const Member *members;
+    const Meta *meta;
+    float *part_ml;                   // [columns, H, 2]: (reference max, sum)
+    float *part_o;                    // [columns, H, D]
+    int max_blocks_per_seq;
+    int num_heads;
+    int block_size;
+    int num_blocks;
+    float qk_scale_log2;              // softmax scale * log2(e), > 0
+    unsigned int *error_word;
+};
+
+struct Item {
+    Chunk c;
+    int h;
+    int k;  // item index, -1 = no more items
+};
+
+// softmax -> epilogue hand-off of one finished item
+struct Epi {
+    Chunk c;
+    int h;
+    int end;
+    float m[kNQ];      // reference max per column (base-2 units)
+    float l[4][kNQ];   // per-warp partial sums per column
+};
+
+struct Shared {
+    uint64_t item_full[kItemRing], item_empty[kItemRing];
+    uint64_t q_full[kQSlots], q_empty[kQSlots];
+    uint64_t kv_full[kSlots], kv_empty[kSlots];
+    uint64_t s_full[2], s_empty[2];
+    uint64_t p_full[kPBufs], p_empty[kPBufs];
+    uint64_t o_full[2], o_empty[2], e_full[2];
+    uint64_t drain;
+    Item item[kItemRing];
+    Epi epi[2];
+    float red[2][4][kNQ];
+    uint32_t tmem;
+    int abort;
+};
+
+__device__ __forceinline__ bool gwait(uint32_t bar, uint32_t parity, volatile int *abort,
+                                      unsigned int *err)
+{
+    if (mbar_try_wait(bar, parity))
+        return true;
+    const uint64_t t0 = global_timer_ns();
+    while (!mbar_try_wait(bar, parity)) {
+        if (*abort)
+            return false;
+        if (global_timer_ns() - t0 > kWaitLimitNs) {
+            atomicOr(err, PA_DEVERR_TIMEOUT);
+            *abort = 1;
+            return false;
+        }
+    }
+    return true;
+}
+
+__device__ __forceinline__ int chunk_tiles(const Chunk &c)
+{
+    return (c.t1 - c.t0 + kT - 1) / kT;
+}
+
+__device__ __forceinline__ float ex2f(float x)
+{
+    float y;
+    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
+}
+
+__device__ __forceinline__ float warp_max(float x)
+{
+    float r;
+    asm volatile("redux.sync.max.f32 %0, %1, 0xffffffff;" : "=f"(r) : "f"(x));
+    return r;
+}
+
+// Barrier over the four softmax warps (named barrier 1) that also ANDs a
+// flag across them, so that all four take the same branch afterwards.
+__device__ __forceinline__ bool softmax_bar_and(bool v)
+{
+    uint32_t r;
+    asm volatile(
+        "{\n\t.reg .pred p, q;\n\t"
+        "setp.ne.u32 p, %1, 0;\n\t"
+        "barrier.cta.red.and.pred q, 1, 128, p;\n\t"
+        "selp.u32 %0, 1, 0, q;\n\t}"
+        : "=r"(r)
+        : "r"(uint32_t(v))
+        : "memory");
+    return r != 0;
+}
+
+__device__ __forceinline__ float warp_sum(float x)
+{
+#pragma unroll
+    for (int off = 16; off >= 1; off >>= 1)
+        x += __shfl_xor_sync(kFullMask, x, off);
+    return x;
+}
+
+// ---------------------------------------------------------------- loads
+// Chunk field f (0..7) of the descriptor a lane holds.
+__device__ __forceinline__ Chunk shfl_chunk(const Chunk &c, int src)
+{
+    Chunk r;
+    r.table_row = __shfl_sync(kFullMask, c.table_row, src);
+    r.q_row0 = __shfl_sync(kFullMask, c.q_row0, src);
+    r.nq = __shfl_sync(kFullMask, c.nq, src);
+    r.t0 = __shfl_sync(kFullMask, c.t0, src);
+    r.t1 = __shfl_sync(kFullMask, c.t1, src);
+    r.group = __shfl_sync(kFullMask, c.group, src);
+    r.col = __shfl_sync(kFullMask, c.col, src);
+    r.pad = 0;
+    return r;
+}
+
+// Block ids of a whole chunk (at most 512 / 8 = 64 runs of `box` tokens):
+// lane l holds runs l and l + 32.
+__device__ __forceinline__ void load_chunk_ids(const Params &p, const Chunk &c, int box, int lane,
+                                               int (&ids)[2])
+{
+    const int runs = (c.t1 - c.t0 + box - 1) / box;
+    const int32_t *row = p.block_tables + size_t(c.table_row) * p.max_blocks_per_seq;
+#pragma unroll
+    for (int r = 0; r < 2; ++r) {
+        const int run = lane + 32 * r;
+        ids[r] = run < runs ? row[(c.t0 + run * box) / p.block_size] : 0;
+    }
+}
+
+// Which loads a load warp issues: both kinds (one load warp), or only the K
+// tiles with the item hand-off and the Q rows, or only the V tiles (two).
+enum LoadPart { kLoadAll = 0, kLoadK = 1, kLoadV = 2 };
+
+// This CTA's items are blockIdx.x, blockIdx.x + gridDim.x, ... (numbered
+// chunk-major, prefix chunks first, so every CTA gets a like mix).  The
+// descriptors of 32 items at a time sit in the lanes' registers; the block
+// ids of the next item and the Q rows of the next item are fetched while the
+// current item's tiles are issued, so no dependent load stalls the stream.
+// Every load takes the shared-memory slot of its position: K(m) is at
+// position 2m and V(n) at 2n + 2 kVLag + 1, so slots 0, 2, 4 only ever hold
+// K tiles and slots 1, 3, 5 V tiles; positions 1, 3, .., 2 kVLag - 1 carry no
+// tile and complete their slot's phases at once.
+template <int kPart>
+__device__ __forceinline__ void load_role(const CUtensorMap *tm_q, const CUtensorMap *tm_k,
+                                          const CUtensorMap *tm_v, const Params &p, Shared &sh,
+                                          uint32_t sbase, int lane, int total)
+{
+    constexpr bool kDoK = kPart != kLoadV, kDoV = kPart != kLoadK;
+    volatile int *abort = &sh.abort;
+    unsigned int *err = p.error_word;
+    const int H = p.num_heads, bs = p.block_size;
+    const int box = bs < kT ? bs : kT;
+    const int stride = int(gridDim.x), first = int(blockIdx.x);
+    const int nitems = first < total ? (total - first + stride - 1) / stride : 0;
+    int last_use[kSlots];
+#pragma unroll
+    for (int i = 0; i < kSlots; ++i)
+        last_use[i] = -1;
+    int last_q[kQSlots];
+#pragma unroll
+    for (int i = 0; i < kQSlots; ++i)
+        last_q[i] = -1;
+    int batch = 0;  // descriptors of items batch .. batch+31 are in the lanes
+    Chunk mine{};
+    auto fetch = [&](int b0) {
+        const int it = b0 + lane;
+        if (it < nitems)
+            mine = p.chunks[(first + it * stride) / H];
+    };
+    auto chunk_of = [&](int it) {
+        if (it - batch >= 32) {
+            batch += 32;
+            fetch(batch);
+        }
+        return shfl_chunk(mine, it - batch);
+    };
+    // the Q rows of item `it` into Q slot it % kQSlots (once its previous
+    // user's score products are done)
+    auto issue_q = [&](int it, const Chunk &c) {
+        const int qs = it % kQSlots, use = it / kQSlots;
+        bool ok = true;
+        if (use > 0 && lane == 0)
+            ok = gwait(smem_u32(&sh.q_empty[qs]), uint32_t(use - 1) & 1u, abort, err);
+        if (!__shfl_sync(kFullMask, int(ok), 0))
+            return false;
+        if (lane == 0) {
+            const int h = (first + it * stride) % H;
+            const uint32_t bar = smem_u32(&sh.q_full[qs]);
+            mbar_arrive_expect_tx(bar, kQTile);
+            const uint32_t dst = sbase + kOffQ + uint32_t(qs) * kQTile;
+            tma_load_2d(dst, tm_q, h * kD, c.q_row0, bar);
+            tma_load_2d(dst + kQHalf, tm_q, h * kD + 64, c.q_row0, bar);
+        }
+        last_q[qs] = use;
+        return true;
+    };
+    struct TileRef {
+        int y8;     // this lane's run: first 8-row group (valid when ok)
+        int runs;   // 0: no tile
+        bool ok;    // this lane has a run and its block id is in range
+    };
+    auto issue = [&](int kind, const TileRef &t, int i) {
+        const int s = i % kSlots, use = i / kSlots;
+        const uint32_t full = smem_u32(&sh.kv_full[s]);
+        if (use > 0) {
+            const bool ok = lane == 0 ? gwait(smem_u32(&sh.kv_empty[s]), uint32_t(use - 1) & 1u, abort, err)
+                                      : true;
+            if (!__shfl_sync(kFullMask, int(ok), 0))
+                return false;
+        }
+        const uint32_t bytes = uint32_t(__popc(__ballot_sync(kFullMask, t.ok))) * uint32_t(box) * 256u;
+        if (lane == 0) {
+            if (t.runs > 0) {
+                mbar_arrive_expect_tx(full, bytes);
+            } else {
+                mbar_arrive(full);
+                mbar_arrive(smem_u32(&sh.kv_empty[s]));
+            }
+        }
+        last_use[s] = use;
+        __syncwarp();
+        if (t.ok)
+            tma_load_4d(sbase + uint32_t(s) * kTile + uint32_t(lane * box) * 256u, kind == 0 ? tm_k : tm_v,
+                        0, 0, 0, t.y8, full);
+        return true;
+    };
+    const TileRef none{0, 0, false};
+    TileRef hist[kVLag + 1];
+    int m = 0;  // tiles seen
+    bool go = true;
+    if (kPart == kLoadV)  // the V positions before V(0) carry no tile
+        for (int f = 0; go && f < kVLag; ++f)
+            go = issue(1, none, 2 * f + 1);
+    fetch(0);
+    Chunk c{};
+    int ids[2] = {0, 0};
+    if (nitems > 0) {
+        c = chunk_of(0);
+        load_chunk_ids(p, c, box, lane, ids);
+        if (kDoK)
+            go = go && issue_q(0, c);
+    }
+    int items = 0;
+    for (; go; ++items) {
+        const int kk = items < nitems && !*abort ? first + items * stride : -1;
+        const int h = kk >= 0 ? kk % H : 0;
+        // prefetch the next item's descriptor and block ids
+        Chunk cn{};
+        int ids_n[2] = {0, 0};
+        const bool has_next = kk >= 0 && items + 1 < nitems;
+        if (has_next) {
+            cn = chunk_of(items + 1);
+            load_chunk_ids(p, cn, box, lane, ids_n);
+        }
+        if (kDoK) {
+            const int slot = items % kItemRing, use = items / kItemRing;
+            bool ok = true;
+            if (use > 0 && lane == 0)
+                ok = gwait(smem_u32(&sh.item_empty[slot]), uint32_t(use - 1) & 1u, abort, err);
+            if (!__shfl_sync(kFullMask, int(ok), 0))
+                break;
+            if (lane == 0) {
+                sh.item[slot].c = c;
+                sh.item[slot].h = h;
+                sh.item[slot].k = kk;
+                mbar_arrive(smem_u32(&sh.item_full[slot]));
+            }
+            __syncwarp();
+        }
+        if (kk < 0) {
+            // one load warp: the V loads still owed to the last tiles
+            if (kPart == kLoadAll)
+                for (int f = 0; go && f < kVLag; ++f, ++m)
+                    go = issue(0, none, 2 * m) &&
+                         issue(1, m - kVLag >= 0 ? hist[(m - kVLag) % (kVLag + 1)] : none, 2 * m + 1);
+            break;
+        }
+        const int nt = chunk_tiles(c);
+        const int runs_per_tile = kT / box;
+        for (int j = 0; go && j < nt; ++j, ++m) {
+            const int valid = min(kT, c.t1 - (c.t0 + j * kT));
+            const int runs = (valid + box - 1) / box;
+            const int run = j * runs_per_tile + lane;  // this lane's run within the chunk
+            const int a = __shfl_sync(kFullMask, ids[0], run & 31);
+            const int b = __shfl_sync(kFullMask, ids[1], run & 31);
+            const int id = (run >> 5) ? b : a;
+            TileRef t;
+            t.runs = runs;
+            t.ok = lane < runs && unsigned(id) < unsigned(p.num_blocks);
+            if (kDoK && lane < runs && !t.ok)
+                atomicOr(err, PA_DEVERR_BLOCK_ID);
+            t.y8 = (id * H + h) * (bs / 8);  // first 8-row group of the run
+            if (kPart == kLoadAll) {
+                hist[m % (kVLag + 1)] = t;
+                go = issue(0, t, 2 * m) &&
+                     issue(1, m >= kVLag ? hist[(m - kVLag) % (kVLag + 1)] : none, 2 * m + 1);
+            } else if (kPart == kLoadK) {
+                go = issue(0, t, 2 * m);
+            } else {
+                go = issue(1, t, 2 * m + 2 * kVLag + 1);
+            }
+        }
+        if (kDoK && go && has_next)
+            go = issue_q(items + 1, cn);
+        c = cn;
+        ids[0] = ids_n[0];
+        ids[1] = ids_n[1];
+    }
+    // After an abort, let the copies already issued land before the CTA (and
+    // its shared memory) goes away.
+    if (*abort && lane == 0) {
+        for (int i = 0; i < kSlots; ++i)
+            if (last_use[i] >= 0)
+                mbar_wait_bounded(smem_u32(&sh.kv_full[i]), uint32_t(last_use[i]) & 1u);
+        for (int i = 0; i < kQSlots; ++i)
+            if (last_q[i] >= 0)
+                mbar_wait_bounded(smem_u32(&sh.q_full[i]), uint32_t(last_q[i]) & 1u);
+    }
+}
+
+// ------------------------------------------------------------ matrix unit
+// One thread.  Two streams of tensor-core work: S^T(n) = K_n Q^T once K_n has
+// landed and score buffer n % 2 is free, and O^T += V_n^T P_n^T once the
+// softmax has written P_n and V_n has landed.  The thread polls both and
+// issues whichever is ready, so a P.V never waits behind a later tile's K.
+// A tile with fewer than 128 valid rows takes only the P.V steps that hold
+// valid rows; the V rows past the end inside the last step are zeroed first.
+struct PvInfo {
+    int u, j, nt, valid;
+};
+
+__device__ __forceinline__ void mma_role(const Params &p, Shared &sh, uint32_t sbase, unsigned char *smem)
+{
+    constexpr uint32_t kIdS = idesc_f16_f32_mn(kT, kNQ, false, false);  // K-major K, K-major Q
+    constexpr uint32_t kIdO = idesc_f16_f32_mn(kD, kNQ, true, false);   // M-major V, K-major P^T
+    volatile int *abort = &sh.abort;
+    const uint32_t tmem = sh.tmem;
+    int u = -1, j = 0, nt = 0, t0 = 0, t1 = 0;  // item and tile of the next score product
+    bool need_item = true, more = true;
+    int ns = 0, np = 0;                         // score products / P.V products issued
+    PvInfo pend[4];
+    uint64_t idle_since = 0;
+    while (!*abort) {
+        bool prog = false;
+        if (need_item && more) {
+            const int slot = (u + 1) % kItemRing;
+            if (mbar_test_wait(smem_u32(&sh.item_full[slot]), uint32_t((u + 1) / kItemRing) & 1u)) {
+                const Item it = sh.item[slot];
+                mbar_arrive(smem_u32(&sh.item_empty[slot]));
+                if (it.k < 0) {
+                    more = false;
+                } else {
+                    ++u;
+                    j = 0;
+                    nt = chunk_tiles(it.c);
+                    t0 = it.c.t0;
+                    t1 = it.c.t1;
+                    need_item = false;
+                }
+                prog = true;
+            }
+        }
+        if (!need_item && ns - np < 4) {
+            const int sb = ns & 1, ks = (2 * ns) % kSlots;
+            if ((ns < 2 || mbar_test_wait(smem_u32(&sh.s_empty[sb]), uint32_t((ns >> 1) - 1) & 1u)) &&
+                mbar_test_wait(smem_u32(&sh.q_full[u % kQSlots]), uint32_t(u / kQSlots) & 1u) &&
+                mbar_test_wait(smem_u32(&sh.kv_full[ks]), uint32_t((2 * ns) / kSlots) & 1u)) {
+                tc_fence_after_sync();
+                const uint32_t ka = sbase + uint32_t(ks) * kTile;
+                const uint32_t qa = sbase + kOffQ + uint32_t(u % kQSlots) * kQTile;
+#pragma unroll
+                for (int k = 0; k < kD / 16; ++k) {
+                    const uint32_t kb = uint32_t(k >> 2), kk = uint32_t(k & 3) * 32u;
+                    umma_f16(tmem + uint32_t(sb) * kNQ,
+                             smem_desc_sw128(ka + kb * kAtom + kk, 16, kGroupStride),
+                             smem_desc_sw128(qa + kb * kQHalf + kk, 16, 1024), kIdS, k > 0);
+                }
+                umma_commit(smem_u32(&sh.s_full[sb]));
+                umma_commit(smem_u32(&sh.kv_empty[ks]));
+                if (j == nt - 1)
+                    umma_commit(smem_u32(&sh.q_empty[u % kQSlots]));
+                pend[ns & 3] = PvInfo{u, j, nt, min(kT, t1 - (t0 + j * kT))};
+                ++ns;
+                if (++j == nt)
+                    need_item = true;
+                prog = true;
+            }
+        }
+        if (np < ns) {
+            const PvInfo f = pend[np & 3];
+            const int vpos = 2 * np + 2 * kVLag + 1;  // V(np)'s load position
+            const int pb = np % kPBufs, ob = f.u & 1, vs = vpos % kSlots;
+            if (mbar_test_wait(smem_u32(&sh.p_full[pb]), uint32_t(np / kPBufs) & 1u) &&
+                mbar_test_wait(smem_u32(&sh.kv_full[vs]), uint32_t(vpos / kSlots) & 1u) &&
+                (f.j > 0 || f.u < 2 ||
+                 mbar_test_wait(smem_u32(&sh.o_empty[ob]), uint32_t((f.u >> 1) - 1) & 1u))) {
+                const int steps = (f.valid + 15) / 16;
+                if (f.valid < steps * 16) {  // zero V rows past the end inside the last step
+                    unsigned char *vt = smem + uint32_t(vs) * kTile;
+                    for (int r = f.valid; r < steps * 16; ++r) {
+                        unsigned char *row = vt + uint32_t(r >> 3) * kGroupStride + uint32_t(r & 7) * 128u;
+#pragma unroll
+                        for (int c16 = 0; c16 < 8; ++c16) {
+                            *reinterpret_cast<uint4 *>(row + c16 * 16) = make_uint4(0, 0, 0, 0);
+                            *reinterpret_cast<uint4 *>(row + kAtom + c16 * 16) = make_uint4(0, 0, 0, 0);
+                        }
+                    }
+                    fence_proxy_async_smem();
+                }
+                tc_fence_after_sync();
+                const uint32_t va = sbase + uint32_t(vs) * kTile;
+                const uint32_t pa = sbase + kOffP + uint32_t(pb) * kQTile;
+                for (int k = 0; k < steps; ++k) {
+                    const uint32_t kb = uint32_t(k >> 2), kk = uint32_t(k & 3) * 32u;
+                    umma_f16(tmem + kTmemO + uint32_t(ob) * kNQ,
+                             smem_desc_sw128(va + uint32_t(k) * 2u * kGroupStride, kAtom, kGroupStride),
+                             smem_desc_sw128(pa + kb * kQHalf + kk, 16, 1024), kIdO, f.j > 0 || k > 0);
+                }
+                umma_commit(smem_u32(&sh.p_empty[pb]));
+                umma_commit(smem_u32(&sh.kv_empty[vs]));
+                if (f.j == f.nt - 1)
+                    umma_commit(smem_u32(&sh.o_full[ob]));
+                ++np;
+                prog = true;
+            }
+        }
+        if (!more && need_item && np == ns)
+            break;
+        if (prog) {
+            idle_since = 0;
+        } else {
+            const uint64_t t = global_timer_ns();
+            if (idle_since == 0) {
+                idle_since = t;
+            } else if (t - idle_since > kWaitLimitNs) {
+                atomicOr(p.error_word, PA_DEVERR_TIMEOUT);
+                *abort = 1;
+            }
+        }
+    }
+    // every matrix operation issued has finished before TMEM and the shared
+    // tiles are released
+    umma_commit(smem_u32(&sh.drain));
+    mbar_wait_bounded(smem_u32(&sh.drain), 0u);
+}
+
+// ---------------------------------------------------------------- softmax
+// One tile for a thread holding token `row`.  NQ = 1 (a tail), 8 or 16 (a
+// prefix slice, of which the first nq columns are real).  Returns false once
+// a wait has failed; the next tile's (or item's) barrier then ends the role
+// in all four warps together.
+template <int NQ>
+__device__ __forceinline__ bool softmax_tile(const Params &p, Shared &sh, unsigned char *smem,
+                                             int warp, int lane, int n, int u, int j, int nq,
+                                             int valid, float (&m_ref)[kNQ], float (&l)[kNQ])
+{
+    volatile int *abort = &sh.abort;
+    unsigned int *err = p.error_word;
+    const int row = warp * 32 + lane;
+    const uint32_t lane_base = uint32_t(warp * 32) << 16;
+    const int sb = n & 1;
+    bool ok = gwait(smem_u32(&sh.s_full[sb]), uint32_t(n >> 1) & 1u, abort, err);
+    tc_fence_after_sync();
+    uint32_t s[16];
+    tmem_load16_async(sh.tmem + uint32_t(sb) * kNQ + lane_base, s);
+    tmem_wait_ld();
+    tc_fence_before_sync();
+    __syncwarp();
+    if (lane == 0)
+        mbar_arrive(smem_u32(&sh.s_empty[sb]));
+
+    const bool live = row < valid;
+    const float c = p.qk_scale_log2;
+    float x[NQ];
+#pragma unroll
+    for (int q = 0; q < NQ; ++q)
+        x[q] = live ? __uint_as_float(s[q]) * c : -INFINITY;
+    // tile max per column: warp reduction, then the four warps' maxima
+    // through shared memory (double-buffered by tile parity) behind one
+    // named barrier
+#pragma unroll
+    for (int q = 0; q < NQ; ++q) {
+        const float wm = warp_max(x[q]);
+        if (lane == q)
+            sh.red[sb][warp][q] = wm;
+    }
+    if (!softmax_bar_and(ok))
+        return false;
+    float tm[NQ];
+#pragma unroll
+    for (int q = 0; q < NQ; ++q)
+        tm[q] = fmaxf(fmaxf(sh.red[sb][0][q], sh.red[sb][1][q]), fmaxf(sh.red[sb][2][q], sh.red[sb][3][q]));
+    if (j == 0) {
+#pragma unroll
+        for (int q = 0; q < NQ; ++q)
+            m_ref[q] = tm[q];
+    } else {
+        bool need = false;
+#pragma unroll
+        for (int q = 0; q < NQ; ++q)
+            need |= q < nq && tm[q] > m_ref[q] + kRescaleLog2;
+        if (need) {  // uniform: every thread sees the same maxima
+            // move the reference: O (rows = head dims, one per thread) and the
+            // partial sums are rescaled once the previous P.V has completed
+            ok = gwait(smem_u32(&sh.p_empty[(n - 1) % kPBufs]), uint32_t((n - 1) / kPBufs) & 1u, abort, err) &&
+                 ok;
+            tc_fence_after_sync();
+            float alpha[NQ];
+#pragma unroll
+            for (int q = 0; q < NQ; ++q) {
+                const float mn = fmaxf(m_ref[q], tm[q]);
+                alpha[q] = ex2f(m_ref[q] - mn);
+                m_ref[q] = mn;
+                l[q] *= alpha[q];
+            }
+            const uint32_t tO = sh.tmem + kTmemO + uint32_t(u & 1) * kNQ + lane_base;
+            uint32_t o[16];
+            tmem_load16_async(tO, o);
+            tmem_wait_ld();
+#pragma unroll
+            for (int q = 0; q < NQ; ++q)
+                o[q] = __float_as_uint(__uint_as_float(o[q]) * alpha[q]);
+            tmem_store16(tO, o);
+            tmem_wait_st();
+        }
+    }
+    float pv[NQ];
+#pragma unroll
+    for (int q = 0; q < NQ; ++q) {
+        pv[q] = live ? ex2f(x[q] - m_ref[q]) : 0.f;
+        l[q] += pv[q];
+    }
+    // P^T (row q = query column, 128 tokens as K, 128-byte swizzle) into the
+    // tile's operand buffer once the P.V two tiles back has read it
+    const int pb = n % kPBufs;
+    if (n >= kPBufs)
+        ok = gwait(smem_u32(&sh.p_empty[pb]), uint32_t(n / kPBufs - 1) & 1u, abort, err) && ok;
+    {
+        unsigned char *pt = smem + kOffP + uint32_t(pb) * kQTile + uint32_t(row >> 6) * kQHalf;
+        const int tt = row & 63;
+#pragma unroll
+        for (int q = 0; q < NQ; ++q)
+            if (q < nq)
+                *reinterpret_cast<__half *>(pt + q * 128 + ((((tt >> 3) ^ (q & 7))) << 4) + (tt & 7) * 2) =
+                    __float2half_rn(pv[q]);
+    }
+    fence_proxy_async_smem();
+    tc_fence_before_sync();
+    __syncwarp();
+    if (lane == 0)
+        mbar_arrive(smem_u32(&sh.p_full[pb]));
+    return ok;
+}
+
+__device__ __forceinline__ void softmax_role(const Params &p, Shared &sh, unsigned char *smem, int warp,
+                                             int lane)
+{
+    volatile int *abort = &sh.abort;
+    unsigned int *err = p.error_word;
+    int n = 0;
+    for (int u = 0;; ++u) {
+        const int slot = u % kItemRing;
+        const bool got = gwait(smem_u32(&sh.item_full[slot]), uint32_t(u / kItemRing) & 1u, abort, err);
+        if (!softmax_bar_and(got))
+            break;
+        const Item it = sh.item[slot];
+        __syncwarp();
+        if (lane == 0)
+            mbar_arrive(smem_u32(&sh.item_empty[slot]));
+        float m_ref[kNQ], l[kNQ];
+#pragma unroll
+        for (int q = 0; q < kNQ; ++q) {
+            m_ref[q] = -INFINITY;
+            l[q] = 0.f;
+        }
+        bool ok = true;
+        if (it.k >= 0) {
+            const int nt = chunk_tiles(it.c), nq = it.c.nq;
+            for (int j = 0; j < nt; ++j, ++n) {
+                const int valid = min(kT, it.c.t1 - (it.c.t0 + j * kT));
+                const bool r = nq == 1   ? softmax_tile<1>(p, sh, smem, warp, lane, n, u, j, 1, valid, m_ref, l)
+                               : nq <= 8 ? softmax_tile<8>(p, sh, smem, warp, lane, n, u, j, nq, valid, m_ref, l)
+                                         : softmax_tile<kNQ>(p, sh, smem, warp, lane, n, u, j, nq, valid, m_ref, l);
+                ok = ok && r;
+            }
+        }
+        // hand the item to the epilogue once it has taken the item two back
+        Epi &e = sh.epi[u & 1];
+        if (u >= 2)
+            ok = gwait(smem_u32(&sh.o_empty[u & 1]), uint32_t((u >> 1) - 1) & 1u, abort, err) && ok;
+        if (!softmax_bar_and(ok))
+            break;
+        if (it.k >= 0) {
+#pragma unroll
+            for (int q = 0; q < kNQ; ++q) {
+                if (q < it.c.nq) {
+                    const float sm = warp_sum(l[q]);
+                    if (lane == 0)
+                        e.l[warp][q] = sm;
+                }
+            }
+        }
+        if (warp == 0 && lane == 0) {
+            e.c = it.c;
+            e.h = it.h;
+            e.end = it.k < 0;
+#pragma unroll
+            for (int q = 0; q < kNQ; ++q)
+                e.m[q] = m_ref[q];
+        }
+        __syncwarp();
+        if (lane == 0)
+            mbar_arrive(smem_u32(&sh.e_full[u & 1]));
+        if (it.k < 0)
+            break;
+    }
+}
+
+// ---------------------------------------------------------------- epilogue
+// Barrier over the four epilogue warps (named barrier 2) with an AND of a
+// flag, so that all four take the same branch afterwards.
+__device__ __forceinline__ bool epilogue_bar_and(bool v)
+{
+    uint32_t r;
+    asm volatile(
+        "{\n\t.reg .pred p, q;\n\t"
+        "setp.ne.u32 p, %1, 0;\n\t"
+        "barrier.cta.red.and.pred q, 2, 128, p;\n\t"
+        "selp.u32 %0, 1, 0, q;\n\t}"
+        : "=r"(r)
+        : "r"(uint32_t(v))
+        : "memory");
+    return r != 0;
+}
+
+// Thread d (head dimension d, TMEM lane d) of the four epilogue warps: per
+// item, the O^T columns and the per-column (m, l) go to the workspace.
+__device__ __forceinline__ void epilogue_role(const Params &p, Shared &sh, int ew, int lane)
+{
+    volatile int *abort = &sh.abort;
+    unsigned int *err = p.error_word;
+    const int d = ew * 32 + lane;
+    const uint32_t lane_base = uint32_t(ew * 32) << 16;
+    const int H = p.num_heads;
+    for (int u = 0;; ++u) {
+        const bool got = gwait(smem_u32(&sh.e_full[u & 1]), uint32_t(u >> 1) & 1u, abort, err);
+        if (!epilogue_bar_and(got))
+            break;
+        const Epi &e = sh.epi[u & 1];
+        if (e.end)
+            break;
+        const Chunk c = e.c;
+        const int h = e.h;
+        const int qd = d < kNQ ? d : 0;
+        const float m_d = e.m[qd];
+        const float l_d = (e.l[0][qd] + e.l[1][qd]) + (e.l[2][qd] + e.l[3][qd]);
+        const bool ok = gwait(smem_u32(&sh.o_full[u & 1]), uint32_t(u >> 1) & 1u, abort, err);
+        tc_fence_after_sync();
+        uint32_t o[16];
+        tmem_load16_async(sh.tmem + kTmemO + uint32_t(u & 1) * kNQ + lane_base, o);
+        tmem_wait_ld();
+        tc_fence_before_sync();
+        __syncwarp();
+        if (lane == 0)
+            mbar_arrive(smem_u32(&sh.o_empty[u & 1]));
+        if (!epilogue_bar_and(ok))
+            break;
+#pragma unroll
+        for (int q = 0; q < kNQ; ++q)
+            if (q < c.nq)
+                p.part_o[(size_t(c.col + q) * H + h) * kD + d] = __uint_as_float(o[q]);
+        if (d < c.nq)
+            reinterpret_cast<float2 *>(p.part_ml)[size_t(c.col + d) * H + h] = make_float2(m_d, l_d);
+    }
+}
+
+__global__ void __launch_bounds__(kThreads, 1)
+    grouped_decode_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+                          const __grid_constant__ CUtensorMap tm_v, const Params p)
+{
+    extern __shared__ unsigned char smem_raw[];
+    __shared__ __align__(16) Shared sh;
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+
+    const uint32_t raw = smem_u32(smem_raw);
+    const uint32_t sbase = (raw + 1023u) & ~1023u;
+    unsigned char *smem = smem_raw + (sbase - raw);
+    if (tid == 0) {
+        for (int i = 0; i < kItemRing; ++i) {
+            mbar_init(smem_u32(&sh.item_full[i]), 1);
+            mbar_init(smem_u32(&sh.item_empty[i]), 1 + 4);  // the MMA thread and the softmax warps
+        }
+        for (int i = 0; i < kQSlots; ++i) {
+            mbar_init(smem_u32(&sh.q_full[i]), 1);
+            mbar_init(smem_u32(&sh.q_empty[i]), 1);
+        }
+        for (int i = 0; i < kPBufs; ++i) {
+            mbar_init(smem_u32(&sh.p_full[i]), 4);
+            mbar_init(smem_u32(&sh.p_empty[i]), 1);
+        }
+        for (int i = 0; i < 2; ++i) {
+            mbar_init(smem_u32(&sh.s_full[i]), 1);
+            mbar_init(smem_u32(&sh.s_empty[i]), 4);
+            mbar_init(smem_u32(&sh.o_full[i]), 1);
+            mbar_init(smem_u32(&sh.o_empty[i]), 4);
+            mbar_init(smem_u32(&sh.e_full[i]), 4);
+        }
+        for (int i = 0; i < kSlots; ++i) {
+            mbar_init(smem_u32(&sh.kv_full[i]), 1);
+            mbar_init(smem_u32(&sh.kv_empty[i]), 1);
+        }
+        mbar_init(smem_u32(&sh.drain), 1);
+        sh.abort = 0;
+        fence_mbar_init();
+    }
+    if (warp == kMmaWarp)
+        tmem_alloc(smem_u32(&sh.tmem), kTmemCols);
+    tc_fence_before_sync();
+    __syncthreads();
+    tc_fence_after_sync();
+
+    // the work list comes from the set-up kernel that precedes this one
+    grid_dependency_wait();
+    allow_dependent_launch();
+    const int total = p.meta->nchunks * p.num_heads;
+
+    if (warp == kLoadWarp) {
+        if (kLoadWarps == 2)
+            load_role<kLoadK>(&tm_q, &tm_k, &tm_v, p, sh, sbase, lane, total);
+        else
+            load_role<kLoadAll>(&tm_q, &tm_k, &tm_v, p, sh, sbase, lane, total);
+    } else if (kLoadWarps == 2 && warp == kLoadWarpV) {
+        load_role<kLoadV>(&tm_q, &tm_k, &tm_v, p, sh, sbase, lane, total);
+    } else if (warp == kMmaWarp) {
+        if (lane == 0)
+            mma_role(p, sh, sbase, smem);
+        __syncwarp();
+    } else if (warp < 4) {
+        softmax_role(p, sh, smem, warp, lane);
+    } else {
+        epilogue_role(p, sh, warp - 4, lane);
+    }
+
+    tc_fence_before_sync();
+    __syncthreads();
+    if (warp == kMmaWarp) {
+        tc_fence_after_sync();
+        tmem_free(sh.tmem, kTmemCols);
+    }
+}
+
+} // namespace grp
+} // namespace pa

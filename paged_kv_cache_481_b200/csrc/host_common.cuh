@@ -25,6 +25,10 @@ pa_status decode_with_lse(void *out, const void *q, const void *k_cache, const v
                           int num_heads, int head_dim, int block_size, int num_blocks, float scale,
                           void *workspace, size_t workspace_bytes, float *lse, pa_stream_t stream);
 
+// Byte offset of the merge tickets (one unsigned per (sequence, head), zero
+// between calls) inside pa_decode's workspace for these sizes.
+size_t decode_ticket_offset(int num_seqs, int num_heads, int head_dim);
+
 } // namespace pa_host
 
 namespace {

@@ -169,6 +169,14 @@ __host__ __device__ constexpr uint32_t idesc_f16_f32(int m, int n, bool b_mn_maj
            | (uint32_t(m >> 4) << 24);       // M / 16
 }
 
+// The same with the major-ness of both operands chosen: a_mn_major reads A
+// (M x K) from an M-major layout (transposed), b_mn_major B from an N-major one.
+__host__ __device__ constexpr uint32_t idesc_f16_f32_mn(int m, int n, bool a_mn_major,
+                                                        bool b_mn_major)
+{
+    return idesc_f16_f32(m, n, b_mn_major) | (uint32_t(a_mn_major) << 15);
+}
+
 // D[tmem] (+)= A[smem] * B[smem]^T, issued by a single thread.
 __device__ __forceinline__ void umma_f16(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc,
                                          uint32_t idesc, uint32_t accumulate)
@@ -212,6 +220,17 @@ __device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap *map
     asm volatile(
         "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%3, %4}], [%2];" ::"r"(dst),
         "l"(map), "r"(bar), "r"(x), "r"(y)
+        : "memory");
+}
+
+// Box of a 4-D tensor map at (x0, x1, x2, x3) into shared memory; x0 times
+// the element size must be a multiple of 16 bytes.
+__device__ __forceinline__ void tma_load_4d(uint32_t dst, const CUtensorMap *map, int x0, int x1, int x2,
+                                            int x3, uint32_t bar)
+{
+    asm volatile(
+        "cp.async.bulk.tensor.4d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%3, %4, %5, %6}], [%2];" ::"r"(dst),
+        "l"(map), "r"(bar), "r"(x0), "r"(x1), "r"(x2), "r"(x3)
         : "memory");
 }
 

@@ -177,7 +177,8 @@ def measure_grouped(iters: int):
         ws = binding.new_workspace(wl.num_seqs, h, d, wl.max_context_len)
         ms_plain = _time_ms(lambda: binding.pa_decode(out, q, kc, vc, t, lens, wl.max_context_len,
                                                       wl.scale, ws), iters)
-        gws = binding.new_grouped_workspace(wl.num_seqs, h, d, tables.shape[1])
+        gws = binding.new_grouped_workspace(wl.num_seqs, wl.num_seqs // 8, h, d,
+                                            wl.max_context_len, tables.shape[1])
         gs = torch.arange(0, wl.num_seqs + 1, 8, dtype=torch.int32, device=dev)
         pl = torch.full((wl.num_seqs // 8,), prefix, dtype=torch.int32, device=dev)
         ms_grp = _time_ms(lambda: binding.pa_decode_grouped(out, q, kc, vc, t, lens,
