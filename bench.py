@@ -49,6 +49,14 @@ def _peak_hbm():
 
 
 KERNEL_SOURCES = {
+    "grouped": ("paged_kv_cache_481_b200/csrc/grouped_kernel.cuh",
+                "paged_kv_cache_481_b200/csrc/grouped.cu",
+                "paged_kv_cache_481_b200/csrc/tcgen05.cuh",
+                "paged_kv_cache_481_b200/csrc/tma_host.cuh",
+                "paged_kv_cache_481_b200/csrc/decode_kernel.cuh",
+                "paged_kv_cache_481_b200/csrc/decode.cu",
+                "paged_kv_cache_481_b200/csrc/ptx.cuh",
+                "paged_kv_cache_481_b200/csrc/host_common.cuh"),
     "decode": ("paged_kv_cache_481_b200/csrc/decode_kernel.cuh",
                "paged_kv_cache_481_b200/csrc/quant.cuh",
                "paged_kv_cache_481_b200/csrc/ptx.cuh",
@@ -511,6 +519,20 @@ def run_gpu(args):
             binding.pa_copy_blocks(kc, vc, pairs, stream=stream)
 
     fused = not args.unfused
+    # the shared-prefix workload decodes its groups with pa_decode_grouped
+    # (each shared prefix read once per group and head); --no-grouped: pa_decode
+    grouped = wl.group_start is not None and not args.no_grouped and not int8
+    if grouped:
+        d_gs = torch.from_numpy(wl.group_start).to(dev)
+        d_pl = torch.from_numpy(wl.prefix_lens).to(dev)
+        max_group = int(np.diff(wl.group_start).max())
+        gws = binding.new_grouped_workspace(b, len(wl.prefix_lens), h, d, mcl, tables.shape[1],
+                                            device=dev)
+        fused = False
+
+    def grouped_step(o, q_, tables_, lens_, gs_, pl_):
+        binding.pa_decode_grouped(o, q_, kc, vc, tables_, lens_, mcl, gs_, pl_, max_group,
+                                  wl.scale, gws, stream=stream)
 
     def append_step(o, q_, key_, value_, slots_, tables_, lens_):
         if int8:
@@ -527,14 +549,17 @@ def run_gpu(args):
             write_step(key, value, slots)
         if ev_pair is not None:
             ev_pair[0].record(stream)
-        if fused:
+        if grouped:
+            grouped_step(out, q, tables, lens, d_gs, d_pl)
+        elif fused:
             append_step(out, q, key, value, slots, tables, lens)
         else:
             decode_step(out, q, tables, lens)
         if ev_pair is not None:
             ev_pair[1].record(stream)
 
-    launches_per_step = (1 if fused else 2) + ((4 if int8 else 1) if pairs is not None else 0)
+    launches_per_step = ((1 if fused else 2) + ((4 if int8 else 1) if pairs is not None else 0)
+                         + (3 if grouped else 0))
     with torch.cuda.stream(stream):
         for _ in range(args.warmup):
             step()
@@ -573,17 +598,21 @@ def run_gpu(args):
     # tables, context lengths) leave pinned host memory and out comes back to
     # it, pipelined with the decode; the KV pool stays resident.
     def decode_from(views, o):
-        d_q, d_key, d_value, d_slots, d_tables, d_lens = views
+        d_q, d_key, d_value, d_slots, d_tables, d_lens = views[:6]
         if pairs is not None:
             copy_step()
-        if fused:
+        if grouped:
+            write_step(d_key, d_value, d_slots)
+            grouped_step(o, d_q, d_tables, d_lens, views[6], views[7])
+        elif fused:
             append_step(o, d_q, d_key, d_value, d_slots, d_tables, d_lens)
         else:
             write_step(d_key, d_value, d_slots)
             decode_step(o, d_q, d_tables, d_lens)
 
-    e2e_ms, h2d, d2h = pipelined_e2e([q, key, value, slots, tables, lens], out, decode_from,
-                                     stream, args.warmup, args.steps, world)
+    e2e_parts = [q, key, value, slots, tables, lens] + ([d_gs, d_pl] if grouped else [])
+    e2e_ms, h2d, d2h = pipelined_e2e(e2e_parts, out, decode_from, stream, args.warmup, args.steps,
+                                     world)
     assert binding.pa_get_last_device_error() == 0
 
     dec_bytes = (accounting.decode_bytes_int8(wl.context_lens, h, d) if int8
@@ -615,7 +644,10 @@ def run_gpu(args):
         kv_bytes = dec_bytes
         desc.update({
             "step": ("pa_copy_blocks + " if pairs is not None else "")
-                    + (f"pa_decode_append{'_int8' if int8 else ''} (cache write of {b} tokens "
+                    + (f"pa_reshape_and_cache({b} tokens) + pa_decode_grouped "
+                       f"({len(wl.prefix_lens)} groups, prefixes of {int(wl.prefix_lens[0])} tokens)"
+                       if grouped else
+                       f"pa_decode_append{'_int8' if int8 else ''} (cache write of {b} tokens "
                        f"fused into the decode)"
                        if fused else f"pa_reshape_and_cache({b} tokens) + pa_decode"),
             "l2": f"inputs larger than L2: {kv_bytes / 1e9:.2f} GB of K/V read per step "
@@ -643,10 +675,16 @@ def run_gpu(args):
                 "decode_us_max": max(decode_ms) * 1e3,
                 "decode_us_argmax": int(np.argmax(decode_ms))}),
             "roofline": {
-                "kernel": "paged_decode_kernel" + ("<int8>" if int8 else ""), "bound": "hbm",
+                "kernel": ("pa_decode_grouped (set-up, grouped_decode_kernel, paged_decode_kernel "
+                           "over the tails, merge)" if grouped else
+                           "paged_decode_kernel" + ("<int8>" if int8 else "")), "bound": "hbm",
                 "achieved": achieved,
                 "peak": peak, "peak_kind": f"{peak_kind} (hbm_gbs)", "unit": "GB/s",
-                "frac": achieved / peak, "traffic": None if int8 else _recorded_traffic(desc["workload"], "pa_decode_append" if fused else "pa_decode"),
+                "frac": achieved / peak,
+                "traffic": None if int8 else _recorded_traffic(
+                    desc["workload"], "pa_decode_grouped" if grouped else
+                    "pa_decode_append" if fused else "pa_decode",
+                    "grouped" if grouped else "decode"),
                 "algorithmic_bytes_per_launch": roof_bytes,
                 "logical_bytes_per_launch": dec_bytes,
             },
@@ -869,6 +907,8 @@ def main(argv=None):
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--unfused", action="store_true",
                     help="time the cache write and the decode as two launches")
+    ap.add_argument("--no-grouped", action="store_true",
+                    help="shared-prefix workload: plain pa_decode instead of pa_decode_grouped")
     ap.add_argument("--path", choices=["decode", "prefill"], default="decode",
                     help="prefill: the prompt cache write + pa_prefill step instead of decode")
     ap.add_argument("--prompts", type=int, default=8, help="prefill: prompts per step")

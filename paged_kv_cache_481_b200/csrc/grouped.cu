@@ -47,6 +47,7 @@ struct SetupParams {
     Chunk *chunks;
     int32_t *tail_tables;         // [B, MB]
     int32_t *tail_lens;           // [B]
+    int32_t *group_of;            // [B] each member's group (-1: none)
     unsigned int *dec_tickets;    // [B, H] merge tickets of the tail decode, cleared here
     unsigned int *err;
 };
@@ -119,6 +120,7 @@ __global__ void __launch_bounds__(kSetupThreads) grouped_setup_kernel(const Setu
     for (int b = tid; b < B; b += kSetupThreads) {
         p.members[b] = Member{-1, 0, 0, 0};
         p.tail_lens[b] = 0;
+        p.group_of[b] = -1;
     }
     for (int i = tid; i < B * H; i += kSetupThreads)
         p.dec_tickets[i] = 0u;
@@ -148,7 +150,7 @@ __global__ void __launch_bounds__(kSetupThreads) grouped_setup_kernel(const Setu
         const int slices = (n + 15) / 16;
         for (int b = g0 + lane; b < g0 + n; b += 32) {
             const int L = clamped_len(p, b);
-            p.members[b] = Member{g, L - P, 0, 0};
+            p.group_of[b] = g;
             p.tail_lens[b] = L - P;
             if (L == 0) {  // nothing to attend to: the output is zero
                 uint4 *o = reinterpret_cast<uint4 *>(p.out + size_t(b) * H * kD);
@@ -176,7 +178,8 @@ __global__ void __launch_bounds__(kSetupThreads) grouped_setup_kernel(const Setu
         return;
     }
 
-    // C: the chunk descriptors, and the tail tables
+    // C: the chunk descriptors, the member records, and the tail tables (a
+    // warp per member: its table row from block P / bs on)
     for (int g = warp; g < G; g += kSetupThreads / 32) {
         const Group gg = gr[g];
         const int slices = (gg.n + 15) / 16;
@@ -188,11 +191,16 @@ __global__ void __launch_bounds__(kSetupThreads) grouped_setup_kernel(const Setu
         }
     }
     const int MB = p.max_blocks;
-    for (size_t i = tid; i < size_t(B) * MB; i += kSetupThreads) {
-        const int b = int(i / MB), k = int(i % MB);
-        const int g = p.members[b].group;
-        const int pb = g >= 0 ? gr[g].P / bs : 0;
-        p.tail_tables[i] = pb + k < MB ? p.block_tables[size_t(b) * MB + pb + k] : -1;
+    for (int b = warp; b < B; b += kSetupThreads / 32) {
+        const int g = p.group_of[b];
+        const Group gg = g >= 0 ? gr[g] : Group{0, 0, 0, 0, 0, 0, 0, 0};
+        if (lane == 0 && g >= 0)
+            p.members[b] = Member{p.tail_lens[b], gg.cp, gg.colbase + (b - gg.g0), gg.n};
+        const int pb = gg.P / bs;
+        const int32_t *row = p.block_tables + size_t(b) * MB;
+        int32_t *trow = p.tail_tables + size_t(b) * MB;
+        for (int k = lane; k < MB; k += 32)
+            trow[k] = pb + k < MB ? row[pb + k] : -1;
     }
     if (tid == 0)
         *p.meta = Meta{nchunks, ncols, 0, 0};
@@ -204,9 +212,9 @@ __global__ void __launch_bounds__(kSetupThreads) grouped_setup_kernel(const Setu
 // tail's normalised fp16 result with its log-normaliser lse_t.  An empty
 // part has weight 0.  One warp per (member, head), four dims per lane.
 __global__ void __launch_bounds__(256) grouped_merge_kernel(
-    __half *__restrict__ out, const Group *__restrict__ groups, const Member *__restrict__ members,
-    const float *__restrict__ part_ml, const float *__restrict__ part_o,
-    const __half *__restrict__ o_t, const float *__restrict__ lse_t, int num_heads, int units)
+    __half *__restrict__ out, const Member *__restrict__ members, const float *__restrict__ part_ml,
+    const float *__restrict__ part_o, const __half *__restrict__ o_t, const float *__restrict__ lse_t,
+    int num_heads, int units)
 {
     pa::grid_dependency_wait();
     pa::allow_dependent_launch();
@@ -214,12 +222,12 @@ __global__ void __launch_bounds__(256) grouped_merge_kernel(
     if (unit >= units)
         return;
     const int b = unit / num_heads, h = unit % num_heads;
+    // the tail's result does not depend on the member record: load both at once
+    const uint2 raw = reinterpret_cast<const uint2 *>(o_t + size_t(unit) * kD)[lane];
+    const float lse = lse_t[unit];
     const Member mb = members[b];
-    if (mb.group < 0)
-        return;
-    const Group G = groups[mb.group];
-    if (G.P + mb.tail == 0)
-        return;  // empty context: zeroed by the set-up kernel
+    if (mb.tail < 0 || mb.cp + mb.tail == 0)
+        return;  // in no group, or an empty context (zeroed by the set-up kernel)
     constexpr int kBatch = 4;
     float M = -INFINITY, den = 0.f, num[4] = {0.f, 0.f, 0.f, 0.f};
     auto add = [&](float m, float l, const float (&x)[4]) {
@@ -231,31 +239,30 @@ __global__ void __launch_bounds__(256) grouped_merge_kernel(
         for (int e = 0; e < 4; ++e)
             num[e] = fmaf(num[e], a, f * x[e]);
     };
-    for (int j0 = 0; j0 < G.cp; j0 += kBatch) {
+    for (int j0 = 0; j0 < mb.cp; j0 += kBatch) {
         float2 v[kBatch];
         float4 o[kBatch];
 #pragma unroll
         for (int c = 0; c < kBatch; ++c) {
-            if (j0 + c < G.cp) {
-                const size_t ix = size_t(G.colbase + (j0 + c) * G.n + (b - G.g0)) * num_heads + h;
+            if (j0 + c < mb.cp) {
+                const size_t ix = size_t(mb.col0 + (j0 + c) * mb.stride) * num_heads + h;
                 v[c] = reinterpret_cast<const float2 *>(part_ml)[ix];
                 o[c] = reinterpret_cast<const float4 *>(part_o + ix * kD)[lane];
             }
         }
 #pragma unroll
         for (int c = 0; c < kBatch; ++c) {
-            if (j0 + c < G.cp) {
+            if (j0 + c < mb.cp) {
                 const float x[4] = {o[c].x, o[c].y, o[c].z, o[c].w};
                 add(v[c].x, v[c].y, x);
             }
         }
     }
     if (mb.tail > 0) {
-        const uint2 raw = reinterpret_cast<const uint2 *>(o_t + size_t(unit) * kD)[lane];
         const float2 t01 = __half22float2(*reinterpret_cast<const __half2 *>(&raw.x));
         const float2 t23 = __half22float2(*reinterpret_cast<const __half2 *>(&raw.y));
         const float x[4] = {t01.x, t01.y, t23.x, t23.y};
-        add(lse_t[unit], 1.f, x);
+        add(lse, 1.f, x);
     }
     const float inv = 1.f / den;
     const __half2 r01 = __floats2half2_rn(num[0] * inv, num[1] * inv);
@@ -274,8 +281,8 @@ __global__ void __launch_bounds__(256) grouped_merge_kernel(
 // B ceil(max_context_len / 512): at most one column per member per 512
 // prefix tokens.
 struct Layout {
-    size_t meta, groups, members, chunks, part_ml, part_o, tail_tables, tail_lens, dec, o_t,
-        lse_t, total;
+    size_t meta, groups, members, group_of, chunks, part_ml, part_o, tail_tables, tail_lens, dec,
+        o_t, lse_t, total;
     int max_chunks;
 };
 
@@ -289,7 +296,8 @@ Layout layout(int num_seqs, int num_groups, int num_heads, int max_context_len, 
     w.meta = 0;
     w.groups = align256(sizeof(Meta));
     w.members = w.groups + align256(size_t(num_groups) * sizeof(Group));
-    w.chunks = w.members + align256(size_t(num_seqs) * sizeof(Member));
+    w.group_of = w.members + align256(size_t(num_seqs) * sizeof(Member));
+    w.chunks = w.group_of + align256(size_t(num_seqs) * sizeof(int32_t));
     w.part_ml = w.chunks + align256(cap * sizeof(Chunk));
     w.part_o = w.part_ml + align256(cap * num_heads * 2 * sizeof(float));
     w.tail_tables = w.part_o + align256(cap * num_heads * kD * sizeof(float));
@@ -410,6 +418,7 @@ extern "C" pa_status pa_decode_grouped(void *out, const void *q, const void *k_c
     sp.chunks = reinterpret_cast<Chunk *>(ws + w.chunks);
     sp.tail_tables = tail_tables;
     sp.tail_lens = tail_lens;
+    sp.group_of = reinterpret_cast<int32_t *>(ws + w.group_of);
     sp.dec_tickets = reinterpret_cast<unsigned int *>(
         ws + w.dec + pa_host::decode_ticket_offset(num_seqs, num_heads, kD));
     sp.err = err;
@@ -421,8 +430,6 @@ extern "C" pa_status pa_decode_grouped(void *out, const void *q, const void *k_c
     p.out = static_cast<__half *>(out);
     p.block_tables = block_tables;
     p.chunks = sp.chunks;
-    p.groups = groups;
-    p.members = members;
     p.meta = meta;
     p.part_ml = part_ml;
     p.part_o = part_o;
@@ -447,8 +454,8 @@ extern "C" pa_status pa_decode_grouped(void *out, const void *q, const void *k_c
     // 4. merge the parts
     const int units = num_seqs * num_heads;
     return launch_pdl(grouped_merge_kernel, dim3(unsigned((units + 7) / 8)), dim3(256), 0, s,
-                      static_cast<__half *>(out), static_cast<const Group *>(groups),
-                      static_cast<const Member *>(members), static_cast<const float *>(part_ml),
+                      static_cast<__half *>(out), static_cast<const Member *>(members),
+                      static_cast<const float *>(part_ml),
                       static_cast<const float *>(part_o), static_cast<const __half *>(o_t),
                       static_cast<const float *>(lse_t), num_heads, units) == cudaSuccess
                ? PA_OK

@@ -74,14 +74,8 @@ constexpr int kPBufs = 2;                   // P^T operand tiles
 constexpr uint32_t kOffQ = kSlots * kTile;
 constexpr uint32_t kOffP = kOffQ + kQSlots * kQTile;
 constexpr uint32_t kSmem = kOffP + kPBufs * kQTile + 1024;  // + 1024-byte alignment slack
-constexpr int kLoadWarps = 1;               // 2: K tiles and V tiles from separate warps
-constexpr int kLoadWarp = 8, kMmaWarp = 9, kLoadWarpV = 10;
-constexpr int kThreads = (kLoadWarps == 2 ? 11 : 10) * 32;
-// The loads are issued K(m), V(m - kVLag), K(m + 1), ...: a V tile is only
-// needed by its P.V, after the tile's score product and softmax, so issuing
-// it later lets it land about when it is used and keeps the shared-memory
-// slots holding data in flight rather than data waiting to be used.
-constexpr int kVLag = 0;
+constexpr int kLoadWarp = 8, kMmaWarp = 9;
+constexpr int kThreads = 10 * 32;
 constexpr uint32_t kTmemCols = 64;          // S0, S1, O0, O1: 16 columns each
 constexpr uint32_t kTmemO = 32;
 constexpr float kRescaleLog2 = 8.f;         // move a reference max only past this growth
@@ -104,9 +98,11 @@ struct Group {
     int g0, n, cp, P, colbase, pstart, pad0, pad1;
 };
 
-// A member: its group (-1: in none) and its tail length L_b - P.
+// A member b of group g: its tail length L_b - P_g (-1: in no group), its
+// number of prefix chunks cp_g, and the partial column of its first prefix
+// chunk (chunk j is column col0 + j * stride).
 struct Member {
-    int group, tail, pad0, pad1;
+    int tail, cp, col0, stride;
 };
 
 struct Meta {
@@ -119,8 +115,6 @@ struct Params {
     __half *out;                      // [B, H, D]
     const int32_t *block_tables;      // [B, MB]
     const Chunk *chunks;
-    const Group *groups;
-    const Member *members;
     const Meta *meta;
     float *part_ml;                   // [columns, H, 2]: (reference max, sum)
     float *part_o;                    // [columns, H, D]
@@ -253,25 +247,17 @@ __device__ __forceinline__ void load_chunk_ids(const Params &p, const Chunk &c, 
     }
 }
 
-// Which loads a load warp issues: both kinds (one load warp), or only the K
-// tiles with the item hand-off and the Q rows, or only the V tiles (two).
-enum LoadPart { kLoadAll = 0, kLoadK = 1, kLoadV = 2 };
-
 // This CTA's items are blockIdx.x, blockIdx.x + gridDim.x, ... (numbered
-// chunk-major, prefix chunks first, so every CTA gets a like mix).  The
-// descriptors of 32 items at a time sit in the lanes' registers; the block
-// ids of the next item and the Q rows of the next item are fetched while the
-// current item's tiles are issued, so no dependent load stalls the stream.
-// Every load takes the shared-memory slot of its position: K(m) is at
-// position 2m and V(n) at 2n + 2 kVLag + 1, so slots 0, 2, 4 only ever hold
-// K tiles and slots 1, 3, 5 V tiles; positions 1, 3, .., 2 kVLag - 1 carry no
-// tile and complete their slot's phases at once.
-template <int kPart>
+// chunk-major, so every CTA gets a like mix).  The descriptors of 32 items at
+// a time sit in the lanes' registers; the block ids of the next item and the
+// Q rows of the next item are fetched while the current item's tiles are
+// issued, so no dependent load stalls the stream.  Tile m's K goes to slot
+// (2m) % kSlots and its V to slot (2m + 1) % kSlots, so slots 0, 2, 4 only
+// ever hold K tiles and slots 1, 3, 5 V tiles.
 __device__ __forceinline__ void load_role(const CUtensorMap *tm_q, const CUtensorMap *tm_k,
                                           const CUtensorMap *tm_v, const Params &p, Shared &sh,
                                           uint32_t sbase, int lane, int total)
 {
-    constexpr bool kDoK = kPart != kLoadV, kDoV = kPart != kLoadK;
     volatile int *abort = &sh.abort;
     unsigned int *err = p.error_word;
     const int H = p.num_heads, bs = p.block_size;
@@ -322,7 +308,6 @@ __device__ __forceinline__ void load_role(const CUtensorMap *tm_q, const CUtenso
     };
     struct TileRef {
         int y8;     // this lane's run: first 8-row group (valid when ok)
-        int runs;   // 0: no tile
         bool ok;    // this lane has a run and its block id is in range
     };
     auto issue = [&](int kind, const TileRef &t, int i) {
@@ -335,14 +320,8 @@ __device__ __forceinline__ void load_role(const CUtensorMap *tm_q, const CUtenso
                 return false;
         }
         const uint32_t bytes = uint32_t(__popc(__ballot_sync(kFullMask, t.ok))) * uint32_t(box) * 256u;
-        if (lane == 0) {
-            if (t.runs > 0) {
-                mbar_arrive_expect_tx(full, bytes);
-            } else {
-                mbar_arrive(full);
-                mbar_arrive(smem_u32(&sh.kv_empty[s]));
-            }
-        }
+        if (lane == 0)
+            mbar_arrive_expect_tx(full, bytes);
         last_use[s] = use;
         __syncwarp();
         if (t.ok)
@@ -350,21 +329,15 @@ __device__ __forceinline__ void load_role(const CUtensorMap *tm_q, const CUtenso
                         0, 0, 0, t.y8, full);
         return true;
     };
-    const TileRef none{0, 0, false};
-    TileRef hist[kVLag + 1];
-    int m = 0;  // tiles seen
+    int m = 0;  // tiles issued
     bool go = true;
-    if (kPart == kLoadV)  // the V positions before V(0) carry no tile
-        for (int f = 0; go && f < kVLag; ++f)
-            go = issue(1, none, 2 * f + 1);
     fetch(0);
     Chunk c{};
     int ids[2] = {0, 0};
     if (nitems > 0) {
         c = chunk_of(0);
         load_chunk_ids(p, c, box, lane, ids);
-        if (kDoK)
-            go = go && issue_q(0, c);
+        go = issue_q(0, c);
     }
     int items = 0;
     for (; go; ++items) {
@@ -378,7 +351,7 @@ __device__ __forceinline__ void load_role(const CUtensorMap *tm_q, const CUtenso
             cn = chunk_of(items + 1);
             load_chunk_ids(p, cn, box, lane, ids_n);
         }
-        if (kDoK) {
+        {
             const int slot = items % kItemRing, use = items / kItemRing;
             bool ok = true;
             if (use > 0 && lane == 0)
@@ -393,14 +366,8 @@ __device__ __forceinline__ void load_role(const CUtensorMap *tm_q, const CUtenso
             }
             __syncwarp();
         }
-        if (kk < 0) {
-            // one load warp: the V loads still owed to the last tiles
-            if (kPart == kLoadAll)
-                for (int f = 0; go && f < kVLag; ++f, ++m)
-                    go = issue(0, none, 2 * m) &&
-                         issue(1, m - kVLag >= 0 ? hist[(m - kVLag) % (kVLag + 1)] : none, 2 * m + 1);
+        if (kk < 0)
             break;
-        }
         const int nt = chunk_tiles(c);
         const int runs_per_tile = kT / box;
         for (int j = 0; go && j < nt; ++j, ++m) {
@@ -411,22 +378,13 @@ __device__ __forceinline__ void load_role(const CUtensorMap *tm_q, const CUtenso
             const int b = __shfl_sync(kFullMask, ids[1], run & 31);
             const int id = (run >> 5) ? b : a;
             TileRef t;
-            t.runs = runs;
             t.ok = lane < runs && unsigned(id) < unsigned(p.num_blocks);
-            if (kDoK && lane < runs && !t.ok)
+            if (lane < runs && !t.ok)
                 atomicOr(err, PA_DEVERR_BLOCK_ID);
             t.y8 = (id * H + h) * (bs / 8);  // first 8-row group of the run
-            if (kPart == kLoadAll) {
-                hist[m % (kVLag + 1)] = t;
-                go = issue(0, t, 2 * m) &&
-                     issue(1, m >= kVLag ? hist[(m - kVLag) % (kVLag + 1)] : none, 2 * m + 1);
-            } else if (kPart == kLoadK) {
-                go = issue(0, t, 2 * m);
-            } else {
-                go = issue(1, t, 2 * m + 2 * kVLag + 1);
-            }
+            go = issue(0, t, 2 * m) && issue(1, t, 2 * m + 1);
         }
-        if (kDoK && go && has_next)
+        if (go && has_next)
             go = issue_q(items + 1, cn);
         c = cn;
         ids[0] = ids_n[0];
@@ -514,7 +472,7 @@ __device__ __forceinline__ void mma_role(const Params &p, Shared &sh, uint32_t s
         }
         if (np < ns) {
             const PvInfo f = pend[np & 3];
-            const int vpos = 2 * np + 2 * kVLag + 1;  // V(np)'s load position
+            const int vpos = 2 * np + 1;  // V(np)'s load position
             const int pb = np % kPBufs, ob = f.u & 1, vs = vpos % kSlots;
             if (mbar_test_wait(smem_u32(&sh.p_full[pb]), uint32_t(np / kPBufs) & 1u) &&
                 mbar_test_wait(smem_u32(&sh.kv_full[vs]), uint32_t(vpos / kSlots) & 1u) &&
@@ -851,12 +809,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int total = p.meta->nchunks * p.num_heads;
 
     if (warp == kLoadWarp) {
-        if (kLoadWarps == 2)
-            load_role<kLoadK>(&tm_q, &tm_k, &tm_v, p, sh, sbase, lane, total);
-        else
-            load_role<kLoadAll>(&tm_q, &tm_k, &tm_v, p, sh, sbase, lane, total);
-    } else if (kLoadWarps == 2 && warp == kLoadWarpV) {
-        load_role<kLoadV>(&tm_q, &tm_k, &tm_v, p, sh, sbase, lane, total);
+        load_role(&tm_q, &tm_k, &tm_v, p, sh, sbase, lane, total);
     } else if (warp == kMmaWarp) {
         if (lane == 0)
             mma_role(p, sh, sbase, smem);

@@ -73,6 +73,8 @@ class PagedWorkload:
     slot_mapping: np.ndarray          # [N] int64
     copy_pairs: np.ndarray = field(default_factory=lambda: np.zeros((0, 2), np.int64))
     alias_block_tables: np.ndarray | None = None   # config 4: tables before the CoW copy
+    group_start: np.ndarray | None = None   # config 4: [G + 1] first sequence of each group
+    prefix_lens: np.ndarray | None = None   # config 4: [G] tokens the copy-on-write tables share
     logical_k: list | None = None     # per sequence [H, L, D] fp16 (small configs only)
     logical_v: list | None = None
     device_k: list | None = None      # per sequence [H, L, D] fp16 on the device (on request)
@@ -318,12 +320,16 @@ def make_shared_prefix(device="cpu", seed: int = 4, num_groups: int = 8,
                 lk.append(torch.cat([pk, tk], dim=1).cpu())
                 lv.append(torch.cat([pv, tv], dim=1).cpu())
     slots = _newest_token_slots(lens, cow_tables, bs)
+    # after the copy-on-write, a group's members share all prefix blocks but the last
+    group_start = (np.arange(num_groups + 1) * group_size).astype(np.int32)
+    prefix_lens = np.full(num_groups, prefix_len - bs, dtype=np.int32)
     return PagedWorkload(name=WORKLOAD_NAMES[4], seed=seed, num_heads=h, head_dim=d,
                          block_size=bs, num_blocks=nb, scale=1.0 / math.sqrt(d),
                          context_lens=lens, block_tables=cow_tables, q=q, k_cache=k_cache,
                          v_cache=v_cache, new_key=new_key, new_value=new_value,
                          slot_mapping=slots, copy_pairs=pairs,
-                         alias_block_tables=alias_tables, logical_k=lk, logical_v=lv)
+                         alias_block_tables=alias_tables, group_start=group_start,
+                         prefix_lens=prefix_lens, logical_k=lk, logical_v=lv)
 
 
 def make_random(seed: int, lens, num_heads: int, head_dim: int, block_size: int,
