@@ -34,33 +34,34 @@ WorkspaceLayout workspace_layout(int num_seqs, int num_heads, int head_dim)
     return w;
 }
 
-template <int D, bool kInt8, int NW, int S>
-pa_status launch_decode(const pa::DecodeParams &p, const pa::DecodeExtras &x, cudaStream_t stream)
+template <int D, bool kInt8, int NW, int S, bool kLateDepWait = false>
+pa_status launch_decode(const pa::DecodeParams &p, const pa::DecodeExtras &x, cudaStream_t stream,
+                        int max_ctas = 0)
 {
     using Sm = pa::DecodeSmem<D, kInt8, NW, S>;
+    constexpr auto kernel = pa::paged_decode_kernel<D, kInt8, NW, S, kLateDepWait>;
     static std::atomic<int> grid_for[kMaxDevices];  // 0 = not configured yet
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices)
         return PA_ERR_CUDA;
     int grid = grid_for[dev].load(std::memory_order_acquire);
     if (grid == 0) {
-        if (cudaFuncSetAttribute(pa::paged_decode_kernel<D, kInt8, NW, S>,
-                                 cudaFuncAttributeMaxDynamicSharedMemorySize,
+        if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  int(Sm::kBytes)) != cudaSuccess)
             return PA_ERR_CUDA;
         int sms = 0, per_sm = 0;
         if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess ||
-            cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm,
-                                                          pa::paged_decode_kernel<D, kInt8, NW, S>,
-                                                          Sm::kThreads, Sm::kBytes) != cudaSuccess)
+            cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kernel, Sm::kThreads, Sm::kBytes) !=
+                cudaSuccess)
             return PA_ERR_CUDA;
         grid = sms * (per_sm > 0 ? per_sm : 1);
         if (grid * NW > pa::kMaxWorkers)
             grid = pa::kMaxWorkers / NW;
         grid_for[dev].store(grid, std::memory_order_release);
     }
-    return launch_pdl(pa::paged_decode_kernel<D, kInt8, NW, S>, dim3(grid), dim3(Sm::kThreads),
-                      Sm::kBytes, stream, p, x) == cudaSuccess
+    if (max_ctas > 0 && max_ctas < grid)
+        grid = max_ctas;
+    return launch_pdl(kernel, dim3(grid), dim3(Sm::kThreads), Sm::kBytes, stream, p, x) == cudaSuccess
                ? PA_OK
                : PA_ERR_CUDA;
 }
@@ -143,7 +144,8 @@ pa_status decode_common(void *out, const void *q, const void *k_cache, const voi
                         int num_heads, int head_dim, int block_size, int num_blocks, float scale,
                         void *workspace, size_t workspace_bytes, pa_stream_t stream,
                         const void *new_k = nullptr, const void *new_v = nullptr,
-                        const int64_t *new_slots = nullptr, float *lse = nullptr)
+                        const int64_t *new_slots = nullptr, float *lse = nullptr,
+                        int max_ctas = 0, bool late_dep_wait = false)
 {
     if (num_seqs < 0 || num_heads <= 0 || num_blocks <= 0 || max_context_len < 0 ||
         max_blocks_per_seq < 0)
@@ -200,9 +202,14 @@ pa_status decode_common(void *out, const void *q, const void *k_cache, const voi
             return launch_decode<128, true, kDecodeWarps, kDecodeStages>(p, x, s);
         return launch_decode<64, true, kDecodeWarps, kDecodeStages>(p, x, s);
     }
+    if (late_dep_wait) {
+        if (head_dim == 128)
+            return launch_decode<128, false, kDecodeWarps, kDecodeStages, true>(p, x, s, max_ctas);
+        return launch_decode<64, false, kDecodeWarps, kDecodeStages, true>(p, x, s, max_ctas);
+    }
     if (head_dim == 128)
-        return launch_decode<128, false, kDecodeWarps, kDecodeStages>(p, x, s);
-    return launch_decode<64, false, kDecodeWarps, kDecodeStages>(p, x, s);
+        return launch_decode<128, false, kDecodeWarps, kDecodeStages>(p, x, s, max_ctas);
+    return launch_decode<64, false, kDecodeWarps, kDecodeStages>(p, x, s, max_ctas);
 }
 
 } // namespace
@@ -346,10 +353,24 @@ pa_status pa_host::decode_with_lse(void *out, const void *q, const void *k_cache
                                    int max_blocks_per_seq, const int32_t *context_lens,
                                    int max_context_len, int num_seqs, int num_heads, int head_dim,
                                    int block_size, int num_blocks, float scale, void *workspace,
-                                   size_t workspace_bytes, float *lse, pa_stream_t stream)
+                                   size_t workspace_bytes, float *lse, pa_stream_t stream,
+                                   int max_ctas, bool late_dep_wait)
 {
     return decode_common(out, q, k_cache, v_cache, nullptr, nullptr, false, block_tables,
                          max_blocks_per_seq, context_lens, max_context_len, num_seqs, num_heads,
                          head_dim, block_size, num_blocks, scale, workspace, workspace_bytes, stream,
-                         nullptr, nullptr, nullptr, lse);
+                         nullptr, nullptr, nullptr, lse, max_ctas, late_dep_wait);
+}
+
+int pa_host::decode_ctas_per_sm()
+{
+    constexpr auto kernel = pa::paged_decode_kernel<128, false, kDecodeWarps, kDecodeStages, true>;
+    using Sm = pa::DecodeSmem<128, false, kDecodeWarps, kDecodeStages>;
+    int per_sm = 0;
+    if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, int(Sm::kBytes)) !=
+            cudaSuccess ||
+        cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kernel, Sm::kThreads, Sm::kBytes) !=
+            cudaSuccess)
+        return 0;
+    return per_sm;
 }

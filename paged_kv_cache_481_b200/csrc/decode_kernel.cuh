@@ -623,7 +623,7 @@ __device__ __forceinline__ void merge_partials(const DecodeParams &p, const Deco
 }
 
 template <int D, bool kInt8, int NW, int S>
-__global__ void __launch_bounds__(NW * 32) paged_decode_kernel(const DecodeParams p, const DecodeExtras x)
+__device__ __forceinline__ void paged_decode_body(const DecodeParams &p, const DecodeExtras &x)
 {
     using Sh = DecodeShape<D, kInt8>;
     using Sm = DecodeSmem<D, kInt8, NW, S>;
@@ -645,11 +645,6 @@ __global__ void __launch_bounds__(NW * 32) paged_decode_kernel(const DecodeParam
             raise_device_error(kErrTimeout);
         return;
     }
-
-    // Inputs may come from the previous kernel in the stream: read none before
-    // it has finished.  The next kernel may start launching meanwhile.
-    grid_dependency_wait();
-    allow_dependent_launch();
 
     // Bring the small inputs every worker looks up (context lengths, block
     // tables, q) into L2 while the scan below runs; the CTAs split the lines.
@@ -964,6 +959,25 @@ __global__ void __launch_bounds__(NW * 32) paged_decode_kernel(const DecodeParam
         if (r == 0)
             merge_partials<D, kDims>(p, x, out_row, c, u_start, w_first, w_last, total, workers);
     }
+}
+
+// kLateDepWait = false: inputs may come from the previous kernel in the
+// stream, so none is read before it has finished; the next kernel may start
+// launching meanwhile.  kLateDepWait = true: the caller guarantees the
+// inputs are ready (they were written two launches back and the previous
+// kernel only starts this one after it has itself waited for them), so the
+// work starts at once, running beside the previous kernel, and the wait for
+// that kernel comes at the end: this grid then completes only after the
+// previous one, and the next kernel that waits for this grid sees both.
+template <int D, bool kInt8, int NW, int S, bool kLateDepWait = false>
+__global__ void __launch_bounds__(NW * 32) paged_decode_kernel(const DecodeParams p, const DecodeExtras x)
+{
+    if (!kLateDepWait)
+        grid_dependency_wait();
+    allow_dependent_launch();
+    paged_decode_body<D, kInt8, NW, S>(p, x);
+    if (kLateDepWait && threadIdx.x == 0)
+        grid_dependency_wait();
 }
 
 } // namespace pa

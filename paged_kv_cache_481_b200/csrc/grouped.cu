@@ -5,15 +5,19 @@
 //      tail table (its block-table row from the first block past the shared
 //      prefix) and tail length, zero outputs for empty contexts;
 //   2. the persistent tensor-core kernel of grouped_kernel.cuh over the
-//      prefix chunks, leaving (m, l, o) per member, head and chunk;
+//      prefix chunks, leaving (m, l, o) per member, head and chunk, on a
+//      share of the SMs (kPrefixSmShare);
 //   3. the paged decode kernel over the tails, with each (member, head)'s
-//      base-2 log-normaliser;
+//      base-2 log-normaliser, on the other SMs at the same time: it starts as
+//      soon as every prefix CTA is resident (programmatic dependent launch)
+//      and waits for the prefix kernel only at its end;
 //   4. a merge kernel: the prefix partials and the tail result combined by
 //      their softmax normalisers.
 // Nothing here allocates device memory.
 #include <cuda.h>
 #include <cuda_runtime.h>
 
+#include <algorithm>
 #include <atomic>
 #include <climits>
 #include <cmath>
@@ -53,6 +57,14 @@ struct SetupParams {
 };
 
 constexpr int kSetupThreads = 1024;
+
+// Share of the SMs the prefix kernel runs on; the tail decode takes the
+// rest.  Which part is larger is known only on the device, so the split is
+// fixed: a prefix SM streams a little slower than a decode SM (its pipeline
+// holds fewer tiles in flight), and this share balances prefixes and tails
+// of similar size (parallel samples of a prompt with tails of a few
+// hundred tokens).
+constexpr float kPrefixSmShare = 0.55f;
 
 __device__ __forceinline__ int clamped_len(const SetupParams &p, int b)
 {
@@ -439,15 +451,24 @@ extern "C" pa_status pa_decode_grouped(void *out, const void *q, const void *k_c
     p.num_blocks = num_blocks;
     p.qk_scale_log2 = float(double(scale) * 1.4426950408889634);
     p.error_word = err;
-    if (launch_pdl(pa::grp::grouped_decode_kernel, dim3(unsigned(sms)), dim3(pa::grp::kThreads),
-                   pa::grp::kSmem, s, tm_q, tm_k, tm_v, p) != cudaSuccess)
+    const int prefix_ctas = std::max(1, std::min(sms - 1, int(float(sms) * kPrefixSmShare + 0.5f)));
+    if (launch_pdl(pa::grp::grouped_decode_kernel, dim3(unsigned(prefix_ctas)),
+                   dim3(pa::grp::kThreads), pa::grp::kSmem, s, tm_q, tm_k, tm_v, p) != cudaSuccess)
         return PA_ERR_CUDA;
 
-    // 3. each member's own tail
+    // 3. each member's own tail, on the remaining SMs at the same time
+    static std::atomic<int> dec_per_sm[kMaxDevices];  // 0 = not configured yet
+    int per_sm = dec_per_sm[dev].load(std::memory_order_acquire);
+    if (per_sm == 0) {
+        per_sm = pa_host::decode_ctas_per_sm();
+        if (per_sm <= 0)
+            return PA_ERR_CUDA;
+        dec_per_sm[dev].store(per_sm, std::memory_order_release);
+    }
     const pa_status st = pa_host::decode_with_lse(
         o_t, q, k_cache, v_cache, tail_tables, max_blocks_per_seq, tail_lens, max_context_len,
         num_seqs, num_heads, head_dim, block_size, num_blocks, scale, ws + w.dec, w.o_t - w.dec, lse_t,
-        stream);
+        stream, per_sm * (sms - prefix_ctas), true);
     if (st != PA_OK)
         return st;
 

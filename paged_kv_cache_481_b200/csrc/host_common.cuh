@@ -19,11 +19,17 @@ unsigned int *device_error_word();
 // pa_decode that also writes each (sequence, head)'s softmax log-normaliser
 // lse = max + log2(sum) in base-2 units ([num_seqs, num_heads] fp32), so the
 // result can be merged with attention over other parts of the context.
+// max_ctas > 0 caps the persistent grid (to share the GPU with the kernel
+// launched before it); late_dep_wait: see paged_decode_kernel's kLateDepWait.
 pa_status decode_with_lse(void *out, const void *q, const void *k_cache, const void *v_cache,
                           const int32_t *block_tables, int max_blocks_per_seq,
                           const int32_t *context_lens, int max_context_len, int num_seqs,
                           int num_heads, int head_dim, int block_size, int num_blocks, float scale,
-                          void *workspace, size_t workspace_bytes, float *lse, pa_stream_t stream);
+                          void *workspace, size_t workspace_bytes, float *lse, pa_stream_t stream,
+                          int max_ctas = 0, bool late_dep_wait = false);
+
+// CTAs of the fp16, head-dim-128 decode kernel that fit on one SM (0 on error).
+int decode_ctas_per_sm();
 
 // Byte offset of the merge tickets (one unsigned per (sequence, head), zero
 // between calls) inside pa_decode's workspace for these sizes.
