@@ -3,6 +3,9 @@
     python bench.py [--gpus N] [--steps K] [--warmup W] [--workload C] [--block-size BS]
     python bench.py --kv-dtype int8 ...      # the same step over the int8 cache
     python bench.py --path prefill ...       # prompt cache write + pa_prefill, TFLOP/s
+    python bench.py --workload 4 ...         # shared prefixes through pa_decode_grouped
+    python bench.py --decode-only ...        # pa_decode alone over the paged pool
+    python bench.py --layout contiguous ...  # the same decode, contiguous K / V, no block table
     python bench.py --impl reference ...     # the fp64 CPU oracle, same metric
 
 One step = one decode iteration of the whole hot path over one batch: the
@@ -10,7 +13,8 @@ cache write of each sequence's newest token and the decode over all
 (sequence, head) pairs -- fused into one pa_decode_append launch
 (pa_decode_append_int8 for the int8 cache; --unfused: the cache write, then
 the decode) -- and, for the shared-prefix workload, the
-copy-on-write pa_copy_blocks before them.  The default workload is the LLaMA-13B-shaped
+copy-on-write pa_copy_blocks before them and the decode done by pa_decode_grouped
+(each shared prefix read once per group and head).  The default workload is the LLaMA-13B-shaped
 single-layer decode batch (B=32, H=40, D=128, bs=16, context U[256, 2048]).
 
 Under torchrun each rank runs its own batch (a different seed) on its own GPU:
@@ -530,6 +534,33 @@ def run_gpu(args):
                                             device=dev)
         fused = False
 
+    # decode alone (the newest tokens written once before timing): over the
+    # paged pool (--decode-only), or over a contiguous copy of the same
+    # values with no block table (--layout contiguous)
+    contig = args.layout == "contiguous"
+    decode_only = (args.decode_only or contig) and not grouped
+    if decode_only:
+        if pairs is not None or int8:
+            raise SystemExit("--decode-only / --layout contiguous: workloads 1, 2, 3 and 5, fp16")
+        write_step(key, value, slots)
+        fused = False
+    if contig:
+        # gather each sequence's blocks into [B, H, Lmax, D] (the same values)
+        kcont = torch.zeros((b, h, mcl, d), dtype=torch.float16, device=dev)
+        vcont = torch.zeros_like(kcont)
+        bsz = wl.block_size
+        for i, length in enumerate(wl.context_lens):
+            length = int(length)
+            nblk = (length + bsz - 1) // bsz
+            ids = tables[i, :nblk].long()
+            for src, dst in ((kc, kcont), (vc, vcont)):
+                dst[i, :, :length] = src.index_select(0, ids).permute(1, 0, 2, 3).reshape(
+                    h, nblk * bsz, d)[:, :length]
+        torch.cuda.synchronize()
+
+    def contig_step(o, q_, lens_):
+        binding.pa_decode_contiguous(o, q_, kcont, vcont, lens_, mcl, wl.scale, ws, stream=stream)
+
     def grouped_step(o, q_, tables_, lens_, gs_, pl_):
         binding.pa_decode_grouped(o, q_, kc, vc, tables_, lens_, mcl, gs_, pl_, max_group,
                                   wl.scale, gws, stream=stream)
@@ -545,11 +576,13 @@ def run_gpu(args):
     def step(ev_pair=None):
         if pairs is not None:
             copy_step()
-        if not fused:
+        if not fused and not decode_only:
             write_step(key, value, slots)
         if ev_pair is not None:
             ev_pair[0].record(stream)
-        if grouped:
+        if contig:
+            contig_step(out, q, lens)
+        elif grouped:
             grouped_step(out, q, tables, lens, d_gs, d_pl)
         elif fused:
             append_step(out, q, key, value, slots, tables, lens)
@@ -558,7 +591,8 @@ def run_gpu(args):
         if ev_pair is not None:
             ev_pair[1].record(stream)
 
-    launches_per_step = ((1 if fused else 2) + ((4 if int8 else 1) if pairs is not None else 0)
+    launches_per_step = (1 if decode_only else
+                         (1 if fused else 2) + ((4 if int8 else 1) if pairs is not None else 0)
                          + (3 if grouped else 0))
     with torch.cuda.stream(stream):
         for _ in range(args.warmup):
@@ -601,7 +635,11 @@ def run_gpu(args):
         d_q, d_key, d_value, d_slots, d_tables, d_lens = views[:6]
         if pairs is not None:
             copy_step()
-        if grouped:
+        if contig:
+            contig_step(o, d_q, d_lens)
+        elif decode_only:
+            decode_step(o, d_q, d_tables, d_lens)
+        elif grouped:
             write_step(d_key, d_value, d_slots)
             grouped_step(o, d_q, d_tables, d_lens, views[6], views[7])
         elif fused:
@@ -611,6 +649,8 @@ def run_gpu(args):
             decode_step(o, d_q, d_tables, d_lens)
 
     e2e_parts = [q, key, value, slots, tables, lens] + ([d_gs, d_pl] if grouped else [])
+    if decode_only:  # the step's inputs: q, (tables,) context lengths
+        e2e_parts = [q, key[:1], value[:1], slots[:1], tables if not contig else tables[:1], lens]
     e2e_ms, h2d, d2h = pipelined_e2e(e2e_parts, out, decode_from, stream, args.warmup, args.steps,
                                      world)
     assert binding.pa_get_last_device_error() == 0
@@ -625,7 +665,8 @@ def run_gpu(args):
                                                     wl.block_size)
     if fused:  # the fused launch also writes each new K and V row to the cache
         roof_bytes += 2 * b * h * (d + 8) if int8 else 2 * b * h * d * 2
-    step_bytes = dec_bytes + (b * h * (2 * d * 2 + 2 * (d + 8)) if int8
+    step_bytes = dec_bytes + (0 if decode_only else
+                              b * h * (2 * d * 2 + 2 * (d + 8)) if int8
                               else accounting.cache_write_bytes(b, h, d))
     if pairs is not None:
         step_bytes += accounting.copy_blocks_bytes(len(wl.copy_pairs), h, d, wl.block_size)
@@ -643,7 +684,9 @@ def run_gpu(args):
         desc = _workload_desc(wl, cfg)
         kv_bytes = dec_bytes
         desc.update({
-            "step": ("pa_copy_blocks + " if pairs is not None else "")
+            "step": "pa_decode_contiguous (K / V [B, H, Lmax, D], no block table)" if contig else
+                    "pa_decode (the newest tokens written before timing)" if decode_only else
+                    ("pa_copy_blocks + " if pairs is not None else "")
                     + (f"pa_reshape_and_cache({b} tokens) + pa_decode_grouped "
                        f"({len(wl.prefix_lens)} groups, prefixes of {int(wl.prefix_lens[0])} tokens)"
                        if grouped else
@@ -654,6 +697,7 @@ def run_gpu(args):
                   f"vs {L2_BYTES / 2**20:.0f} MiB L2 (no flush)",
             "parallelism": f"dp{world} (independent batches per GPU)",
             "placement": args.placement,
+            "layout": args.layout,
             "kv_cache": ("int8 codes + fp32 (s, z) per row" if int8 else "fp16"),
         })
         result = {
@@ -677,11 +721,12 @@ def run_gpu(args):
             "roofline": {
                 "kernel": ("pa_decode_grouped (set-up, grouped_decode_kernel, paged_decode_kernel "
                            "over the tails, merge)" if grouped else
+                           "paged_decode_kernel<contiguous>" if contig else
                            "paged_decode_kernel" + ("<int8>" if int8 else "")), "bound": "hbm",
                 "achieved": achieved,
                 "peak": peak, "peak_kind": f"{peak_kind} (hbm_gbs)", "unit": "GB/s",
                 "frac": achieved / peak,
-                "traffic": None if int8 else _recorded_traffic(
+                "traffic": None if int8 or contig else _recorded_traffic(
                     desc["workload"], "pa_decode_grouped" if grouped else
                     "pa_decode_append" if fused else "pa_decode",
                     "grouped" if grouped else "decode"),
@@ -907,6 +952,11 @@ def main(argv=None):
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--unfused", action="store_true",
                     help="time the cache write and the decode as two launches")
+    ap.add_argument("--layout", choices=["paged", "contiguous"], default="paged",
+                    help="contiguous: the same decode over K / V [B, H, Lmax, D] with no block "
+                         "table (the baseline for the indirection's cost); times the decode alone")
+    ap.add_argument("--decode-only", action="store_true",
+                    help="time pa_decode alone (the newest tokens written before timing)")
     ap.add_argument("--no-grouped", action="store_true",
                     help="shared-prefix workload: plain pa_decode instead of pa_decode_grouped")
     ap.add_argument("--path", choices=["decode", "prefill"], default="decode",

@@ -161,6 +161,24 @@ PA_API pa_status pa_copy_blocks(void *k_cache, void *v_cache, const int64_t *blo
                          int num_blocks, pa_stream_t stream);
 
 /*
+ * Contiguous-cache baseline (polomodov.tech "vLLM and PagedAttention", slide
+ * 19: the paged kernel against one that reads a contiguous cache).  The same
+ * decode as pa_decode, but over K / V kept contiguous per (sequence, head):
+ *   k, v  [num_seqs, num_heads, seq_stride, head_dim] fp16, token t of
+ *         sequence b, head h at ((b * H + h) * seq_stride + t) * D,
+ * so every address follows from the position and no block table is read.
+ * It exists to measure what the paged layout's indirection costs; results
+ * equal pa_decode's over the same values.  max_context_len <= seq_stride;
+ * the workspace is pa_decode's (pa_decode_workspace_size, zeroed once).
+ * Other rules as pa_decode.
+ */
+PA_API pa_status pa_decode_contiguous(void *out, const void *q, const void *k, const void *v,
+                                      const int32_t *context_lens, int max_context_len,
+                                      int seq_stride, int num_seqs, int num_heads, int head_dim,
+                                      float scale, void *workspace, size_t workspace_bytes,
+                                      pa_stream_t stream);
+
+/*
  * pa_decode without a caller-supplied workspace, for callers that cannot
  * allocate device memory at decode time (for example a serving engine that
  * has reserved nearly all free HBM for its KV block pool, or a loop that

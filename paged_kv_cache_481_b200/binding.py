@@ -36,7 +36,7 @@ EXPORTED = ("pa_reshape_and_cache", "pa_decode_workspace_size", "pa_decode_works
             "pa_copy_blocks_raw", "pa_prefill", "pa_swap_blocks", "pa_bm_create_with_swap",
             "pa_bm_num_free_cpu", "pa_bm_cpu_refcount", "pa_bm_is_swapped", "pa_bm_swap_out",
             "pa_bm_swap_in", "pa_decode_append", "pa_decode_grouped_workspace_size",
-            "pa_decode_grouped")
+            "pa_decode_grouped", "pa_decode_contiguous")
 
 _lock = threading.Lock()
 _lib = None
@@ -102,6 +102,9 @@ def load(path: str | None = None):
         lib.pa_copy_blocks_raw.argtypes = [vp, sz, vp, i32, i32, vp]
         lib.pa_copy_blocks_raw.restype = i32
         lib.pa_decode_grouped_workspace_size.argtypes = [i32, i32, i32, i32, i32, i32]
+        lib.pa_decode_contiguous.argtypes = [vp, vp, vp, vp, vp, i32, i32, i32, i32, i32,
+                                             ctypes.c_float, vp, sz, vp]
+        lib.pa_decode_contiguous.restype = i32
         lib.pa_decode_grouped_workspace_size.restype = sz
         lib.pa_decode_grouped.argtypes = [vp, vp, vp, vp, vp, i32, vp, i32, vp, vp, i32, i32, i32,
                                           i32, i32, i32, i32, ctypes.c_float, vp, sz, vp]
@@ -301,6 +304,22 @@ def pa_decode_grouped(out, q, k_cache, v_cache, block_tables, context_lens, max_
                                     _ptr(workspace), workspace.numel() * workspace.element_size(),
                                     _stream(stream)),
            "pa_decode_grouped")
+
+
+def pa_decode_contiguous(out, q, k, v, context_lens, max_context_len, scale, workspace,
+                         stream=None):
+    """The contiguous-cache baseline: decode over K / V [B, H, Lmax, D] laid
+    out contiguously per (sequence, head), no block table."""
+    b, h, d = q.shape
+    bk, hk, lmax, dk = k.shape
+    assert q.dtype == out.dtype == k.dtype == v.dtype == torch.float16
+    assert out.shape == q.shape and (bk, hk, dk) == (b, h, d) and v.shape == k.shape
+    assert context_lens.dtype == torch.int32
+    _check(load().pa_decode_contiguous(_ptr(out), _ptr(q), _ptr(k), _ptr(v), _ptr(context_lens),
+                                       int(max_context_len), lmax, b, h, d, float(scale),
+                                       _ptr(workspace), workspace.numel() * workspace.element_size(),
+                                       _stream(stream)),
+           "pa_decode_contiguous")
 
 
 def pa_decode_no_alloc(out, q, k_cache, v_cache, block_tables, context_lens, max_context_len,

@@ -34,12 +34,12 @@ WorkspaceLayout workspace_layout(int num_seqs, int num_heads, int head_dim)
     return w;
 }
 
-template <int D, bool kInt8, int NW, int S, bool kLateDepWait = false>
+template <int D, bool kInt8, int NW, int S, bool kLateDepWait = false, bool kContig = false>
 pa_status launch_decode(const pa::DecodeParams &p, const pa::DecodeExtras &x, cudaStream_t stream,
                         int max_ctas = 0)
 {
     using Sm = pa::DecodeSmem<D, kInt8, NW, S>;
-    constexpr auto kernel = pa::paged_decode_kernel<D, kInt8, NW, S, kLateDepWait>;
+    constexpr auto kernel = pa::paged_decode_kernel<D, kInt8, NW, S, kLateDepWait, kContig>;
     static std::atomic<int> grid_for[kMaxDevices];  // 0 = not configured yet
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices)
@@ -272,6 +272,59 @@ pa_status pa_decode_int8(void *out, const void *q, const void *k_codes, const vo
 }
 
 } // extern "C"
+
+// ---------------------------------------------------------------------------
+// The contiguous-cache baseline: the same decode over per-(sequence, head)
+// contiguous K / V, [B, H, seq_stride, D], addresses computed from the
+// position with no block table.
+
+extern "C" pa_status pa_decode_contiguous(void *out, const void *q, const void *k, const void *v,
+                                          const int32_t *context_lens, int max_context_len,
+                                          int seq_stride, int num_seqs, int num_heads, int head_dim,
+                                          float scale, void *workspace, size_t workspace_bytes,
+                                          pa_stream_t stream)
+{
+    if (num_seqs < 0 || num_heads <= 0 || max_context_len < 0 || seq_stride <= 0 ||
+        max_context_len > seq_stride)
+        return PA_ERR_INVALID_ARG;
+    if (!supported_head_dim(head_dim))
+        return PA_ERR_UNSUPPORTED;
+    if (!std::isfinite(scale))
+        return PA_ERR_INVALID_ARG;
+    if (num_seqs == 0)
+        return PA_OK;
+    if (!out || !q || !k || !v || !context_lens)
+        return PA_ERR_INVALID_ARG;
+    if (!aligned16(out) || !aligned16(q) || !aligned16(k) || !aligned16(v) ||
+        (reinterpret_cast<uintptr_t>(context_lens) & 3u))
+        return PA_ERR_INVALID_ARG;
+    const WorkspaceLayout w = workspace_layout(num_seqs, num_heads, head_dim);
+    if (!workspace || workspace_bytes < w.total || !aligned16(workspace))
+        return PA_ERR_WORKSPACE;
+    unsigned char *ws = static_cast<unsigned char *>(workspace);
+    pa::DecodeParams p{};
+    p.out = static_cast<__half *>(out);
+    p.q = static_cast<const __half *>(q);
+    p.k_cache = k;
+    p.v_cache = v;
+    p.block_tables = nullptr;
+    p.context_lens = context_lens;
+    p.ws_o = reinterpret_cast<float *>(ws + w.o_off);
+    p.ws_ml = reinterpret_cast<float *>(ws + w.ml_off);
+    p.ws_count = reinterpret_cast<unsigned *>(ws + w.count_off);
+    p.num_seqs = num_seqs;
+    p.max_blocks_per_seq = 0;
+    p.max_context_len = max_context_len;
+    p.num_heads = num_heads;
+    p.block_size = seq_stride;  // rows per (sequence, head)
+    p.num_blocks = num_seqs;
+    p.qk_scale_log2 = float(double(scale) * 1.4426950408889634);
+    const pa::DecodeExtras x{};
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    if (head_dim == 128)
+        return launch_decode<128, false, kDecodeWarps, kDecodeStages, false, true>(p, x, s);
+    return launch_decode<64, false, kDecodeWarps, kDecodeStages, false, true>(p, x, s);
+}
 
 // ---------------------------------------------------------------------------
 // Allocation-free variant of pa_decode.

@@ -353,10 +353,16 @@ struct TileCursor {
 
 // Block ids of the tile under the cursor, loaded one tile ahead of their use;
 // they are range-checked when the copies are issued.
-template <class Sh>
+template <class Sh, bool kContig = false>
 __device__ __forceinline__ void load_tile_ids(const DecodeParams &p, const TileCursor &cur,
                                               int (&ids)[Sh::kMaxIds])
 {
+    if constexpr (kContig) {  // no table: addresses follow from the position
+#pragma unroll
+        for (int s = 0; s < Sh::kMaxIds; ++s)
+            ids[s] = 0;
+        return;
+    }
     const int bs = p.block_size;
     const int t0 = cur.i * Sh::kTokens;
     const int nv = min(Sh::kTokens, cur.len - t0);
@@ -404,7 +410,7 @@ __device__ __forceinline__ uint32_t rows_tx_bytes(int rows)
 // `with_q`).  K and V are read exactly once, so they go through L2 with an
 // evict-first policy that keeps the small reused data (block tables, q, split
 // partials) resident.
-template <int D, bool kInt8, class Sm>
+template <int D, bool kInt8, class Sm, bool kContig = false>
 __device__ __forceinline__ void issue_tile(const DecodeParams &p, const DecodeExtras &x,
                                            const TileCursor &cur,
                                            const int (&ids)[DecodeShape<D, kInt8>::kMaxIds],
@@ -427,6 +433,17 @@ __device__ __forceinline__ void issue_tile(const DecodeParams &p, const DecodeEx
     int nf = nv;
     if (x.new_slots && cur.i == cur.nt - 1 && x.new_slots[cur.b] >= 0)
         nf = nv - 1;
+    if constexpr (kContig) {
+        // contiguous layout [B, H, Lmax, D] (Lmax = block_size): the tile is
+        // one run of rows at ((b H + h) Lmax + t0)
+        mbar_arrive_expect_tx(bar, (with_q ? uint32_t(D * 2) : 0u) + rows_tx_bytes<D, kInt8>(nf));
+        if (with_q)
+            bulk_copy_g2s(dst + Sm::kOffQ, p.q + (size_t(cur.b) * p.num_heads + cur.h) * D, D * 2, bar);
+        if (nf > 0)
+            copy_rows<D, kInt8, Sm>(p, (size_t(cur.b) * p.num_heads + cur.h) * size_t(bs) + size_t(t0), nf,
+                                    dst, 0, bar, stream_policy);
+        return;
+    }
     // an id outside the pool is recorded and its rows are not fetched
     bool ok[Sh::kMaxIds];
 #pragma unroll
@@ -622,7 +639,7 @@ __device__ __forceinline__ void merge_partials(const DecodeParams &p, const Deco
         x.lse[(reinterpret_cast<const __half *>(out_row) - p.out) / D] = gmax + log2f(den);
 }
 
-template <int D, bool kInt8, int NW, int S>
+template <int D, bool kInt8, int NW, int S, bool kContig>
 __device__ __forceinline__ void paged_decode_body(const DecodeParams &p, const DecodeExtras &x)
 {
     using Sh = DecodeShape<D, kInt8>;
@@ -650,7 +667,7 @@ __device__ __forceinline__ void paged_decode_body(const DecodeParams &p, const D
     // tables, q) into L2 while the scan below runs; the CTAs split the lines.
     {
         const size_t g = size_t(blockIdx.x) * kThreads + tid, stride = size_t(gridDim.x) * kThreads;
-        const size_t table_lines = (size_t(B) * p.max_blocks_per_seq * 4 + 127) / 128;
+        const size_t table_lines = kContig ? 0 : (size_t(B) * p.max_blocks_per_seq * 4 + 127) / 128;
         const size_t q_lines = (size_t(B) * H * D * 2 + 127) / 128;
         const size_t len_lines = (size_t(B) * 4 + 127) / 128;
         for (size_t i = g; i < table_lines + q_lines + len_lines; i += stride) {
@@ -777,7 +794,7 @@ __device__ __forceinline__ void paged_decode_body(const DecodeParams &p, const D
             if (s < lane)
                 mc.template advance<T>(p);
         if (lane < first)
-            load_tile_ids<Sh>(p, mc, ids);
+            load_tile_ids<Sh, kContig>(p, mc, ids);
         __syncwarp();
         for (int s = 0; s < first; ++s) {
             TileCursor cs;
@@ -792,7 +809,7 @@ __device__ __forceinline__ void paged_decode_body(const DecodeParams &p, const D
             for (int e = 0; e < Sh::kMaxIds; ++e)
                 ids_s[e] = __shfl_sync(kFullMask, ids[e], s);
             if (lane == 0)
-                issue_tile<D, kInt8, Sm>(p, x, cs, ids_s, cs.i == 0 || cs.k == lo,
+                issue_tile<D, kInt8, Sm, kContig>(p, x, cs, ids_s, cs.i == 0 || cs.k == lo,
                                          my_buf + size_t(s) * Sm::kStageBytes, my_bar + 8 * s,
                                          my_meta + s, policy);
             if constexpr (!kInt8)
@@ -805,7 +822,7 @@ __device__ __forceinline__ void paged_decode_body(const DecodeParams &p, const D
     int issued = first;
     if (issued < ntiles) {
         prod.template advance<T>(p);
-        load_tile_ids<Sh>(p, prod, ids);
+        load_tile_ids<Sh, kContig>(p, prod, ids);
     }
 
     // ---- 5. stream --------------------------------------------------------
@@ -882,7 +899,7 @@ __device__ __forceinline__ void paged_decode_body(const DecodeParams &p, const D
         if (issued < ntiles) {  // refill the stage just consumed
             if (lane == 0) {
                 fence_proxy_async_smem();
-                issue_tile<D, kInt8, Sm>(p, x, prod, ids, prod.i == 0 || prod.k == lo,
+                issue_tile<D, kInt8, Sm, kContig>(p, x, prod, ids, prod.i == 0 || prod.k == lo,
                                          my_buf + size_t(stage) * Sm::kStageBytes,
                                          my_bar + 8 * stage, my_meta + stage, policy);
             }
@@ -891,7 +908,7 @@ __device__ __forceinline__ void paged_decode_body(const DecodeParams &p, const D
                     append_new_row<D, Sm>(p, x, prod, my_buf + size_t(stage) * Sm::kStageBytes, lane);
             if (++issued < ntiles) {
                 prod.template advance<T>(p);
-                load_tile_ids<Sh>(p, prod, ids);
+                load_tile_ids<Sh, kContig>(p, prod, ids);
             }
         }
         if (!(mt.i == nt - 1 || mt.k == hi - 1))
@@ -969,13 +986,16 @@ __device__ __forceinline__ void paged_decode_body(const DecodeParams &p, const D
 // work starts at once, running beside the previous kernel, and the wait for
 // that kernel comes at the end: this grid then completes only after the
 // previous one, and the next kernel that waits for this grid sees both.
-template <int D, bool kInt8, int NW, int S, bool kLateDepWait = false>
+// kContig: the cache is contiguous per (sequence, head), [B, H, Lmax, D]
+// with Lmax in block_size, and no block table is read (the baseline that
+// measures what the paged layout's indirection costs).
+template <int D, bool kInt8, int NW, int S, bool kLateDepWait = false, bool kContig = false>
 __global__ void __launch_bounds__(NW * 32) paged_decode_kernel(const DecodeParams p, const DecodeExtras x)
 {
     if (!kLateDepWait)
         grid_dependency_wait();
     allow_dependent_launch();
-    paged_decode_body<D, kInt8, NW, S>(p, x);
+    paged_decode_body<D, kInt8, NW, S, kContig>(p, x);
     if (kLateDepWait && threadIdx.x == 0)
         grid_dependency_wait();
 }

@@ -40,13 +40,13 @@ unsigned int *next_sched_slot(int dev)
 }
 
 // Encode the tensor maps and launch the persistent kernel (arguments already
-// validated).  grouped / o_f32 / lse: see PrefillParams.
+// validated).
 pa_status launch_prefill(void *out, const void *q, const void *k_cache, const void *v_cache,
                          const int32_t *block_tables, int max_blocks_per_seq,
                          const int32_t *context_lens, int max_context_len,
                          const int32_t *query_start_loc, int num_tokens, int max_query_len,
                          int num_seqs, int num_heads, int head_dim, int block_size, int num_blocks,
-                         float scale, bool grouped, float *o_f32, float *lse, cudaStream_t stream)
+                         float scale, cudaStream_t stream)
 {
     CUtensorMap tm_q, tm_k, tm_v;
     const uint64_t cache_rows = uint64_t(num_blocks) * num_heads * block_size;
@@ -84,10 +84,7 @@ pa_status launch_prefill(void *out, const void *q, const void *k_cache, const vo
     if (!p.error_word)
         return PA_ERR_CUDA;
     p.qk_scale_log2 = float(double(scale) * 1.4426950408889634);
-    p.grouped = grouped ? 1 : 0;
     p.num_rows = num_tokens;
-    p.o_f32 = o_f32;
-    p.lse = lse;
     // persistent: one CTA per SM (the shared-memory footprint allows one),
     // never more CTAs than items
     constexpr int kRowsPerItem = pa::kQTiles * pa::kPM;
@@ -137,6 +134,6 @@ extern "C" pa_status pa_prefill(void *out, const void *q, const void *k_cache, c
         return PA_ERR_INVALID_ARG;
     return launch_prefill(out, q, k_cache, v_cache, block_tables, max_blocks_per_seq, context_lens,
                           max_context_len, query_start_loc, num_tokens, max_query_len, num_seqs,
-                          num_heads, head_dim, block_size, num_blocks, scale, false, nullptr,
-                          nullptr, reinterpret_cast<cudaStream_t>(stream));
+                          num_heads, head_dim, block_size, num_blocks, scale,
+                          reinterpret_cast<cudaStream_t>(stream));
 }

@@ -68,15 +68,7 @@ struct PrefillParams {
     int num_seqs;
     int num_pairs;                    // query-tile pairs per sequence: ceil(max_query_len / 256)
     unsigned int *sched;              // [2]: next item to hand out, CTAs finished (both 0 at launch)
-    // Grouped mode (shared-prefix decode of a group of sequences): "sequence"
-    // g is a group whose queries are rows query_start_loc[g] ..
-    // query_start_loc[g+1] - 1 and whose context is the first
-    // context_lens[g] tokens of the block-table row query_start_loc[g]; every
-    // query sees the whole context (no causal mask).
-    int grouped;
     int num_rows;                     // T: rows of q and out
-    float *o_f32;                     // optional [T, H, D]: fp32 outputs instead of out
-    float *lse;                       // optional [T, H]: max + log2(sum), base-2 units
 };
 
 constexpr int kPM = 128;              // query rows per tile (MMA M)
@@ -248,7 +240,7 @@ __device__ __forceinline__ bool prefill_item(const PrefillParams &p, int k, Pref
     }
     it.L = L;
     it.row0 = pair * kQTiles * kPM;
-    it.table_row = p.grouped ? it.q_first : it.b;
+    it.table_row = it.b;
     if (n <= 0 || it.row0 >= n)
         return false;
     if (it.q_first < 0 || n > p.num_rows - it.q_first) {  // rows outside q / out
@@ -256,10 +248,7 @@ __device__ __forceinline__ bool prefill_item(const PrefillParams &p, int k, Pref
             prefill_error(p, PA_DEVERR_CONTEXT_LEN);
         return false;
     }
-    if (p.grouped) {
-        if (L == 0)
-            return false;  // nothing shared: the group's tails hold everything
-    } else if (n > L) {  // more new tokens than the context holds: nothing sensible to do
+    if (n > L) {  // more new tokens than the context holds: nothing sensible to do
         if (first)
             prefill_error(p, PA_DEVERR_CONTEXT_LEN);
         return false;
@@ -270,7 +259,7 @@ __device__ __forceinline__ bool prefill_item(const PrefillParams &p, int k, Pref
         const int r0 = it.row0 + t * kPM;
         it.rows[t] = max(0, min(kPM, n - r0));
         it.pos0[t] = L - n + r0;
-        const int last = p.grouped ? L - 1 : it.pos0[t] + it.rows[t] - 1;  // last position seen
+        const int last = it.pos0[t] + it.rows[t] - 1;  // last position seen
         it.nt[t] = it.rows[t] > 0 ? last / kPN + 1 : 0;
         it.ntiles = max(it.ntiles, it.nt[t]);
     }
@@ -570,7 +559,7 @@ __device__ __forceinline__ void prefill_softmax_role(const PrefillParams &p, Pre
             tc_fence_after_sync();
             const int t0 = j * kPN;
             // columns of this tile this row may see: t <= my_pos and t < L
-            const int lim = (p.grouped ? L - 1 : min(my_pos, L - 1)) - t0 + 1;
+            const int lim = min(my_pos, L - 1) - t0 + 1;
             const bool masked = __any_sync(kFullMask, lim < kPN);
             ScoreRow row;
             load_score_row(tS, row);
@@ -643,21 +632,12 @@ __device__ __forceinline__ void prefill_softmax_role(const PrefillParams &p, Pre
         const size_t out_row = size_t(it.q_first + it.row0 + t * kPM + r) * H + it.h;
         uint4 *dst = reinterpret_cast<uint4 *>(p.out + out_row * kPD);
         const bool store = r < it.rows[t];
-        if (store && p.lse)
-            p.lse[out_row] = m_ref + log2f(l);
 #pragma unroll 1
         for (int cc = 0; cc < kPD / 32; ++cc) {
             uint32_t o[32];
             tmem_load32_async(tO + uint32_t(cc * 32), o);
             tmem_wait_ld();
-            if (store && p.o_f32) {
-                float4 *d32 = reinterpret_cast<float4 *>(p.o_f32 + out_row * kPD) + cc * 8;
-#pragma unroll
-                for (int g4 = 0; g4 < 8; ++g4)
-                    d32[g4] = make_float4(__uint_as_float(o[4 * g4]) * inv, __uint_as_float(o[4 * g4 + 1]) * inv,
-                                          __uint_as_float(o[4 * g4 + 2]) * inv,
-                                          __uint_as_float(o[4 * g4 + 3]) * inv);
-            } else if (store) {
+            if (store) {
 #pragma unroll
                 for (int g = 0; g < 4; ++g) {
                     __half2 v[4];
