@@ -46,29 +46,44 @@ struct SetupParams {
     int max_chunks;               // capacity of `chunks` and of the partial columns
     __half *out;                  // rows of empty contexts are zeroed here
     Meta *meta;
-    Group *groups;
+    Group *groups;                // used without the shared-memory working set
     Member *members;
     Chunk *chunks;
     int32_t *tail_tables;         // [B, MB]
     int32_t *tail_lens;           // [B]
-    int32_t *group_of;            // [B] each member's group (-1: none)
+    int32_t *group_of;            // [B] each member's group (-1: none); likewise
     unsigned int *dec_tickets;    // [B, H] merge tickets of the tail decode, cleared here
     unsigned int *err;
 };
 
 constexpr int kSetupThreads = 1024;
 
+// Dynamic shared memory of the set-up kernel when its whole working set --
+// the group records, bounds and prefixes, each member's group, tail length
+// and context length, and the block-table rows -- fits in it (0: it does
+// not, and the workspace and the inputs serve instead).
+constexpr size_t kSetupSmemMax = 200u * 1024u;
+
+size_t setup_smem_bytes(int num_groups, int num_seqs, int max_blocks)
+{
+    const size_t bytes = size_t(num_groups) * (sizeof(Group) + 2 * sizeof(int32_t)) + sizeof(int32_t) +
+                         size_t(num_seqs) * 3 * sizeof(int32_t) +
+                         size_t(num_seqs) * size_t(max_blocks) * sizeof(int32_t);
+    return bytes <= kSetupSmemMax ? bytes : 0;
+}
+
 // Share of the SMs the prefix kernel runs on; the tail decode takes the
 // rest.  Which part is larger is known only on the device, so the split is
 // fixed: a prefix SM streams a little slower than a decode SM (its pipeline
 // holds fewer tiles in flight), and this share balances prefixes and tails
 // of similar size (parallel samples of a prompt with tails of a few
-// hundred tokens).
-constexpr float kPrefixSmShare = 0.55f;
+// hundred tokens).  On 8 groups of 8 with ~1000-token prefixes and tails
+// of 1-256 tokens, 0.50 suits copy-on-write tables (each tail also holds
+// the copied last prefix block) and 0.55 fully aliased ones.
+constexpr float kPrefixSmShare = 0.53f;
 
-__device__ __forceinline__ int clamped_len(const SetupParams &p, int b)
+__device__ __forceinline__ int clamp_len(const SetupParams &p, int raw)
 {
-    const int raw = p.context_lens[b];
     if (raw < 0 || raw > p.max_context_len) {
         atomicOr(p.err, PA_DEVERR_CONTEXT_LEN);
         return raw < 0 ? 0 : p.max_context_len;
@@ -76,44 +91,32 @@ __device__ __forceinline__ int clamped_len(const SetupParams &p, int b)
     return raw;
 }
 
-// Exclusive scan of get(i), i < n, over the whole CTA; put(i, prefix).
-// Returns the total.  All threads of the CTA must call it.
-template <class Get, class Put>
-__device__ int block_exclusive_scan(int n, Get get, Put put, int *s_warp)
+// Exclusive scans of the groups' chunk counts (pstart) and partial-column
+// counts (colbase) by one warp, 32 groups a step; returns the totals.
+__device__ int2 warp_scan_groups(Group *gr, int G, int lane)
 {
-    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    int carry = 0;
-    for (int base = 0; base < n; base += kSetupThreads) {
-        const int i = base + tid;
-        const int v = i < n ? get(i) : 0;
-        int x = v;
+    int carry_p = 0, carry_c = 0;
+    for (int base = 0; base < G; base += 32) {
+        const int i = base + lane;
+        const int vp = i < G ? gr[i].pstart : 0, vc = i < G ? gr[i].colbase : 0;
+        int xp = vp, xc = vc;
 #pragma unroll
         for (int off = 1; off < 32; off <<= 1) {
-            const int y = __shfl_up_sync(pa::kFullMask, x, off);
-            if (lane >= off)
-                x += y;
-        }
-        if (lane == 31)
-            s_warp[warp] = x;
-        __syncthreads();
-        if (warp == 0) {
-            int w = s_warp[lane];
-#pragma unroll
-            for (int off = 1; off < 32; off <<= 1) {
-                const int y = __shfl_up_sync(pa::kFullMask, w, off);
-                if (lane >= off)
-                    w += y;
+            const int yp = __shfl_up_sync(pa::kFullMask, xp, off);
+            const int yc = __shfl_up_sync(pa::kFullMask, xc, off);
+            if (lane >= off) {
+                xp += yp;
+                xc += yc;
             }
-            s_warp[lane] = w;
         }
-        __syncthreads();
-        const int before = carry + (warp > 0 ? s_warp[warp - 1] : 0);
-        if (i < n)
-            put(i, before + x - v);
-        carry += s_warp[31];
-        __syncthreads();
+        if (i < G) {
+            gr[i].pstart = carry_p + xp - vp;
+            gr[i].colbase = carry_c + xc - vc;
+        }
+        carry_p += __shfl_sync(pa::kFullMask, xp, 31);
+        carry_c += __shfl_sync(pa::kFullMask, xc, 31);
     }
-    return carry;
+    return make_int2(carry_p, carry_c);
 }
 
 // Group g with members g0 .. g0+n-1 and a valid prefix P (a multiple of the
@@ -122,36 +125,99 @@ __device__ int block_exclusive_scan(int n, Get get, Put put, int *s_warp)
 // table.  A prefix that breaks the rules is recorded (PA_DEVERR_CONTEXT_LEN)
 // and the group decodes without one.  Member b's tail is tokens P .. L_b - 1
 // of its own table: its tail table is that row from block P / bs on.
+// The work is a few dependent steps over small arrays, so its time is set by
+// round trips to memory, and a CTA barrier waits for every load and store
+// its threads have outstanding.  With the working set in shared memory
+// (kSmem) every input -- lengths, group bounds and prefixes, table rows --
+// comes in at once in the first step, the groups are settled in shared
+// memory, and every output is written after the last barrier: one round
+// trip in all.  With at most 32 groups each warp scans the groups' counts
+// itself (lane g holds group g) and needs no further barrier.
+template <bool kSmem>
 __global__ void __launch_bounds__(kSetupThreads) grouped_setup_kernel(const SetupParams p)
 {
-    __shared__ int s_warp[32];
+    extern __shared__ int4 setup_smem[];
     pa::grid_dependency_wait();
     pa::allow_dependent_launch();
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int B = p.num_seqs, G = p.num_groups, bs = p.block_size, H = p.num_heads;
-    for (int b = tid; b < B; b += kSetupThreads) {
-        p.members[b] = Member{-1, 0, 0, 0};
-        p.tail_lens[b] = 0;
-        p.group_of[b] = -1;
+    const int MB = p.max_blocks;
+    Group *gr;
+    int32_t *gof, *tl, *len = nullptr, *gs = nullptr, *pl = nullptr, *rows = nullptr;
+    if constexpr (kSmem) {
+        gr = reinterpret_cast<Group *>(setup_smem);
+        gs = reinterpret_cast<int32_t *>(gr + G);  // group bounds [G + 1]
+        pl = gs + G + 1;                           // prefixes [G]
+        gof = pl + G;                              // each member's group [B]
+        tl = gof + B;                              // tail lengths [B]
+        len = tl + B;                              // clamped context lengths [B]
+        rows = len + B;                            // block-table rows [B, MB]
+    } else {
+        gr = p.groups;
+        gof = p.group_of;
+        tl = p.tail_lens;
     }
-    for (int i = tid; i < B * H; i += kSetupThreads)
-        p.dec_tickets[i] = 0u;
-    __syncthreads();
 
-    // A: per group (a warp each): bounds, prefix, tails
+    // 1: the inputs in (one round trip)
+    for (int b = tid; b < B; b += kSetupThreads) {
+        gof[b] = -1;
+        tl[b] = 0;
+        if constexpr (kSmem)
+            len[b] = clamp_len(p, p.context_lens[b]);
+    }
+    if constexpr (kSmem) {
+        for (int g = tid; g <= G; g += kSetupThreads) {
+            gs[g] = p.group_start[g];
+            if (g < G)
+                pl[g] = p.prefix_lens[g];
+        }
+        // loads before stores, so all go out at once
+        const int entries = B * MB;
+        constexpr int kBatch = 8;
+        for (int base = 0; base < entries; base += kBatch * kSetupThreads) {
+            int32_t v[kBatch];
+#pragma unroll
+            for (int r = 0; r < kBatch; ++r) {
+                const int i = base + r * kSetupThreads + tid;
+                v[r] = i < entries ? p.block_tables[i] : 0;
+            }
+#pragma unroll
+            for (int r = 0; r < kBatch; ++r) {
+                const int i = base + r * kSetupThreads + tid;
+                if (i < entries)
+                    rows[i] = v[r];
+            }
+        }
+    }
+    __syncthreads();
+    auto length = [&](int b) {
+        if constexpr (kSmem)
+            return len[b];
+        else
+            return clamp_len(p, p.context_lens[b]);
+    };
+
+    // 2: per group (a warp each): bounds, prefix, tails
     for (int g = warp; g < G; g += kSetupThreads / 32) {
-        int g0 = p.group_start[g];
-        const int g1 = p.group_start[g + 1];
+        int g0, g1, P;
+        if constexpr (kSmem) {
+            g0 = gs[g];
+            g1 = gs[g + 1];
+            P = pl[g];
+        } else {
+            g0 = p.group_start[g];
+            g1 = p.group_start[g + 1];
+            P = p.prefix_lens[g];
+        }
         const bool okg = 0 <= g0 && g0 <= g1 && g1 <= B;
         if (!okg && lane == 0)
             atomicOr(p.err, PA_DEVERR_CONTEXT_LEN);
         const int n = okg ? g1 - g0 : 0;
         if (!okg)
             g0 = 0;
-        int P = p.prefix_lens[g];
         int min_len = INT_MAX;
         for (int b = g0 + lane; b < g0 + n; b += 32)
-            min_len = min(min_len, clamped_len(p, b));
+            min_len = min(min_len, length(b));
         min_len = __reduce_min_sync(pa::kFullMask, min_len);
         if (n == 0 || P < 0 || P % bs != 0 || P > min_len) {
             if (n > 0 && P != 0 && lane == 0)
@@ -161,26 +227,51 @@ __global__ void __launch_bounds__(kSetupThreads) grouped_setup_kernel(const Setu
         const int cp = (P + kChunk - 1) / kChunk;
         const int slices = (n + 15) / 16;
         for (int b = g0 + lane; b < g0 + n; b += 32) {
-            const int L = clamped_len(p, b);
-            p.group_of[b] = g;
-            p.tail_lens[b] = L - P;
-            if (L == 0) {  // nothing to attend to: the output is zero
-                uint4 *o = reinterpret_cast<uint4 *>(p.out + size_t(b) * H * kD);
-                for (int e = 0; e < H * kD / 8; ++e)
-                    o[e] = make_uint4(0, 0, 0, 0);
-            }
+            gof[b] = g;
+            tl[b] = length(b) - P;
         }
-        if (lane == 0)  // colbase and pstart hold counts until the scans turn them into offsets
-            p.groups[g] = Group{g0, n, cp, P, n * cp, slices * cp, 0, 0};
+        if (lane == 0)  // colbase and pstart hold counts until the scan turns them into offsets
+            gr[g] = Group{g0, n, cp, P, n * cp, slices * cp, 0, 0};
     }
     __syncthreads();
 
-    // B: offsets of every group's chunks and partial columns
-    Group *gr = p.groups;
-    const int nchunks = block_exclusive_scan(
-        G, [&](int i) { return gr[i].pstart; }, [&](int i, int x) { gr[i].pstart = x; }, s_warp);
-    const int ncols = block_exclusive_scan(
-        G, [&](int i) { return gr[i].colbase; }, [&](int i, int x) { gr[i].colbase = x; }, s_warp);
+    // 3: the offsets: lane g of every warp holds group g's (at most 32
+    // groups), else one warp scans in place behind a barrier
+    const bool small = G <= 32;
+    int xp = 0, xc = 0, nchunks, ncols;
+    if (small) {
+        const int vp = lane < G ? gr[lane].pstart : 0, vc = lane < G ? gr[lane].colbase : 0;
+        xp = vp;
+        xc = vc;
+#pragma unroll
+        for (int off = 1; off < 32; off <<= 1) {
+            const int yp = __shfl_up_sync(pa::kFullMask, xp, off);
+            const int yc = __shfl_up_sync(pa::kFullMask, xc, off);
+            if (lane >= off) {
+                xp += yp;
+                xc += yc;
+            }
+        }
+        nchunks = __shfl_sync(pa::kFullMask, xp, 31);
+        ncols = __shfl_sync(pa::kFullMask, xc, 31);
+        xp -= vp;  // exclusive
+        xc -= vc;
+    } else {
+        __shared__ int2 s_tot;
+        if (warp == 0) {
+            const int2 tot = warp_scan_groups(gr, G, lane);
+            if (lane == 0)
+                s_tot = tot;
+        }
+        __syncthreads();
+        nchunks = s_tot.x;
+        ncols = s_tot.y;
+    }
+    // group g's (first chunk, first partial column)
+    auto offsets = [&](int g) {
+        return small ? make_int2(__shfl_sync(pa::kFullMask, xp, g & 31), __shfl_sync(pa::kFullMask, xc, g & 31))
+                     : make_int2(gr[g].pstart, gr[g].colbase);
+    };
     const bool fits = nchunks <= p.max_chunks && ncols <= p.max_chunks;
     if (!fits) {  // cannot happen with the host's bound; refuse rather than overrun
         if (tid == 0) {
@@ -190,30 +281,63 @@ __global__ void __launch_bounds__(kSetupThreads) grouped_setup_kernel(const Setu
         return;
     }
 
-    // C: the chunk descriptors, the member records, and the tail tables (a
-    // warp per member: its table row from block P / bs on)
+    // 4: every output: per member (a warp each) its record, tail length and
+    // tail table (entry k is entry P / bs + k of its table row), zero rows
+    // for empty contexts; the chunk descriptors; the decode's merge tickets;
+    // the header
+    for (int b = warp; b < B; b += kSetupThreads / 32) {
+        const int g = gof[b];
+        const Group gg = g >= 0 ? gr[g] : Group{0, 0, 0, 0, 0, 0, 0, 0};
+        const int2 off = offsets(g >= 0 ? g : 0);
+        const int tail = tl[b];
+        const int pb = gg.P / bs;
+        int32_t *trow = p.tail_tables + size_t(b) * MB;
+        if constexpr (kSmem) {
+            const int32_t *row = rows + b * MB;
+            for (int k = lane; k < MB; k += 32)
+                trow[k] = pb + k < MB ? row[pb + k] : -1;
+        } else {  // loads before stores
+            const int32_t *__restrict__ row = p.block_tables + size_t(b) * MB;
+            constexpr int kBatch = 4;
+            for (int k0 = 0; k0 < MB; k0 += 32 * kBatch) {
+                int32_t v[kBatch];
+#pragma unroll
+                for (int r = 0; r < kBatch; ++r) {
+                    const int k = k0 + r * 32 + lane;
+                    v[r] = k < MB && pb + k < MB ? row[pb + k] : -1;
+                }
+#pragma unroll
+                for (int r = 0; r < kBatch; ++r) {
+                    const int k = k0 + r * 32 + lane;
+                    if (k < MB)
+                        trow[k] = v[r];
+                }
+            }
+        }
+        if (lane == 0) {
+            p.members[b] = g >= 0 ? Member{tail, gg.cp, off.y + (b - gg.g0), gg.n} : Member{-1, 0, 0, 0};
+            if constexpr (kSmem)
+                p.tail_lens[b] = tail;
+        }
+        if (g >= 0 && tail + gg.P == 0) {  // nothing to attend to: the output is zero
+            uint4 *o = reinterpret_cast<uint4 *>(p.out + size_t(b) * H * kD);
+            for (int e = lane; e < H * kD / 8; e += 32)
+                o[e] = make_uint4(0, 0, 0, 0);
+        }
+    }
     for (int g = warp; g < G; g += kSetupThreads / 32) {
         const Group gg = gr[g];
+        const int2 off = offsets(g);
         const int slices = (gg.n + 15) / 16;
         for (int idx = lane; idx < slices * gg.cp; idx += 32) {
             const int j = idx / slices, s = idx % slices;
-            p.chunks[gg.pstart + idx] =
+            p.chunks[off.x + idx] =
                 Chunk{gg.g0, gg.g0 + 16 * s, min(16, gg.n - 16 * s), j * kChunk,
-                      min((j + 1) * kChunk, gg.P), g, gg.colbase + j * gg.n + 16 * s, 0};
+                      min((j + 1) * kChunk, gg.P), g, off.y + j * gg.n + 16 * s, 0};
         }
     }
-    const int MB = p.max_blocks;
-    for (int b = warp; b < B; b += kSetupThreads / 32) {
-        const int g = p.group_of[b];
-        const Group gg = g >= 0 ? gr[g] : Group{0, 0, 0, 0, 0, 0, 0, 0};
-        if (lane == 0 && g >= 0)
-            p.members[b] = Member{p.tail_lens[b], gg.cp, gg.colbase + (b - gg.g0), gg.n};
-        const int pb = gg.P / bs;
-        const int32_t *row = p.block_tables + size_t(b) * MB;
-        int32_t *trow = p.tail_tables + size_t(b) * MB;
-        for (int k = lane; k < MB; k += 32)
-            trow[k] = pb + k < MB ? row[pb + k] : -1;
-    }
+    for (int i = tid; i < B * H; i += kSetupThreads)
+        p.dec_tickets[i] = 0u;
     if (tid == 0)
         *p.meta = Meta{nchunks, ncols, 0, 0};
 }
@@ -305,19 +429,21 @@ Layout layout(int num_seqs, int num_groups, int num_heads, int max_context_len, 
     const size_t cap = size_t(num_seqs) * (per_member > 0 ? per_member : 1);
     const size_t units = size_t(num_seqs) * size_t(num_heads);
     w.max_chunks = cap > size_t(INT_MAX) ? INT_MAX : int(cap);
+    // what the set-up kernel writes first and together, the large partial
+    // buffers after it
     w.meta = 0;
     w.groups = align256(sizeof(Meta));
     w.members = w.groups + align256(size_t(num_groups) * sizeof(Group));
     w.group_of = w.members + align256(size_t(num_seqs) * sizeof(Member));
     w.chunks = w.group_of + align256(size_t(num_seqs) * sizeof(int32_t));
-    w.part_ml = w.chunks + align256(cap * sizeof(Chunk));
-    w.part_o = w.part_ml + align256(cap * num_heads * 2 * sizeof(float));
-    w.tail_tables = w.part_o + align256(cap * num_heads * kD * sizeof(float));
+    w.tail_tables = w.chunks + align256(cap * sizeof(Chunk));
     w.tail_lens = w.tail_tables + align256(size_t(num_seqs) * size_t(max_blocks) * sizeof(int32_t));
-    w.dec = w.tail_lens + align256(size_t(num_seqs) * sizeof(int32_t));
-    w.o_t = w.dec + align256(pa_decode_workspace_size(num_seqs, num_heads, kD, max_context_len));
-    w.lse_t = w.o_t + align256(units * kD * 2);
-    w.total = w.lse_t + align256(units * sizeof(float));
+    w.part_ml = w.tail_lens + align256(size_t(num_seqs) * sizeof(int32_t));
+    w.lse_t = w.part_ml + align256(cap * num_heads * 2 * sizeof(float));
+    w.o_t = w.lse_t + align256(units * sizeof(float));
+    w.part_o = w.o_t + align256(units * kD * 2);
+    w.dec = w.part_o + align256(cap * num_heads * kD * sizeof(float));
+    w.total = w.dec + align256(pa_decode_workspace_size(num_seqs, num_heads, kD, max_context_len));
     return w;
 }
 
@@ -365,7 +491,7 @@ extern "C" pa_status pa_decode_grouped(void *out, const void *q, const void *k_c
     if (num_seqs > 65535 || num_heads > 65535 || max_group_size > 65535 ||
         int64_t(num_blocks) * num_heads * block_size > INT32_MAX ||
         int64_t(num_heads) * ((max_context_len + kChunk - 1) / kChunk + 1) * num_seqs > INT32_MAX ||
-        int64_t(num_seqs) * max_blocks_per_seq > INT32_MAX)
+        int64_t(num_seqs) * max_blocks_per_seq > INT32_MAX - 65536)
         return PA_ERR_INVALID_ARG;
     const Layout w = layout(num_seqs, num_groups, num_heads, max_context_len, max_blocks_per_seq);
     if (!workspace || workspace_bytes < w.total || !aligned16(workspace))
@@ -385,6 +511,8 @@ extern "C" pa_status pa_decode_grouped(void *out, const void *q, const void *k_c
         if (cudaFuncSetAttribute(pa::grp::grouped_decode_kernel,
                                  cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  int(pa::grp::kSmem)) != cudaSuccess ||
+            cudaFuncSetAttribute(grouped_setup_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 int(kSetupSmemMax)) != cudaSuccess ||
             cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess ||
             sms <= 0)
             return PA_ERR_CUDA;
@@ -423,6 +551,7 @@ extern "C" pa_status pa_decode_grouped(void *out, const void *q, const void *k_c
     sp.num_heads = num_heads;
     sp.max_blocks = max_blocks_per_seq;
     sp.max_chunks = w.max_chunks;
+    const size_t setup_smem = setup_smem_bytes(num_groups, num_seqs, max_blocks_per_seq);
     sp.out = static_cast<__half *>(out);
     sp.meta = meta;
     sp.groups = groups;
@@ -434,7 +563,9 @@ extern "C" pa_status pa_decode_grouped(void *out, const void *q, const void *k_c
     sp.dec_tickets = reinterpret_cast<unsigned int *>(
         ws + w.dec + pa_host::decode_ticket_offset(num_seqs, num_heads, kD));
     sp.err = err;
-    if (launch_pdl(grouped_setup_kernel, dim3(1), dim3(kSetupThreads), 0, s, sp) != cudaSuccess)
+    if ((setup_smem > 0 ? launch_pdl(grouped_setup_kernel<true>, dim3(1), dim3(kSetupThreads), setup_smem, s, sp)
+                        : launch_pdl(grouped_setup_kernel<false>, dim3(1), dim3(kSetupThreads), 0, s, sp)) !=
+        cudaSuccess)
         return PA_ERR_CUDA;
 
     // 2. the shared prefixes, once per (group, head), on the tensor cores
@@ -443,6 +574,7 @@ extern "C" pa_status pa_decode_grouped(void *out, const void *q, const void *k_c
     p.block_tables = block_tables;
     p.chunks = sp.chunks;
     p.meta = meta;
+    p.max_chunks = w.max_chunks;
     p.part_ml = part_ml;
     p.part_o = part_o;
     p.max_blocks_per_seq = max_blocks_per_seq;
@@ -467,7 +599,7 @@ extern "C" pa_status pa_decode_grouped(void *out, const void *q, const void *k_c
     }
     const pa_status st = pa_host::decode_with_lse(
         o_t, q, k_cache, v_cache, tail_tables, max_blocks_per_seq, tail_lens, max_context_len,
-        num_seqs, num_heads, head_dim, block_size, num_blocks, scale, ws + w.dec, w.o_t - w.dec, lse_t,
+        num_seqs, num_heads, head_dim, block_size, num_blocks, scale, ws + w.dec, w.total - w.dec, lse_t,
         stream, per_sm * (sms - prefix_ctas), true);
     if (st != PA_OK)
         return st;

@@ -15,31 +15,37 @@
 //
 // How: the score product is computed transposed, S^T = K Q^T, so the MMA's
 // M dimension is 128 context tokens and N is 16 query columns (up to 16
-// members); O^T = V^T P^T accumulates in TMEM with the head dimension as M.
-// A softmax thread then owns one token (one TMEM lane) and handles its <= 16
-// scores, so the per-tile softmax stays short.
+// members); a softmax thread then owns one token (one TMEM lane) and handles
+// its <= 16 scores, so the per-tile softmax stays short.  The output
+// O = P V accumulates in TMEM with the queries as M (rows 0-15 of 128; the
+// other rows of the A operand are whatever follows P in shared memory and
+// their results are never read) and the head dimension as N = 128: P is a
+// K-major operand and V an N-major one, both as the loads left them.  (A
+// small tcgen05.mma costs about the same for any N up to 64, and taking V
+// as an M-major A operand instead costs about twice as much per
+// instruction, so this orientation halves the P.V's tensor-pipe time.)
 //   * Work items ("chunks", built by a set-up kernel): up to 512 tokens of a
 //     group's prefix for a slice of up to 16 members, read through the first
 //     member's table.  Items are (chunk, head) pairs; persistent CTAs (one per
-//     SM) take every gridDim-th item.
-//   * warp 8 (loads): walks the CTA's items, passes each to the other roles
+//     SM) start with one each and claim the rest from a counter.
+//   * warp 5 (loads): walks the CTA's items, passes each to the other roles
 //     through a small shared-memory ring, and issues the TMA loads: the 16 Q
 //     rows of the next item, and per 128-token tile K and V through the block
 //     table, one 4-D box per (block, head) run, into six 32 KB slots.
-//   * warp 9 (one thread): S^T(n) = K_n Q^T into one of two TMEM score
-//     buffers and O^T += V_n^T P_n^T (V as an M-major operand, P^T from shared
-//     memory), each issued as soon as its inputs are ready; a K slot is
-//     released when its score product completes, a V slot when its P.V does.
+//   * warp 6 (one thread): S^T(n) = K_n Q^T into one of two TMEM score
+//     buffers and O += P_n V_n, each issued as soon as its inputs are ready;
+//     a K slot is released when its score product completes, a V slot when
+//     its P.V does.
 //   * warps 0-3 (softmax, thread = token): the tile maximum per query column
 //     (warp reduction, then the four warps' maxima through shared memory
 //     behind one named barrier), exp2 against a reference max per column that
-//     only moves when a tile's max exceeds it by more than 2^8 (then the
-//     column of O and the partial sums are rescaled), P^T as fp16 into a
-//     shared-memory operand tile; rows past the prefix end get P = 0 and
-//     their V rows are zeroed (by the MMA thread) so garbage never meets a
-//     zero weight.
-//   * warps 4-7 (epilogue, thread = head dimension): O^T columns and the
-//     per-column sums are written to the workspace as (m, l, o).
+//     only moves when a tile's max exceeds it by more than 2^8 (then warp 0
+//     rescales the rows of O and every thread its partial sums), P as fp16
+//     into one of four shared-memory operand tiles; tokens past the prefix
+//     end get P = 0 and their V rows are zeroed (by the MMA thread) so
+//     garbage never meets a zero weight.
+//   * warp 4 (epilogue, thread = query row of O): the rows of O and the
+//     per-query sums are written to the workspace as (m, l, o).
 // Every wait is bounded (1 s); the first to run out records PA_DEVERR_TIMEOUT
 // and raises an abort flag that ends every role; copies and matrix
 // operations in flight are drained (bounded) before TMEM is released.
@@ -69,15 +75,21 @@ constexpr uint32_t kAtom = 1024u;           // 8 rows x 128 bytes
 constexpr uint32_t kGroupStride = 2048u;    // between 8-row groups
 constexpr uint32_t kQHalf = kNQ * 128u;     // [16 rows x 64 fp16]
 constexpr uint32_t kQTile = 2 * kQHalf;     // Q rows of an item, or P^T of a tile (4 KB)
-constexpr int kQSlots = 4;                  // Q rows of the items in flight
-constexpr int kPBufs = 2;                   // P^T operand tiles
-constexpr uint32_t kOffQ = kSlots * kTile;
-constexpr uint32_t kOffP = kOffQ + kQSlots * kQTile;
-constexpr uint32_t kSmem = kOffP + kPBufs * kQTile + 1024;  // + 1024-byte alignment slack
-constexpr int kLoadWarp = 8, kMmaWarp = 9;
-constexpr int kThreads = 10 * 32;
-constexpr uint32_t kTmemCols = 64;          // S0, S1, O0, O1: 16 columns each
-constexpr uint32_t kTmemO = 32;
+constexpr int kQSlots = 2;                  // Q rows of the items in flight
+constexpr int kPBufs = 4;                   // P operand tiles
+// P tiles first: the P.V's A operand spans 128 rows (16 KB from a P tile's
+// start), of which only the first 16 are P, so what follows a P tile must
+// still be this CTA's shared memory.
+constexpr uint32_t kOffP = 0;
+constexpr uint32_t kOffQ = kOffP + kPBufs * kQTile;
+constexpr uint32_t kOffKV = kOffQ + kQSlots * kQTile;
+constexpr uint32_t kSmem = kOffKV + kSlots * kTile + 1024;  // + 1024-byte alignment slack
+static_assert(kOffP + (kPBufs - 1) * kQTile + kQHalf + 16u * 1024u <= kOffKV + kSlots * kTile,
+              "the P.V's A operand must stay inside the CTA's shared memory");
+constexpr int kEpiWarp = 4, kLoadWarp = 5, kMmaWarp = 6;
+constexpr int kThreads = 7 * 32;
+constexpr uint32_t kTmemCols = 512;         // S0, S1 (16 columns each); O0, O1 (128 each)
+constexpr uint32_t kTmemO = 128;            // O buffer b at kTmemO + 128 b
 constexpr float kRescaleLog2 = 8.f;         // move a reference max only past this growth
 
 // One work item's context part (head-independent): tokens [t0, t1) of
@@ -108,14 +120,16 @@ struct Member {
 struct Meta {
     int nchunks;      // prefix chunks of all groups
     int ncols;        // partial columns they use
-    int pad0, pad1;
+    int claimed;      // work items handed out past the first gridDim.x (zeroed by the set-up)
+    int pad;
 };
 
 struct Params {
     __half *out;                      // [B, H, D]
     const int32_t *block_tables;      // [B, MB]
-    const Chunk *chunks;
-    const Meta *meta;
+    const Chunk *chunks;              // capacity max_chunks
+    Meta *meta;
+    int max_chunks;
     float *part_ml;                   // [columns, H, 2]: (reference max, sum)
     float *part_o;                    // [columns, H, D]
     int max_blocks_per_seq;
@@ -247,23 +261,24 @@ __device__ __forceinline__ void load_chunk_ids(const Params &p, const Chunk &c, 
     }
 }
 
-// This CTA's items are blockIdx.x, blockIdx.x + gridDim.x, ... (numbered
-// chunk-major, so every CTA gets a like mix).  The descriptors of 32 items at
-// a time sit in the lanes' registers; the block ids of the next item and the
-// Q rows of the next item are fetched while the current item's tiles are
-// issued, so no dependent load stalls the stream.  Tile m's K goes to slot
-// (2m) % kSlots and its V to slot (2m + 1) % kSlots, so slots 0, 2, 4 only
-// ever hold K tiles and slots 1, 3, 5 V tiles.
+// Items are numbered chunk-major (k = chunk * H + head).  CTA c starts with
+// item c and then claims one item at a time from a counter in the work-list
+// header, so a CTA that streams faster takes more items and all CTAs finish
+// within about one item of each other.  Every step that waits on memory is
+// started a stage ahead: while item u's tiles are issued, item u + 1's
+// descriptor is loaded (its index was claimed during item u - 1), then its
+// block ids (after u's first tile), the index of item u + 2 is being
+// claimed, and u + 1's Q rows go out after u's last tile.
+// Tile m's K goes to slot (2m) % kSlots and its V to slot (2m + 1) % kSlots,
+// so slots 0, 2, 4 only ever hold K tiles and slots 1, 3, 5 V tiles.
 __device__ __forceinline__ void load_role(const CUtensorMap *tm_q, const CUtensorMap *tm_k,
                                           const CUtensorMap *tm_v, const Params &p, Shared &sh,
-                                          uint32_t sbase, int lane, int total)
+                                          uint32_t sbase, int lane)
 {
     volatile int *abort = &sh.abort;
     unsigned int *err = p.error_word;
     const int H = p.num_heads, bs = p.block_size;
     const int box = bs < kT ? bs : kT;
-    const int stride = int(gridDim.x), first = int(blockIdx.x);
-    const int nitems = first < total ? (total - first + stride - 1) / stride : 0;
     int last_use[kSlots];
 #pragma unroll
     for (int i = 0; i < kSlots; ++i)
@@ -272,23 +287,19 @@ __device__ __forceinline__ void load_role(const CUtensorMap *tm_q, const CUtenso
 #pragma unroll
     for (int i = 0; i < kQSlots; ++i)
         last_q[i] = -1;
-    int batch = 0;  // descriptors of items batch .. batch+31 are in the lanes
-    Chunk mine{};
-    auto fetch = [&](int b0) {
-        const int it = b0 + lane;
-        if (it < nitems)
-            mine = p.chunks[(first + it * stride) / H];
+    // the descriptor of item k (a broadcast load), or an empty one past the
+    // work-list capacity
+    auto descriptor = [&](int k) {
+        Chunk c{};
+        if (k >= 0 && k / H < p.max_chunks)
+            c = p.chunks[k / H];
+        return c;
     };
-    auto chunk_of = [&](int it) {
-        if (it - batch >= 32) {
-            batch += 32;
-            fetch(batch);
-        }
-        return shfl_chunk(mine, it - batch);
-    };
-    // the Q rows of item `it` into Q slot it % kQSlots (once its previous
-    // user's score products are done)
-    auto issue_q = [&](int it, const Chunk &c) {
+    // the next item index: one atomic by lane 0, not waited for here
+    auto claim = [&]() { return lane == 0 ? int(gridDim.x) + atomicAdd(&p.meta->claimed, 1) : 0; };
+    // the Q rows of item `it` (index k) into Q slot it % kQSlots, once its
+    // previous user's score products are done
+    auto issue_q = [&](int it, int k, const Chunk &c) {
         const int qs = it % kQSlots, use = it / kQSlots;
         bool ok = true;
         if (use > 0 && lane == 0)
@@ -296,7 +307,7 @@ __device__ __forceinline__ void load_role(const CUtensorMap *tm_q, const CUtenso
         if (!__shfl_sync(kFullMask, int(ok), 0))
             return false;
         if (lane == 0) {
-            const int h = (first + it * stride) % H;
+            const int h = k % H;
             const uint32_t bar = smem_u32(&sh.q_full[qs]);
             mbar_arrive_expect_tx(bar, kQTile);
             const uint32_t dst = sbase + kOffQ + uint32_t(qs) * kQTile;
@@ -325,32 +336,36 @@ __device__ __forceinline__ void load_role(const CUtensorMap *tm_q, const CUtenso
         last_use[s] = use;
         __syncwarp();
         if (t.ok)
-            tma_load_4d(sbase + uint32_t(s) * kTile + uint32_t(lane * box) * 256u, kind == 0 ? tm_k : tm_v,
+            tma_load_4d(sbase + kOffKV + uint32_t(s) * kTile + uint32_t(lane * box) * 256u, kind == 0 ? tm_k : tm_v,
                         0, 0, 0, t.y8, full);
         return true;
     };
     int m = 0;  // tiles issued
     bool go = true;
-    fetch(0);
-    Chunk c{};
+    // item 0 of this CTA: its descriptor and the item count come in together
+    int kk = int(blockIdx.x);
+    Chunk c = descriptor(kk);
+    const int total = p.meta->nchunks * H;
+    if (kk >= total)
+        kk = -1;
+    int kn = -1, kclaim = 0;  // the next item; the claim after it (lane 0)
     int ids[2] = {0, 0};
-    if (nitems > 0) {
-        c = chunk_of(0);
+    if (kk >= 0) {
+        kclaim = claim();
         load_chunk_ids(p, c, box, lane, ids);
-        go = issue_q(0, c);
+        go = issue_q(0, kk, c);
+        kn = __shfl_sync(kFullMask, kclaim, 0);
+        kclaim = claim();
     }
-    int items = 0;
-    for (; go; ++items) {
-        const int kk = items < nitems && !*abort ? first + items * stride : -1;
-        const int h = kk >= 0 ? kk % H : 0;
-        // prefetch the next item's descriptor and block ids
-        Chunk cn{};
+    for (int items = 0; go; ++items) {
+        if (*abort)
+            kk = -1;
+        const bool has_next = kk >= 0 && kn < total;
+        // the next item's descriptor; its block ids are loaded after this
+        // item's first tile, when the descriptor has arrived
+        const Chunk cn = has_next ? descriptor(kn) : Chunk{};
         int ids_n[2] = {0, 0};
-        const bool has_next = kk >= 0 && items + 1 < nitems;
-        if (has_next) {
-            cn = chunk_of(items + 1);
-            load_chunk_ids(p, cn, box, lane, ids_n);
-        }
+        bool ids_pending = has_next;
         {
             const int slot = items % kItemRing, use = items / kItemRing;
             bool ok = true;
@@ -360,7 +375,7 @@ __device__ __forceinline__ void load_role(const CUtensorMap *tm_q, const CUtenso
                 break;
             if (lane == 0) {
                 sh.item[slot].c = c;
-                sh.item[slot].h = h;
+                sh.item[slot].h = kk >= 0 ? kk % H : 0;
                 sh.item[slot].k = kk;
                 mbar_arrive(smem_u32(&sh.item_full[slot]));
             }
@@ -368,6 +383,7 @@ __device__ __forceinline__ void load_role(const CUtensorMap *tm_q, const CUtenso
         }
         if (kk < 0)
             break;
+        const int h = kk % H;
         const int nt = chunk_tiles(c);
         const int runs_per_tile = kT / box;
         for (int j = 0; go && j < nt; ++j, ++m) {
@@ -383,12 +399,22 @@ __device__ __forceinline__ void load_role(const CUtensorMap *tm_q, const CUtenso
                 atomicOr(err, PA_DEVERR_BLOCK_ID);
             t.y8 = (id * H + h) * (bs / 8);  // first 8-row group of the run
             go = issue(0, t, 2 * m) && issue(1, t, 2 * m + 1);
+            if (ids_pending) {
+                load_chunk_ids(p, cn, box, lane, ids_n);
+                ids_pending = false;
+            }
         }
         if (go && has_next)
-            go = issue_q(items + 1, cn);
+            go = issue_q(items + 1, kn, cn);
+        kk = has_next ? kn : -1;
         c = cn;
         ids[0] = ids_n[0];
         ids[1] = ids_n[1];
+        if (kk >= 0) {  // the claim started one item ago becomes the next item; start another
+            kn = __shfl_sync(kFullMask, kclaim, 0);
+            if (kn < total)
+                kclaim = claim();
+        }
     }
     // After an abort, let the copies already issued land before the CTA (and
     // its shared memory) goes away.
@@ -404,8 +430,8 @@ __device__ __forceinline__ void load_role(const CUtensorMap *tm_q, const CUtenso
 
 // ------------------------------------------------------------ matrix unit
 // One thread.  Two streams of tensor-core work: S^T(n) = K_n Q^T once K_n has
-// landed and score buffer n % 2 is free, and O^T += V_n^T P_n^T once the
-// softmax has written P_n and V_n has landed.  The thread polls both and
+// landed and score buffer n % 2 is free, and O += P_n V_n once the softmax
+// has written P_n and V_n has landed.  The thread polls both and
 // issues whichever is ready, so a P.V never waits behind a later tile's K.
 // A tile with fewer than 128 valid rows takes only the P.V steps that hold
 // valid rows; the V rows past the end inside the last step are zeroed first.
@@ -416,7 +442,7 @@ struct PvInfo {
 __device__ __forceinline__ void mma_role(const Params &p, Shared &sh, uint32_t sbase, unsigned char *smem)
 {
     constexpr uint32_t kIdS = idesc_f16_f32_mn(kT, kNQ, false, false);  // K-major K, K-major Q
-    constexpr uint32_t kIdO = idesc_f16_f32_mn(kD, kNQ, true, false);   // M-major V, K-major P^T
+    constexpr uint32_t kIdO = idesc_f16_f32_mn(128, kD, false, true);   // K-major P, N-major V
     volatile int *abort = &sh.abort;
     const uint32_t tmem = sh.tmem;
     int u = -1, j = 0, nt = 0, t0 = 0, t1 = 0;  // item and tile of the next score product
@@ -450,7 +476,7 @@ __device__ __forceinline__ void mma_role(const Params &p, Shared &sh, uint32_t s
                 mbar_test_wait(smem_u32(&sh.q_full[u % kQSlots]), uint32_t(u / kQSlots) & 1u) &&
                 mbar_test_wait(smem_u32(&sh.kv_full[ks]), uint32_t((2 * ns) / kSlots) & 1u)) {
                 tc_fence_after_sync();
-                const uint32_t ka = sbase + uint32_t(ks) * kTile;
+                const uint32_t ka = sbase + kOffKV + uint32_t(ks) * kTile;
                 const uint32_t qa = sbase + kOffQ + uint32_t(u % kQSlots) * kQTile;
 #pragma unroll
                 for (int k = 0; k < kD / 16; ++k) {
@@ -480,7 +506,7 @@ __device__ __forceinline__ void mma_role(const Params &p, Shared &sh, uint32_t s
                  mbar_test_wait(smem_u32(&sh.o_empty[ob]), uint32_t((f.u >> 1) - 1) & 1u))) {
                 const int steps = (f.valid + 15) / 16;
                 if (f.valid < steps * 16) {  // zero V rows past the end inside the last step
-                    unsigned char *vt = smem + uint32_t(vs) * kTile;
+                    unsigned char *vt = smem + kOffKV + uint32_t(vs) * kTile;
                     for (int r = f.valid; r < steps * 16; ++r) {
                         unsigned char *row = vt + uint32_t(r >> 3) * kGroupStride + uint32_t(r & 7) * 128u;
 #pragma unroll
@@ -492,13 +518,17 @@ __device__ __forceinline__ void mma_role(const Params &p, Shared &sh, uint32_t s
                     fence_proxy_async_smem();
                 }
                 tc_fence_after_sync();
-                const uint32_t va = sbase + uint32_t(vs) * kTile;
+                const uint32_t va = sbase + kOffKV + uint32_t(vs) * kTile;
                 const uint32_t pa = sbase + kOffP + uint32_t(pb) * kQTile;
                 for (int k = 0; k < steps; ++k) {
                     const uint32_t kb = uint32_t(k >> 2), kk = uint32_t(k & 3) * 32u;
-                    umma_f16(tmem + kTmemO + uint32_t(ob) * kNQ,
+                    // A: P rows (8-row groups 1 KB apart), tokens 16k .. 16k+15;
+                    // B: V rows 16k .. 16k+15 (8-row groups kGroupStride apart),
+                    // the head dimension in two 64-wide halves kAtom apart
+                    umma_f16(tmem + kTmemO + uint32_t(ob) * kD,
+                             smem_desc_sw128(pa + kb * kQHalf + kk, 16, 1024),
                              smem_desc_sw128(va + uint32_t(k) * 2u * kGroupStride, kAtom, kGroupStride),
-                             smem_desc_sw128(pa + kb * kQHalf + kk, 16, 1024), kIdO, f.j > 0 || k > 0);
+                             kIdO, f.j > 0 || k > 0);
                 }
                 umma_commit(smem_u32(&sh.p_empty[pb]));
                 umma_commit(smem_u32(&sh.kv_empty[vs]));
@@ -584,28 +614,36 @@ __device__ __forceinline__ bool softmax_tile(const Params &p, Shared &sh, unsign
         for (int q = 0; q < NQ; ++q)
             need |= q < nq && tm[q] > m_ref[q] + kRescaleLog2;
         if (need) {  // uniform: every thread sees the same maxima
-            // move the reference: O (rows = head dims, one per thread) and the
-            // partial sums are rescaled once the previous P.V has completed
+            // move the reference: the partial sums (every thread) and the rows
+            // of O (warp 0: TMEM lane q holds query q) are rescaled once the
+            // previous P.V has completed
             ok = gwait(smem_u32(&sh.p_empty[(n - 1) % kPBufs]), uint32_t((n - 1) / kPBufs) & 1u, abort, err) &&
                  ok;
             tc_fence_after_sync();
-            float alpha[NQ];
+            float a_lane = 1.f;
 #pragma unroll
             for (int q = 0; q < NQ; ++q) {
                 const float mn = fmaxf(m_ref[q], tm[q]);
-                alpha[q] = ex2f(m_ref[q] - mn);
+                const float alpha = ex2f(m_ref[q] - mn);
                 m_ref[q] = mn;
-                l[q] *= alpha[q];
+                l[q] *= alpha;
+                if (lane == q)
+                    a_lane = alpha;
             }
-            const uint32_t tO = sh.tmem + kTmemO + uint32_t(u & 1) * kNQ + lane_base;
-            uint32_t o[16];
-            tmem_load16_async(tO, o);
-            tmem_wait_ld();
+            if (warp == 0) {
+                const uint32_t tO = sh.tmem + kTmemO + uint32_t(u & 1) * kD;
+#pragma unroll 1
+                for (int c = 0; c < kD / 16; ++c) {
+                    uint32_t o[16];
+                    tmem_load16_async(tO + uint32_t(c) * 16u, o);
+                    tmem_wait_ld();
 #pragma unroll
-            for (int q = 0; q < NQ; ++q)
-                o[q] = __float_as_uint(__uint_as_float(o[q]) * alpha[q]);
-            tmem_store16(tO, o);
-            tmem_wait_st();
+                    for (int e = 0; e < 16; ++e)
+                        o[e] = __float_as_uint(__uint_as_float(o[e]) * a_lane);
+                    tmem_store16(tO + uint32_t(c) * 16u, o);
+                }
+                tmem_wait_st();
+            }
         }
     }
     float pv[NQ];
@@ -614,8 +652,8 @@ __device__ __forceinline__ bool softmax_tile(const Params &p, Shared &sh, unsign
         pv[q] = live ? ex2f(x[q] - m_ref[q]) : 0.f;
         l[q] += pv[q];
     }
-    // P^T (row q = query column, 128 tokens as K, 128-byte swizzle) into the
-    // tile's operand buffer once the P.V two tiles back has read it
+    // P (row q = query, 128 tokens as K, 128-byte swizzle) into the tile's
+    // operand buffer once the P.V kPBufs tiles back has read it
     const int pb = n % kPBufs;
     if (n >= kPBufs)
         ok = gwait(smem_u32(&sh.p_empty[pb]), uint32_t(n / kPBufs - 1) & 1u, abort, err) && ok;
@@ -701,60 +739,48 @@ __device__ __forceinline__ void softmax_role(const Params &p, Shared &sh, unsign
 }
 
 // ---------------------------------------------------------------- epilogue
-// Barrier over the four epilogue warps (named barrier 2) with an AND of a
-// flag, so that all four take the same branch afterwards.
-__device__ __forceinline__ bool epilogue_bar_and(bool v)
-{
-    uint32_t r;
-    asm volatile(
-        "{\n\t.reg .pred p, q;\n\t"
-        "setp.ne.u32 p, %1, 0;\n\t"
-        "barrier.cta.red.and.pred q, 2, 128, p;\n\t"
-        "selp.u32 %0, 1, 0, q;\n\t}"
-        : "=r"(r)
-        : "r"(uint32_t(v))
-        : "memory");
-    return r != 0;
-}
-
-// Thread d (head dimension d, TMEM lane d) of the four epilogue warps: per
-// item, the O^T columns and the per-column (m, l) go to the workspace.
-__device__ __forceinline__ void epilogue_role(const Params &p, Shared &sh, int ew, int lane)
+// Warp 4 (TMEM lanes 0-31), thread q = query row q of O: per item, the row
+// (128 head dimensions) and the query's (m, l) go to the workspace.
+__device__ __forceinline__ void epilogue_role(const Params &p, Shared &sh, int lane)
 {
     volatile int *abort = &sh.abort;
     unsigned int *err = p.error_word;
-    const int d = ew * 32 + lane;
-    const uint32_t lane_base = uint32_t(ew * 32) << 16;
     const int H = p.num_heads;
+    const int q = lane < kNQ ? lane : 0;
     for (int u = 0;; ++u) {
         const bool got = gwait(smem_u32(&sh.e_full[u & 1]), uint32_t(u >> 1) & 1u, abort, err);
-        if (!epilogue_bar_and(got))
+        if (!__all_sync(kFullMask, got))
             break;
         const Epi &e = sh.epi[u & 1];
         if (e.end)
             break;
         const Chunk c = e.c;
         const int h = e.h;
-        const int qd = d < kNQ ? d : 0;
-        const float m_d = e.m[qd];
-        const float l_d = (e.l[0][qd] + e.l[1][qd]) + (e.l[2][qd] + e.l[3][qd]);
+        const float m_q = e.m[q];
+        const float l_q = (e.l[0][q] + e.l[1][q]) + (e.l[2][q] + e.l[3][q]);
         const bool ok = gwait(smem_u32(&sh.o_full[u & 1]), uint32_t(u >> 1) & 1u, abort, err);
+        if (!__all_sync(kFullMask, ok))
+            break;
         tc_fence_after_sync();
-        uint32_t o[16];
-        tmem_load16_async(sh.tmem + kTmemO + uint32_t(u & 1) * kNQ + lane_base, o);
+        const uint32_t tO = sh.tmem + kTmemO + uint32_t(u & 1) * kD;
+        uint32_t o[kD];
+        tmem_load32_into(tO, o);
+        tmem_load32_into(tO + 32u, o + 32);
+        tmem_load32_into(tO + 64u, o + 64);
+        tmem_load32_into(tO + 96u, o + 96);
         tmem_wait_ld();
         tc_fence_before_sync();
         __syncwarp();
         if (lane == 0)
             mbar_arrive(smem_u32(&sh.o_empty[u & 1]));
-        if (!epilogue_bar_and(ok))
-            break;
+        if (lane < c.nq) {
+            float4 *dst = reinterpret_cast<float4 *>(p.part_o + (size_t(c.col + q) * H + h) * kD);
 #pragma unroll
-        for (int q = 0; q < kNQ; ++q)
-            if (q < c.nq)
-                p.part_o[(size_t(c.col + q) * H + h) * kD + d] = __uint_as_float(o[q]);
-        if (d < c.nq)
-            reinterpret_cast<float2 *>(p.part_ml)[size_t(c.col + d) * H + h] = make_float2(m_d, l_d);
+            for (int i = 0; i < kD / 4; ++i)
+                dst[i] = make_float4(__uint_as_float(o[4 * i]), __uint_as_float(o[4 * i + 1]),
+                                     __uint_as_float(o[4 * i + 2]), __uint_as_float(o[4 * i + 3]));
+            reinterpret_cast<float2 *>(p.part_ml)[size_t(c.col + q) * H + h] = make_float2(m_q, l_q);
+        }
     }
 }
 
@@ -786,7 +812,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             mbar_init(smem_u32(&sh.s_full[i]), 1);
             mbar_init(smem_u32(&sh.s_empty[i]), 4);
             mbar_init(smem_u32(&sh.o_full[i]), 1);
-            mbar_init(smem_u32(&sh.o_empty[i]), 4);
+            mbar_init(smem_u32(&sh.o_empty[i]), 1);
             mbar_init(smem_u32(&sh.e_full[i]), 4);
         }
         for (int i = 0; i < kSlots; ++i) {
@@ -806,18 +832,17 @@ __global__ void __launch_bounds__(kThreads, 1)
     // the work list comes from the set-up kernel that precedes this one
     grid_dependency_wait();
     allow_dependent_launch();
-    const int total = p.meta->nchunks * p.num_heads;
 
     if (warp == kLoadWarp) {
-        load_role(&tm_q, &tm_k, &tm_v, p, sh, sbase, lane, total);
+        load_role(&tm_q, &tm_k, &tm_v, p, sh, sbase, lane);
     } else if (warp == kMmaWarp) {
         if (lane == 0)
             mma_role(p, sh, sbase, smem);
         __syncwarp();
     } else if (warp < 4) {
         softmax_role(p, sh, smem, warp, lane);
-    } else {
-        epilogue_role(p, sh, warp - 4, lane);
+    } else if (warp == kEpiWarp) {
+        epilogue_role(p, sh, lane);
     }
 
     tc_fence_before_sync();
