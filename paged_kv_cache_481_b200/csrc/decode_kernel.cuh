@@ -37,11 +37,16 @@
 //     lets its copies in flight land and stops.
 //   * Storage: fp16 rows, or int8 codes with one affine (s, z) per (token,
 //     head) row (brentwoodlivery.com 5.3.18: r_hat = s (q - z)).  For int8 a
-//     tile is 32 rows; the QK dot runs on the widened codes with the same
-//     mixed-precision FMA, and the zero point enters once per row:
-//       q.K = s (sum_d q_d (1024 + c_d) - (1024 + z) sum_d q_d),
-//     sum_t w_t V_t = sum_t w_t s_t (1024 + c_t) - sum_t w_t s_t (1024 + z_t),
-//     the codes being widened exactly to fp16 as 1024 + c by a byte permute.
+//     tile is 32 rows, and the zero point enters once per row:
+//       q.K = s (q . c - z sum_d q_d),
+//       sum_t w_t V_t = sum_t w_t s_t (1024 + c_t) - sum_t w_t s_t (1024 + z_t).
+//     q . c is exact integer arithmetic (dp4a) on the query in 16-bit fixed
+//     point (q = s_q q16, s_q = max |q| / 32767, set once per segment), so
+//     the only rounding the int8 path adds to the score is q's to 16 bits.
+//     For the P.V sum the codes are widened exactly to fp16 as 1024 + c by a
+//     byte permute and multiplied by w_t s_t rounded once to fp16 (the same
+//     rounded value in both sums, so the bias cancels exactly), with the
+//     products and sums in fp32 (mixed-precision FMA).
 //   * Fused append (DecodeExtras, fp16): the worker that issues a unit's last
 //     tile fetches one row fewer and its warp copies the new token's K / V
 //     rows from the input into the stage and into the cache slot (the decode
@@ -52,6 +57,7 @@
 
 #include <cuda_fp16.h>
 #include <cstdint>
+#include <type_traits>
 
 #include "ptx.cuh"
 #include "quant.cuh"
@@ -180,27 +186,35 @@ __device__ __forceinline__ uint32_t codes_to_h2(uint32_t word, uint32_t selector
     return __byte_perm(word, 0x64646464u, selector);
 }
 
-// q . k over one 16-byte chunk: 8 fp16 of K, or 16 int8 codes (as 1024 + c).
-template <bool kInt8>
-__device__ __forceinline__ float dot_chunk(const uint4 (&q)[kInt8 ? 2 : 1], const uint4 &k)
+// q . k over one 16-byte chunk of 8 fp16 values of K.
+__device__ __forceinline__ float dot_chunk(const uint4 (&q)[1], const uint4 &k)
 {
-    if constexpr (!kInt8) {
-        float s0 = fma2_f16_f32(q[0].x, k.x, 0.f);
-        float s1 = fma2_f16_f32(q[0].y, k.y, 0.f);
-        s0 = fma2_f16_f32(q[0].z, k.z, s0);
-        s1 = fma2_f16_f32(q[0].w, k.w, s1);
-        return s0 + s1;
-    } else {
-        float s0 = fma2_f16_f32(q[0].x, codes_to_h2(k.x, 0x5140u), 0.f);
-        float s1 = fma2_f16_f32(q[0].y, codes_to_h2(k.x, 0x5342u), 0.f);
-        s0 = fma2_f16_f32(q[0].z, codes_to_h2(k.y, 0x5140u), s0);
-        s1 = fma2_f16_f32(q[0].w, codes_to_h2(k.y, 0x5342u), s1);
-        s0 = fma2_f16_f32(q[1].x, codes_to_h2(k.z, 0x5140u), s0);
-        s1 = fma2_f16_f32(q[1].y, codes_to_h2(k.z, 0x5342u), s1);
-        s0 = fma2_f16_f32(q[1].z, codes_to_h2(k.w, 0x5140u), s0);
-        s1 = fma2_f16_f32(q[1].w, codes_to_h2(k.w, 0x5342u), s1);
-        return s0 + s1;
-    }
+    float s0 = fma2_f16_f32(q[0].x, k.x, 0.f);
+    float s1 = fma2_f16_f32(q[0].y, k.y, 0.f);
+    s0 = fma2_f16_f32(q[0].z, k.z, s0);
+    s1 = fma2_f16_f32(q[0].w, k.w, s1);
+    return s0 + s1;
+}
+
+// q . codes over one 16-byte chunk of 16 int8 codes, exactly, in int32: the
+// query in 16-bit fixed point split into a signed high byte and an unsigned
+// low byte per dimension (qw[0] = the high bytes of the chunk's 16 dims,
+// four per word; qw[1] = the low bytes), q16 . c = 256 (hi . c) + (lo . c).
+__device__ __forceinline__ int dot_codes_q16(const uint4 (&qw)[2], const uint4 &k)
+{
+    int hi = 0, lo = 0;
+    asm("dp4a.s32.u32 %0, %2, %3, %0;\n\t"
+        "dp4a.s32.u32 %0, %4, %5, %0;\n\t"
+        "dp4a.s32.u32 %0, %6, %7, %0;\n\t"
+        "dp4a.s32.u32 %0, %8, %9, %0;\n\t"
+        "dp4a.u32.u32 %1, %10, %3, %1;\n\t"
+        "dp4a.u32.u32 %1, %11, %5, %1;\n\t"
+        "dp4a.u32.u32 %1, %12, %7, %1;\n\t"
+        "dp4a.u32.u32 %1, %13, %9, %1;"
+        : "+r"(hi), "+r"(lo)
+        : "r"(qw[0].x), "r"(k.x), "r"(qw[0].y), "r"(k.y), "r"(qw[0].z), "r"(k.z), "r"(qw[0].w), "r"(k.w),
+          "r"(qw[1].x), "r"(qw[1].y), "r"(qw[1].z), "r"(qw[1].w));
+    return hi * 256 + lo;
 }
 
 __device__ __forceinline__ void axpy_h2(float &a0, float &a1, float w, uint32_t h2)
@@ -210,31 +224,43 @@ __device__ __forceinline__ void axpy_h2(float &a0, float &a1, float w, uint32_t 
     a1 = fmaf(w, v.y, a1);
 }
 
-// acc += w * chunk (8 fp16 values, or 16 int8 codes as 1024 + c).
-template <bool kInt8>
-__device__ __forceinline__ void axpy_chunk(float (&acc)[kInt8 ? 16 : 8], float w, const uint4 &u)
+// acc += w * chunk (8 fp16 values).
+__device__ __forceinline__ void axpy_chunk(float (&acc)[8], float w, const uint4 &u)
 {
-    if constexpr (!kInt8) {
-        axpy_h2(acc[0], acc[1], w, u.x);
-        axpy_h2(acc[2], acc[3], w, u.y);
-        axpy_h2(acc[4], acc[5], w, u.z);
-        axpy_h2(acc[6], acc[7], w, u.w);
-    } else {
-        axpy_h2(acc[0], acc[1], w, codes_to_h2(u.x, 0x5140u));
-        axpy_h2(acc[2], acc[3], w, codes_to_h2(u.x, 0x5342u));
-        axpy_h2(acc[4], acc[5], w, codes_to_h2(u.y, 0x5140u));
-        axpy_h2(acc[6], acc[7], w, codes_to_h2(u.y, 0x5342u));
-        axpy_h2(acc[8], acc[9], w, codes_to_h2(u.z, 0x5140u));
-        axpy_h2(acc[10], acc[11], w, codes_to_h2(u.z, 0x5342u));
-        axpy_h2(acc[12], acc[13], w, codes_to_h2(u.w, 0x5140u));
-        axpy_h2(acc[14], acc[15], w, codes_to_h2(u.w, 0x5342u));
+    axpy_h2(acc[0], acc[1], w, u.x);
+    axpy_h2(acc[2], acc[3], w, u.y);
+    axpy_h2(acc[4], acc[5], w, u.z);
+    axpy_h2(acc[6], acc[7], w, u.w);
+}
+
+// acc[2j], acc[2j + 1] += w * (1024 + code) for the 16 codes of a chunk, with
+// the weight w in fp16 (both halves of w2) and the products and sums in fp32
+// (mixed-precision FMA: no conversion of the codes' fp16 form to fp32).
+__device__ __forceinline__ void axpy_codes_f16w(float (&acc)[16], uint32_t w2, const uint4 &u)
+{
+    const uint32_t words[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+        const uint32_t lo = codes_to_h2(words[j], 0x5140u), hi = codes_to_h2(words[j], 0x5342u);
+        asm("{\n\t.reg .f16 w0, w1, a0, a1, b0, b1;\n\t"
+            "mov.b32 {w0, w1}, %4;\n\t"
+            "mov.b32 {a0, a1}, %5;\n\t"
+            "mov.b32 {b0, b1}, %6;\n\t"
+            "fma.rn.f32.f16 %0, w0, a0, %0;\n\t"
+            "fma.rn.f32.f16 %1, w0, a1, %1;\n\t"
+            "fma.rn.f32.f16 %2, w0, b0, %2;\n\t"
+            "fma.rn.f32.f16 %3, w0, b1, %3;\n\t}"
+            : "+f"(acc[4 * j]), "+f"(acc[4 * j + 1]), "+f"(acc[4 * j + 2]), "+f"(acc[4 * j + 3])
+            : "r"(w2), "r"(lo), "r"(hi));
     }
 }
 
 // Consume one staged tile: scores, online-softmax update and PV accumulate.
 // Lane (r, c) = (lane / kChunks, lane % kChunks) handles rows i*kRowsPerStep + r
 // and dims [kDims c, kDims (c + 1)).  For int8, kp / vp are the tile's (s, z)
-// rows, qsum = sum_d q_d, and corr accumulates sum_t w_t s_t (1024 + z_t).
+// rows, qh the query in 16-bit fixed point (dot_codes_q16), qsum = sum_d q16_d,
+// qk_scale_log2 includes the query's fixed-point scale s_q, and corr
+// accumulates sum_t w_t s_t (1024 + z_t).
 template <int D, bool kInt8, bool kFull>
 __device__ __forceinline__ void consume_tile(const uint4 *__restrict__ ks, const uint4 *__restrict__ vs,
                                              const float2 *__restrict__ kp, const float2 *__restrict__ vp,
@@ -244,10 +270,16 @@ __device__ __forceinline__ void consume_tile(const uint4 *__restrict__ ks, const
                                              float (&acc)[DecodeShape<D, kInt8>::kDims], float &corr)
 {
     using S = DecodeShape<D, kInt8>;
-    float v[S::kIters];
+    // int8: exact integer partial dot products (query in 16-bit fixed point)
+    using Part = typename std::conditional<kInt8, int, float>::type;
+    Part v[S::kIters];
 #pragma unroll
-    for (int i = 0; i < S::kIters; ++i)
-        v[i] = dot_chunk<kInt8>(qh, ks[(i * S::kRowsPerStep + r) * S::kChunks + c]);
+    for (int i = 0; i < S::kIters; ++i) {
+        if constexpr (kInt8)
+            v[i] = dot_codes_q16(qh, ks[(i * S::kRowsPerStep + r) * S::kChunks + c]);
+        else
+            v[i] = dot_chunk(qh, ks[(i * S::kRowsPerStep + r) * S::kChunks + c]);
+    }
 
     // Transposing reduction over the kChunks lanes of a row group: each step
     // halves the number of values a lane holds while summing across lanes.
@@ -259,8 +291,8 @@ __device__ __forceinline__ void consume_tile(const uint4 *__restrict__ ks, const
             const bool upper = (c & off) != 0;
 #pragma unroll
             for (int j = 0; j < n / 2; ++j) {
-                const float send = upper ? v[j] : v[j + n / 2];
-                const float keep = upper ? v[j + n / 2] : v[j];
+                const Part send = upper ? v[j] : v[j + n / 2];
+                const Part keep = upper ? v[j + n / 2] : v[j];
                 v[j] = keep + __shfl_xor_sync(kFullMask, send, off);
             }
         } else {
@@ -270,8 +302,10 @@ __device__ __forceinline__ void consume_tile(const uint4 *__restrict__ ks, const
     const int my_row = (c / S::kDup) * S::kRowsPerStep + r;
     float s;
     if constexpr (kInt8) {
+        // q . k_t = s_t (q . c_t - z_t sum_d q_d), q = s_q q16; qsum is
+        // sum_d q16_d and qk_scale_log2 carries s_q
         const float2 pz = kp[my_row];  // (s, z) of this lane's row
-        s = pz.x * fmaf(-(pz.y + kCodeBias), qsum, v[0]) * qk_scale_log2;
+        s = pz.x * fmaf(-pz.y, qsum, float(v[0])) * qk_scale_log2;
     } else {
         s = v[0] * qk_scale_log2;
     }
@@ -298,12 +332,15 @@ __device__ __forceinline__ void consume_tile(const uint4 *__restrict__ ks, const
         const int row = i * S::kRowsPerStep + r;
         if (kFull || row < valid_rows) {
             if constexpr (kInt8) {
+                // the row's weight times its scale, rounded once to fp16 and
+                // used as such by both sums, so the code bias cancels exactly
                 const float2 pz = vp[row];
-                const float ws = wi * pz.x;
-                corr = fmaf(ws, pz.y + kCodeBias, corr);
-                axpy_chunk<true>(acc, ws, vs[row * S::kChunks + c]);
+                const __half2 ws2 = __float2half2_rn(wi * pz.x);
+                const uint32_t w2 = *reinterpret_cast<const uint32_t *>(&ws2);
+                corr = fmaf(__low2float(ws2), pz.y + kCodeBias, corr);
+                axpy_codes_f16w(acc, w2, vs[row * S::kChunks + c]);
             } else {
-                axpy_chunk<false>(acc, wi, vs[row * S::kChunks + c]);
+                axpy_chunk(acc, wi, vs[row * S::kChunks + c]);
             }
         }
     }
@@ -830,7 +867,7 @@ __device__ __forceinline__ void paged_decode_body(const DecodeParams &p, const D
 #pragma unroll
     for (int k = 0; k < Sh::kQWords; ++k)
         qh[k] = make_uint4(0, 0, 0, 0);
-    float qsum = 0.f;
+    float qsum = 0.f, qscale = p.qk_scale_log2;
     float m = -INFINITY, l_part = 0.f, corr = 0.f;
     float acc[kDims];
 #pragma unroll
@@ -862,20 +899,48 @@ __device__ __forceinline__ void paged_decode_body(const DecodeParams &p, const D
             for (int k = 0; k < Sh::kQWords; ++k)
                 qh[k] = qs[Sh::kQWords * c + k];
             if constexpr (kInt8) {
-                float part = 0.f;
+                // the query row in 16-bit fixed point: q_d = s_q q16_d with
+                // s_q = max_d |q_d| / 32767, q16 split into a signed high
+                // byte and an unsigned low byte (dot_codes_q16)
+                float qf[16];
+                float amax = 0.f;
 #pragma unroll
-                for (int k = 0; k < Sh::kQWords; ++k) {
+                for (int k = 0; k < 2; ++k) {
                     const uint32_t w4[4] = {qh[k].x, qh[k].y, qh[k].z, qh[k].w};
 #pragma unroll
                     for (int e = 0; e < 4; ++e) {
                         const float2 f = h2f(w4[e]);
-                        part += f.x + f.y;
+                        qf[8 * k + 2 * e] = f.x;
+                        qf[8 * k + 2 * e + 1] = f.y;
+                        amax = fmaxf(amax, fmaxf(fabsf(f.x), fabsf(f.y)));
                     }
                 }
 #pragma unroll
                 for (int off = Sh::kChunks >> 1; off >= 1; off >>= 1)
-                    part += __shfl_xor_sync(kFullMask, part, off);
-                qsum = part;
+                    amax = fmaxf(amax, __shfl_xor_sync(kFullMask, amax, off));
+                const float inv = amax > 0.f ? 32767.f / amax : 0.f;
+                int isum = 0;
+                uint32_t hw[4], lw[4];
+#pragma unroll
+                for (int w = 0; w < 4; ++w) {
+                    uint32_t hb = 0, lb = 0;
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) {
+                        const int q16 = __float2int_rn(qf[4 * w + e] * inv);
+                        isum += q16;
+                        hb |= uint32_t((q16 >> 8) & 0xff) << (8 * e);
+                        lb |= uint32_t(q16 & 0xff) << (8 * e);
+                    }
+                    hw[w] = hb;
+                    lw[w] = lb;
+                }
+                qh[0] = make_uint4(hw[0], hw[1], hw[2], hw[3]);
+                qh[1] = make_uint4(lw[0], lw[1], lw[2], lw[3]);
+#pragma unroll
+                for (int off = Sh::kChunks >> 1; off >= 1; off >>= 1)
+                    isum += __shfl_xor_sync(kFullMask, isum, off);
+                qsum = float(isum);
+                qscale = (amax / 32767.f) * p.qk_scale_log2;
             }
 #pragma unroll
             for (int k = 0; k < kDims; ++k)
@@ -890,11 +955,11 @@ __device__ __forceinline__ void paged_decode_body(const DecodeParams &p, const D
         const float2 *kp = reinterpret_cast<const float2 *>(buf + Sm::kOffKP);
         const float2 *vp = reinterpret_cast<const float2 *>(buf + Sm::kOffVP);
         if (nv == T)
-            consume_tile<D, kInt8, true>(ks, vs, kp, vp, nv, r, c, qh, qsum, p.qk_scale_log2, m,
-                                         l_part, acc, corr);
+            consume_tile<D, kInt8, true>(ks, vs, kp, vp, nv, r, c, qh, qsum, qscale, m, l_part,
+                                         acc, corr);
         else
-            consume_tile<D, kInt8, false>(ks, vs, kp, vp, nv, r, c, qh, qsum, p.qk_scale_log2, m,
-                                          l_part, acc, corr);
+            consume_tile<D, kInt8, false>(ks, vs, kp, vp, nv, r, c, qh, qsum, qscale, m, l_part,
+                                          acc, corr);
         __syncwarp();
         if (issued < ntiles) {  // refill the stage just consumed
             if (lane == 0) {
