@@ -4,8 +4,10 @@
     python bench.py --kv-dtype int8 ...      # the same step over the int8 cache
     python bench.py --path prefill ...       # prompt cache write + pa_prefill, TFLOP/s
     python bench.py --workload 4 ...         # shared prefixes through pa_decode_grouped
-    python bench.py --decode-only ...        # pa_decode alone over the paged pool
+    python bench.py --decode-only ...        # the decode alone (pa_decode / pa_decode_grouped)
     python bench.py --layout contiguous ...  # the same decode, contiguous K / V, no block table
+    python bench.py --path prefill --new-tokens 512 --prompt-len 4096 ...  # chunked prefill
+    python bench.py --path cache-write|copy-blocks|swap ...  # those entry points alone, GB/s
     python bench.py --impl reference ...     # the fp64 CPU oracle, same metric
 
 One step = one decode iteration of the whole hot path over one batch: the
@@ -534,14 +536,18 @@ def run_gpu(args):
                                             device=dev)
         fused = False
 
-    # decode alone (the newest tokens written once before timing): over the
-    # paged pool (--decode-only), or over a contiguous copy of the same
-    # values with no block table (--layout contiguous)
+    # decode alone (the newest tokens written, and the shared-prefix workload's
+    # blocks copied, once before timing): over the paged pool (--decode-only;
+    # pa_decode_grouped for the shared-prefix workload), or over a contiguous
+    # copy of the same values with no block table (--layout contiguous)
     contig = args.layout == "contiguous"
-    decode_only = (args.decode_only or contig) and not grouped
+    decode_only = args.decode_only or contig
     if decode_only:
-        if pairs is not None or int8:
-            raise SystemExit("--decode-only / --layout contiguous: workloads 1, 2, 3 and 5, fp16")
+        if int8 or (contig and pairs is not None):
+            raise SystemExit("--decode-only: fp16 only; --layout contiguous: workloads 1, 2, 3 "
+                             "and 5")
+        if pairs is not None:
+            copy_step()
         write_step(key, value, slots)
         fused = False
     if contig:
@@ -574,7 +580,7 @@ def run_gpu(args):
                                      wl.scale, ws, stream=stream)
 
     def step(ev_pair=None):
-        if pairs is not None:
+        if pairs is not None and not decode_only:
             copy_step()
         if not fused and not decode_only:
             write_step(key, value, slots)
@@ -591,7 +597,7 @@ def run_gpu(args):
         if ev_pair is not None:
             ev_pair[1].record(stream)
 
-    launches_per_step = (1 if decode_only else
+    launches_per_step = ((4 if grouped else 1) if decode_only else
                          (1 if fused else 2) + ((4 if int8 else 1) if pairs is not None else 0)
                          + (3 if grouped else 0))
     with torch.cuda.stream(stream):
@@ -601,10 +607,11 @@ def run_gpu(args):
     assert binding.pa_get_last_device_error() == 0
 
     sampler = ClockSampler(local).start()
-    # a step of one launch is timed as K back-to-back launches between two
-    # events (the region's mean is that launch's mean duration, gaps included);
-    # a step of several launches brackets each decode with its own events
-    single_launch = launches_per_step == 1
+    # a step of one call (one launch, or the decode alone) is timed as K
+    # back-to-back calls between two events (the region's mean is that call's
+    # mean duration, gaps included); a step of several calls brackets each
+    # decode with its own events
+    single_launch = launches_per_step == 1 or decode_only
     evs = [None if single_launch else
            (torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
            for _ in range(args.steps)]
@@ -633,10 +640,12 @@ def run_gpu(args):
     # it, pipelined with the decode; the KV pool stays resident.
     def decode_from(views, o):
         d_q, d_key, d_value, d_slots, d_tables, d_lens = views[:6]
-        if pairs is not None:
+        if pairs is not None and not decode_only:
             copy_step()
         if contig:
             contig_step(o, d_q, d_lens)
+        elif decode_only and grouped:
+            grouped_step(o, d_q, d_tables, d_lens, views[6], views[7])
         elif decode_only:
             decode_step(o, d_q, d_tables, d_lens)
         elif grouped:
@@ -649,8 +658,9 @@ def run_gpu(args):
             decode_step(o, d_q, d_tables, d_lens)
 
     e2e_parts = [q, key, value, slots, tables, lens] + ([d_gs, d_pl] if grouped else [])
-    if decode_only:  # the step's inputs: q, (tables,) context lengths
-        e2e_parts = [q, key[:1], value[:1], slots[:1], tables if not contig else tables[:1], lens]
+    if decode_only:  # the step's inputs: q, (tables,) context lengths (, groups)
+        e2e_parts = ([q, key[:1], value[:1], slots[:1], tables if not contig else tables[:1], lens]
+                     + ([d_gs, d_pl] if grouped else []))
     e2e_ms, h2d, d2h = pipelined_e2e(e2e_parts, out, decode_from, stream, args.warmup, args.steps,
                                      world)
     assert binding.pa_get_last_device_error() == 0
@@ -668,7 +678,7 @@ def run_gpu(args):
     step_bytes = dec_bytes + (0 if decode_only else
                               b * h * (2 * d * 2 + 2 * (d + 8)) if int8
                               else accounting.cache_write_bytes(b, h, d))
-    if pairs is not None:
+    if pairs is not None and not decode_only:
         step_bytes += accounting.copy_blocks_bytes(len(wl.copy_pairs), h, d, wl.block_size)
 
     # max over ranks of the device-timed regions; totals over ranks
@@ -685,7 +695,10 @@ def run_gpu(args):
         kv_bytes = dec_bytes
         desc.update({
             "step": "pa_decode_contiguous (K / V [B, H, Lmax, D], no block table)" if contig else
-                    "pa_decode (the newest tokens written before timing)" if decode_only else
+                    (f"pa_decode_grouped ({len(wl.prefix_lens)} groups, prefixes of "
+                     f"{int(wl.prefix_lens[0])} tokens; blocks copied and newest tokens written "
+                     f"before timing)" if grouped else
+                     "pa_decode (the newest tokens written before timing)") if decode_only else
                     ("pa_copy_blocks + " if pairs is not None else "")
                     + (f"pa_reshape_and_cache({b} tokens) + pa_decode_grouped "
                        f"({len(wl.prefix_lens)} groups, prefixes of {int(wl.prefix_lens[0])} tokens)"
@@ -712,7 +725,7 @@ def run_gpu(args):
             "seq_heads_per_s": total_units * args.steps / (ms * 1e-3),
             "hbm_frac": achieved / peak,
             "decode_us_mean": mean_dec_ms * 1e3,
-            "launch_timing": ("events around the K back-to-back launches of the timed region"
+            "launch_timing": ("events around the K back-to-back calls of the timed region"
                               if single_launch else "events around each decode launch"),
             **({} if single_launch else {
                 "decode_us_median": statistics.median(decode_ms) * 1e3,
@@ -774,8 +787,8 @@ def prefill_cpu_baseline(q, key, value, n, length, num_heads, head_dim, block_si
     nblk = length // block_size
 
     def sample(heads):
-        k = key[:n, :heads].reshape(nblk, block_size, heads, head_dim).transpose(0, 2, 1, 3)
-        v = value[:n, :heads].reshape(nblk, block_size, heads, head_dim).transpose(0, 2, 1, 3)
+        k = key[:length, :heads].reshape(nblk, block_size, heads, head_dim).transpose(0, 2, 1, 3)
+        v = value[:length, :heads].reshape(nblk, block_size, heads, head_dim).transpose(0, 2, 1, 3)
         return (np.ascontiguousarray(q[:n, :heads]), np.ascontiguousarray(k),
                 np.ascontiguousarray(v), np.arange(nblk, dtype=np.int32)[None],
                 np.array([length], np.int32), np.array([0, n], np.int32))
@@ -809,36 +822,46 @@ def run_prefill(args):
 
     b, length, h, d = args.prompts, args.prompt_len, 40, 128
     bs = args.block_size or 16
-    n = length
+    n = args.new_tokens or length
     if length % bs:
         raise SystemExit("--prompt-len must be a multiple of the block size")
+    if not 0 < n <= length:
+        raise SystemExit("--new-tokens must be in [1, --prompt-len]")
     seed = 7 + 100 * rank
     rng = np.random.default_rng(seed)
     gen = torch.Generator().manual_seed(seed)
     tokens = b * n
-    # inputs drawn on the host (seeded), as the oracle sample needs them there too
+    # inputs drawn on the host (seeded), as the oracle sample needs them there too;
+    # K / V of every context token, of which the last n per sequence are new
     q_h = torch.randn((tokens, h, d), generator=gen).half()
-    key_h = torch.randn((tokens, h, d), generator=gen).half()
-    value_h = torch.randn((tokens, h, d), generator=gen).half()
+    key_h = torch.randn((b * length, h, d), generator=gen).half()
+    value_h = torch.randn((b * length, h, d), generator=gen).half()
     per_seq = length // bs
     nb = b * per_seq
     tables_h = rng.permutation(nb).astype(np.int32).reshape(b, per_seq)
-    pos = np.arange(n)
-    slots_h = np.concatenate([tables_h[i, pos // bs].astype(np.int64) * bs + pos % bs
-                              for i in range(b)])
+    pos = np.arange(length)
+    slots_all = np.stack([tables_h[i, pos // bs].astype(np.int64) * bs + pos % bs
+                          for i in range(b)])
+    slots_h = np.ascontiguousarray(slots_all[:, length - n:]).reshape(-1)
     scale = d ** -0.5
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         cpu = prefill_cpu_baseline(q_h.numpy(), key_h.numpy(), value_h.numpy(), n, length, h, d,
                                    bs, scale, target_s=args.cpu_seconds)
 
-    q, key, value = q_h.to(dev), key_h.to(dev), value_h.to(dev)
+    q = q_h.to(dev)
+    key = key_h.view(b, length, h, d)[:, length - n:].reshape(tokens, h, d).to(dev)
+    value = value_h.view(b, length, h, d)[:, length - n:].reshape(tokens, h, d).to(dev)
     slots = torch.from_numpy(slots_h).to(dev)
     tables = torch.from_numpy(tables_h).to(dev)
     lens = torch.full((b,), length, dtype=torch.int32, device=dev)
     qsl = torch.arange(b + 1, dtype=torch.int32, device=dev) * n
     kc = torch.zeros((nb, h, bs, d), dtype=torch.float16, device=dev)
     vc = torch.zeros_like(kc)
+    if n < length:  # the earlier chunks' K / V are in the cache before the step
+        binding.pa_reshape_and_cache(key_h.to(dev), value_h.to(dev), kc, vc,
+                                     torch.from_numpy(slots_all.reshape(-1)).to(dev))
+        torch.cuda.synchronize()
     out = torch.empty_like(q)
     stream = torch.cuda.Stream(device=dev)
     flops = _prefill_flops([length] * b, [n] * b, h, d)
@@ -895,15 +918,20 @@ def run_prefill(args):
             peak, peak_sus, kind = 1590.0, 1400.0, "fallback"
         mean_ms = statistics.fmean(launch_ms)
         achieved = flops / (mean_ms * 1e-3) / 1e12
-        workload = (f"13B prefill: {b} prompts x {length} tokens, H={h} D={d} bs={bs}, "
-                    f"shuffled blocks, causal")
+        if n == length:
+            workload = (f"13B prefill: {b} prompts x {length} tokens, H={h} D={d} bs={bs}, "
+                        f"shuffled blocks, causal")
+        else:
+            workload = (f"13B chunked prefill: {b} sequences, {n} new of {length} tokens, "
+                        f"H={h} D={d} bs={bs}, shuffled blocks, causal")
         result = {
             "metric": PREFILL_METRIC, "value": total_flops * args.steps / (ms * 1e-3) / 1e12,
             "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
             "ms_per_step": ms / args.steps, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "f16", "data": "synthetic",
             "config": {"workload": workload,
-                       "num_seqs": b, "prompt_len": length, "num_heads": h, "head_dim": d,
+                       "num_seqs": b, "prompt_len": length, "new_tokens": n,
+                       "num_heads": h, "head_dim": d,
                        "block_size": bs, "seed": seed,
                        "step": f"pa_reshape_and_cache({tokens} tokens) + pa_prefill",
                        "l2": f"K/V {2 * nb * h * bs * d * 2 / 1e9:.2f} GB and q/out "
@@ -936,6 +964,235 @@ def run_prefill(args):
     return 0
 
 
+BLOCK_OP_METRIC = {
+    "cache-write": "pa_reshape_and_cache: GB/s (new K/V read + cache rows written; % of HBM peak)",
+    "copy-blocks": "pa_copy_blocks: GB/s (blocks read + written; % of HBM peak)",
+    "swap": "pa_swap_blocks: GB/s over the host link (% of a plain copy of the same bytes)",
+}
+
+
+def _graph_ms(launch, stream, warmup, steps):
+    """Device time of `steps` calls launch(0), ..., launch(steps - 1) captured
+    in one CUDA graph and replayed once.  These kernels run for a few
+    microseconds, less than a host launch takes, so issuing them one by one
+    would time the host; the replay times the device.  Warm-up: one replay
+    of a graph of `warmup` calls."""
+    import torch
+
+    def capture(n):
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=stream):
+            for i in range(n):
+                launch(i, stream)
+        return g
+
+    with torch.cuda.stream(stream):
+        for i in range(3):  # outside any capture: the library's first launches
+            launch(i, stream)
+    torch.cuda.synchronize()
+    warm, timed = capture(warmup), capture(steps)
+    with torch.cuda.stream(stream):  # a graph replays on the current stream
+        warm.replay()
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        timed.replay()
+        e1.record(stream)
+    torch.cuda.synchronize()
+    return e0.elapsed_time(e1)
+
+
+def _host_fed_ms(parts, launch, stream, warmup, steps):
+    """The same calls issued one by one through the public API, each step's
+    inputs (`parts`) copied from pinned host memory just before it on the
+    launching stream; returns (ms for `steps` steps, h2d bytes per step)."""
+    import torch
+    hosts = [p.cpu().pin_memory() for p in parts]
+    devs = [torch.empty_like(p) for p in parts]
+
+    def one(i):
+        with torch.cuda.stream(stream):
+            for h_, d_ in zip(hosts, devs):
+                d_.copy_(h_, non_blocking=True)
+            launch(devs, stream)
+
+    for i in range(warmup):
+        one(i)
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for i in range(steps):
+        one(i)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    return e0.elapsed_time(e1), sum(p.numel() * p.element_size() for p in parts)
+
+
+def run_block_ops(args):
+    """The cache-management entry points, one JSON line each.
+
+    cache-write: one decode step's pa_reshape_and_cache of --tokens new
+    tokens (13B shapes, H=40, D=128, bs=16) into random slots of an 8192-block
+    pool.  copy-blocks: pa_copy_blocks of --pairs copy-on-write pairs.  A
+    step's inputs (new K/V and slots; the pairs) rotate through enough
+    distinct sets that they and the rows they touch do not stay in L2 from
+    one step to the next.  Timed as a CUDA graph of the K calls.
+
+    swap: pa_swap_blocks of --swap-blocks blocks (160 KB each at 13B shapes)
+    between the device pool and a page-locked host pool, in the direction
+    --direction, to a permuted set of blocks, against a plain copy of the
+    same number of contiguous bytes over the same link; events per call."""
+    import torch
+    import torch.distributed as dist
+    from paged_kv_cache_481_b200 import accounting, binding
+
+    world, rank, local = _init_ranks(args)
+    dev = torch.device("cuda", local)
+    h, d, bs = 40, 128, args.block_size or 16
+    seed = 11 + 100 * rank
+    g = torch.Generator(device=dev).manual_seed(seed)
+    stream = torch.cuda.Stream(device=dev)
+    peak_hbm, peak_kind = _peak_hbm()
+    sampler = ClockSampler(local).start()
+    extra = {}
+    if args.path == "swap":
+        nblk = args.swap_blocks
+        pool = torch.randn((nblk, h, bs, d), generator=g, device=dev).half()
+        host = torch.empty((nblk, h, bs, d), dtype=torch.float16).pin_memory()
+        perm = torch.randperm(nblk, generator=g, device=dev)
+        pairs = torch.stack([torch.arange(nblk, device=dev), perm], 1).contiguous()
+        src, dst = (pool, host) if args.direction == "d2h" else (host, pool)
+        nbytes = pool.numel() * pool.element_size()
+
+        def timed(fn):
+            with torch.cuda.stream(stream):
+                for _ in range(args.warmup):
+                    fn()
+            torch.cuda.synchronize()
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record(stream)
+            with torch.cuda.stream(stream):
+                for _ in range(args.steps):
+                    fn()
+            e1.record(stream)
+            torch.cuda.synchronize()
+            return e0.elapsed_time(e1)
+
+        if world > 1:
+            dist.barrier()
+        w0 = time.perf_counter()
+        ms = timed(lambda: binding.pa_swap_blocks(src, dst, pairs, stream=stream))
+        w1 = time.perf_counter()
+        ms_link = timed(lambda: dst.copy_(src, non_blocking=True))
+        unit_bytes = nbytes
+        launches = args.steps
+        workload = (f"13B swap {'device -> host' if args.direction == 'd2h' else 'host -> device'}"
+                    f": {nblk} blocks of {nbytes // nblk // 1024} KB (H={h} D={d} bs={bs}), "
+                    f"permuted destination blocks")
+        link_gbs = nbytes * args.steps / (ms_link * 1e-3) / 1e9
+        roof = {"kernel": "copy_blocks_kernel (host pool)", "bound": "link",
+                "achieved": nbytes * args.steps / (ms * 1e-3) / 1e9, "peak": link_gbs,
+                "peak_kind": "measured in this run: a plain cudaMemcpyAsync of the same bytes "
+                             "over the same link (torch copy_)",
+                "unit": "GB/s", "traffic": None}
+        roof["frac"] = roof["achieved"] / roof["peak"]
+        config = {"workload": workload, "blocks": nblk, "block_bytes": nbytes // nblk,
+                  "direction": args.direction, "seed": seed,
+                  "l2": "host link bound; the pool (one copy per step) is "
+                        f"{nbytes / 2**20:.0f} MiB vs {L2_BYTES / 2**20:.0f} MiB L2"}
+        e2e = {"value": roof["achieved"], "unit": "GB/s",
+               "note": "the call is itself the host <-> device transfer",
+               "h2d_bytes_per_step": nbytes if args.direction == "h2d" else 0,
+               "d2h_bytes_per_step": nbytes if args.direction == "d2h" else 0}
+    else:
+        nb = 8192
+        kc = torch.randn((nb, h, bs, d), generator=g, device=dev).half()
+        vc = torch.randn_like(kc)
+        if args.path == "cache-write":
+            n = args.tokens
+            unit_bytes = accounting.cache_write_bytes(n, h, d)
+            # distinct sets of inputs and target rows: 2x L2 of inputs, at most 1024
+            sets = int(min(1024, max(8, math.ceil(2 * L2_BYTES / (4 * n * h * d)))))
+            key = torch.randn((sets, n, h, d), generator=g, device=dev).half()
+            value = torch.randn_like(key)
+            slots = (torch.randint(0, nb, (sets, n), generator=g, device=dev) * bs
+                     + torch.randint(0, bs, (sets, n), generator=g, device=dev)).long()
+
+            def launch(i, st):
+                j = i % sets
+                binding.pa_reshape_and_cache(key[j], value[j], kc, vc, slots[j], stream=st)
+
+            parts = [key[0], value[0], slots[0]]
+
+            def fed(views, st):
+                binding.pa_reshape_and_cache(views[0], views[1], kc, vc, views[2], stream=st)
+
+            kernel = "reshape_and_cache_kernel"
+            workload = (f"13B decode-step cache write: {n} new tokens (H={h} D={d} bs={bs}) "
+                        f"into random slots of an {nb}-block pool")
+            config_extra = {"tokens": n, "input_sets": sets}
+        else:
+            p = args.pairs
+            unit_bytes = accounting.copy_blocks_bytes(p, h, d, bs)
+            sets = int(min(1024, max(4, math.ceil(2 * L2_BYTES / (unit_bytes / 2)))))
+            sets = min(sets, nb // (2 * p))
+            pairs = torch.stack([torch.randperm(nb, generator=g, device=dev)[:2 * p].view(p, 2)
+                                 for _ in range(sets)]).long().contiguous()
+
+            def launch(i, st):
+                binding.pa_copy_blocks(kc, vc, pairs[i % sets], stream=st)
+
+            parts = [pairs[0]]
+
+            def fed(views, st):
+                binding.pa_copy_blocks(kc, vc, views[0], stream=st)
+
+            kernel = "copy_blocks_kernel"
+            workload = (f"13B copy-on-write: {p} block pairs (H={h} D={d} bs={bs}, K and V) "
+                        f"in an {nb}-block pool")
+            config_extra = {"pairs": p, "pair_sets": sets}
+        if world > 1:
+            dist.barrier()
+        w0 = time.perf_counter()
+        ms = _graph_ms(launch, stream, args.warmup, args.steps)
+        w1 = time.perf_counter()
+        e2e_ms, h2d = _host_fed_ms(parts, fed, stream, args.warmup, args.steps)
+        launches = args.steps
+        achieved = unit_bytes * args.steps / (ms * 1e-3) / 1e9
+        roof = {"kernel": kernel, "bound": "hbm", "achieved": achieved, "peak": peak_hbm,
+                "peak_kind": peak_kind, "unit": "GB/s", "frac": achieved / peak_hbm,
+                "traffic": None, "algorithmic_bytes_per_launch": unit_bytes}
+        config = {"workload": workload, "num_heads": h, "head_dim": d, "block_size": bs,
+                  "seed": seed, **config_extra,
+                  "timing": f"one CUDA graph of the {args.steps} calls, replayed once",
+                  "l2": f"inputs rotate through {sets} distinct sets (no flush)"}
+        e2e = {"value": unit_bytes * args.steps / (e2e_ms * 1e-3) / 1e9, "unit": "GB/s",
+               "copies": "the step's inputs from pinned host memory each step, calls issued "
+                         "one by one from the host",
+               "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": 0,
+               "ms_per_step": e2e_ms / args.steps}
+        extra["us_per_call"] = ms * 1e3 / args.steps
+    sampler.stop()
+    assert binding.pa_get_last_device_error() == 0
+    (ms,), (total,) = reduce_over_ranks([ms], [unit_bytes * args.steps], dev)
+    result = None
+    if rank == 0:
+        result = {
+            "metric": BLOCK_OP_METRIC[args.path], "value": total / (ms * 1e-3) / 1e9,
+            "unit": "GB/s", "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": ms / args.steps, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "f16", "data": "synthetic", "config": config,
+            **extra, "roofline": roof, "e2e": e2e, "gpu_launches": launches,
+            "clocks": sampler.summary(w0, w1),
+        }
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    if result is not None:
+        print(json.dumps(result), flush=True)
+    return 0
+
+
 def main(argv=None):
     ap = argparse.ArgumentParser(description=__doc__.splitlines()[0])
     ap.add_argument("--gpus", type=int, default=1)
@@ -956,13 +1213,24 @@ def main(argv=None):
                     help="contiguous: the same decode over K / V [B, H, Lmax, D] with no block "
                          "table (the baseline for the indirection's cost); times the decode alone")
     ap.add_argument("--decode-only", action="store_true",
-                    help="time pa_decode alone (the newest tokens written before timing)")
+                    help="time the decode alone, K back-to-back calls (pa_decode; pa_decode_grouped "
+                         "for the shared-prefix workload; the newest tokens written and the blocks "
+                         "copied before timing)")
     ap.add_argument("--no-grouped", action="store_true",
                     help="shared-prefix workload: plain pa_decode instead of pa_decode_grouped")
-    ap.add_argument("--path", choices=["decode", "prefill"], default="decode",
-                    help="prefill: the prompt cache write + pa_prefill step instead of decode")
+    ap.add_argument("--path", choices=["decode", "prefill", "cache-write", "copy-blocks", "swap"],
+                    default="decode",
+                    help="prefill: the prompt cache write + pa_prefill step instead of decode; "
+                         "cache-write / copy-blocks / swap: those entry points alone")
     ap.add_argument("--prompts", type=int, default=8, help="prefill: prompts per step")
     ap.add_argument("--prompt-len", type=int, default=2048, help="prefill: tokens per prompt")
+    ap.add_argument("--new-tokens", type=int, default=None,
+                    help="prefill: new tokens per sequence (the last ones of its --prompt-len "
+                         "context; the earlier ones already cached): chunked prefill")
+    ap.add_argument("--tokens", type=int, default=256, help="cache-write: new tokens per step")
+    ap.add_argument("--pairs", type=int, default=64, help="copy-blocks: block pairs per step")
+    ap.add_argument("--swap-blocks", type=int, default=1024, help="swap: blocks per step")
+    ap.add_argument("--direction", choices=["d2h", "h2d"], default="d2h", help="swap direction")
     ap.add_argument("--cpu-threads", type=int, default=None,
                     help="host threads for the oracle (CPU baseline / reference arm); default all")
     args = ap.parse_args(argv)
@@ -980,6 +1248,8 @@ def main(argv=None):
         return run_reference(args)
     if args.path == "prefill":
         return run_prefill(args)
+    if args.path in BLOCK_OP_METRIC:
+        return run_block_ops(args)
     return run_gpu(args)
 
 
