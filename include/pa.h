@@ -337,8 +337,8 @@ PA_API pa_status pa_prefill(void *out, const void *q, const void *k_cache, const
  * Same result as pa_decode over the same arguments, but each shared prefix
  * is read from memory once per (group, head): the group's queries are scored
  * against it together on the tensor cores, each member's own tail is scored
- * alone, and the parts are merged by their softmax normalisers, all in one
- * persistent kernel after a small set-up kernel.
+ * alone by the decode kernel on the other SMs at the same time, and the
+ * parts are merged by their softmax normalisers.
  *   group_start [num_groups + 1] int32 (device): group g = sequences
  *     group_start[g] .. group_start[g+1] - 1; group_start[0] = 0 and
  *     group_start[num_groups] = num_seqs, nondecreasing (every sequence in
@@ -348,9 +348,10 @@ PA_API pa_status pa_prefill(void *out, const void *q, const void *k_cache, const
  *     members' block tables must agree on those blocks (0 = nothing shared).
  *   max_group_size: host bound on group sizes (<= 65535).
  *   workspace: pa_decode_grouped_workspace_size(num_seqs, num_groups,
- *     num_heads, head_dim, max_context_len) bytes, 16-byte aligned; no
- *     initialisation needed (each call clears what it uses), and one
- *     workspace serves any smaller problem too.  Calls that share a
+ *     num_heads, head_dim, max_context_len, max_blocks_per_seq) bytes,
+ *     16-byte aligned, all zero before its first use (cudaMemsetAsync, or
+ *     pa_decode_workspace_init); every call leaves it ready for the next,
+ *     and one workspace serves any smaller problem too.  Calls that share a
  *     workspace must not overlap on the GPU.
  * head_dim must be 128 (else PA_ERR_UNSUPPORTED), scale > 0.  A prefix that
  * breaks these rules is recorded (PA_DEVERR_CONTEXT_LEN) and its group is

@@ -277,7 +277,7 @@ def pa_decode_append_int8(out, q, key, value, k_codes, v_codes, k_params, v_para
 
 def new_grouped_workspace(num_seqs, num_groups, num_heads, head_dim, max_context_len,
                           max_blocks_per_seq, device="cuda"):
-    """Workspace for pa_decode_grouped (needs no initialisation)."""
+    """Workspace for pa_decode_grouped, zero-filled as its first use requires."""
     n = load().pa_decode_grouped_workspace_size(num_seqs, num_groups, num_heads, head_dim,
                                                 max_context_len, max_blocks_per_seq)
     return torch.zeros(max(int(n), 16), dtype=torch.uint8, device=device)

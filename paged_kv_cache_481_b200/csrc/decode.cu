@@ -145,7 +145,8 @@ pa_status decode_common(void *out, const void *q, const void *k_cache, const voi
                         void *workspace, size_t workspace_bytes, pa_stream_t stream,
                         const void *new_k = nullptr, const void *new_v = nullptr,
                         const int64_t *new_slots = nullptr, float *lse = nullptr,
-                        int max_ctas = 0, bool late_dep_wait = false)
+                        int max_ctas = 0, bool late_dep_wait = false,
+                        const unsigned int *ready = nullptr)
 {
     if (num_seqs < 0 || num_heads <= 0 || num_blocks <= 0 || max_context_len < 0 ||
         max_blocks_per_seq < 0)
@@ -195,6 +196,7 @@ pa_status decode_common(void *out, const void *q, const void *k_cache, const voi
     x.new_v = static_cast<const __half *>(new_v);
     x.new_slots = new_slots;
     x.lse = lse;
+    x.ready = late_dep_wait ? ready : nullptr;
 
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
     if (int8) {
@@ -407,12 +409,12 @@ pa_status pa_host::decode_with_lse(void *out, const void *q, const void *k_cache
                                    int max_context_len, int num_seqs, int num_heads, int head_dim,
                                    int block_size, int num_blocks, float scale, void *workspace,
                                    size_t workspace_bytes, float *lse, pa_stream_t stream,
-                                   int max_ctas, bool late_dep_wait)
+                                   int max_ctas, bool late_dep_wait, const unsigned int *ready)
 {
     return decode_common(out, q, k_cache, v_cache, nullptr, nullptr, false, block_tables,
                          max_blocks_per_seq, context_lens, max_context_len, num_seqs, num_heads,
                          head_dim, block_size, num_blocks, scale, workspace, workspace_bytes, stream,
-                         nullptr, nullptr, nullptr, lse, max_ctas, late_dep_wait);
+                         nullptr, nullptr, nullptr, lse, max_ctas, late_dep_wait, ready);
 }
 
 int pa_host::decode_ctas_per_sm()

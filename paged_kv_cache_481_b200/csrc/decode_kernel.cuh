@@ -114,6 +114,10 @@ struct DecodeExtras {
     // optional [B, H]: log2 of each unit's softmax denominator relative to
     // 2^0, i.e. max + log2(sum) in base-2 units (to merge with other parts)
     float *lse;
+    // optional, kLateDepWait instances only: the inputs are written by a
+    // kernel that may still be running, which sets *ready non-zero once they
+    // are all visible; every CTA waits for it (bounded) before it starts
+    const unsigned int *ready;
 };
 
 constexpr int ilog2(int x)
@@ -1046,11 +1050,13 @@ __device__ __forceinline__ void paged_decode_body(const DecodeParams &p, const D
 // kLateDepWait = false: inputs may come from the previous kernel in the
 // stream, so none is read before it has finished; the next kernel may start
 // launching meanwhile.  kLateDepWait = true: the caller guarantees the
-// inputs are ready (they were written two launches back and the previous
-// kernel only starts this one after it has itself waited for them), so the
+// inputs are ready -- they were written two launches back and the previous
+// kernel only starts this one after it has itself waited for them, or
+// x.ready is set and the kernel that writes them raises that flag -- so the
 // work starts at once, running beside the previous kernel, and the wait for
-// that kernel comes at the end: this grid then completes only after the
-// previous one, and the next kernel that waits for this grid sees both.
+// that kernel comes at the end: this grid then completes only after
+// everything before it, and the next kernel that waits for this grid sees
+// all of it.
 // kContig: the cache is contiguous per (sequence, head), [B, H, Lmax, D]
 // with Lmax in block_size, and no block table is read (the baseline that
 // measures what the paged layout's indirection costs).
@@ -1060,6 +1066,23 @@ __global__ void __launch_bounds__(NW * 32) paged_decode_kernel(const DecodeParam
     if (!kLateDepWait)
         grid_dependency_wait();
     allow_dependent_launch();
+    if constexpr (kLateDepWait) {
+        if (x.ready) {
+            if (threadIdx.x == 0) {
+                const volatile unsigned int *flag = x.ready;
+                bool ok = *flag != 0u;
+                if (!ok) {
+                    const uint64_t t0 = global_timer_ns();
+                    while (!(ok = *flag != 0u) && global_timer_ns() - t0 < kWaitLimitNs)
+                        __nanosleep(64);
+                }
+                if (!ok)
+                    raise_device_error(kErrTimeout);
+                __threadfence();
+            }
+            __syncthreads();
+        }
+    }
     paged_decode_body<D, kInt8, NW, S, kContig>(p, x);
     if (kLateDepWait && threadIdx.x == 0)
         grid_dependency_wait();

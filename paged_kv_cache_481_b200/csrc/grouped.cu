@@ -1,19 +1,27 @@
 // libpa, shared-prefix decode: C ABI of pa_decode_grouped.  Host code here
 // validates arguments, lays out the workspace, encodes the TMA tensor maps
 // and launches four kernels on the caller's stream:
-//   1. a one-CTA set-up kernel: the prefix work list (chunks), each member's
-//      tail table (its block-table row from the first block past the shared
-//      prefix) and tail length, zero outputs for empty contexts;
-//   2. the persistent tensor-core kernel of grouped_kernel.cuh over the
-//      prefix chunks, leaving (m, l, o) per member, head and chunk, on a
-//      share of the SMs (kPrefixSmShare);
-//   3. the paged decode kernel over the tails, with each (member, head)'s
-//      base-2 log-normaliser, on the other SMs at the same time: it starts as
-//      soon as every prefix CTA is resident (programmatic dependent launch)
-//      and waits for the prefix kernel only at its end;
-//   4. a merge kernel: the prefix partials and the tail result combined by
-//      their softmax normalisers.
-// Nothing here allocates device memory.
+//   * a one-CTA set-up kernel: each member's tail table (its block-table row
+//     from the first block past the shared prefix), tail length and merge
+//     record, zero outputs for empty contexts, and (beyond 32 groups) the
+//     prefix work list (chunks);
+//   * the persistent tensor-core kernel of grouped_kernel.cuh over the
+//     prefix chunks, leaving (m, l, o) per member, head and chunk, on a
+//     share of the SMs;
+//   * the paged decode kernel over the tails, with each (member, head)'s
+//     base-2 log-normaliser, on the other SMs at the same time;
+//   * a merge kernel: the prefix partials and the tail result combined by
+//     their softmax normalisers, once every prefix CTA has counted itself
+//     done.
+// The order is set-up, prefix, tails, merge, each launched as a programmatic
+// dependent of the one before.  The tails start as soon as every prefix CTA
+// is resident and wait for the prefix kernel only at their end.  With at
+// most 32 groups the prefix kernel works out its own work list and does not
+// wait for the set-up kernel, so it streams while the set-up kernel works out
+// the tails; the tail decode then waits for the set-up kernel's `ready`
+// flag before it starts (a dependency wait there would wait for the prefix
+// kernel too: such a wait covers everything launched before).  Nothing here
+// allocates device memory.
 #include <cuda.h>
 #include <cuda_runtime.h>
 
@@ -44,6 +52,8 @@ struct SetupParams {
     const int32_t *block_tables;  // [B, MB]
     int num_groups, num_seqs, max_context_len, block_size, num_heads, max_blocks;
     int max_chunks;               // capacity of `chunks` and of the partial columns
+    int self_list;                // the prefix kernel builds its own work list and runs
+                                  // beside this kernel: leave the header alone, raise `ready`
     __half *out;                  // rows of empty contexts are zeroed here
     Meta *meta;
     Group *groups;                // used without the shared-memory working set
@@ -81,6 +91,12 @@ size_t setup_smem_bytes(int num_groups, int num_seqs, int max_blocks)
 // of 1-256 tokens, 0.50 suits copy-on-write tables (each tail also holds
 // the copied last prefix block) and 0.55 fully aliased ones.
 constexpr float kPrefixSmShare = 0.53f;
+
+// With its own work list (at most kSelfListMaxGroups groups: one per lane of
+// its load warp) the prefix kernel streams several microseconds before the
+// tails start, and takes a smaller share.
+constexpr int kSelfListMaxGroups = 32;
+constexpr float kSelfListSmShare = 0.49f;
 
 __device__ __forceinline__ int clamp_len(const SetupParams &p, int raw)
 {
@@ -212,26 +228,20 @@ __global__ void __launch_bounds__(kSetupThreads) grouped_setup_kernel(const Setu
         const bool okg = 0 <= g0 && g0 <= g1 && g1 <= B;
         if (!okg && lane == 0)
             atomicOr(p.err, PA_DEVERR_CONTEXT_LEN);
-        const int n = okg ? g1 - g0 : 0;
-        if (!okg)
-            g0 = 0;
         int min_len = INT_MAX;
-        for (int b = g0 + lane; b < g0 + n; b += 32)
-            min_len = min(min_len, length(b));
+        if (okg)
+            for (int b = g0 + lane; b < g1; b += 32)
+                min_len = min(min_len, length(b));
         min_len = __reduce_min_sync(pa::kFullMask, min_len);
-        if (n == 0 || P < 0 || P % bs != 0 || P > min_len) {
-            if (n > 0 && P != 0 && lane == 0)
-                atomicOr(p.err, PA_DEVERR_CONTEXT_LEN);
-            P = 0;
-        }
-        const int cp = (P + kChunk - 1) / kChunk;
-        const int slices = (n + 15) / 16;
-        for (int b = g0 + lane; b < g0 + n; b += 32) {
+        const pa::grp::GroupPlan gp = pa::grp::plan_group(g0, g1, P, min_len, B, bs);
+        if (!gp.prefix_ok && gp.n > 0 && P != 0 && lane == 0)
+            atomicOr(p.err, PA_DEVERR_CONTEXT_LEN);
+        for (int b = gp.g0 + lane; b < gp.g0 + gp.n; b += 32) {
             gof[b] = g;
-            tl[b] = length(b) - P;
+            tl[b] = length(b) - gp.P;
         }
         if (lane == 0)  // colbase and pstart hold counts until the scan turns them into offsets
-            gr[g] = Group{g0, n, cp, P, n * cp, slices * cp, 0, 0};
+            gr[g] = Group{gp.g0, gp.n, gp.cp, gp.P, gp.n * gp.cp, gp.slices * gp.cp, 0, 0};
     }
     __syncthreads();
 
@@ -276,7 +286,12 @@ __global__ void __launch_bounds__(kSetupThreads) grouped_setup_kernel(const Setu
     if (!fits) {  // cannot happen with the host's bound; refuse rather than overrun
         if (tid == 0) {
             atomicOr(p.err, PA_DEVERR_CONTEXT_LEN);
-            *p.meta = Meta{0, 0, 0, 0};
+            if (!p.self_list) {
+                p.meta->nchunks = 0;
+                p.meta->ncols = 0;
+            } else {
+                atomicExch(&p.meta->ready, 1u);
+            }
         }
         return;
     }
@@ -338,8 +353,18 @@ __global__ void __launch_bounds__(kSetupThreads) grouped_setup_kernel(const Setu
     }
     for (int i = tid; i < B * H; i += kSetupThreads)
         p.dec_tickets[i] = 0u;
-    if (tid == 0)
-        *p.meta = Meta{nchunks, ncols, 0, 0};
+    if (!p.self_list) {  // the prefix kernel's work list; it starts after this kernel
+        if (tid == 0) {
+            p.meta->nchunks = nchunks;
+            p.meta->ncols = ncols;
+            p.meta->claimed = 0;
+        }
+    } else {  // the tail decode is already running and waits for this flag
+        __threadfence();
+        __syncthreads();
+        if (tid == 0)
+            atomicExch(&p.meta->ready, 1u);
+    }
 }
 
 // out[b, h] = (sum_j 2^(m_j - M) o_j + 2^(lse_t - M) o_t) /
@@ -347,16 +372,11 @@ __global__ void __launch_bounds__(kSetupThreads) grouped_setup_kernel(const Setu
 // the prefix chunks' partials (m_j, l_j, o_j unnormalised, fp32) and the
 // tail's normalised fp16 result with its log-normaliser lse_t.  An empty
 // part has weight 0.  One warp per (member, head), four dims per lane.
-__global__ void __launch_bounds__(256) grouped_merge_kernel(
-    __half *__restrict__ out, const Member *__restrict__ members, const float *__restrict__ part_ml,
-    const float *__restrict__ part_o, const __half *__restrict__ o_t, const float *__restrict__ lse_t,
-    int num_heads, int units)
+__device__ __forceinline__ void merge_unit(__half *__restrict__ out, const Member *__restrict__ members,
+                                           const float *__restrict__ part_ml, const float *__restrict__ part_o,
+                                           const __half *__restrict__ o_t, const float *__restrict__ lse_t,
+                                           int num_heads, int unit, int lane)
 {
-    pa::grid_dependency_wait();
-    pa::allow_dependent_launch();
-    const int unit = blockIdx.x * 8 + (threadIdx.x >> 5), lane = threadIdx.x & 31;
-    if (unit >= units)
-        return;
     const int b = unit / num_heads, h = unit % num_heads;
     // the tail's result does not depend on the member record: load both at once
     const uint2 raw = reinterpret_cast<const uint2 *>(o_t + size_t(unit) * kD)[lane];
@@ -407,6 +427,43 @@ __global__ void __launch_bounds__(256) grouped_merge_kernel(
     res.x = *reinterpret_cast<const uint32_t *>(&r01);
     res.y = *reinterpret_cast<const uint32_t *>(&r23);
     reinterpret_cast<uint2 *>(out + size_t(unit) * kD)[lane] = res;
+}
+
+// The merge runs after the tail decode (programmatic dependent launch), which
+// itself completes only after the prefix kernel.  Each CTA also checks (with
+// a bounded wait) that all tc_ctas prefix CTAs have counted themselves done
+// before it reads their partials.  Once every merge CTA is past that check,
+// the last one sets the work-list counters and flag back to zero for the
+// next call.
+__global__ void __launch_bounds__(256) grouped_merge_kernel(
+    __half *__restrict__ out, const Member *__restrict__ members, const float *__restrict__ part_ml,
+    const float *__restrict__ part_o, const __half *__restrict__ o_t, const float *__restrict__ lse_t,
+    int num_heads, int units, Meta *meta, unsigned int tc_ctas, unsigned int *err)
+{
+    pa::grid_dependency_wait();
+    pa::allow_dependent_launch();
+    if (threadIdx.x == 0) {
+        volatile unsigned int *done = &meta->tc_done;
+        bool ok = *done >= tc_ctas;
+        if (!ok) {
+            const uint64_t t0 = pa::global_timer_ns();
+            while (!(ok = *done >= tc_ctas) && pa::global_timer_ns() - t0 < pa::kWaitLimitNs)
+                __nanosleep(64);
+        }
+        if (!ok)
+            atomicOr(err, PA_DEVERR_TIMEOUT);
+        __threadfence();
+    }
+    __syncthreads();
+    const int unit = blockIdx.x * 8 + (threadIdx.x >> 5), lane = threadIdx.x & 31;
+    if (unit < units)
+        merge_unit(out, members, part_ml, part_o, o_t, lse_t, num_heads, unit, lane);
+    if (threadIdx.x == 0 && atomicAdd(&meta->merge_done, 1u) == gridDim.x - 1) {
+        meta->claimed = 0;
+        meta->tc_done = 0u;
+        meta->ready = 0u;
+        meta->merge_done = 0u;
+    }
 }
 
 // Workspace of pa_decode_grouped: work-list header, group and member
@@ -538,7 +595,13 @@ extern "C" pa_status pa_decode_grouped(void *out, const void *q, const void *k_c
     __half *o_t = reinterpret_cast<__half *>(ws + w.o_t);
     float *lse_t = reinterpret_cast<float *>(ws + w.lse_t);
 
-    // 1. the prefix work list and the tails
+    // With at most 32 groups the prefix kernel builds its own work list and
+    // starts without waiting for the set-up kernel, so it streams while the
+    // set-up kernel works out the tails; the tail decode then waits for the
+    // set-up kernel's `ready` flag instead.  Otherwise the prefix kernel runs
+    // on the set-up kernel's list, after it.
+    const bool self_list = num_groups <= kSelfListMaxGroups;
+
     SetupParams sp{};
     sp.group_start = group_start;
     sp.prefix_lens = prefix_lens;
@@ -551,6 +614,7 @@ extern "C" pa_status pa_decode_grouped(void *out, const void *q, const void *k_c
     sp.num_heads = num_heads;
     sp.max_blocks = max_blocks_per_seq;
     sp.max_chunks = w.max_chunks;
+    sp.self_list = self_list ? 1 : 0;
     const size_t setup_smem = setup_smem_bytes(num_groups, num_seqs, max_blocks_per_seq);
     sp.out = static_cast<__half *>(out);
     sp.meta = meta;
@@ -563,18 +627,27 @@ extern "C" pa_status pa_decode_grouped(void *out, const void *q, const void *k_c
     sp.dec_tickets = reinterpret_cast<unsigned int *>(
         ws + w.dec + pa_host::decode_ticket_offset(num_seqs, num_heads, kD));
     sp.err = err;
-    if ((setup_smem > 0 ? launch_pdl(grouped_setup_kernel<true>, dim3(1), dim3(kSetupThreads), setup_smem, s, sp)
-                        : launch_pdl(grouped_setup_kernel<false>, dim3(1), dim3(kSetupThreads), 0, s, sp)) !=
-        cudaSuccess)
-        return PA_ERR_CUDA;
+    auto launch_setup = [&]() {
+        return (setup_smem > 0
+                    ? launch_pdl(grouped_setup_kernel<true>, dim3(1), dim3(kSetupThreads), setup_smem, s, sp)
+                    : launch_pdl(grouped_setup_kernel<false>, dim3(1), dim3(kSetupThreads), 0, s, sp)) ==
+               cudaSuccess;
+    };
 
-    // 2. the shared prefixes, once per (group, head), on the tensor cores
     pa::grp::Params p{};
     p.out = static_cast<__half *>(out);
     p.block_tables = block_tables;
     p.chunks = sp.chunks;
     p.meta = meta;
     p.max_chunks = w.max_chunks;
+    if (self_list) {
+        p.group_start = group_start;
+        p.prefix_lens = prefix_lens;
+        p.context_lens = context_lens;
+        p.num_groups = num_groups;
+        p.num_seqs = num_seqs;
+        p.max_context_len = max_context_len;
+    }
     p.part_ml = part_ml;
     p.part_o = part_o;
     p.max_blocks_per_seq = max_blocks_per_seq;
@@ -583,12 +656,22 @@ extern "C" pa_status pa_decode_grouped(void *out, const void *q, const void *k_c
     p.num_blocks = num_blocks;
     p.qk_scale_log2 = float(double(scale) * 1.4426950408889634);
     p.error_word = err;
-    const int prefix_ctas = std::max(1, std::min(sms - 1, int(float(sms) * kPrefixSmShare + 0.5f)));
-    if (launch_pdl(pa::grp::grouped_decode_kernel, dim3(unsigned(prefix_ctas)),
-                   dim3(pa::grp::kThreads), pa::grp::kSmem, s, tm_q, tm_k, tm_v, p) != cudaSuccess)
+    const float share = self_list ? kSelfListSmShare : kPrefixSmShare;
+    const int prefix_ctas = std::max(1, std::min(sms - 1, int(float(sms) * share + 0.5f)));
+    auto launch_prefix = [&]() {
+        return launch_pdl(pa::grp::grouped_decode_kernel, dim3(unsigned(prefix_ctas)),
+                          dim3(pa::grp::kThreads), pa::grp::kSmem, s, tm_q, tm_k, tm_v, p) == cudaSuccess;
+    };
+
+    // 1. the tails (and the work list); 2. the shared prefixes, once per
+    // (group, head), on the tensor cores
+    if (!launch_setup() || !launch_prefix())
         return PA_ERR_CUDA;
 
-    // 3. each member's own tail, on the remaining SMs at the same time
+    // 3. each member's own tail, on the remaining SMs at the same time: it
+    // starts as soon as every prefix CTA is resident and waits for the
+    // prefix kernel only at its end (and, beside a prefix kernel on its own
+    // list, for the set-up kernel's `ready` flag first)
     static std::atomic<int> dec_per_sm[kMaxDevices];  // 0 = not configured yet
     int per_sm = dec_per_sm[dev].load(std::memory_order_acquire);
     if (per_sm == 0) {
@@ -600,17 +683,18 @@ extern "C" pa_status pa_decode_grouped(void *out, const void *q, const void *k_c
     const pa_status st = pa_host::decode_with_lse(
         o_t, q, k_cache, v_cache, tail_tables, max_blocks_per_seq, tail_lens, max_context_len,
         num_seqs, num_heads, head_dim, block_size, num_blocks, scale, ws + w.dec, w.total - w.dec, lse_t,
-        stream, per_sm * (sms - prefix_ctas), true);
+        stream, per_sm * (sms - prefix_ctas), true, self_list ? &meta->ready : nullptr);
     if (st != PA_OK)
         return st;
 
-    // 4. merge the parts
+    // 4. merge the parts, once the prefix kernel's CTAs are all done
     const int units = num_seqs * num_heads;
     return launch_pdl(grouped_merge_kernel, dim3(unsigned((units + 7) / 8)), dim3(256), 0, s,
                       static_cast<__half *>(out), static_cast<const Member *>(members),
                       static_cast<const float *>(part_ml),
                       static_cast<const float *>(part_o), static_cast<const __half *>(o_t),
-                      static_cast<const float *>(lse_t), num_heads, units) == cudaSuccess
+                      static_cast<const float *>(lse_t), num_heads, units, meta,
+                      unsigned(prefix_ctas), err) == cudaSuccess
                ? PA_OK
                : PA_ERR_CUDA;
 }

@@ -53,6 +53,7 @@
 
 #include <cuda.h>
 #include <cuda_fp16.h>
+#include <climits>
 #include <cstdint>
 
 #include "../../include/pa.h"
@@ -117,12 +118,42 @@ struct Member {
     int tail, cp, col0, stride;
 };
 
+// Work-list header at the start of the workspace.  The counters and the
+// flag are zero when a call starts: the workspace is zeroed before its first
+// use and every call's merge kernel sets them back to zero once it no longer
+// needs them.
 struct Meta {
-    int nchunks;      // prefix chunks of all groups
-    int ncols;        // partial columns they use
-    int claimed;      // work items handed out past the first gridDim.x (zeroed by the set-up)
-    int pad;
+    int nchunks;            // prefix chunks of all groups (from the set-up kernel)
+    int ncols;              // partial columns they use
+    int claimed;            // work items handed out past the first gridDim.x
+    unsigned int tc_done;   // prefix CTAs finished (their partials written)
+    unsigned int merge_done;// merge CTAs past their wait for the prefix kernel
+    unsigned int ready;     // the set-up kernel's outputs are all visible
+    int pad0, pad1;
 };
+
+// What a group contributes, by the same rules wherever it is worked out (the
+// set-up kernel, or the prefix kernel itself when it builds its own work
+// list): members g0 .. g0+n-1 when 0 <= g0 <= g1 <= B (else none); the prefix
+// P when it is a multiple of the block size and at most every member's
+// context (else 0); ceil(P / 512) chunks per slice of up to 16 members.
+struct GroupPlan {
+    int g0, n, P, cp, slices;
+    bool bounds_ok, prefix_ok;
+};
+
+__host__ __device__ __forceinline__ GroupPlan plan_group(int g0, int g1, int P, int min_len, int B, int bs)
+{
+    GroupPlan r{};
+    r.bounds_ok = 0 <= g0 && g0 <= g1 && g1 <= B;
+    r.n = r.bounds_ok ? g1 - g0 : 0;
+    r.g0 = r.bounds_ok ? g0 : 0;
+    r.prefix_ok = r.n > 0 && P >= 0 && P % bs == 0 && P <= min_len;
+    r.P = r.prefix_ok ? P : 0;
+    r.cp = (r.P + kChunk - 1) / kChunk;
+    r.slices = (r.n + 15) / 16;
+    return r;
+}
 
 struct Params {
     __half *out;                      // [B, H, D]
@@ -130,6 +161,14 @@ struct Params {
     const Chunk *chunks;              // capacity max_chunks
     Meta *meta;
     int max_chunks;
+    // Set (at most 32 groups): the kernel builds its own work list from these
+    // inputs instead of reading the set-up kernel's `chunks`, and so does not
+    // wait for that kernel (which was launched before it and let it start
+    // only after its own wait for the inputs).
+    const int32_t *group_start;       // [G + 1]
+    const int32_t *prefix_lens;       // [G]
+    const int32_t *context_lens;      // [B]
+    int num_groups, num_seqs, max_context_len;
     float *part_ml;                   // [columns, H, 2]: (reference max, sum)
     float *part_o;                    // [columns, H, D]
     int max_blocks_per_seq;
@@ -289,10 +328,68 @@ __device__ __forceinline__ void load_role(const CUtensorMap *tm_q, const CUtenso
         last_q[i] = -1;
     // the descriptor of item k (a broadcast load), or an empty one past the
     // work-list capacity
+    // Self-built work list: lane g holds group g's plan and the exclusive
+    // prefix sums of the groups' chunk and column counts.
+    const bool self_list = p.group_start != nullptr;
+    int sg0 = 0, sn = 0, sP = 0, sslices = 0, scount = 0, spstart = 0, scolbase = 0;
+    int self_chunks = 0, self_cols = 0;
+    if (self_list) {
+        const int G = p.num_groups, B = p.num_seqs;
+        if (lane < G) {
+            const int g0 = p.group_start[lane], g1 = p.group_start[lane + 1], P = p.prefix_lens[lane];
+            int min_len = INT_MAX;
+            if (0 <= g0 && g0 <= g1 && g1 <= B)
+                for (int b = g0; b < g1; ++b) {
+                    const int L = p.context_lens[b];
+                    min_len = min(min_len, L < 0 ? 0 : (L > p.max_context_len ? p.max_context_len : L));
+                }
+            const GroupPlan gp = plan_group(g0, g1, P, min_len, B, bs);
+            sg0 = gp.g0;
+            sn = gp.n;
+            sP = gp.P;
+            sslices = gp.slices;
+            scount = gp.slices * gp.cp;
+            scolbase = gp.n * gp.cp;
+        }
+        int xp = scount, xc = scolbase;
+#pragma unroll
+        for (int off = 1; off < 32; off <<= 1) {
+            const int yp = __shfl_up_sync(kFullMask, xp, off), yc = __shfl_up_sync(kFullMask, xc, off);
+            if (lane >= off) {
+                xp += yp;
+                xc += yc;
+            }
+        }
+        self_chunks = __shfl_sync(kFullMask, xp, 31);
+        self_cols = __shfl_sync(kFullMask, xc, 31);
+        spstart = xp - scount;
+        scolbase = xc - scolbase;
+        if (self_chunks > p.max_chunks || self_cols > p.max_chunks) {  // not with the host's bound
+            if (lane == 0)
+                atomicOr(err, PA_DEVERR_CONTEXT_LEN);
+            self_chunks = 0;
+        }
+    }
+    // the descriptor of item k (all lanes, k uniform): from the self-built
+    // list, or a broadcast load of the set-up kernel's (an empty one past the
+    // work-list capacity)
     auto descriptor = [&](int k) {
         Chunk c{};
-        if (k >= 0 && k / H < p.max_chunks)
+        if (self_list) {
+            const int ci = k / H;
+            const unsigned mask = __ballot_sync(kFullMask, scount > 0 && spstart <= ci);
+            if (k >= 0 && mask != 0u) {
+                const int g = 31 - __clz(int(mask));
+                const int g0 = __shfl_sync(kFullMask, sg0, g), n = __shfl_sync(kFullMask, sn, g);
+                const int P = __shfl_sync(kFullMask, sP, g), sl = __shfl_sync(kFullMask, sslices, g);
+                const int ps = __shfl_sync(kFullMask, spstart, g), cb = __shfl_sync(kFullMask, scolbase, g);
+                const int idx = ci - ps, j = idx / sl, sli = idx - j * sl;
+                c = Chunk{g0, g0 + 16 * sli, min(16, n - 16 * sli), j * kChunk, min((j + 1) * kChunk, P), g,
+                          cb + j * n + 16 * sli, 0};
+            }
+        } else if (k >= 0 && k / H < p.max_chunks) {
             c = p.chunks[k / H];
+        }
         return c;
     };
     // the next item index: one atomic by lane 0, not waited for here
@@ -345,7 +442,7 @@ __device__ __forceinline__ void load_role(const CUtensorMap *tm_q, const CUtenso
     // item 0 of this CTA: its descriptor and the item count come in together
     int kk = int(blockIdx.x);
     Chunk c = descriptor(kk);
-    const int total = p.meta->nchunks * H;
+    const int total = (self_list ? self_chunks : p.meta->nchunks) * H;
     if (kk >= total)
         kk = -1;
     int kn = -1, kclaim = 0;  // the next item; the claim after it (lane 0)
@@ -782,6 +879,8 @@ __device__ __forceinline__ void epilogue_role(const Params &p, Shared &sh, int l
             reinterpret_cast<float2 *>(p.part_ml)[size_t(c.col + q) * H + h] = make_float2(m_q, l_q);
         }
     }
+    // the partials are visible device-wide before the CTA counts itself done
+    __threadfence();
 }
 
 __global__ void __launch_bounds__(kThreads, 1)
@@ -829,8 +928,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     __syncthreads();
     tc_fence_after_sync();
 
-    // the work list comes from the set-up kernel that precedes this one
-    grid_dependency_wait();
+    // the work list comes from the set-up kernel that precedes this one,
+    // unless the kernel builds its own
+    if (p.group_start == nullptr)
+        grid_dependency_wait();
     allow_dependent_launch();
 
     if (warp == kLoadWarp) {
@@ -847,6 +948,10 @@ __global__ void __launch_bounds__(kThreads, 1)
 
     tc_fence_before_sync();
     __syncthreads();
+    if (tid == 0) {  // this CTA's partials are all written (the merge waits for every CTA)
+        __threadfence();
+        atomicAdd(&p.meta->tc_done, 1u);
+    }
     if (warp == kMmaWarp) {
         tc_fence_after_sync();
         tmem_free(sh.tmem, kTmemCols);

@@ -26,7 +26,8 @@ pa_status decode_with_lse(void *out, const void *q, const void *k_cache, const v
                           const int32_t *context_lens, int max_context_len, int num_seqs,
                           int num_heads, int head_dim, int block_size, int num_blocks, float scale,
                           void *workspace, size_t workspace_bytes, float *lse, pa_stream_t stream,
-                          int max_ctas = 0, bool late_dep_wait = false);
+                          int max_ctas = 0, bool late_dep_wait = false,
+                          const unsigned int *ready = nullptr);
 
 // CTAs of the fp16, head-dim-128 decode kernel that fit on one SM (0 on error).
 int decode_ctas_per_sm();

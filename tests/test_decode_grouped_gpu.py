@@ -91,6 +91,37 @@ def test_grouped_equals_plain_decode(seed, sizes, prefix_blocks, max_tail, bs):
     assert binding.pa_get_last_device_error() == 0
 
 
+def test_grouped_many_groups_and_both_work_lists_on_one_workspace():
+    """More groups (40) than the prefix kernel builds a work list for by
+    itself (32): the set-up kernel's list, the set-up launched first.  Then a
+    3-group call (the prefix kernel first, on its own list) and the 40-group
+    call again on the same workspace: each call leaves the work-list counters
+    at zero for the next, whichever order it ran in."""
+    rng = np.random.default_rng(512)
+    sizes = [int(x) for x in rng.integers(1, 4, 40)]
+    prefix_blocks = [int(x) for x in rng.integers(0, 6, 40)]
+    many = _groups(512, sizes, prefix_blocks, 30, 16)
+    few = _groups(513, [5, 2, 7], [6, 3, 9], 60, 16)
+    dev = "cuda"
+    cap = max(many["q"].shape[0], few["q"].shape[0])
+    ws = binding.new_grouped_workspace(cap, 40, 4, 128, int(max(many["lens"].max(), few["lens"].max())),
+                                       max(many["tables"].shape[1], few["tables"].shape[1]))
+    for c in (many, few, many):
+        b, h, d = c["q"].shape
+        out = torch.full((b, h, d), float("nan"), dtype=torch.float16, device=dev)
+        binding.pa_decode_grouped(out, c["q"].to(dev), c["kc"].to(dev), c["vc"].to(dev),
+                                  torch.from_numpy(c["tables"]).to(dev),
+                                  torch.from_numpy(c["lens"]).to(dev), int(c["lens"].max()),
+                                  torch.from_numpy(c["gs"]).to(dev), torch.from_numpy(c["pl"]).to(dev),
+                                  c["max_group"], c["scale"], ws)
+        torch.cuda.synchronize()
+        ref = oracle.paged_decode(c["q"].numpy(), c["kc"].numpy(), c["vc"].numpy(), c["tables"],
+                                  c["lens"], c["scale"])
+        assert not torch.isnan(out).any()
+        assert max_abs_err(out, ref) <= ATOL
+    assert binding.pa_get_last_device_error() == 0
+
+
 def test_grouped_prefix_breaking_the_rules_falls_back():
     c = _groups(507, [3, 2], [4, 3], 30, 16)
     bad = c["pl"].copy()
