@@ -530,6 +530,80 @@ __device__ __forceinline__ void issue_tile(const DecodeParams &p, const DecodeEx
     }
 }
 
+// The int8 tile under the cursor, issued by the whole warp: lane 4 s + k
+// issues copy k (K codes, V codes, K (s, z), V (s, z)) of the tile's s-th
+// block run, lane 16 the q row.  A 32-row int8 tile is two block runs at
+// bs 16 (eight copies) and four at bs 8 (sixteen); one lane issuing them in
+// turn spent several hundred cycles on each, and lanes issuing side by side
+// took the int8 kernel from 80.6 to 82.6 % of the copy peak on the 13B batch
+// and from 69.8 to 73.1 % on the serving batch (same box).  Arguments are
+// the same in every lane.
+template <int D, class Sm>
+__device__ __forceinline__ void issue_tile_int8_warp(const DecodeParams &p, const DecodeExtras &x,
+                                                     const TileCursor &cur,
+                                                     const int (&ids)[DecodeShape<D, true>::kMaxIds],
+                                                     bool with_q, unsigned char *stage_buf, uint32_t bar,
+                                                     TileMeta *meta, uint64_t stream_policy, int lane)
+{
+    using Sh = DecodeShape<D, true>;
+    const int bs = p.block_size;
+    const int t0 = cur.i * Sh::kTokens;
+    const int nv = min(Sh::kTokens, cur.len - t0);
+    int nf = nv;  // the appended token's row comes from the input (append_new_row_int8)
+    if (x.new_slots && cur.i == cur.nt - 1 && x.new_slots[cur.b] >= 0)
+        nf = nv - 1;
+    const bool one = bs >= Sh::kTokens;  // the tile lies inside one block
+    const int nsub = one ? (nf > 0 ? 1 : 0) : (nf + bs - 1) / bs;
+    uint32_t total = with_q ? uint32_t(D * 2) : 0u;
+    bool bad = false;
+#pragma unroll
+    for (int s = 0; s < Sh::kMaxIds; ++s) {
+        if (s < nsub) {
+            if (unsigned(ids[s]) < unsigned(p.num_blocks))
+                total += rows_tx_bytes<D, true>(one ? nf : min(bs, nf - s * bs));
+            else
+                bad = true;  // recorded; that run's rows are not fetched
+        }
+    }
+    if (lane == 0) {
+        meta->b = cur.b;
+        meta->h = cur.h;
+        meta->i = cur.i;
+        meta->len = cur.len;
+        meta->k = cur.k;
+        if (bad)
+            raise_device_error(kErrBlockId);
+        mbar_arrive_expect_tx(bar, total);
+    }
+    __syncwarp();
+    const uint32_t dst = smem_u32(stage_buf);
+    const int s = lane >> 2, kind = lane & 3;
+    const int id = s == 0 ? ids[0] : s == 1 ? ids[1] : s == 2 ? ids[2] : ids[3];
+    if (lane < 4 * Sh::kMaxIds && s < nsub && unsigned(id) < unsigned(p.num_blocks)) {
+        const int rows = one ? nf : min(bs, nf - s * bs);
+        const size_t row0 = (size_t(id) * p.num_heads + cur.h) * bs + (one ? size_t(t0 % bs) : size_t(0));
+        const uint32_t dst_row = one ? 0u : uint32_t(s * bs);
+        fence_proxy_async_smem();
+        if (kind == 0) {
+            bulk_copy_g2s_hint(dst + dst_row * Sh::kRowBytes,
+                               static_cast<const char *>(p.k_cache) + row0 * Sh::kRowBytes,
+                               uint32_t(rows) * Sh::kRowBytes, bar, stream_policy);
+        } else if (kind == 1) {
+            bulk_copy_g2s_hint(dst + Sm::kOffV + dst_row * Sh::kRowBytes,
+                               static_cast<const char *>(p.v_cache) + row0 * Sh::kRowBytes,
+                               uint32_t(rows) * Sh::kRowBytes, bar, stream_policy);
+        } else {
+            const uint32_t pbytes = uint32_t((rows + 1) & ~1) * 8u;
+            bulk_copy_g2s(dst + (kind == 2 ? Sm::kOffKP : Sm::kOffVP) + dst_row * 8u,
+                          (kind == 2 ? p.k_params : p.v_params) + row0 * 2, pbytes, bar);
+        }
+    }
+    if (with_q && lane == 16) {
+        fence_proxy_async_smem();
+        bulk_copy_g2s(dst + Sm::kOffQ, p.q + (size_t(cur.b) * p.num_heads + cur.h) * D, D * 2, bar);
+    }
+}
+
 // Fused append, whole warp, right after the tile under the cursor was issued:
 // if it is the last tile of its unit and the sequence appends a token, put
 // the new K / V rows (position len - 1) into the stage from the new-token
@@ -828,6 +902,8 @@ __device__ __forceinline__ void paged_decode_body(const DecodeParams &p, const D
     prod.k = lo;
     const int first = min(S, ntiles);
     const uint64_t policy = l2_policy_evict_first();
+    // int8 tiles: the whole warp issues the copies (issue_tile_int8_warp)
+    constexpr bool warp_issue = kInt8;
     int ids[Sh::kMaxIds];
     {
         TileCursor mc = prod;
@@ -849,7 +925,11 @@ __device__ __forceinline__ void paged_decode_body(const DecodeParams &p, const D
 #pragma unroll
             for (int e = 0; e < Sh::kMaxIds; ++e)
                 ids_s[e] = __shfl_sync(kFullMask, ids[e], s);
-            if (lane == 0)
+            if constexpr (warp_issue && !kContig)
+                issue_tile_int8_warp<D, Sm>(p, x, cs, ids_s, cs.i == 0 || cs.k == lo,
+                                            my_buf + size_t(s) * Sm::kStageBytes, my_bar + 8 * s,
+                                            my_meta + s, policy, lane);
+            else if (lane == 0)
                 issue_tile<D, kInt8, Sm, kContig>(p, x, cs, ids_s, cs.i == 0 || cs.k == lo,
                                          my_buf + size_t(s) * Sm::kStageBytes, my_bar + 8 * s,
                                          my_meta + s, policy);
@@ -966,7 +1046,11 @@ __device__ __forceinline__ void paged_decode_body(const DecodeParams &p, const D
                                           acc, corr);
         __syncwarp();
         if (issued < ntiles) {  // refill the stage just consumed
-            if (lane == 0) {
+            if constexpr (warp_issue && !kContig) {
+                issue_tile_int8_warp<D, Sm>(p, x, prod, ids, prod.i == 0 || prod.k == lo,
+                                            my_buf + size_t(stage) * Sm::kStageBytes, my_bar + 8 * stage,
+                                            my_meta + stage, policy, lane);
+            } else if (lane == 0) {
                 fence_proxy_async_smem();
                 issue_tile<D, kInt8, Sm, kContig>(p, x, prod, ids, prod.i == 0 || prod.k == lo,
                                          my_buf + size_t(stage) * Sm::kStageBytes,
