@@ -100,3 +100,24 @@ def test_cpu_baselines_of_the_other_paths():
     line = bench.prefill_cpu_baseline(q, k, v, n, n, h, d, bs, d ** -0.5, target_s=0.05)
     assert line["unit"] == "TFLOP/s" and line["value"] > 0 and line["cores"] >= 1
     assert bench._prefill_flops([n], [n], h, d) == 4 * d * h * n * (n + 1) / 2
+    # chunked prefill (--new-tokens): the last 16 of 64 context tokens are new;
+    # token p of them attends to p + 1 cached tokens
+    m = 16
+    line = bench.prefill_cpu_baseline(q[:m], k, v, m, n, h, d, bs, d ** -0.5, target_s=0.05)
+    assert line["value"] > 0 and f"({m} new tokens)" in line["sample"]
+    assert bench._prefill_flops([n], [m], h, d) == 4 * d * h * sum(p + 1 for p in range(n - m, n))
+
+
+def test_secondary_bench_paths_parse_and_refuse_bad_combinations():
+    """The cache-write / copy-blocks / swap and chunked-prefill options parse,
+    and combinations the bench does not measure are refused before any GPU
+    work."""
+    ap_help = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--help"],
+                             capture_output=True, text=True, timeout=120)
+    assert ap_help.returncode == 0
+    for opt in ("cache-write", "copy-blocks", "swap", "--new-tokens", "--direction", "--decode-only"):
+        assert opt in ap_help.stdout
+    r = _run_bench(["--impl", "reference", "--path", "swap", "--steps", "3", "--warmup", "3"])
+    assert r.returncode != 0 and "times the decode path" in (r.stdout + r.stderr)
+    r = _run_bench(["--kv-dtype", "int8", "--workload", "4", "--steps", "3", "--warmup", "3"])
+    assert r.returncode != 0 and "int8" in (r.stdout + r.stderr)
